@@ -1,0 +1,171 @@
+"""CPU oracle for the BinaryAttention forward pass (ctypes wrapper).
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE. Only the tests, the smoke check and the
+benchmark's CPU-baseline / reference arm import this module; the GPU library
+never does, and this module imports nothing from the GPU package.
+
+The arithmetic lives in ``binattn_oracle.c`` (plain C, fp64, OpenMP over query
+rows). This file only marshals numpy arrays. See the C file's header for the
+steps and the passages of "BinaryAttention: One-Bit QK-Attention for Vision and
+Diffusion Transformers" that each step follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "binattn_oracle.c")
+LIBRARY = os.path.join(_HERE, "liboracle.so")
+
+F32 = 0
+BF16 = 1
+
+_i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+def build(source: str = SOURCE, out: str = LIBRARY, extra_flags=()) -> str:
+    """Compile the oracle with gcc (-O2, no fast-math, OpenMP). Returns the path."""
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+           *extra_flags, "-o", out, source, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _needs_build(src: str, lib: str) -> bool:
+    return (not os.path.exists(lib)) or os.path.getmtime(lib) < os.path.getmtime(src)
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+class Oracle:
+    """One loaded copy of the oracle library."""
+
+    def __init__(self, lib_path: str = LIBRARY):
+        if lib_path == LIBRARY and _needs_build(SOURCE, LIBRARY):
+            build()
+        self.path = lib_path
+        lib = ctypes.CDLL(lib_path)
+        L, I, D, V = ctypes.c_long, ctypes.c_int, ctypes.c_double, ctypes.c_void_p
+        lib.oracle_pack.argtypes = [V, I, L, L, L, L, V, V]
+        lib.oracle_scores_rows.argtypes = [V, V, I, L, L, L, L, L, _i64p, V]
+        lib.oracle_probs_rows.argtypes = [V, V, I, V, D, L, L, L, L, L, _i64p, V]
+        lib.oracle_forward_rows.argtypes = [V, V, I, V, V, D, L, L, L, L, L, _i64p, V]
+        lib.oracle_forward.argtypes = [V, V, I, V, V, D, L, L, L, L, V]
+        lib.oracle_num_threads.restype = I
+        lib.oracle_set_num_threads.argtypes = [I]
+        for f in ("oracle_pack", "oracle_scores_rows", "oracle_probs_rows",
+                  "oracle_forward_rows", "oracle_forward"):
+            getattr(lib, f).restype = I
+        self.lib = lib
+
+    # ---------------------------------------------------------------- helpers
+    @staticmethod
+    def _dtype_code(x: np.ndarray) -> int:
+        if x.dtype == np.float32:
+            return F32
+        if x.dtype == np.uint16:  # bf16 bit patterns
+            return BF16
+        raise TypeError(f"oracle takes float32 or bf16-as-uint16, got {x.dtype}")
+
+    @staticmethod
+    def _rows(rows) -> np.ndarray:
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
+        return r
+
+    def num_threads(self) -> int:
+        return int(self.lib.oracle_num_threads())
+
+    def set_num_threads(self, n: int) -> None:
+        self.lib.oracle_set_num_threads(int(n))
+
+    # -------------------------------------------------------------- functions
+    def pack(self, x: np.ndarray):
+        """Sign bits uint32 [B,H,N,ceil(d/32)] and alpha fp64 [B,H,N]."""
+        B, H, N, d = x.shape
+        W = (d + 31) // 32
+        bits = np.zeros((B, H, N, W), dtype=np.uint32)
+        alpha = np.zeros((B, H, N), dtype=np.float64)
+        x = np.ascontiguousarray(x)
+        rc = self.lib.oracle_pack(_ptr(x), self._dtype_code(x), B, H, N, d,
+                                  _ptr(bits), _ptr(alpha))
+        if rc:
+            raise RuntimeError(f"oracle_pack failed ({rc})")
+        return bits, alpha
+
+    def scores_rows(self, q: np.ndarray, k: np.ndarray, rows) -> np.ndarray:
+        """Integer scores S[r, j] for flat query-row ids rows[r] = (b*H+h)*N+i."""
+        B, H, N, d = q.shape
+        r = self._rows(rows)
+        S = np.zeros((r.size, N), dtype=np.int32)
+        q = np.ascontiguousarray(q); k = np.ascontiguousarray(k)
+        rc = self.lib.oracle_scores_rows(_ptr(q), _ptr(k), self._dtype_code(q), B, H, N, d,
+                                         r.size, r.ctypes.data_as(_i64p), _ptr(S))
+        if rc:
+            raise RuntimeError(f"oracle_scores_rows failed ({rc})")
+        return S
+
+    def scores(self, q: np.ndarray, k: np.ndarray) -> np.ndarray:
+        """All integer scores int32 [B,H,N,N]."""
+        B, H, N, _ = q.shape
+        return self.scores_rows(q, k, np.arange(B * H * N)).reshape(B, H, N, N)
+
+    def probs_rows(self, q, k, bias, softmax_scale, rows) -> np.ndarray:
+        B, H, N, d = q.shape
+        r = self._rows(rows)
+        P = np.zeros((r.size, N), dtype=np.float64)
+        q = np.ascontiguousarray(q); k = np.ascontiguousarray(k)
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16)
+        rc = self.lib.oracle_probs_rows(_ptr(q), _ptr(k), self._dtype_code(q), _ptr(b),
+                                        float(softmax_scale), B, H, N, d,
+                                        r.size, r.ctypes.data_as(_i64p), _ptr(P))
+        if rc:
+            raise RuntimeError(f"oracle_probs_rows failed ({rc})")
+        return P
+
+    def forward_rows(self, q, k, bias, v, softmax_scale, rows) -> np.ndarray:
+        """O rows (fp64, unrounded) for flat query-row ids."""
+        B, H, N, d = q.shape
+        r = self._rows(rows)
+        O = np.zeros((r.size, d), dtype=np.float64)
+        q = np.ascontiguousarray(q); k = np.ascontiguousarray(k)
+        v = np.ascontiguousarray(v, dtype=np.uint16)
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16)
+        rc = self.lib.oracle_forward_rows(_ptr(q), _ptr(k), self._dtype_code(q), _ptr(b),
+                                          _ptr(v), float(softmax_scale), B, H, N, d,
+                                          r.size, r.ctypes.data_as(_i64p), _ptr(O))
+        if rc:
+            raise RuntimeError(f"oracle_forward_rows failed ({rc})")
+        return O
+
+    def forward(self, q, k, bias, v, softmax_scale) -> np.ndarray:
+        """O fp64 [B,H,N,d] for every row."""
+        B, H, N, d = q.shape
+        O = np.zeros((B, H, N, d), dtype=np.float64)
+        q = np.ascontiguousarray(q); k = np.ascontiguousarray(k)
+        v = np.ascontiguousarray(v, dtype=np.uint16)
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16)
+        rc = self.lib.oracle_forward(_ptr(q), _ptr(k), self._dtype_code(q), _ptr(b), _ptr(v),
+                                     float(softmax_scale), B, H, N, d, _ptr(O))
+        if rc:
+            raise RuntimeError(f"oracle_forward failed ({rc})")
+        return O
+
+
+_default: Oracle | None = None
+
+
+def get() -> Oracle:
+    """The oracle built from this directory's source (compiled on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default

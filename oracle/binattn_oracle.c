@@ -1,0 +1,328 @@
+/*
+ * CPU oracle for the BinaryAttention forward pass.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE. Only the test suite, the smoke check
+ * and the benchmark's CPU-baseline / reference arm load this library. The GPU
+ * path never calls it and shares no code with it: no headers, no helpers, no
+ * tables. It is plain, slow and written to be checked against the pages by eye.
+ *
+ * Sources (cited by page title and section):
+ *   [ES] "BinaryAttention: One-Bit QK-Attention for Vision and Diffusion
+ *        Transformers", Spanish technical summary ("Resumen técnico"),
+ *        §2 Metodología.
+ *   [KO] the same title, Korean technical summary ("기술 요약"),
+ *        §2 방법론 나 (core components) and 다 (hardware-aware implementation).
+ *
+ * What is computed, for every (b, h, i) query row of an [B, H, N, d] problem:
+ *   1. sigma(x) = +1 if x >= 0 else -1                  ([ES] §2, scaled binary
+ *      representations: s_i = mu_q * sign(q_i), t_j = mu_k * sign(k_j)).
+ *      x >= 0 is evaluated on the stored value, so +0.0 and -0.0 both give +1.
+ *   2. alpha(token) = (1/d) * sum_c |x_c| over the d real channels: the scale
+ *      mu of [ES] §2, read as the per-token mean absolute value ([KO] §2 나-1
+ *      names a token-axis mean used as the scaling factor).
+ *   3. S_ij = sum_c sigma(q_ic) * sigma(k_jc): an explicit +-1 dot product
+ *      (what XNOR + popcount evaluate, [ES] §2 and [KO] §2 나-1).
+ *   4. logit_ij = softmax_scale * alpha_q_i * alpha_k_j * S_ij + bias[h, i, j]
+ *      (learnable additive bias b_ij, [ES] §2 "Mejora mediante Sesgo";
+ *      [KO] §2 나-2). The bias is not multiplied by softmax_scale; a NULL bias
+ *      means zero. The bias is shared by every batch index b.
+ *   5. P_ij = exp(logit_ij - max_j logit_ij) / sum_j exp(...) over all N keys
+ *      (ordinary softmax attention; no mask).
+ *   6. O_i = sum_j P_ij * V_j, dense, fp64 ([ES] §2 implementation follows
+ *      FlashAttention2, whose tiling gives exactly this result).
+ *
+ * All arithmetic is IEEE double. bf16 inputs are widened exactly (the 16 bits
+ * become the top half of a float). Rows are processed in parallel with OpenMP;
+ * each row's arithmetic is sequential in the order written above.
+ *
+ * Parity pins for each function live in the CPU test suite (exhaustive sign
+ * predicate, packbits layout, Hamming identity, closed forms, invariants and an
+ * independent numpy formulation on small cases).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_F32 0
+#define ORACLE_BF16 1
+
+/* Exact widening of one stored element to double. */
+static double load_elem(const void *x, int dtype, size_t idx)
+{
+    if (dtype == ORACLE_BF16) {
+        uint32_t u = ((uint32_t)((const uint16_t *)x)[idx]) << 16;
+        float f;
+        memcpy(&f, &u, sizeof f);
+        return (double)f;
+    }
+    return (double)((const float *)x)[idx];
+}
+
+/* Step 1: the sign used by the method. x >= 0 maps to +1 (so -0.0 -> +1). */
+static double sign_pm1(double x)
+{
+    return x >= 0.0 ? 1.0 : -1.0;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/*
+ * Signs and scales of every token of one [T, d] tensor (T = B*H*N):
+ * sig[t*d + c] = sigma(x[t, c]) as +-1.0 and alpha[t] = mean_c |x[t, c]|.
+ */
+static void signs_and_scales(const void *x, int dtype, size_t T, long d,
+                             double *sig, double *alpha)
+{
+    long t;
+#pragma omp parallel for schedule(static)
+    for (t = 0; t < (long)T; t++) {
+        double sum_abs = 0.0;
+        for (long c = 0; c < d; c++) {
+            double v = load_elem(x, dtype, (size_t)t * d + c);
+            if (sig)
+                sig[(size_t)t * d + c] = sign_pm1(v);
+            sum_abs += fabs(v);
+        }
+        alpha[t] = sum_abs / (double)d;
+    }
+}
+
+/*
+ * a1 + a2: sign bits and per-token scale.
+ * bits[t*W + w], W = ceil(d/32): bit (c % 32) of word (c / 32) is 1 exactly
+ * when sigma(x[t, c]) = +1. Bits for channels c >= d are 0. Built one bit at a
+ * time with shifts from the +-1 value.
+ */
+int oracle_pack(const void *x, int dtype, long B, long H, long N, long d,
+                uint32_t *bits, double *alpha)
+{
+    if (!x || !bits || !alpha || d < 1 || B < 0 || H < 0 || N < 0)
+        return 1;
+    const long W = (d + 31) / 32;
+    const size_t T = (size_t)B * H * N;
+    signs_and_scales(x, dtype, T, d, NULL, alpha);
+    long t;
+#pragma omp parallel for schedule(static)
+    for (t = 0; t < (long)T; t++) {
+        for (long w = 0; w < W; w++)
+            bits[(size_t)t * W + w] = 0u;
+        for (long c = 0; c < d; c++) {
+            double s = sign_pm1(load_elem(x, dtype, (size_t)t * d + c));
+            if (s > 0.0)
+                bits[(size_t)t * W + c / 32] |= (uint32_t)1u << (c % 32);
+        }
+    }
+    return 0;
+}
+
+/* Shared preparation for the row functions below: signs and scales of Q and K. */
+typedef struct {
+    long B, H, N, d;
+    double *sq, *sk; /* [B*H*N*d] +-1 */
+    double *aq, *ak; /* [B*H*N]      */
+} prep_t;
+
+static int prep_init(prep_t *p, const void *q, const void *k, int qk_dtype,
+                     long B, long H, long N, long d)
+{
+    size_t T = (size_t)B * H * N;
+    p->B = B; p->H = H; p->N = N; p->d = d;
+    p->sq = (double *)malloc(sizeof(double) * (T * d + 1));
+    p->sk = (double *)malloc(sizeof(double) * (T * d + 1));
+    p->aq = (double *)malloc(sizeof(double) * (T + 1));
+    p->ak = (double *)malloc(sizeof(double) * (T + 1));
+    if (!p->sq || !p->sk || !p->aq || !p->ak)
+        return 1;
+    signs_and_scales(q, qk_dtype, T, d, p->sq, p->aq);
+    signs_and_scales(k, qk_dtype, T, d, p->sk, p->ak);
+    return 0;
+}
+
+static void prep_free(prep_t *p)
+{
+    free(p->sq); free(p->sk); free(p->aq); free(p->ak);
+}
+
+/* Step 3 for one pair: explicit +-1 dot product over the d real channels. */
+static double score_pm1(const prep_t *p, size_t qtok, size_t ktok)
+{
+    double s = 0.0;
+    for (long c = 0; c < p->d; c++)
+        s += p->sq[qtok * p->d + c] * p->sk[ktok * p->d + c];
+    return s;
+}
+
+static int check_rows(long nrows, const int64_t *rows, long B, long H, long N)
+{
+    for (long r = 0; r < nrows; r++)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * H * N)
+            return 1;
+    return 0;
+}
+
+/*
+ * a3: integer scores for selected query rows. rows[r] = (b*H + h)*N + i.
+ * S_rows[r*N + j] = S_ij as int32 (each value is an exact integer in [-d, d]).
+ */
+int oracle_scores_rows(const void *q, const void *k, int qk_dtype,
+                       long B, long H, long N, long d,
+                       long nrows, const int64_t *rows, int32_t *S_rows)
+{
+    if (!q || !k || !rows || !S_rows || d < 1 || N < 1)
+        return 1;
+    if (check_rows(nrows, rows, B, H, N))
+        return 2;
+    prep_t p;
+    if (prep_init(&p, q, k, qk_dtype, B, H, N, d)) {
+        prep_free(&p);
+        return 3;
+    }
+    long r;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (r = 0; r < nrows; r++) {
+        size_t qtok = (size_t)rows[r];
+        size_t bh = qtok / (size_t)N;
+        for (long j = 0; j < N; j++) {
+            double s = score_pm1(&p, qtok, bh * (size_t)N + (size_t)j);
+            S_rows[(size_t)r * N + j] = (int32_t)s;
+        }
+    }
+    prep_free(&p);
+    return 0;
+}
+
+/* Steps 3-5 for one query row: attention probabilities P[j], j < N. */
+static void probs_row(const prep_t *p, size_t qtok, const uint16_t *bias,
+                      double softmax_scale, double *P)
+{
+    const long N = p->N, H = p->H;
+    size_t bh = qtok / (size_t)N;
+    long i = (long)(qtok % (size_t)N);
+    long h = (long)(bh % (size_t)H);
+    double aq = p->aq[qtok];
+    double m = -INFINITY;
+    for (long j = 0; j < N; j++) {
+        size_t ktok = bh * (size_t)N + (size_t)j;
+        double s = score_pm1(p, qtok, ktok);
+        double logit = softmax_scale * aq * p->ak[ktok] * s;
+        if (bias)
+            logit += load_elem(bias, ORACLE_BF16, ((size_t)h * N + i) * N + j);
+        P[j] = logit;
+        if (logit > m)
+            m = logit;
+    }
+    double z = 0.0;
+    for (long j = 0; j < N; j++) {
+        P[j] = exp(P[j] - m);
+        z += P[j];
+    }
+    for (long j = 0; j < N; j++)
+        P[j] /= z;
+}
+
+/*
+ * a5: softmax probabilities for selected rows: P_rows[r*N + j] (fp64).
+ * bias: bf16 [H, N, N] or NULL.
+ */
+int oracle_probs_rows(const void *q, const void *k, int qk_dtype,
+                      const uint16_t *bias, double softmax_scale,
+                      long B, long H, long N, long d,
+                      long nrows, const int64_t *rows, double *P_rows)
+{
+    if (!q || !k || !rows || !P_rows || d < 1 || N < 1)
+        return 1;
+    if (check_rows(nrows, rows, B, H, N))
+        return 2;
+    prep_t p;
+    if (prep_init(&p, q, k, qk_dtype, B, H, N, d)) {
+        prep_free(&p);
+        return 3;
+    }
+    long r;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (r = 0; r < nrows; r++)
+        probs_row(&p, (size_t)rows[r], bias, softmax_scale, P_rows + (size_t)r * N);
+    prep_free(&p);
+    return 0;
+}
+
+/*
+ * Steps 1-6: attention output for selected rows, O_rows[r*d + c] (fp64,
+ * unrounded). V is bf16 [B, H, N, d]; bias is bf16 [H, N, N] or NULL.
+ */
+int oracle_forward_rows(const void *q, const void *k, int qk_dtype,
+                        const uint16_t *bias, const uint16_t *v,
+                        double softmax_scale, long B, long H, long N, long d,
+                        long nrows, const int64_t *rows, double *O_rows)
+{
+    if (!q || !k || !v || !rows || !O_rows || d < 1 || N < 1)
+        return 1;
+    if (check_rows(nrows, rows, B, H, N))
+        return 2;
+    prep_t p;
+    if (prep_init(&p, q, k, qk_dtype, B, H, N, d)) {
+        prep_free(&p);
+        return 3;
+    }
+    int err = 0;
+    long r;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (r = 0; r < nrows; r++) {
+        double *P = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!P) {
+#pragma omp atomic write
+            err = 3;
+            continue;
+        }
+        size_t qtok = (size_t)rows[r];
+        size_t bh = qtok / (size_t)N;
+        probs_row(&p, qtok, bias, softmax_scale, P);
+        for (long c = 0; c < d; c++) {
+            double o = 0.0;
+            for (long j = 0; j < N; j++)
+                o += P[j] * load_elem(v, ORACLE_BF16, (bh * (size_t)N + (size_t)j) * d + c);
+            O_rows[(size_t)r * d + c] = o;
+        }
+        free(P);
+    }
+    prep_free(&p);
+    return err;
+}
+
+/* All rows: O[B, H, N, d] in fp64. */
+int oracle_forward(const void *q, const void *k, int qk_dtype,
+                   const uint16_t *bias, const uint16_t *v, double softmax_scale,
+                   long B, long H, long N, long d, double *O)
+{
+    size_t T = (size_t)B * H * N;
+    int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (T + 1));
+    if (!rows)
+        return 3;
+    for (size_t t = 0; t < T; t++)
+        rows[t] = (int64_t)t;
+    int rc = oracle_forward_rows(q, k, qk_dtype, bias, v, softmax_scale,
+                                 B, H, N, d, (long)T, rows, O);
+    free(rows);
+    return rc;
+}

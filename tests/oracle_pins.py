@@ -1,0 +1,315 @@
+"""Checks that pin the CPU oracle to facts outside itself.
+
+Each ``pin_*`` function takes a loaded ``oracle.Oracle`` and raises
+AssertionError when the oracle disagrees with what "BinaryAttention: One-Bit
+QK-Attention for Vision and Diffusion Transformers" fixes or with textbook
+mathematics: an exhaustive sign predicate, numpy's packbits layout, the
+Hamming identity behind XNOR/popcount, closed forms, invariants, special cases
+that reduce to scipy's softmax, a hand-worked example, and an independent
+matrix-form formulation on tiny inputs.
+
+They are run against the real oracle (test_oracle_pins.py) and against
+deliberately broken copies of it (test_oracle_mutants.py), where at least one
+of them must fail.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+from scipy.special import softmax as scipy_softmax
+
+from diffusion_transformers_b200.synthetic import (bf16_bits_to_f32, f32_to_bf16_bits,
+                                                  make_custom)
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _f64(x: np.ndarray) -> np.ndarray:
+    """Exact float64 view of a float32 or bf16-bits array."""
+    if x.dtype == np.uint16:
+        return bf16_bits_to_f32(x).astype(np.float64)
+    return x.astype(np.float64)
+
+
+# ----------------------------------------------------------------- a1: bits
+def pin_sign_predicate_exhaustive(orc):
+    """Every non-NaN bf16 pattern (one channel per token): bit == (x >= 0) as
+    evaluated by numpy; +0.0 and -0.0 both give 1 (sign of the stored value,
+    'sign' of the scaled binary representation)."""
+    pats = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    f = bf16_bits_to_f32(pats)
+    keep = ~np.isnan(f)
+    x = pats[keep].reshape(1, 1, -1, 1)
+    bits, _ = orc.pack(x)
+    want = (f[keep] >= np.float32(0)).astype(np.uint32)
+    assert np.array_equal(bits.reshape(-1), want), "sign predicate differs from x >= 0"
+    # the same for fp32 special values
+    specials = np.array([0.0, -0.0, 1e-45, -1e-45, 1.17e-38, -1.17e-38, np.inf, -np.inf,
+                         3.4e38, -3.4e38, 1.0, -1.0], dtype=np.float32)
+    b2, _ = orc.pack(specials.reshape(1, 1, -1, 1))
+    assert np.array_equal(b2.reshape(-1), (specials >= 0).astype(np.uint32))
+
+
+def pin_pack_layout_packbits(orc):
+    """Word c//32, bit c%32, LSB first, pad bits zero: equal to numpy's
+    little-endian packbits of (x >= 0) read back as little-endian uint32."""
+    rng = np.random.default_rng(11)
+    for d in (1, 5, 31, 32, 33, 64, 72, 96, 100, 128, 200):
+        x = rng.standard_normal((2, 3, 7, d)).astype(np.float32)
+        bits, _ = orc.pack(x)
+        W = (d + 31) // 32
+        pb = np.packbits(x >= 0, axis=-1, bitorder="little")
+        pad = np.zeros(pb.shape[:-1] + (W * 4 - pb.shape[-1],), dtype=np.uint8)
+        want = np.concatenate([pb, pad], axis=-1).copy().view("<u4")
+        assert bits.shape == (2, 3, 7, W)
+        assert np.array_equal(bits, want), f"bit layout differs at d={d}"
+
+
+# ---------------------------------------------------------------- a2: alpha
+def pin_alpha_mean_abs(orc):
+    """alpha = mean |x| over the d real channels: numpy's fp64 mean of |x|,
+    exact closed form |c| for x = c * (+-1), and exact scaling by powers of 2
+    (bits unchanged)."""
+    rng = np.random.default_rng(12)
+    for d in (1, 7, 64, 72, 128):
+        x = rng.standard_normal((2, 2, 9, d)).astype(np.float32)
+        _, a = orc.pack(x)
+        want = np.mean(np.abs(x.astype(np.float64)), axis=-1)
+        assert np.allclose(a, want, rtol=1e-14, atol=0), f"alpha != mean|x| at d={d}"
+        # closed form: x = c * s with s in {+1,-1}
+        c = rng.uniform(0.1, 4.0, size=(2, 2, 9, 1)).astype(np.float32)
+        s = np.where(rng.random((2, 2, 9, d)) < 0.5, -1.0, 1.0).astype(np.float32)
+        _, a2 = orc.pack(c * s)
+        assert np.array_equal(a2, np.broadcast_to(c[..., 0].astype(np.float64), a2.shape)), \
+            "alpha of c*(+-1) is not |c|"
+        # power-of-two scaling: alpha scales exactly, bits do not change
+        b1, a1 = orc.pack(x)
+        b4, a4 = orc.pack(x * np.float32(4.0))
+        assert np.array_equal(b1, b4) and np.array_equal(a4, 4.0 * a1)
+    # bf16 storage path gives the same as the exactly widened fp32 values
+    xb = f32_to_bf16_bits(rng.standard_normal((1, 2, 5, 72)).astype(np.float32))
+    _, ab = orc.pack(xb)
+    _, af = orc.pack(bf16_bits_to_f32(xb))
+    assert np.array_equal(ab, af)
+
+
+# --------------------------------------------------------------- a3: scores
+def pin_hamming_identity_exhaustive(orc):
+    """<sign q, sign k> = d - 2 * Hamming(q, k) (XNOR/popcount similarity) for
+    every pair of sign vectors at d = 1..10."""
+    for d in range(1, 11):
+        n = 1 << d
+        idx = np.arange(n)
+        signs = np.where((idx[:, None] >> np.arange(d)[None, :]) & 1, 1.0, -1.0)
+        x = signs.astype(np.float32).reshape(1, 1, n, d)
+        S = orc.scores(x, x)[0, 0].astype(np.int64)
+        ham = np.array([[bin(a ^ b).count("1") for b in range(n)] for a in range(n)]) \
+            if d <= 6 else _popcount_table(idx[:, None] ^ idx[None, :])
+        assert np.array_equal(S, d - 2 * ham), f"Hamming identity fails at d={d}"
+
+
+def _popcount_table(z: np.ndarray) -> np.ndarray:
+    z = z.astype(np.uint32)
+    return np.unpackbits(z.view(np.uint8).reshape(z.shape + (4,)), axis=-1).sum(-1).astype(np.int64)
+
+
+def pin_scores_matmul(orc):
+    """S equals an int64 matrix product of the +-1 sign matrices (numpy), per
+    (b, h), for several d including padded ones."""
+    rng = np.random.default_rng(13)
+    for d in (33, 64, 72, 128):
+        q = f32_to_bf16_bits(rng.standard_normal((2, 3, 17, d)).astype(np.float32))
+        k = f32_to_bf16_bits(rng.standard_normal((2, 3, 17, d)).astype(np.float32))
+        S = orc.scores(q, k).astype(np.int64)
+        sq = np.where(_f64(q) >= 0, 1, -1).astype(np.int64)
+        sk = np.where(_f64(k) >= 0, 1, -1).astype(np.int64)
+        want = np.einsum("bhic,bhjc->bhij", sq, sk)
+        assert np.array_equal(S, want), f"scores differ from +-1 matmul at d={d}"
+
+
+def pin_scores_special_cases(orc):
+    """All-equal signs give S == d; K = -Q (no zeros) gives S_ii = -d; negating
+    Q negates S; +0.0 and -0.0 both count as +1."""
+    rng = np.random.default_rng(14)
+    d = 72
+    pos = np.abs(rng.standard_normal((1, 2, 9, d))).astype(np.float32) + 0.1
+    S = orc.scores(pos, pos * np.float32(3.0))
+    assert np.all(S == d)
+    q = rng.standard_normal((1, 2, 9, d)).astype(np.float32)
+    q[q == 0] = 1.0
+    S2 = orc.scores(q, -q)
+    assert np.all(np.diagonal(S2, axis1=2, axis2=3) == -d)
+    k = rng.standard_normal((1, 2, 9, d)).astype(np.float32)
+    k[k == 0] = 1.0
+    assert np.array_equal(orc.scores(-q, k), -orc.scores(q, k))
+    z = np.zeros((1, 1, 2, d), dtype=np.float32)
+    z[0, 0, 1] = -0.0
+    assert np.all(orc.scores(z, np.ones_like(z)) == d)
+
+
+# -------------------------------------------------------------- a4/a5: softmax
+def pin_softmax_rows_sum_to_one(orc):
+    c = make_custom(2, 3, 37, 72, seed=15, bias_std=0.5)
+    rows = np.arange(2 * 3 * 37)
+    P = orc.probs_rows(c["q"], c["k"], c["bias"], c["softmax_scale"], rows)
+    assert np.all(P >= 0)
+    assert np.allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+
+
+def pin_softmax_bias_only(orc):
+    """softmax_scale = 0 leaves only the bias: each row of P is scipy's softmax
+    of bias[h, i, :], the same for every b (bias broadcast over the batch)."""
+    B, H, N = 2, 3, 23
+    c = make_custom(B, H, N, 40, seed=16, bias_std=1.0)
+    rows = np.arange(B * H * N)
+    P = orc.probs_rows(c["q"], c["k"], c["bias"], 0.0, rows).reshape(B, H, N, N)
+    bias = _f64(c["bias"])
+    want = scipy_softmax(bias, axis=-1)
+    for b in range(B):
+        assert np.allclose(P[b], want, rtol=1e-12, atol=1e-15), "P != softmax(bias)"
+
+
+def pin_softmax_shift_invariance(orc):
+    """Adding a per-row constant to the logits (through the bias, exactly
+    representable in bf16) leaves P unchanged."""
+    B, H, N, d = 1, 2, 19, 64
+    c = make_custom(B, H, N, d, seed=17, with_bias=False)
+    rng = np.random.default_rng(18)
+    k8 = rng.integers(-16, 17, size=(H, N, N)).astype(np.float32) / 8.0
+    shift = (np.arange(N) % 4).astype(np.float32)[None, :, None] * 8.0
+    b0 = f32_to_bf16_bits(k8)
+    b1 = f32_to_bf16_bits(k8 + shift)
+    assert np.array_equal(_f64(b1) - _f64(b0), np.broadcast_to(shift, (H, N, N)).astype(np.float64))
+    rows = np.arange(B * H * N)
+    P0 = orc.probs_rows(c["q"], c["k"], b0, c["softmax_scale"], rows)
+    P1 = orc.probs_rows(c["q"], c["k"], b1, c["softmax_scale"], rows)
+    assert np.allclose(P0, P1, rtol=1e-12, atol=1e-15)
+
+
+def pin_scale_invariances(orc):
+    """Scaling Q (or K) by 2 multiplies alpha_q (alpha_k) by 2 and leaves the
+    signs alone, so halving softmax_scale gives the same O; the bias is not
+    scaled, so this holds with a bias present."""
+    c = make_custom(2, 2, 21, 72, seed=19, qk_dtype="f32", bias_std=0.3)
+    rows = np.arange(2 * 2 * 21)
+    s = c["softmax_scale"] * 4.0
+    O = orc.forward_rows(c["q"], c["k"], c["bias"], c["v"], s, rows)
+    Oq = orc.forward_rows(c["q"] * np.float32(2), c["k"], c["bias"], c["v"], s / 2, rows)
+    Ok = orc.forward_rows(c["q"], c["k"] * np.float32(2), c["bias"], c["v"], s / 2, rows)
+    assert np.allclose(O, Oq, rtol=1e-12, atol=1e-13), "alpha_q does not enter the logit"
+    assert np.allclose(O, Ok, rtol=1e-12, atol=1e-13), "alpha_k does not enter the logit"
+    # and the logits do depend on the scale (guards against a constant result)
+    O2 = orc.forward_rows(c["q"], c["k"], c["bias"], c["v"], s * 3, rows)
+    assert not np.allclose(O, O2, rtol=1e-6, atol=1e-8)
+
+
+# ------------------------------------------------------------ a6: P.V and O
+def pin_uniform_scores_mean_v(orc):
+    """Every key row identical within a head (different across heads) and no
+    bias: scores are constant along j, P is uniform, and O_i = mean_j V_j."""
+    B, H, N, d = 2, 3, 13, 72
+    rng = np.random.default_rng(20)
+    q = rng.standard_normal((B, H, N, d)).astype(np.float32)
+    krow = rng.standard_normal((B, H, 1, d)).astype(np.float32)
+    k = np.ascontiguousarray(np.broadcast_to(krow, (B, H, N, d)))
+    v = f32_to_bf16_bits(rng.standard_normal((B, H, N, d)).astype(np.float32))
+    O = orc.forward(q, k, None, v, 0.7)
+    want = np.broadcast_to(_f64(v).mean(axis=2, keepdims=True), O.shape)
+    assert np.allclose(O, want, rtol=1e-12, atol=1e-14)
+
+
+def pin_onehot_bias_gather(orc):
+    """softmax_scale = 0 and bias[h, i, pi(i)] = 40 (others 0): P puts all but
+    (N-1)e^-40 of its mass on key pi(i), so O_i = V[pi(i)] (a permutation
+    gather, different per head and batch index)."""
+    B, H, N, d = 2, 2, 11, 33
+    rng = np.random.default_rng(21)
+    c = make_custom(B, H, N, d, seed=22, with_bias=False)
+    bias = np.zeros((H, N, N), dtype=np.float32)
+    perms = [rng.permutation(N) for _ in range(H)]
+    for h in range(H):
+        bias[h, np.arange(N), perms[h]] = 40.0
+    O = orc.forward(c["q"], c["k"], f32_to_bf16_bits(bias), c["v"], 0.0)
+    v = _f64(c["v"])
+    tol = N * math.exp(-40) * np.abs(v).max() * 2
+    for b in range(B):
+        for h in range(H):
+            assert np.allclose(O[b, h], v[b, h, perms[h]], rtol=0, atol=tol)
+
+
+def pin_convex_hull(orc):
+    """Each O_i[c] lies between min_j V_jc and max_j V_jc (P is a probability
+    vector)."""
+    c = make_custom(2, 2, 31, 72, seed=23, bias_std=1.0)
+    O = orc.forward(c["q"], c["k"], c["bias"], c["v"], c["softmax_scale"])
+    v = _f64(c["v"])
+    lo = v.min(axis=2, keepdims=True) - 1e-12
+    hi = v.max(axis=2, keepdims=True) + 1e-12
+    assert np.all(O >= lo) and np.all(O <= hi)
+
+
+def pin_bruteforce_matrix_form(orc):
+    """Tiny cases (N <= 8) against a second, matrix-form fp64 formulation:
+    S = sign(Q) sign(K)^T, L = scale * a_q a_k^T * S + bias, P = scipy softmax,
+    O = P V."""
+    rng = np.random.default_rng(24)
+    for (B, H, N, d) in [(1, 1, 1, 1), (2, 2, 3, 5), (1, 3, 8, 72), (2, 1, 8, 33), (1, 2, 7, 64)]:
+        for with_bias in (False, True):
+            c = make_custom(B, H, N, d, seed=int(rng.integers(1 << 30)), qk_dtype="bf16",
+                            with_bias=with_bias, bias_std=0.7, zeros_frac=0.1)
+            q, k, v = _f64(c["q"]), _f64(c["k"]), _f64(c["v"])
+            sq, sk = np.where(q >= 0, 1.0, -1.0), np.where(k >= 0, 1.0, -1.0)
+            aq, ak = np.abs(q).mean(-1), np.abs(k).mean(-1)
+            S = sq @ np.swapaxes(sk, -1, -2)
+            L = c["softmax_scale"] * aq[..., :, None] * ak[..., None, :] * S
+            if with_bias:
+                L = L + _f64(c["bias"])[None]
+            want = scipy_softmax(L, axis=-1) @ v
+            O = orc.forward(c["q"], c["k"], c["bias"], c["v"], c["softmax_scale"])
+            assert np.allclose(O, want, rtol=1e-12, atol=1e-14), f"brute force fails at {B,H,N,d}"
+
+
+def pin_worked_example(orc):
+    """Hand-worked example (tests/golden/worked_example.json): sign bits,
+    alphas, integer scores and logits derived by hand as rationals; O from the
+    closed-form two-key softmax."""
+    with open(os.path.join(GOLDEN, "worked_example.json")) as f:
+        g = json.load(f)
+    q = np.array(g["Q"], dtype=np.float32).reshape(1, 1, 2, 3)
+    k = np.array(g["K"], dtype=np.float32).reshape(1, 1, 2, 3)
+    v = f32_to_bf16_bits(np.array(g["V"], dtype=np.float32).reshape(1, 1, 2, 3))
+    bias = f32_to_bf16_bits(np.array(g["bias"], dtype=np.float32).reshape(1, 2, 2))
+    bits, aq = orc.pack(q)
+    assert bits.reshape(-1).tolist() == g["q_bits"]
+    assert np.allclose(aq.reshape(-1), [eval(a) for a in g["alpha_q"]], rtol=1e-15)
+    S = orc.scores(q, k)[0, 0]
+    assert S.tolist() == g["S"]
+    logits = np.array([[eval(x) for x in row] for row in g["logits"]])
+    # two keys: P_i0 = 1 / (1 + exp(l_i1 - l_i0))
+    p0 = 1.0 / (1.0 + np.exp(logits[:, 1] - logits[:, 0]))
+    V = np.array(g["V"], dtype=np.float64)
+    want = p0[:, None] * V[0][None, :] + (1 - p0)[:, None] * V[1][None, :]
+    O = orc.forward(q, k, bias, v, g["softmax_scale"])[0, 0]
+    assert np.allclose(O, want, rtol=1e-14, atol=1e-15)
+
+
+ALL_PINS = [
+    pin_sign_predicate_exhaustive,
+    pin_pack_layout_packbits,
+    pin_alpha_mean_abs,
+    pin_hamming_identity_exhaustive,
+    pin_scores_matmul,
+    pin_scores_special_cases,
+    pin_softmax_rows_sum_to_one,
+    pin_softmax_bias_only,
+    pin_softmax_shift_invariance,
+    pin_scale_invariances,
+    pin_uniform_scores_mean_v,
+    pin_onehot_bias_gather,
+    pin_convex_hull,
+    pin_bruteforce_matrix_form,
+    pin_worked_example,
+]

@@ -1,0 +1,73 @@
+"""Pins are strong enough: each plausible mistake, planted in a temporary copy
+of the CPU oracle, is caught by at least one pin (no GPU).
+
+Every mutant is a one-line textual change of ``oracle/binattn_oracle.c``
+compiled into a temporary directory. The committed oracle is never modified.
+"""
+import os
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS
+
+MUTANTS = [
+    ("sign(0) = -1",
+     "return x >= 0.0 ? 1.0 : -1.0;", "return x > 0.0 ? 1.0 : -1.0;"),
+    ("signed mean instead of mean |x|",
+     "sum_abs += fabs(v);", "sum_abs += v;"),
+    ("alpha divided by the padded width",
+     "alpha[t] = sum_abs / (double)d;", "alpha[t] = sum_abs / (double)(((d + 31) / 32) * 32);"),
+    ("bit order MSB first",
+     "|= (uint32_t)1u << (c % 32);", "|= (uint32_t)1u << (31 - c % 32);"),
+    ("score sign flipped",
+     "s += p->sq[qtok * p->d + c] * p->sk[ktok * p->d + c];",
+     "s -= p->sq[qtok * p->d + c] * p->sk[ktok * p->d + c];"),
+    ("first channel dropped from the score",
+     "for (long c = 0; c < p->d; c++)", "for (long c = 1; c < p->d; c++)"),
+    ("scores always against head 0",
+     "double s = score_pm1(&p, qtok, bh * (size_t)N + (size_t)j);",
+     "double s = score_pm1(&p, qtok, (size_t)j);"),
+    ("alpha_k dropped",
+     "double logit = softmax_scale * aq * p->ak[ktok] * s;",
+     "double logit = softmax_scale * aq * s;"),
+    ("alpha_q dropped",
+     "double logit = softmax_scale * aq * p->ak[ktok] * s;",
+     "double logit = softmax_scale * p->ak[ktok] * s;"),
+    ("bias scaled by softmax_scale",
+     "logit += load_elem(bias, ORACLE_BF16, ((size_t)h * N + i) * N + j);",
+     "logit += softmax_scale * load_elem(bias, ORACLE_BF16, ((size_t)h * N + i) * N + j);"),
+    ("bias transposed",
+     "((size_t)h * N + i) * N + j", "((size_t)h * N + j) * N + i"),
+    ("bias head index ignored",
+     "long h = (long)(bh % (size_t)H);", "long h = 0;"),
+    ("keys of the wrong head in the softmax",
+     "size_t ktok = bh * (size_t)N + (size_t)j;", "size_t ktok = (size_t)j;"),
+    ("exp of the negated logit",
+     "P[j] = exp(P[j] - m);", "P[j] = exp(m - P[j]);"),
+    ("softmax not normalised",
+     "P[j] /= z;", "P[j] /= 1.0;"),
+    ("V indexed by the query row",
+     "o += P[j] * load_elem(v, ORACLE_BF16, (bh * (size_t)N + (size_t)j) * d + c);",
+     "o += P[j] * load_elem(v, ORACLE_BF16, qtok * d + c);"),
+    ("last key dropped from P.V",
+     "for (long j = 0; j < N; j++)\n                o +=", "for (long j = 0; j < N - 1; j++)\n                o +="),
+]
+
+
+@pytest.mark.parametrize("name,find,repl", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, name, find, repl):
+    src = open(oracle.SOURCE).read()
+    assert src.count(find) == 1, f"mutation site not unique: {find!r}"
+    mut_src = tmp_path / "mutant.c"
+    mut_src.write_text(src.replace(find, repl))
+    lib = oracle.build(str(mut_src), str(tmp_path / "libmutant.so"))
+    orc = oracle.Oracle(lib)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(orc)
+        except AssertionError:
+            caught.append(pin.__name__)
+            break
+    assert caught, f"no pin catches the mutant '{name}'"
