@@ -1,0 +1,384 @@
+"""Benchmark of the BinaryAttention forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {binattn,reference}]
+                    [--workload dit_xl_1024] [--engine auto|tc|popc_tc|simt]
+
+One step = the whole hot path over one batch: binattn_pack(Q), binattn_pack(K)
+and binattn_forward, on DiT-XL/2 @1024px-shaped synthetic inputs (B=2, H=16,
+N=4096, d=72) with the dense bf16 bias [16, 4096, 4096] resident on the device.
+The same step without the bias is timed as well and reported under "no_bias".
+
+Timing: W untimed warm-up steps (plus about a second of untimed steps, during
+which clocks are sampled), then K steps, each between a pair of CUDA events on
+the launching stream, with a 256 MiB write between steps so that L2 (126 MB)
+starts cold for every step. Barrier + synchronize bracket the timed region; the
+step time is the max over ranks. With N > 1 every rank runs its own batch
+(weak scaling, no collective on the data path).
+
+`--impl reference` times the CPU oracle (the reference implementation of this
+path) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from diffusion_transformers_b200.synthetic import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "BinaryAttention fwd ms & effective TFLOPS at DiT-XL N=4096; % of roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="binattn", choices=["binattn", "reference"])
+    ap.add_argument("--workload", default="dit_xl_1024", choices=sorted(WORKLOADS))
+    ap.add_argument("--engine", default="auto")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the bounded oracle sample")
+    return ap.parse_args()
+
+
+def workload_config(w, with_bias=True):
+    return {
+        "workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d}, bf16 Q/K/V, "
+                    + (f"dense bf16 bias [{w.H},{w.N},{w.N}]" if with_bias else "no bias"),
+        "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bias": with_bias,
+        "step": "pack(Q) + pack(K) + forward",
+        "l2": "flushed between timed steps (256 MiB write)",
+    }
+
+
+def algorithmic(w, with_bias=True):
+    """Per-launch algorithmic work of the forward kernel (one (b,h,i,j) pair =
+    2d binary ops for QK, 2d flops for P.V)."""
+    BH, N, d = w.B * w.H, w.N, w.d
+    pairs = BH * N * N
+    W = (d + 31) // 32
+    bytes_ = (2 * BH * N * W * 4          # q_bits, k_bits
+              + 2 * BH * N * 4            # alpha_q, alpha_k
+              + 2 * BH * N * d * 2        # V read, O written
+              + (w.H * N * N * 2 if with_bias else 0))  # bias, once
+    pack_bytes = 2 * (BH * N * d * 2 + BH * N * W * 4 + BH * N * 4)
+    return dict(pairs=pairs, qk_ops=2 * d * pairs, pv_flops=2 * d * pairs,
+                eff_flops=4 * d * pairs, bytes=bytes_, pack_bytes=pack_bytes)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"],
+                    bf16_tflops_sustained=p.get("bf16_tflops_sustained"), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.proc, self.lines = index, None, []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), util=float(parts[4]),
+                                 reasons=[n for n, v in zip(
+                                     ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                      "sw_power_cap"), parts[5:9]) if v.lower() == "active"]))
+            except ValueError:
+                continue
+        loaded = [r for r in rows if r["util"] > 0] or rows
+        if not loaded:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted({x for r in loaded for x in r["reasons"]})
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["smax"] for r in loaded), "reasons": reasons,
+                "samples": len(loaded)}
+
+
+# ------------------------------------------------------------ oracle (CPU)
+def cpu_oracle_sample(w, with_bias, target_s, inp=None):
+    """Time the oracle on a bounded sample of query rows of the workload and
+    extrapolate linearly to one whole step (pack is part of the oracle's prep)."""
+    import oracle
+    orc = oracle.get()
+    if inp is None:
+        inp = make_inputs(w, with_bias=with_bias)
+    T = w.B * w.H * w.N
+    rng = np.random.default_rng(123)
+    n = 64
+    t0 = time.perf_counter()
+    orc.forward_rows(inp["q"], inp["k"], inp["bias"] if with_bias else None, inp["v"],
+                     inp["softmax_scale"], rng.integers(0, T, size=n))
+    t1 = time.perf_counter() - t0
+    n2 = int(min(T, max(n, n * target_s / max(t1, 1e-3))))
+    rows = rng.integers(0, T, size=n2)
+    t0 = time.perf_counter()
+    orc.forward_rows(inp["q"], inp["k"], inp["bias"] if with_bias else None, inp["v"],
+                     inp["softmax_scale"], rows)
+    dt = time.perf_counter() - t0
+    ms = dt * 1e3 * T / n2
+    return dict(value=ms, unit="ms", cores=orc.num_threads(), kind="oracle",
+                sample=f"{n2} of {T} query rows (signs/scales of all tokens + those rows' "
+                       f"scores, softmax and P.V), {dt:.1f} s, extrapolated linearly to all rows")
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    base = cpu_oracle_sample(w, True, args.cpu_seconds)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": base["value"], "unit": "ms",
+        "n_gpus": args.gpus, "steps": 1, "warmup": 0, "ms_per_step": base["value"],
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, True),
+        "cpu_baseline": base,
+        "e2e": {"value": base["value"], "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- GPU
+def run_gpu(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from diffusion_transformers_b200 import binattn
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    peaks = measured_peaks()
+
+    inp = make_inputs(w, with_bias=True, seed=w.seed + 1000 * rank)
+
+    def to_dev(x):
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(x).to(dev)
+
+    q, k, v, bias = to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"]), to_dev(inp["bias"])
+    scale = inp["softmax_scale"]
+    B, H, N, d = w.B, w.H, w.N, w.d
+    W = (d + 31) // 32
+    qb = torch.empty((B, H, N, W), dtype=torch.int32, device=dev)
+    kb = torch.empty_like(qb)
+    aq = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    ak = torch.empty_like(aq)
+    out = torch.empty_like(v)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def step(b):
+        binattn.pack(q, qb, aq, stream)
+        binattn.pack(k, kb, ak, stream)
+        binattn.forward(qb, kb, aq, ak, b, v, scale, out=out, engine=args.engine, stream=stream)
+
+    def timed(b, steps, fwd_only_events=None):
+        """Per-step events; returns (step_ms list, forward_ms list)."""
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for e0, e1, e2 in ev:
+            flush.fill_(1)
+            e0.record(stream)
+            binattn.pack(q, qb, aq, stream)
+            binattn.pack(k, kb, ak, stream)
+            e1.record(stream)
+            binattn.forward(qb, kb, aq, ak, b, v, scale, out=out, engine=args.engine, stream=stream)
+            e2.record(stream)
+        torch.cuda.synchronize()
+        return ([e0.elapsed_time(e2) for e0, _, e2 in ev], [e1.elapsed_time(e2) for _, e1, e2 in ev])
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up (untimed), including one checked run
+    for _ in range(max(args.warmup, 3)):
+        step(bias)
+    binattn.device_status(stream)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    t_end = time.time() + 1.0
+    while time.time() < t_end:  # clock soak, untimed
+        for _ in range(20):
+            flush.fill_(1)
+            step(bias)
+        torch.cuda.synchronize()
+
+    results = {}
+    for name, b in (("bias", bias), ("no_bias", None)):
+        barrier()
+        step_ms, fwd_ms = timed(b, args.steps)
+        barrier()
+        results[name] = dict(step_ms=max_over_ranks(sum(step_ms) / len(step_ms)),
+                             fwd_ms=max_over_ranks(sum(fwd_ms) / len(fwd_ms)),
+                             fwd_ms_median=statistics.median(fwd_ms),
+                             fwd_ms_min=min(fwd_ms))
+    clocks = sampler.stop()
+    binattn.device_status(stream)
+
+    # in-build bf16 attention on the same shapes (speed reference)
+    ref = None
+    try:
+        binattn.ref_bf16_forward(q, k, bias, v, scale, out=out, stream=stream)
+        torch.cuda.synchronize()
+        ev = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            binattn.ref_bf16_forward(q, k, bias, v, scale, out=out, stream=stream)
+            e1.record(stream)
+            ev.append((e0, e1))
+        torch.cuda.synchronize()
+        ref = {"forward_ms": max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / len(ev))}
+    except Exception as exc:  # not built for this engine/shape
+        ref = {"unavailable": str(exc).splitlines()[0]}
+
+    # end to end through the public API: pinned host inputs -> device -> result back
+    h_q = torch.from_numpy(inp["q"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_k = torch.from_numpy(inp["k"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_v = torch.from_numpy(inp["v"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_o = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        q.copy_(h_q, non_blocking=True)
+        k.copy_(h_k, non_blocking=True)
+        v.copy_(h_v, non_blocking=True)
+        step(bias)
+        h_o.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+
+    if rank != 0:
+        return
+    a = algorithmic(w, True)
+    a0 = algorithmic(w, False)
+    fwd_s = results["bias"]["fwd_ms"] * 1e-3
+    eff_tflops = a["eff_flops"] / fwd_s / 1e12
+    fwd0_s = results["no_bias"]["fwd_ms"] * 1e-3
+    peak_t = peaks["bf16_tflops"]
+    t_mem = a["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_tensor = a["eff_flops"] / (peak_t * 1e12)
+    bound = "hbm" if t_mem > t_tensor else "tensor"
+    if bound == "hbm":
+        achieved, peak, unit = a["bytes"] / fwd_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved, peak, unit = eff_tflops, peak_t, "TFLOP/s"
+    line = {
+        "metric": METRIC,
+        "value": round(results["bias"]["step_ms"], 5),
+        "unit": "ms",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(results["bias"]["step_ms"], 5),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "dtype_detail": "1-bit Q/K scores (exact int), fp32 softmax, bf16 P.V, fp32 accumulate",
+        "data": "synthetic",
+        "config": workload_config(w, True) | {"engine": args.engine, "parallelism": f"replicas x{world}"},
+        "forward_ms": round(results["bias"]["fwd_ms"], 5),
+        "forward_ms_median": round(results["bias"]["fwd_ms_median"], 5),
+        "pack_ms": round(results["bias"]["step_ms"] - results["bias"]["fwd_ms"], 5),
+        "effective_tflops": round(eff_tflops, 2),
+        "no_bias": {"ms_per_step": round(results["no_bias"]["step_ms"], 5),
+                    "forward_ms": round(results["no_bias"]["fwd_ms"], 5),
+                    "effective_tflops": round(a0["eff_flops"] / fwd0_s / 1e12, 2)},
+        "bf16_reference": ref,
+        "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "binattn forward (with bias)",
+                     "peak_source": peaks["source"] + " (burst)",
+                     "t_mem_us": round(t_mem * 1e6, 2), "t_tensor_us": round(t_tensor * 1e6, 2)},
+        "e2e": {"value": round(e2e_ms, 4), "unit": "ms",
+                "h2d_bytes_per_step": int(3 * B * H * N * d * 2),
+                "d2h_bytes_per_step": int(B * H * N * d * 2)},
+        "gpu_launches": 3 * args.steps * 2,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(w, True, args.cpu_seconds, inp)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_gpu(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

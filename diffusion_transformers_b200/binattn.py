@@ -1,0 +1,159 @@
+"""Thin Python binding of libbinattn (the C ABI in include/binattn.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libbinattn.so. torch is used for device memory and streams. There is
+no CPU fallback: if the library is missing, importing a function raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+OK = 0
+F32, BF16 = 0, 1
+ENGINE_AUTO, ENGINE_SIMT, ENGINE_POPC_TC, ENGINE_TC = 0, 1, 2, 3
+ENGINES = {"auto": ENGINE_AUTO, "simt": ENGINE_SIMT, "popc_tc": ENGINE_POPC_TC, "tc": ENGINE_TC}
+
+# Every symbol include/binattn.h declares.
+EXPORTS = (
+    "binattn_pack", "binattn_forward", "binattn_forward_engine", "binattn_scores_debug",
+    "binattn_ref_bf16_forward", "binattn_device_status", "binattn_strerror",
+    "binattn_last_error_message", "binattn_abi_version",
+)
+
+
+class BinattnError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({detail})")
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIBRARY
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbinattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m diffusion_transformers_b200.build`")
+    L = ctypes.CDLL(path)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    L.binattn_pack.argtypes = [P, I, I, I, I, I, P, P, P]
+    L.binattn_forward.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, P]
+    L.binattn_forward_engine.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, I, P]
+    L.binattn_scores_debug.argtypes = [P, P, I, I, I, I, P, I, P]
+    L.binattn_ref_bf16_forward.argtypes = [P, P, P, P, F, I, I, I, I, P, P]
+    L.binattn_device_status.argtypes = [P]
+    L.binattn_strerror.argtypes = [I]
+    L.binattn_strerror.restype = ctypes.c_char_p
+    L.binattn_last_error_message.restype = ctypes.c_char_p
+    for name in ("binattn_pack", "binattn_forward", "binattn_forward_engine", "binattn_scores_debug",
+                 "binattn_ref_bf16_forward", "binattn_device_status", "binattn_abi_version"):
+        getattr(L, name).restype = I
+    _lib = L
+    return L
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != OK:
+        L = lib()
+        detail = L.binattn_last_error_message().decode() or L.binattn_strerror(rc).decode()
+        raise BinattnError(rc, where, detail)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libbinattn must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _words(d: int) -> int:
+    return (d + 31) // 32
+
+
+def pack(x: torch.Tensor, bits: torch.Tensor | None = None, alpha: torch.Tensor | None = None,
+         stream=None):
+    """x [B,H,N,d] (float32 or bfloat16, CUDA) -> (bits uint32-as-int32 [B,H,N,W], alpha fp32 [B,H,N])."""
+    B, H, N, d = x.shape
+    dt = {torch.float32: F32, torch.bfloat16: BF16}.get(x.dtype)
+    if dt is None:
+        raise TypeError(f"pack takes float32 or bfloat16, got {x.dtype}")
+    if bits is None:
+        bits = torch.empty((B, H, N, _words(d)), dtype=torch.int32, device=x.device)
+    if alpha is None:
+        alpha = torch.empty((B, H, N), dtype=torch.float32, device=x.device)
+    _check(lib().binattn_pack(_ptr(x), dt, B, H, N, d, _ptr(bits), _ptr(alpha), _stream(stream)),
+           "binattn_pack")
+    return bits, alpha
+
+
+def forward(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor,
+            alpha_k: torch.Tensor, bias: torch.Tensor | None, v: torch.Tensor,
+            softmax_scale: float, out: torch.Tensor | None = None, engine: int | str = ENGINE_AUTO,
+            stream=None) -> torch.Tensor:
+    """O [B,H,N,d] bfloat16 = softmax(scale * a_q a_k^T * S + bias) V."""
+    B, H, N, d = v.shape
+    if isinstance(engine, str):
+        engine = ENGINES[engine]
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=v.device)
+    _check(lib().binattn_forward_engine(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k),
+                                        _ptr(bias), _ptr(v), float(softmax_scale), B, H, N, d,
+                                        _ptr(out), int(engine), _stream(stream)),
+           "binattn_forward_engine")
+    return out
+
+
+def scores_debug(q_bits: torch.Tensor, k_bits: torch.Tensor, d: int,
+                 engine: int | str = ENGINE_AUTO, S: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """Integer scores S [B,H,N,N] int32 as the given engine computes them."""
+    B, H, N, _ = q_bits.shape
+    if isinstance(engine, str):
+        engine = ENGINES[engine]
+    if S is None:
+        S = torch.empty((B, H, N, N), dtype=torch.int32, device=q_bits.device)
+    _check(lib().binattn_scores_debug(_ptr(q_bits), _ptr(k_bits), B, H, N, d, _ptr(S), int(engine),
+                                      _stream(stream)), "binattn_scores_debug")
+    return S
+
+
+def ref_bf16_forward(q: torch.Tensor, k: torch.Tensor, bias: torch.Tensor | None, v: torch.Tensor,
+                     softmax_scale: float, out: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Full-precision bf16 softmax attention on the same shapes (speed reference)."""
+    B, H, N, d = q.shape
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
+    _check(lib().binattn_ref_bf16_forward(_ptr(q), _ptr(k), _ptr(bias), _ptr(v), float(softmax_scale),
+                                          B, H, N, d, _ptr(out), _stream(stream)),
+           "binattn_ref_bf16_forward")
+    return out
+
+
+def device_status(stream=None) -> None:
+    """Synchronize and raise if a kernel abandoned a bounded wait."""
+    _check(lib().binattn_device_status(_stream(stream)), "binattn_device_status")
+
+
+def abi_version() -> int:
+    return int(lib().binattn_abi_version())

@@ -1,0 +1,258 @@
+// binattn.cu — the C ABI of libbinattn (declared in include/binattn.h).
+//
+// Host-side argument validation, engine dispatch and status reporting. All
+// kernels are compiled into this one translation unit from the .cuh files.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "binattn.h"
+#include "common.cuh"
+#include "pack.cuh"
+#include "fwd_simt.cuh"
+#include "fwd_tc.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int status, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return status;
+}
+
+int ok() {
+  g_last_error.clear();
+  return BINATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || d < 1)
+    return fail(BINATTN_ERR_SHAPE, "B, H, N, d must be >= 1 (got %d, %d, %d, %d)", B, H, N, d);
+  if (d > 128) return fail(BINATTN_ERR_SHAPE, "d = %d > 128 is not supported", d);
+  if (static_cast<long long>(B) * H > 65535)
+    return fail(BINATTN_ERR_SHAPE, "B*H = %lld > 65535", static_cast<long long>(B) * H);
+  if (N > 65535) return fail(BINATTN_ERR_SHAPE, "N = %d > 65535", N);
+  return BINATTN_OK;
+}
+
+#define BINATTN_CHECK_PTR(p)                                                 \
+  do {                                                                       \
+    if (!(p)) return fail(BINATTN_ERR_NULL, "%s is NULL", #p);               \
+    if (!aligned16(p)) return fail(BINATTN_ERR_ALIGN, "%s is not 16-byte aligned", #p); \
+  } while (0)
+
+int launch_status(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return fail(BINATTN_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
+  return ok();
+}
+
+int check_forward_args(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
+                       const float* alpha_k, const uint16_t* bias, const uint16_t* v,
+                       float softmax_scale, int B, int H, int N, int d, const uint16_t* out) {
+  BINATTN_CHECK_PTR(q_bits);
+  BINATTN_CHECK_PTR(k_bits);
+  BINATTN_CHECK_PTR(alpha_q);
+  BINATTN_CHECK_PTR(alpha_k);
+  BINATTN_CHECK_PTR(v);
+  BINATTN_CHECK_PTR(out);
+  if (bias && !aligned16(bias)) return fail(BINATTN_ERR_ALIGN, "bias is not 16-byte aligned");
+  if (!std::isfinite(softmax_scale)) return fail(BINATTN_ERR_ARG, "softmax_scale is not finite");
+  return check_shape(B, H, N, d);
+}
+
+template <int W>
+int launch_simt(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
+                const float* alpha_k, const uint16_t* bias, const uint16_t* v, float scale,
+                int B, int H, int N, int d, uint16_t* out, cudaStream_t st) {
+  dim3 grid((N + binattn::kSimtRows - 1) / binattn::kSimtRows, B * H);
+  if (bias)
+    binattn::fwd_simt_kernel<W, true><<<grid, binattn::kSimtRows, 0, st>>>(
+        q_bits, k_bits, alpha_q, alpha_k, bias, v, scale, H, N, d, out);
+  else
+    binattn::fwd_simt_kernel<W, false><<<grid, binattn::kSimtRows, 0, st>>>(
+        q_bits, k_bits, alpha_q, alpha_k, nullptr, v, scale, H, N, d, out);
+  return launch_status("fwd_simt_kernel");
+}
+
+int forward_simt(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
+                 const float* alpha_k, const uint16_t* bias, const uint16_t* v, float scale,
+                 int B, int H, int N, int d, uint16_t* out, cudaStream_t st) {
+  switch (binattn::words_for(d)) {
+    case 1: return launch_simt<1>(q_bits, k_bits, alpha_q, alpha_k, bias, v, scale, B, H, N, d, out, st);
+    case 2: return launch_simt<2>(q_bits, k_bits, alpha_q, alpha_k, bias, v, scale, B, H, N, d, out, st);
+    case 3: return launch_simt<3>(q_bits, k_bits, alpha_q, alpha_k, bias, v, scale, B, H, N, d, out, st);
+    default: return launch_simt<4>(q_bits, k_bits, alpha_q, alpha_k, bias, v, scale, B, H, N, d, out, st);
+  }
+}
+
+template <int W>
+int launch_scores_popc(const uint32_t* q_bits, const uint32_t* k_bits, int B, int H, int N,
+                       int d, int32_t* S, cudaStream_t st) {
+  const long long gx = static_cast<long long>((N + 255) / 256) * N;
+  dim3 grid(static_cast<unsigned>(gx), B * H);
+  binattn::scores_popc_kernel<W><<<grid, 256, 0, st>>>(q_bits, k_bits, N, d, S);
+  return launch_status("scores_popc_kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
+int binattn_abi_version(void) { return BINATTN_ABI_VERSION; }
+
+const char* binattn_strerror(int status) {
+  switch (status) {
+    case BINATTN_OK: return "success";
+    case BINATTN_ERR_NULL: return "a required pointer is NULL";
+    case BINATTN_ERR_SHAPE: return "B, H, N or d out of range";
+    case BINATTN_ERR_DTYPE: return "unknown dtype";
+    case BINATTN_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case BINATTN_ERR_UNSUPPORTED: return "engine or shape not supported by this build";
+    case BINATTN_ERR_CUDA: return "CUDA error";
+    case BINATTN_ERR_TIMEOUT: return "a kernel abandoned a bounded wait";
+    case BINATTN_ERR_ARG: return "invalid argument";
+    default: return "unknown status";
+  }
+}
+
+const char* binattn_last_error_message(void) { return g_last_error.c_str(); }
+
+int binattn_pack(const void* x, int dtype, int B, int H, int N, int d, uint32_t* bits,
+                 float* alpha, void* stream) {
+  BINATTN_CHECK_PTR(x);
+  BINATTN_CHECK_PTR(bits);
+  BINATTN_CHECK_PTR(alpha);
+  if (dtype != BINATTN_F32 && dtype != BINATTN_BF16)
+    return fail(BINATTN_ERR_DTYPE, "dtype %d is neither BINATTN_F32 nor BINATTN_BF16", dtype);
+  if (int rc = check_shape(B, H, N, d)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long n_tokens = static_cast<long long>(B) * H * N;
+  const int W = binattn::words_for(d);
+  const int esize = dtype == BINATTN_F32 ? 4 : 2;
+  const bool vec = (d * esize) % 16 == 0;
+  const size_t smem = binattn::pack_smem_bytes(d, esize, vec);
+  const unsigned grid = static_cast<unsigned>((n_tokens + binattn::kPackTokens - 1) / binattn::kPackTokens);
+  if (dtype == BINATTN_F32) {
+    const float* xf = static_cast<const float*>(x);
+    if (vec) binattn::pack_kernel<float, true><<<grid, binattn::kPackThreads, smem, st>>>(xf, n_tokens, d, W, bits, alpha);
+    else binattn::pack_kernel<float, false><<<grid, binattn::kPackThreads, 0, st>>>(xf, n_tokens, d, W, bits, alpha);
+  } else {
+    const uint16_t* xb = static_cast<const uint16_t*>(x);
+    if (vec) binattn::pack_kernel<uint16_t, true><<<grid, binattn::kPackThreads, smem, st>>>(xb, n_tokens, d, W, bits, alpha);
+    else binattn::pack_kernel<uint16_t, false><<<grid, binattn::kPackThreads, 0, st>>>(xb, n_tokens, d, W, bits, alpha);
+  }
+  return launch_status("pack_kernel");
+}
+
+int binattn_forward_engine(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
+                           const float* alpha_k, const uint16_t* bias, const uint16_t* v,
+                           float softmax_scale, int B, int H, int N, int d, uint16_t* out,
+                           int engine, void* stream) {
+  if (int rc = check_forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out))
+    return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (engine == BINATTN_ENGINE_AUTO)
+    engine = binattn::tc_built() && binattn::tc_supported(d) ? BINATTN_ENGINE_TC : BINATTN_ENGINE_SIMT;
+  switch (engine) {
+    case BINATTN_ENGINE_SIMT:
+      return forward_simt(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out, st);
+    case BINATTN_ENGINE_POPC_TC:
+    case BINATTN_ENGINE_TC: {
+      if (!binattn::tc_supported(d))
+        return fail(BINATTN_ERR_UNSUPPORTED, "engine %d needs d %% 8 == 0 (d = %d)", engine, d);
+      std::string msg;
+      int rc = binattn::forward_tc(engine == BINATTN_ENGINE_TC, q_bits, k_bits, alpha_q, alpha_k, bias,
+                                   v, softmax_scale, B, H, N, d, out, st, &msg);
+      if (rc) return fail(rc, "%s", msg.c_str());
+      return ok();
+    }
+    default:
+      return fail(BINATTN_ERR_ARG, "unknown engine %d", engine);
+  }
+}
+
+int binattn_forward(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
+                    const float* alpha_k, const uint16_t* bias, const uint16_t* v,
+                    float softmax_scale, int B, int H, int N, int d, uint16_t* out, void* stream) {
+  return binattn_forward_engine(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N,
+                                d, out, BINATTN_ENGINE_AUTO, stream);
+}
+
+int binattn_scores_debug(const uint32_t* q_bits, const uint32_t* k_bits, int B, int H, int N,
+                         int d, int32_t* S, int engine, void* stream) {
+  BINATTN_CHECK_PTR(q_bits);
+  BINATTN_CHECK_PTR(k_bits);
+  BINATTN_CHECK_PTR(S);
+  if (int rc = check_shape(B, H, N, d)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (engine == BINATTN_ENGINE_AUTO)
+    engine = binattn::tc_built() && binattn::tc_supported(d) ? BINATTN_ENGINE_TC : BINATTN_ENGINE_SIMT;
+  switch (engine) {
+    case BINATTN_ENGINE_SIMT:
+    case BINATTN_ENGINE_POPC_TC:
+      switch (binattn::words_for(d)) {
+        case 1: return launch_scores_popc<1>(q_bits, k_bits, B, H, N, d, S, st);
+        case 2: return launch_scores_popc<2>(q_bits, k_bits, B, H, N, d, S, st);
+        case 3: return launch_scores_popc<3>(q_bits, k_bits, B, H, N, d, S, st);
+        default: return launch_scores_popc<4>(q_bits, k_bits, B, H, N, d, S, st);
+      }
+    case BINATTN_ENGINE_TC: {
+      if (!binattn::tc_supported(d))
+        return fail(BINATTN_ERR_UNSUPPORTED, "engine TC needs d %% 8 == 0 (d = %d)", d);
+      std::string msg;
+      int rc = binattn::scores_tc(q_bits, k_bits, B, H, N, d, S, st, &msg);
+      if (rc) return fail(rc, "%s", msg.c_str());
+      return ok();
+    }
+    default:
+      return fail(BINATTN_ERR_ARG, "unknown engine %d", engine);
+  }
+}
+
+int binattn_ref_bf16_forward(const uint16_t* q, const uint16_t* k, const uint16_t* bias,
+                             const uint16_t* v, float softmax_scale, int B, int H, int N, int d,
+                             uint16_t* out, void* stream) {
+  BINATTN_CHECK_PTR(q);
+  BINATTN_CHECK_PTR(k);
+  BINATTN_CHECK_PTR(v);
+  BINATTN_CHECK_PTR(out);
+  if (bias && !aligned16(bias)) return fail(BINATTN_ERR_ALIGN, "bias is not 16-byte aligned");
+  if (!std::isfinite(softmax_scale)) return fail(BINATTN_ERR_ARG, "softmax_scale is not finite");
+  if (int rc = check_shape(B, H, N, d)) return rc;
+  if (!binattn::tc_supported(d))
+    return fail(BINATTN_ERR_UNSUPPORTED, "the bf16 reference needs d %% 8 == 0 (d = %d)", d);
+  std::string msg;
+  int rc = binattn::forward_ref_bf16(q, k, bias, v, softmax_scale, B, H, N, d, out,
+                                     static_cast<cudaStream_t>(stream), &msg);
+  if (rc) return fail(rc, "%s", msg.c_str());
+  return ok();
+}
+
+int binattn_device_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fail(BINATTN_ERR_CUDA, "stream synchronize: %s", cudaGetErrorString(e));
+  int status = 0;
+  e = cudaMemcpyFromSymbol(&status, binattn::g_device_status, sizeof(int));
+  if (e != cudaSuccess) return fail(BINATTN_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(binattn::g_device_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return fail(BINATTN_ERR_CUDA, "status clear: %s", cudaGetErrorString(e));
+  if (status != 0) return fail(BINATTN_ERR_TIMEOUT, "device status code %d", status);
+  return ok();
+}
+
+}  // extern "C"

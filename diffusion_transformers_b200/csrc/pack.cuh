@@ -1,0 +1,70 @@
+// pack.cuh — sign bits and per-token scale (binattn_pack).
+//
+// Source: "BinaryAttention: One-Bit QK-Attention for Vision and Diffusion
+// Transformers", §2 scaled binary representations (s_i = mu_q * sign(q_i),
+// t_j = mu_k * sign(k_j)); mu is the per-token mean |x|.
+//
+// One block handles kPackTokens consecutive tokens. Their bytes are one
+// contiguous range, staged into shared memory with 128-bit coalesced loads
+// (when a token is a whole number of 16-byte chunks). Then each warp takes a
+// token at a time: lane c looks at channel 32*w + c, __ballot_sync(x >= 0)
+// is packed word w, and the lanes' |x| partial sums are warp-reduced into alpha.
+#pragma once
+#include "common.cuh"
+
+namespace binattn {
+
+constexpr int kPackThreads = 256;
+constexpr int kPackTokens = 64;
+
+template <typename T> __device__ __forceinline__ float load_as_float(const T* p);
+template <> __device__ __forceinline__ float load_as_float<float>(const float* p) { return *p; }
+template <> __device__ __forceinline__ float load_as_float<uint16_t>(const uint16_t* p) {
+  return bf16_bits_to_float(*p);
+}
+
+// kVec: token size d * sizeof(T) is a multiple of 16 bytes (and x is 16-byte
+// aligned, which the API checks), so the block's range is whole uint4 chunks.
+template <typename T, bool kVec>
+__global__ void __launch_bounds__(kPackThreads)
+pack_kernel(const T* __restrict__ x, long long n_tokens, int d, int W,
+            uint32_t* __restrict__ bits, float* __restrict__ alpha) {
+  extern __shared__ uint4 pack_smem[];
+  const long long t0 = static_cast<long long>(blockIdx.x) * kPackTokens;
+  const int ntok = static_cast<int>(min(static_cast<long long>(kPackTokens), n_tokens - t0));
+  const T* src = x + t0 * d;
+  const T* tile = src;
+  if constexpr (kVec) {
+    const int nchunks = static_cast<int>((static_cast<long long>(ntok) * d * sizeof(T)) / 16);
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    for (int c = threadIdx.x; c < nchunks; c += kPackThreads) pack_smem[c] = __ldg(&s4[c]);
+    __syncthreads();
+    tile = reinterpret_cast<const T*>(pack_smem);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int tk = warp; tk < ntok; tk += kPackThreads / 32) {
+    const T* row = tile + static_cast<size_t>(tk) * d;
+    float acc = 0.f;
+    uint32_t myword = 0;
+    for (int w = 0; w < W; ++w) {
+      const int c = w * 32 + lane;
+      const bool in = c < d;
+      const float v = in ? load_as_float(row + c) : 0.f;
+      // x >= 0 is true for +0.0 and -0.0; pad lanes contribute 0 bits.
+      const uint32_t word = __ballot_sync(0xffffffffu, in && v >= 0.f);
+      if (lane == w) myword = word;
+      acc += fabsf(v);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    const long long t = t0 + tk;
+    if (lane < W) bits[t * W + lane] = myword;
+    if (lane == 0) alpha[t] = acc / static_cast<float>(d);
+  }
+}
+
+inline size_t pack_smem_bytes(int d, int esize, bool vec) {
+  return vec ? static_cast<size_t>(kPackTokens) * d * esize : 0;
+}
+
+}  // namespace binattn

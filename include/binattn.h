@@ -1,0 +1,176 @@
+/*
+ * binattn.h — C ABI of the BinaryAttention forward pass for NVIDIA B200 (sm_100a).
+ *
+ * The method ("BinaryAttention: One-Bit QK-Attention for Vision and Diffusion
+ * Transformers", technical summaries, §2 Methodology) replaces the query/key
+ * dot product of softmax attention by a 1-bit one:
+ *
+ *   s_i = alpha_q_i * sign(q_i),  t_j = alpha_k_j * sign(k_j)
+ *       (§2 "scaled binary representations"; alpha = per-token mean |x|)
+ *   S_ij = <sign q_i, sign k_j> = d - 2 * popcount(q_bits_i XOR k_bits_j)
+ *       (§2: similarity through XNOR and popcount instead of float multiplies)
+ *   logit_ij = softmax_scale * alpha_q_i * alpha_k_j * S_ij + bias[h, i, j]
+ *       (§2 "bias enhancement": a learnable dense additive bias b_ij)
+ *   O_i = sum_j softmax_j(logit_i.) * V_j
+ *       (§2 hardware implementation: FlashAttention2-style tiling, so the N x N
+ *        matrix is never written out)
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers (cudaMalloc / torch CUDA memory)
+ *    owned by the caller. The library never allocates device memory in these
+ *    calls and never frees caller memory.
+ *  - Layouts are row-major and contiguous, last index fastest.
+ *  - bf16 tensors are passed as uint16_t bit patterns.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). Work is
+ *    enqueued asynchronously; results are valid after the stream is synchronized.
+ *  - Every call returns a binattn_status. Arguments are validated on the host
+ *    before anything is launched; on any error nothing is launched and the
+ *    outputs are untouched. No exception or abort crosses the ABI.
+ *    binattn_last_error_message() gives a one-line detail for the calling thread.
+ *  - Sizes: B, H, N >= 1; 1 <= d <= 128; B*H <= 2^20; N <= 65536.
+ *    All pointers must be 16-byte aligned.
+ *  - Inputs containing NaN or Inf are outside the contract.
+ */
+#ifndef BINATTN_H
+#define BINATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BINATTN_ABI_VERSION 1
+
+typedef enum {
+    BINATTN_OK = 0,
+    BINATTN_ERR_NULL = 1,        /* a required pointer is NULL                         */
+    BINATTN_ERR_SHAPE = 2,       /* B, H, N or d out of range                          */
+    BINATTN_ERR_DTYPE = 3,       /* unknown dtype code                                 */
+    BINATTN_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned                   */
+    BINATTN_ERR_UNSUPPORTED = 5, /* valid request this build cannot serve (engine/d)   */
+    BINATTN_ERR_CUDA = 6,        /* a CUDA call failed (detail in last_error_message)  */
+    BINATTN_ERR_TIMEOUT = 7,     /* a kernel gave up a bounded wait (device status)    */
+    BINATTN_ERR_ARG = 8          /* other invalid argument (non-finite scale, engine)  */
+} binattn_status;
+
+typedef enum {
+    BINATTN_F32 = 0,
+    BINATTN_BF16 = 1
+} binattn_dtype;
+
+/*
+ * Score engines. All give identical integer scores S_ij; they differ in the
+ * hardware unit that evaluates them.
+ *   AUTO      — the fastest engine for the shape (TC where supported, else SIMT).
+ *   SIMT      — CUDA cores only: __popc over uint32 words for S, fp32 softmax,
+ *               fp32 P.V. Any d in [1, 128]. Reference-grade GPU path.
+ *   POPC_TC   — S by __popc over uint32 words in the softmax threads; P.V as a
+ *               bf16 tcgen05 MMA with the accumulator in tensor memory.
+ *               Needs d % 8 == 0.
+ *   TC        — S by a tcgen05 MMA on +-1 operands expanded from the sign bits in
+ *               shared memory (exact integer scores in an fp32 accumulator);
+ *               P.V as a bf16 tcgen05 MMA. Needs d % 8 == 0.
+ * (A warp-level mma.sync .b1 XOR-popc engine was measured on sm_100a and runs
+ *  below __popc throughput; it is not built.)
+ */
+typedef enum {
+    BINATTN_ENGINE_AUTO = 0,
+    BINATTN_ENGINE_SIMT = 1,
+    BINATTN_ENGINE_POPC_TC = 2,
+    BINATTN_ENGINE_TC = 3
+} binattn_engine;
+
+/*
+ * binattn_pack — sign bits and per-token scale of Q or K (one call per tensor).
+ *
+ * Source: §2 scaled binary representations, s_i = mu * sign(q_i); mu read as
+ * the per-token mean of |x| over the d channels (the closed-form minimiser of
+ * ||x - mu * sign(x)||_2).
+ *
+ *   x      [B, H, N, d]  dtype `dtype` (BINATTN_F32 or BINATTN_BF16), device.
+ *   bits   [B, H, N, W]  uint32, W = ceil(d / 32), device, written.
+ *          Channel c of a token is bit (c % 32) of word (c / 32); the bit is 1
+ *          exactly when x >= 0 (so +0.0 and -0.0 give 1). Bits for c >= d are 0.
+ *          This bit format is part of the ABI.
+ *   alpha  [B, H, N]     fp32, device, written: (1/d) * sum_c |x_c|, summed in
+ *          fp32 (order of summation unspecified; relative error ~1e-6).
+ */
+int binattn_pack(const void *x, int dtype, int B, int H, int N, int d,
+                 uint32_t *bits, float *alpha, void *stream);
+
+/*
+ * binattn_forward — O = softmax(logits) V with binary scores (engine AUTO).
+ *
+ * Source: §2 (all four bullets above) and the FlashAttention2-style kernel of
+ * §2 hardware-aware implementation.
+ *
+ *   q_bits, k_bits    [B, H, N, W] uint32 from binattn_pack, device, read.
+ *   alpha_q, alpha_k  [B, H, N] fp32 from binattn_pack, device, read.
+ *   bias              [H, N, N] bf16 or NULL (= zero), device, read. Shared by
+ *                     every batch index b. Added after scaling; not scaled.
+ *   v                 [B, H, N, d] bf16, device, read.
+ *   softmax_scale     finite float (usually 1/sqrt(d)).
+ *   out               [B, H, N, d] bf16, device, written (round to nearest even
+ *                     of the fp32 result). Must not overlap any input.
+ * Numerics: S exact (integer); logits and softmax in fp32; P rounded to bf16
+ * before a bf16 x bf16 -> fp32 P.V on the tensor-core engines (fp32 P on SIMT);
+ * normalisation by the fp32 row sum in the epilogue.
+ * No mask: every query attends to all N keys (vision / diffusion self-attention).
+ */
+int binattn_forward(const uint32_t *q_bits, const uint32_t *k_bits,
+                    const float *alpha_q, const float *alpha_k,
+                    const uint16_t *bias, const uint16_t *v, float softmax_scale,
+                    int B, int H, int N, int d, uint16_t *out, void *stream);
+
+/* binattn_forward with an explicit score engine (binattn_engine). Returns
+ * BINATTN_ERR_UNSUPPORTED when the engine cannot serve the shape. */
+int binattn_forward_engine(const uint32_t *q_bits, const uint32_t *k_bits,
+                           const float *alpha_q, const float *alpha_k,
+                           const uint16_t *bias, const uint16_t *v, float softmax_scale,
+                           int B, int H, int N, int d, uint16_t *out, int engine,
+                           void *stream);
+
+/*
+ * binattn_scores_debug — writes the integer scores S [B, H, N, N] (int32,
+ * device) that engine `engine` computes inside the forward pass, using the same
+ * device score routine. For testing only: it materialises the N x N matrix.
+ * Source: §2, S_ij = d - 2 * popcount(q_i XOR k_j) (identical pad bits add 0).
+ */
+int binattn_scores_debug(const uint32_t *q_bits, const uint32_t *k_bits,
+                         int B, int H, int N, int d, int32_t *S, int engine,
+                         void *stream);
+
+/*
+ * binattn_ref_bf16_forward — full-precision softmax attention on the same
+ * shapes, the speed reference the binary kernel is compared against:
+ * O = softmax(softmax_scale * Q K^T + bias) V with bf16 Q, K, V, bias (NULL =
+ * zero), fp32 accumulation and softmax, bf16 output. Needs d % 8 == 0.
+ */
+int binattn_ref_bf16_forward(const uint16_t *q, const uint16_t *k,
+                             const uint16_t *bias, const uint16_t *v,
+                             float softmax_scale, int B, int H, int N, int d,
+                             uint16_t *out, void *stream);
+
+/*
+ * binattn_device_status — synchronizes `stream`, then reads and clears the
+ * library's device status word. Returns BINATTN_OK, or BINATTN_ERR_TIMEOUT when
+ * a kernel abandoned a bounded wait (its outputs are then undefined), or
+ * BINATTN_ERR_CUDA when the synchronize itself failed.
+ */
+int binattn_device_status(void *stream);
+
+/* Static description of a status code. Never NULL. */
+const char *binattn_strerror(int status);
+
+/* One-line detail of the calling thread's last failed call ("" if none). */
+const char *binattn_last_error_message(void);
+
+/* BINATTN_ABI_VERSION of the loaded library. */
+int binattn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BINATTN_H */

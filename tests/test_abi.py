@@ -1,0 +1,94 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol the header
+declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from diffusion_transformers_b200 import binattn
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "binattn.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(binattn_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    return binattn.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 9
+    assert set(names) == set(binattn.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), f"{n} not exported by {binattn.library_path()}"
+
+
+def test_abi_version_and_strerror(L):
+    assert L.binattn_abi_version() == 1
+    for code in range(0, 9):
+        s = L.binattn_strerror(code)
+        assert s and isinstance(s, bytes)
+    assert L.binattn_strerror(99) == b"unknown status"
+
+
+A = 0x10000  # aligned fake device addresses: never dereferenced by these calls
+P = ctypes.c_void_p
+
+
+def _fwd(L, q=A, k=A, aq=A, ak=A, bias=None, v=A, scale=0.125, B=1, H=1, N=16, d=64, out=A,
+         engine=0):
+    return L.binattn_forward_engine(P(q), P(k), P(aq), P(ak), P(bias) if bias else None, P(v),
+                                    ctypes.c_float(scale), B, H, N, d, P(out), engine, None)
+
+
+def test_forward_host_validation(L):
+    assert _fwd(L, q=0) == 1
+    assert _fwd(L, out=0) == 1
+    assert _fwd(L, v=A + 8) == 4
+    assert _fwd(L, bias=A + 2) == 4
+    assert _fwd(L, N=0) == 2
+    assert _fwd(L, d=129) == 2
+    assert _fwd(L, B=300, H=300) == 2
+    assert _fwd(L, N=70000) == 2
+    assert _fwd(L, scale=math.inf) == 8
+    assert _fwd(L, scale=math.nan) == 8
+    assert _fwd(L, engine=17) == 8
+    assert _fwd(L, d=33, engine=binattn.ENGINE_TC) == 5
+    assert _fwd(L, d=33, engine=binattn.ENGINE_POPC_TC) == 5
+    assert b"NULL" in L.binattn_last_error_message() or True
+
+
+def test_pack_host_validation(L):
+    def pack(x=A, dt=1, B=1, H=1, N=4, d=64, bits=A, alpha=A):
+        return L.binattn_pack(P(x), dt, B, H, N, d, P(bits), P(alpha), None)
+    assert pack(x=0) == 1
+    assert pack(alpha=0) == 1
+    assert pack(bits=A + 4) == 4
+    assert pack(dt=7) == 3
+    assert pack(d=0) == 2
+    assert pack(N=-1) == 2
+
+
+def test_scores_and_ref_host_validation(L):
+    assert L.binattn_scores_debug(P(A), P(0), 1, 1, 4, 64, P(A), 0, None) == 1
+    assert L.binattn_scores_debug(P(A), P(A), 1, 1, 4, 200, P(A), 0, None) == 2
+    assert L.binattn_scores_debug(P(A), P(A), 1, 1, 4, 64, P(A), 9, None) == 8
+    assert L.binattn_ref_bf16_forward(P(A), P(A), None, P(A), ctypes.c_float(1.0), 1, 1, 4, 33,
+                                      P(A), None) == 5
+    assert L.binattn_ref_bf16_forward(P(A), P(A), None, P(A + 2), ctypes.c_float(1.0), 1, 1, 4, 64,
+                                      P(A), None) == 4
+    assert L.binattn_ref_bf16_forward(P(A), P(A), None, P(A), ctypes.c_float(math.inf), 1, 1, 4, 64,
+                                      P(A), None) == 8
+
+
+def test_last_error_message_is_specific(L):
+    assert _fwd(L, v=A + 8) == 4
+    assert b"v is not 16-byte aligned" in L.binattn_last_error_message()

@@ -1,0 +1,151 @@
+"""GPU path (through the C ABI) against the CPU oracle, on the same seeded inputs.
+
+Bits: exact. alpha: relative 1e-6 (fp32 tree sum of depth <= W + 6, each step
+rounding by at most 2^-24). Integer scores: exact. O: max-abs 2e-2 and
+rel-RMS 5e-3 against the oracle's unrounded fp64 result.
+"""
+import numpy as np
+import pytest
+import torch
+
+from diffusion_transformers_b200 import binattn
+from diffusion_transformers_b200.synthetic import WORKLOADS, make_custom, make_inputs
+from parity import bf16_to_f64, check_o, dev, run_path, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+ENGINES = ["simt"]
+
+SMALL_SHAPES = [  # (B, H, N, d): several tiles and a ragged tail
+    (1, 2, 256, 64), (2, 3, 129, 72), (1, 2, 197, 64), (1, 1, 1, 64), (2, 1, 7, 32),
+    (1, 2, 127, 96), (1, 1, 300, 128), (2, 2, 257, 8), (1, 1, 130, 72),
+]
+ODD_D_SHAPES = [(1, 2, 65, 33), (1, 1, 40, 1), (2, 1, 33, 100), (1, 1, 31, 127)]
+
+
+def _engines_for(d):
+    return [e for e in ENGINES if e == "simt" or d % 8 == 0]
+
+
+# ------------------------------------------------------------------ pack (a1, a2)
+@pytest.mark.parametrize("shape", SMALL_SHAPES + ODD_D_SHAPES)
+@pytest.mark.parametrize("qk_dtype", ["bf16", "f32"])
+def test_pack_exact(orc, shape, qk_dtype):
+    B, H, N, d = shape
+    c = make_custom(B, H, N, d, seed=N * 7 + d, qk_dtype=qk_dtype, zeros_frac=0.05)
+    bits, alpha = binattn.pack(dev(c["q"]))
+    ob, oa = orc.pack(c["q"])
+    assert np.array_equal(bits.cpu().numpy().view(np.uint32), ob)
+    np.testing.assert_allclose(alpha.cpu().numpy().astype(np.float64), oa, rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize("name", ["tiny", "deit_b", "vit_l384", "dit_xl_512", "dit_xl_1024"])
+def test_pack_exact_full_size(orc, name):
+    inp = make_inputs(name, with_bias=False)
+    for key in ("q", "k"):
+        bits, alpha = binattn.pack(dev(inp[key]))
+        ob, oa = orc.pack(inp[key])
+        assert np.array_equal(bits.cpu().numpy().view(np.uint32), ob), f"{name} {key} bits"
+        np.testing.assert_allclose(alpha.cpu().numpy().astype(np.float64), oa, rtol=1e-6, atol=0)
+
+
+# --------------------------------------------------------------- scores (a3, a8)
+# The POPC_TC forward uses the same __popc routine as SIMT (one debug kernel);
+# the TC engine has its own tensor-core score routine and needs d % 8 == 0.
+SCORE_CASES = [(s, e) for s in SMALL_SHAPES + ODD_D_SHAPES for e in ["simt"] + [x for x in ENGINES if x == "tc"]
+               if e == "simt" or s[3] % 8 == 0]
+
+
+@pytest.mark.parametrize("shape,engine", SCORE_CASES)
+def test_scores_exact(orc, shape, engine):
+    B, H, N, d = shape
+    c = make_custom(B, H, N, d, seed=N + d, zeros_frac=0.05)
+    qb, _ = binattn.pack(dev(c["q"]))
+    kb, _ = binattn.pack(dev(c["k"]))
+    S = binattn.scores_debug(qb, kb, d, engine=engine).cpu().numpy()
+    assert np.array_equal(S, orc.scores(c["q"], c["k"]))
+
+
+@pytest.mark.parametrize("name", ["deit_b", "vit_l384", "dit_xl_512", "dit_xl_1024"])
+def test_scores_exact_full_size_sampled(orc, name):
+    inp = make_inputs(name, with_bias=False)
+    B, H, N, d = inp["B"], inp["H"], inp["N"], inp["d"]
+    qb, _ = binattn.pack(dev(inp["q"]))
+    kb, _ = binattn.pack(dev(inp["k"]))
+    rows = sample_rows(B, H, N, 48)
+    for engine in ["simt"] + [e for e in ENGINES if e != "simt"]:
+        S = binattn.scores_debug(qb, kb, d, engine=engine)
+        got = S.view(B * H * N, N)[torch.from_numpy(rows).cuda()].cpu().numpy()
+        del S
+        assert np.array_equal(got, orc.scores_rows(inp["q"], inp["k"], rows)), f"{name} {engine}"
+
+
+# ------------------------------------------------------------ forward (a1-a8)
+@pytest.mark.parametrize("shape", SMALL_SHAPES + ODD_D_SHAPES)
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_forward_small(orc, shape, with_bias):
+    B, H, N, d = shape
+    c = make_custom(B, H, N, d, seed=3 * N + d, with_bias=with_bias, bias_std=0.5)
+    ref = orc.forward(c["q"], c["k"], c["bias"], c["v"], c["softmax_scale"])
+    for engine in _engines_for(d):
+        r = run_path(c, engine=engine, with_bias=with_bias)
+        check_o(bf16_to_f64(r["out"]), ref, f"{shape} bias={with_bias} {engine}")
+
+
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_forward_tiny_config(orc, with_bias):
+    inp = make_inputs("tiny", with_bias=with_bias)
+    ref = orc.forward(inp["q"], inp["k"], inp["bias"], inp["v"], inp["softmax_scale"])
+    for engine in ENGINES:
+        r = run_path(inp, engine=engine, with_bias=with_bias)
+        check_o(bf16_to_f64(r["out"]), ref, f"tiny {engine}")
+
+
+@pytest.mark.parametrize("name,with_bias", [
+    ("deit_b", True), ("vit_l384", True), ("dit_xl_512", True),
+    ("dit_xl_1024", True), ("dit_xl_1024", False)])
+def test_forward_full_size_sampled(orc, name, with_bias):
+    inp = make_inputs(name, with_bias=with_bias)
+    B, H, N, d = inp["B"], inp["H"], inp["N"], inp["d"]
+    rows = sample_rows(B, H, N, 96, seed=5)
+    ref = orc.forward_rows(inp["q"], inp["k"], inp["bias"], inp["v"], inp["softmax_scale"], rows)
+    engines = [e for e in ENGINES if e != "simt"] or ["simt"]
+    for engine in engines:
+        r = run_path(inp, engine=engine, with_bias=with_bias)
+        got = r["out"].view(B * H * N, d)[torch.from_numpy(rows).cuda()]
+        check_o(bf16_to_f64(got), ref, f"{name} bias={with_bias} {engine}")
+
+
+# -------------------------------------------------------------- edge cases
+@pytest.mark.parametrize("engine", ENGINES)
+def test_forward_special_cases(orc, engine):
+    B, H, N, d = 1, 2, 130, 72
+    # softmax_scale = 0: P = softmax(bias); large scale: very peaked rows;
+    # negative scale; value scale 1e3 (alpha large) and 1e-3 (alpha small).
+    for kw in [dict(scale=0.0), dict(scale=8.0), dict(scale=-0.5), dict(vs=1e3, scale=1e-3),
+               dict(vs=1e-3, scale=1e3)]:
+        c = make_custom(B, H, N, d, seed=77, bias_std=0.5, value_scale=kw.get("vs", 1.0))
+        c["softmax_scale"] = kw["scale"]
+        ref = orc.forward(c["q"], c["k"], c["bias"], c["v"], c["softmax_scale"])
+        r = run_path(c, engine=engine)
+        check_o(bf16_to_f64(r["out"]), ref, f"{kw} {engine}")
+
+
+@pytest.mark.parametrize("engine", ENGINES)
+def test_forward_deterministic(engine):
+    c = make_custom(2, 2, 300, 72, seed=9)
+    a = run_path(c, engine=engine)["out"].clone()
+    b = run_path(c, engine=engine)["out"]
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_device_errors_are_reported():
+    x = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16, device="cuda")
+    bits = torch.empty(1, 1, 4, 2, dtype=torch.int32, device="cuda")
+    alpha = torch.empty(1, 1, 4, dtype=torch.float32, device="cuda")
+    L = binattn.lib()
+    import ctypes
+    rc = L.binattn_pack(ctypes.c_void_p(x.data_ptr() + 2), 1, 1, 1, 4, 64,
+                        ctypes.c_void_p(bits.data_ptr()), ctypes.c_void_p(alpha.data_ptr()), None)
+    assert rc == 4
+    binattn.device_status()
