@@ -14,7 +14,7 @@ from parity import bf16_to_f64, check_o, dev, run_path, sample_rows
 
 pytestmark = pytest.mark.gpu
 
-ENGINES = ["simt"]
+ENGINES = ["simt", "popc_tc", "tc"]
 
 SMALL_SHAPES = [  # (B, H, N, d): several tiles and a ragged tail
     (1, 2, 256, 64), (2, 3, 129, 72), (1, 2, 197, 64), (1, 1, 1, 64), (2, 1, 7, 32),
