@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the bounded oracle sample")
+    ap.add_argument("--profile-once", action="store_true",
+                    help="run --warmup plain steps (with bias) and exit: the command profiled by ncu")
+    ap.add_argument("--no-bias", action="store_true", help="with --profile-once: steps without bias")
     return ap.parse_args()
 
 
@@ -153,21 +156,29 @@ def cpu_oracle_sample(w, with_bias, target_s, inp=None):
         inp = make_inputs(w, with_bias=with_bias)
     T = w.B * w.H * w.N
     rng = np.random.default_rng(123)
-    n = 64
-    t0 = time.perf_counter()
-    orc.forward_rows(inp["q"], inp["k"], inp["bias"] if with_bias else None, inp["v"],
-                     inp["softmax_scale"], rng.integers(0, T, size=n))
-    t1 = time.perf_counter() - t0
-    n2 = int(min(T, max(n, n * target_s / max(t1, 1e-3))))
-    rows = rng.integers(0, T, size=n2)
-    t0 = time.perf_counter()
-    orc.forward_rows(inp["q"], inp["k"], inp["bias"] if with_bias else None, inp["v"],
-                     inp["softmax_scale"], rows)
-    dt = time.perf_counter() - t0
-    ms = dt * 1e3 * T / n2
+    bias = inp["bias"] if with_bias else None
+
+    def run(n):
+        rows = rng.integers(0, T, size=n)
+        t0 = time.perf_counter()
+        orc.forward_rows(inp["q"], inp["k"], bias, inp["v"], inp["softmax_scale"], rows)
+        return time.perf_counter() - t0
+
+    # t(n) = a + b n: a = signs and scales of every token (done once per call),
+    # b = one query row's scores, softmax and P.V. Two sizes fix a and b.
+    n1 = 256
+    t1 = run(n1)
+    n2 = n1 * 4
+    t2 = run(n2)
+    b = max((t2 - t1) / (n2 - n1), 1e-9)
+    a = max(t1 - b * n1, 0.0)
+    n3 = int(min(T, max(n2, (target_s - a) / b)))
+    t3 = run(n3)
+    b3 = max((t3 - a) / n3, 1e-9)
+    ms = (a + b3 * T) * 1e3
     return dict(value=ms, unit="ms", cores=orc.num_threads(), kind="oracle",
-                sample=f"{n2} of {T} query rows (signs/scales of all tokens + those rows' "
-                       f"scores, softmax and P.V), {dt:.1f} s, extrapolated linearly to all rows")
+                sample=f"{n3} of {T} query rows ({t3:.1f} s; per-call token prep {a:.2f} s, "
+                       f"{b3 * 1e3:.3f} ms per row), extrapolated to all rows as prep + rows x per-row")
 
 
 def run_reference(args, w, rank):
@@ -245,6 +256,13 @@ def run_gpu(args, w, rank, world, local_rank):
         t = torch.tensor([x], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
+
+    if args.profile_once:
+        for _ in range(args.warmup):
+            step(None if args.no_bias else bias)
+        torch.cuda.synchronize()
+        binattn.device_status(stream)
+        return
 
     # warm-up (untimed), including one checked run
     for _ in range(max(args.warmup, 3)):

@@ -10,17 +10,23 @@
 // 128-row tiles t = 0, 1, and streams all keys in tiles of 128:
 //   warps 0-7   softmax: warpgroup t (warps 4t..4t+3), thread = one query row.
 //   warp 8      MMA issuer (one thread): tcgen05.mma, tcgen05.commit.
-//   warps 9-11  producers: per key tile, alpha_k, the key sign bits (expanded to
-//               +-1 bf16 for TC, copied as words for POPC_TC) and V, into a
-//               two-stage shared-memory ring.
-// Tensor memory (512 columns): S_t at column 128t (fp32, 128 keys), P_t written
-// back over the first 64 columns of S_t as bf16 pairs, O_t at 256 + 128t.
+//   warps 9-11  loaders, in one of two modes:
+//     TMA mode (KDIM <= 80, N % 8 == 0): warp 9 issues TMA / bulk copies of V
+//       and alpha_k (and the sign words for POPC_TC); warp 10 issues the bias
+//       tiles, each as soon as its stage is free; warp 11 loads the key sign
+//       words and expands them to +-1 bf16 operand tiles (TC engine). Q_t lives
+//       in tensor memory next to O_t.
+//     load mode (other shapes): warps 9-11 load the same data with batched
+//       plain loads; Q_t lives in shared memory; softmax threads read the bias.
+// Tensor memory (512 columns): S_t at 128t (fp32, 128 keys); P_t written back
+// over the first 64 columns of S_t as bf16 pairs; O_t at 256 + 128t (KDIM
+// columns); in TMA mode Q_t at 256 + 128t + KDIM (KDIM/2 columns of bf16 pairs).
 //
 // TC engine: S_t = Q_t K^T on the tensor core with +-1 bf16 operands. Pad
 // channels of Q are 0, so every product is +-1 or 0 and the fp32 accumulator
 // holds the exact integer score d - 2 popcount(q XOR k).
 // POPC_TC engine: the softmax threads compute S with __popc over the packed
-// words (binary_score), the tensor core does P.V only.
+// words (binary_score); the tensor core does P.V only.
 //
 // Softmax (per row, fp32, online over key tiles): logit = (S * alpha_k) *
 // (scale * alpha_q) + bias; running max m and sum l; O_t in TMEM is rescaled by
@@ -31,6 +37,10 @@
 // records a device status code, leaves its loops, waits for its own MMAs and
 // frees its tensor memory.
 #pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cstring>
+#include <mutex>
 #include <string>
 #include "binattn.h"
 #include "common.cuh"
@@ -51,38 +61,59 @@ constexpr int kStages = 2;
 constexpr int kWarps = 12;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMmaWarp = 8;
-constexpr int kProdWarp0 = 9;
-constexpr int kProdThreads = 96;
+constexpr int kLoadWarp0 = 9;
+constexpr int kLoadThreads = 96;     // load mode: warps 9-11
+constexpr int kBiasWarp = 10;        // TMA mode: bias tile issuer
+constexpr int kExpandWarp0 = 11;     // TMA mode: warp 11 expands signs
+constexpr int kExpandThreads = 32;
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescale = 5.545177444479562f;  // 8 * ln 2: rescale O only past 2^8
 
-// Shared-memory map (byte offsets). An "operand tile" is 128 rows x KDIM bf16.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
+}
+
+__host__ __device__ constexpr bool tma_mode_kdim(int kdim) { return kdim <= 80; }
+
+// Shared-memory map (byte offsets). An operand tile is 128 rows x KDIM bf16.
 //  Q_t, K_s  (K-major, no swizzle): 16-byte chunk (row r, channel group c) at
 //            (r / 8) * (KDIM * 16) + c * 128 + (r % 8) * 16
 //            -> descriptor LBO = 128 (next channel group), SBO = KDIM * 16 (next 8 rows).
 //  V_s       (MN-major, no swizzle): chunk (key j, d group g) at g * 2048 + j * 16
 //            -> descriptor LBO = 128 (next 8 keys), SBO = 2048 (next 8 d values).
-template <int KDIM>
+//            In TMA mode each d group is one TMA box of 8 x 128 elements.
+//  bias_s,t  (TMA mode) 128 rows x 128 keys bf16 as two 128B-swizzled boxes of
+//            64 keys: key k of row r at (k / 64) * 16384 + r * 128 +
+//            (((k % 64) / 8) ^ (r % 8)) * 16 + (k % 8) * 2.
+//  kb_s      sign words of the tile's keys, contiguous: key j word w at j * W + w.
+template <int KDIM, bool kTma>
 struct Layout {
   static constexpr int kTile = kKeys * KDIM * 2;
-  static constexpr int kLut = 0;                               // 256 x 16 B
-  static constexpr int kQ = 4096;                              // 2 tiles
-  static constexpr int kK = kQ + 2 * kTile;                    // kStages tiles
-  static constexpr int kV = kK + kStages * kTile;              // kStages tiles
-  static constexpr int kAk = kV + kStages * kTile;             // kStages x 128 fp32
-  static constexpr int kKb = kAk + kStages * kKeys * 4;        // kStages x 128 x 4 words
-  static constexpr int kBar = kKb + kStages * kKeys * 16;      // mbarriers
-  static constexpr int kNumBars = 2 * kStages + 7;
-  static constexpr int kMisc = kBar + 8 * kNumBars;            // tmem base, abort flag
+  static constexpr int kBiasTile = kRows * kKeys * 2;            // 32 KB
+  static constexpr int kLut = 0;                                 // 256 x 16 B
+  static constexpr int kQ = 4096;                                // load mode: 2 tiles
+  static constexpr int kK = kQ + (kTma ? 0 : 2 * kTile);         // kStages tiles
+  static constexpr int kV = kK + kStages * kTile;                // kStages tiles
+  static constexpr int kBias = (kV + kStages * kTile + 1023) / 1024 * 1024;  // TMA: [kStages][2]
+  static constexpr int kAk = kBias + (kTma ? kStages * 2 * kBiasTile : 0);  // kStages x 128 fp32
+  static constexpr int kKb = kAk + kStages * kKeys * 4;          // kStages x 128 x 4 words
+  static constexpr int kBar = kKb + kStages * kKeys * 16;
+  static constexpr int kNumBars = 32;
+  static constexpr int kMisc = kBar + 8 * kNumBars;              // tmem base, abort flag
   static constexpr int kBytes = kMisc + 16;
-  // at least this much dynamic shared memory, so that one CTA occupies an SM
-  // (each CTA allocates all 512 TMEM columns)
+  // at least this much, so that one CTA occupies an SM (each CTA allocates all
+  // 512 TMEM columns)
   static constexpr int kLaunchBytes = kBytes > 120 * 1024 ? kBytes : 120 * 1024;
 };
 
 struct Params {
   const uint32_t* qb;
   const uint32_t* kb;
+  const uint16_t* q;  // bf16 reference attention: Q [B,H,N,d]
+  const uint16_t* k;  // bf16 reference attention: K [B,H,N,d]
   const float* aq;
   const float* ak;
   const uint16_t* bias;
@@ -90,52 +121,114 @@ struct Params {
   uint16_t* out;
   int32_t* S;  // debug scores (dump mode)
   float scale;
-  int H, N, d;
+  int B, H, N, d;
 };
 
-template <int KDIM, bool kTcQK, bool kBias, bool kDump>
-__global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const Params p) {
-  using L = Layout<KDIM>;
+// Named barrier 1 over the load-mode loader warps with an AND reduction.
+__device__ __forceinline__ bool loaders_all(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "n"(kLoadThreads)
+      : "memory");
+  return r != 0;
+}
+
+// Score sources (template parameter kQK).
+constexpr int kQkPopc = 0;  // __popc in the softmax threads (POPC_TC engine)
+constexpr int kQkTc = 1;    // tcgen05.mma on +-1 operands expanded from sign bits (TC engine)
+constexpr int kQkRef = 2;   // tcgen05.mma on bf16 Q, K: full-precision reference attention
+
+template <int KDIM, bool kTma, int kQK, bool kBias, bool kDump>
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
+              const __grid_constant__ CUtensorMap tm_ak, const __grid_constant__ CUtensorMap tm_bias,
+              const __grid_constant__ CUtensorMap tm_k) {
+  constexpr bool kTcQK = kQK != kQkPopc;  // QK^T on the tensor core
+  constexpr bool kRef = kQK == kQkRef;
+  // K operand layout (K-major, no swizzle): binary = rows of KDIM*16 bytes per
+  // 8 keys (LBO 128, SBO KDIM*16); reference = one TMA box of 8 channels x 128
+  // keys per channel group (LBO 2048, SBO 128).
+  constexpr uint32_t kKLbo = kRef ? 2048 : 128;
+  constexpr uint32_t kKSbo = kRef ? 128 : KDIM * 16;
+  using L = Layout<KDIM, kTma>;
   constexpr int W = (KDIM + 31) / 32;  // packed words per token (= ceil(d / 32))
   constexpr int KCH = KDIM / 8;        // 16-byte channel groups per operand row
   constexpr uint32_t kIdescQK = idesc_bf16(kRows, kKeys, false);
   constexpr uint32_t kIdescPV = idesc_bf16(kRows, KDIM, true);
+  static_assert(!kTma || tma_mode_kdim(KDIM), "TMA mode keeps Q in TMEM: KDIM <= 80");
+  static_assert(KCH % 2 == 0, "KDIM is a multiple of 16");
 
   extern __shared__ __align__(1024) uint8_t smem[];
   uint4* lut = reinterpret_cast<uint4*>(smem + L::kLut);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* kv_full = bars;                  // [kStages] producers -> consumers
-  uint64_t* kv_empty = bars + kStages;       // [kStages] MMA commit -> producers
-  uint64_t* s_full = bars + 2 * kStages;     // [2] QK commit -> softmax t
-  uint64_t* p_full = s_full + 2;             // [2] softmax t (128 arrivals) -> MMA
-  uint64_t* o_done = p_full + 2;             // [2] PV commit -> softmax t
-  uint64_t* drain = o_done + 2;              // error path only
+  uint64_t* kv_full = bars + 0;    // [2] load mode: loaders -> all;  TMA mode: V + alpha_k tx
+  uint64_t* kv_empty = bars + 2;   // [2] MMA commit after PV of the stage
+  uint64_t* kb_full = bars + 4;    // [2] TMA mode: sign-word bulk copy tx
+  uint64_t* k_full = bars + 6;     // [2] TMA mode: expanders -> MMA
+  uint64_t* k_empty = bars + 8;    // [2] TMA mode: MMA commit after QK of the stage
+  uint64_t* b_full = bars + 10;    // [2][2] TMA mode: bias tile tx (stage, t)
+  uint64_t* b_empty = bars + 14;   // [2][2] TMA mode: softmax t done with bias tile
+  uint64_t* s_full = bars + 18;    // [2] QK commit -> softmax t
+  uint64_t* p_full = bars + 20;    // [2] softmax t (128 arrivals) -> MMA
+  uint64_t* o_done = bars + 22;    // [2] PV commit -> softmax t
+  uint64_t* drain = bars + 24;     // error path only
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y, h = bh % p.H;
+  // Batch entries sharing a bias tile (same h and query tile) are adjacent in
+  // launch order, so the bias tile is fetched from HBM once.
+  const int b = blockIdx.x % p.B;
+  const int qt = blockIdx.x / p.B;
+  const int h = blockIdx.y;
+  const int bh = b * p.H + h;
   const int N = p.N, d = p.d;
   const size_t tok0 = static_cast<size_t>(bh) * N;
-  const int q0 = blockIdx.x * 2 * kRows;
+  const int q0 = qt * 2 * kRows;
   const int ntiles = (N + kKeys - 1) / kKeys;
+  const int dgroups = d / 8;
 
   // ---------------------------------------------------------------- setup
   // LUT: 8 sign bits -> 8 bf16 values, element e = +1.0 if bit e is set, else -1.0.
-  for (int b = threadIdx.x; b < 256; b += kThreads) {
+  for (int i = threadIdx.x; i < 256; i += kThreads) {
     uint32_t w[4];
 #pragma unroll
     for (int pr = 0; pr < 4; ++pr) {
-      const uint32_t lo = ((b >> (2 * pr)) & 1) ? 0x3F80u : 0xBF80u;
-      const uint32_t hi = ((b >> (2 * pr + 1)) & 1) ? 0x3F80u : 0xBF80u;
+      const uint32_t lo = ((i >> (2 * pr)) & 1) ? 0x3F80u : 0xBF80u;
+      const uint32_t hi = ((i >> (2 * pr + 1)) & 1) ? 0x3F80u : 0xBF80u;
       w[pr] = lo | (hi << 16);
     }
-    lut[b] = make_uint4(w[0], w[1], w[2], w[3]);
+    lut[i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if constexpr (kTma && !kDump) {
+    // V pad groups (g >= d / 8) are never written by TMA: zero them once (and
+    // the K pad groups of the reference kernel, which would otherwise hold
+    // whatever shared memory held before).
+    const int npad = (KCH - dgroups) * kKeys;
+    for (int e = threadIdx.x; e < kStages * npad; e += kThreads) {
+      const int s = e / npad, rem = e % npad;
+      const int g = dgroups + rem / kKeys, kk = rem % kKeys;
+      *reinterpret_cast<uint4*>(smem + L::kV + s * L::kTile + g * 2048 + kk * 16) = make_uint4(0, 0, 0, 0);
+      if (kRef)
+        *reinterpret_cast<uint4*>(smem + L::kK + s * L::kTile + g * 2048 + kk * 16) = make_uint4(0, 0, 0, 0);
+    }
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&kv_full[s], kProdThreads);
+      mbar_init(&kv_full[s], kTma ? 1 : kLoadThreads);
       mbar_init(&kv_empty[s], 1);
+      mbar_init(&kb_full[s], 1);
+      mbar_init(&k_full[s], kRef ? 1 : kExpandThreads);
+      mbar_init(&k_empty[s], 1);
+      for (int t = 0; t < 2; ++t) {
+        mbar_init(&b_full[s * 2 + t], 1);
+        mbar_init(&b_empty[s * 2 + t], kRows);
+      }
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
@@ -152,81 +245,257 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const Params p) {
     tc_fence_before();
   }
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
 
-  // Softmax threads: this thread's query row, and (TC) its +-1 row of Q_t.
+  // Softmax threads: this thread's query row and its +-1 row of Q_t.
   const int t = warp >> 2;                      // warpgroup (valid for warps 0-7)
   const int r = ((warp & 3) << 5) | lane;       // row within the tile = TMEM lane
   const int row = q0 + t * kRows + r;
   const bool row_valid = warp < 8 && row < N;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   uint32_t qw[W];
 #pragma unroll
-  for (int w = 0; w < W; ++w) qw[w] = row_valid ? p.qb[(tok0 + row) * W + w] : 0u;
-  if (kTcQK && warp < 8) {
-    uint8_t* qs = smem + L::kQ + t * L::kTile;
-#pragma unroll
-    for (int c = 0; c < KCH; ++c) {
-      uint4 val = make_uint4(0, 0, 0, 0);  // pad channels (c >= d) are 0
-      if (8 * c < d) val = lut[(qw[c >> 2] >> (8 * (c & 3))) & 0xFFu];
-      *reinterpret_cast<uint4*>(qs + (r >> 3) * (KDIM * 16) + c * 128 + (r & 7) * 16) = val;
+  for (int w = 0; w < W; ++w) qw[w] = (!kRef && row_valid) ? p.qb[(tok0 + row) * W + w] : 0u;
+  // Channel group c (8 channels, 16 bytes) of this row's Q operand row.
+  auto q_group = [&](int c) -> uint4 {
+    uint4 val = make_uint4(0, 0, 0, 0);  // pad channels (>= d) are 0
+    if (8 * c < d) {
+      if constexpr (kRef) {
+        if (row_valid) val = *reinterpret_cast<const uint4*>(p.q + (tok0 + row) * d + 8 * c);
+      } else {
+        val = lut[(qw[c >> 2] >> (8 * (c & 3))) & 0xFFu];
+      }
     }
-    fence_proxy_async_smem();
+    return val;
+  };
+  if (kTcQK && warp < 8) {
+    if constexpr (kTma) {
+      // Q_t row in TMEM at column 256 + 128t + KDIM: column c2 holds channels
+      // 2*c2 (low half) and 2*c2 + 1, as bf16 +-1 (0 for pad channels).
+      const uint32_t qcol = tmem + lane_base + 256 + 128 * t + KDIM;
+#pragma unroll
+      for (int c = 0; c < KCH; c += 2) {
+        uint32_t wv[8];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const uint4 val = q_group(c + h2);
+          wv[4 * h2 + 0] = val.x;
+          wv[4 * h2 + 1] = val.y;
+          wv[4 * h2 + 2] = val.z;
+          wv[4 * h2 + 3] = val.w;
+        }
+        tmem_st8(qcol + 4 * c, wv);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+    } else {
+      uint8_t* qs = smem + L::kQ + t * L::kTile;
+#pragma unroll
+      for (int c = 0; c < KCH; ++c)
+        *reinterpret_cast<uint4*>(qs + (r >> 3) * (KDIM * 16) + c * 128 + (r & 7) * 16) = q_group(c);
+    }
   }
+  fence_proxy_async_smem();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
 
-  if (warp >= kProdWarp0) {
-    // ------------------------------------------------------------ producers
-    const int pt = threadIdx.x - kProdWarp0 * 32;
-    const int dgroups = d / 8;
-    for (int j = 0; j < ntiles; ++j) {
-      const int s = j % kStages;
-      if (j >= kStages && !mbar_wait(&kv_empty[s], ((j / kStages) - 1) & 1, abort)) break;
-      const int j0 = j * kKeys;
-      if constexpr (!kDump) {  // the debug-scores variant gets no alpha_k / V
-        float* aks = reinterpret_cast<float*>(smem + L::kAk) + s * kKeys;
-        for (int kk = pt; kk < kKeys; kk += kProdThreads)
-          aks[kk] = (j0 + kk < N) ? p.ak[tok0 + j0 + kk] : 0.f;
-      }
-      if constexpr (kTcQK) {
-        uint8_t* ks = smem + L::kK + s * L::kTile;
-        for (int e = pt; e < kKeys * KCH; e += kProdThreads) {
-          const int kk = e / KCH, c = e % KCH, key = j0 + kk;
-          uint4 val = make_uint4(0, 0, 0, 0);
-          if (key < N && 8 * c < d)
-            val = lut[(p.kb[(tok0 + key) * W + (c >> 2)] >> (8 * (c & 3))) & 0xFFu];
-          *reinterpret_cast<uint4*>(ks + (kk >> 3) * (KDIM * 16) + c * 128 + (kk & 7) * 16) = val;
-        }
-      } else {
-        uint32_t* kbs = reinterpret_cast<uint32_t*>(smem + L::kKb) + s * kKeys * 4;
-        for (int e = pt; e < kKeys * W; e += kProdThreads) {
-          const int kk = e / W, w = e % W, key = j0 + kk;
-          kbs[kk * 4 + w] = key < N ? p.kb[(tok0 + key) * W + w] : 0u;
-        }
-      }
-      if constexpr (!kDump) {
-        uint8_t* vs = smem + L::kV + s * L::kTile;
-        constexpr int kVIters = (kKeys * KCH + kProdThreads - 1) / kProdThreads;
-        uint4 vbuf[kVIters];
-#pragma unroll
-        for (int it = 0; it < kVIters; ++it) {
-          const int e = pt + it * kProdThreads;
-          const int kk = e / KCH, g = e % KCH, key = j0 + kk;
-          vbuf[it] = make_uint4(0, 0, 0, 0);
-          if (e < kKeys * KCH && key < N && g < dgroups)
-            vbuf[it] = __ldg(reinterpret_cast<const uint4*>(p.v + (tok0 + key) * d + 8 * g));
-        }
-#pragma unroll
-        for (int it = 0; it < kVIters; ++it) {
-          const int e = pt + it * kProdThreads;
-          if (e < kKeys * KCH) {
-            const int kk = e / KCH, g = e % KCH;
-            *reinterpret_cast<uint4*>(vs + g * 2048 + kk * 16) = vbuf[it];
+  if (warp >= kLoadWarp0) {
+    if constexpr (kTma) {
+      if (warp == kLoadWarp0) {
+        // ------------------------------------------------ TMA issuer (one thread)
+        if (lane == 0) {
+          for (int j = 0; j < ntiles; ++j) {
+            const int s = j % kStages;
+            const uint32_t ph_prev = ((j / kStages) - 1) & 1;
+            const int j0 = j * kKeys;
+            const int nk = min(kKeys, N - j0);
+            // Stage s is free once tile j - kStages is done with it: its QK MMAs
+            // (TC: K operand and sign words) and its P.V MMAs (V, alpha_k, and
+            // for POPC_TC the sign words read by the softmax threads).
+            if (j >= kStages) {
+              if (kRef && !mbar_wait(&k_empty[s], ph_prev, abort)) break;
+              if (!kDump && !mbar_wait(&kv_empty[s], ph_prev, abort)) break;
+            }
+            if constexpr (kRef) {  // bf16 K: one box of 8 channels x 128 keys per group
+              mbar_arrive_expect_tx(&k_full[s], dgroups * 2048);
+              for (int g = 0; g < dgroups; ++g)
+                tma_load_3d(smem + L::kK + s * L::kTile + g * 2048, &tm_k, 8 * g, j0, bh, &k_full[s]);
+            } else if constexpr (!kTcQK) {
+              // POPC_TC: sign words for the softmax threads, nk keys x W words,
+              // contiguous and 16-byte aligned (N % 8 == 0). (For TC the
+              // expander warps load the words themselves.)
+              const uint32_t nbytes = static_cast<uint32_t>(nk * W * 4);
+              mbar_arrive_expect_tx(&kb_full[s], nbytes);
+              bulk_load(smem + L::kKb + s * kKeys * 16, p.kb + (tok0 + j0) * W, nbytes, &kb_full[s]);
+            }
+            if constexpr (!kDump) {
+              mbar_arrive_expect_tx(&kv_full[s], dgroups * 2048 + (kRef ? 0 : kKeys * 4));
+              for (int g = 0; g < dgroups; ++g)
+                tma_load_3d(smem + L::kV + s * L::kTile + g * 2048, &tm_v, 8 * g, j0, bh, &kv_full[s]);
+              if (!kRef) tma_load_2d(smem + L::kAk + s * kKeys * 4, &tm_ak, j0, bh, &kv_full[s]);
+            }
           }
         }
+        __syncwarp();
+      } else if (warp == kBiasWarp) {
+        // ------------------------------------------------ bias issuer (one thread)
+        // The bias tile (128 rows x 128 keys of warpgroup t) is the largest
+        // stream; each is requested as soon as warpgroup t released the stage.
+        if (kBias && !kDump && lane == 0) {
+          for (int j = 0; j < ntiles; ++j) {
+            const int s = j % kStages;
+            const int j0 = j * kKeys;
+            bool ok = true;
+            for (int tt = 0; tt < 2; ++tt) {
+              uint64_t* bf = &b_full[s * 2 + tt];
+              if (j >= kStages && !(ok = mbar_wait(&b_empty[s * 2 + tt], ((j / kStages) - 1) & 1, abort)))
+                break;
+              uint8_t* dst = smem + L::kBias + (s * 2 + tt) * L::kBiasTile;
+              mbar_arrive_expect_tx(bf, L::kBiasTile);
+              tma_load_3d(dst, &tm_bias, j0, q0 + tt * kRows, h, bf);
+              tma_load_3d(dst + L::kBiasTile / 2, &tm_bias, j0 + 64, q0 + tt * kRows, h, bf);
+            }
+            if (!ok) break;
+          }
+        }
+        __syncwarp();
+      } else if (kTcQK && !kRef) {
+        // ------------------------------------------------ sign expanders
+        // Thread et owns keys et + 32u of every tile: it loads their sign words
+        // itself (the next tile's words are in flight while it waits for the
+        // stage) and writes their +-1 rows; consecutive threads write
+        // consecutive keys, which keeps the 16-byte stores conflict-free.
+        constexpr int kPer = kKeys / kExpandThreads;
+        const int et = threadIdx.x - kExpandWarp0 * 32;
+        uint32_t wd[kPer][W];
+        auto load_words = [&](int j) {
+#pragma unroll
+          for (int u = 0; u < kPer; ++u) {
+            const int key = j * kKeys + et + u * kExpandThreads;
+#pragma unroll
+            for (int w = 0; w < W; ++w) wd[u][w] = key < N ? p.kb[(tok0 + key) * W + w] : 0u;
+          }
+        };
+        load_words(0);
+        for (int j = 0; j < ntiles; ++j) {
+          const int s = j % kStages;
+          if (j >= kStages && !mbar_wait(&k_empty[s], ((j / kStages) - 1) & 1, abort)) break;
+          uint8_t* ks = smem + L::kK + s * L::kTile;
+#pragma unroll
+          for (int u = 0; u < kPer; ++u) {
+            const int kk = et + u * kExpandThreads;
+#pragma unroll
+            for (int c = 0; c < KCH; ++c) {
+              uint4 val = make_uint4(0, 0, 0, 0);
+              if (8 * c < d) val = lut[(wd[u][c >> 2] >> (8 * (c & 3))) & 0xFFu];
+              *reinterpret_cast<uint4*>(ks + (kk >> 3) * (KDIM * 16) + c * 128 + (kk & 7) * 16) = val;
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&k_full[s]);
+          if (j + 1 < ntiles) load_words(j + 1);
+        }
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&kv_full[s]);
+    } else {
+      // -------------------------------------------- loaders (load mode)
+      // Per key tile: (A) issue every global load of the tile at once (sign
+      // words, alpha_k, V), (B) store them into the stage, (C, TC) once all
+      // loaders have stored, expand the sign words to +-1 bf16.
+      const int pt = threadIdx.x - kLoadWarp0 * 32;
+      constexpr int kKbIters = (kKeys * W + kLoadThreads - 1) / kLoadThreads;
+      constexpr int kAkIters = (kKeys + kLoadThreads - 1) / kLoadThreads;
+      constexpr int kVIters = (kKeys * KCH + kLoadThreads - 1) / kLoadThreads;
+      for (int j = 0; j < ntiles; ++j) {
+        const int s = j % kStages;
+        // All 96 loaders agree (barrier with AND reduction) so that either all
+        // reach the named barrier below or all leave the loop.
+        const bool ok = j < kStages || mbar_wait(&kv_empty[s], ((j / kStages) - 1) & 1, abort);
+        if (!loaders_all(ok)) break;
+        const int j0 = j * kKeys;
+        const int nk = min(kKeys, N - j0);
+        uint32_t kbuf[kKbIters];
+#pragma unroll
+        for (int it = 0; it < kKbIters; ++it) {
+          const int e = pt + it * kLoadThreads;
+          kbuf[it] = (!kRef && e < nk * W) ? p.kb[(tok0 + j0) * W + e] : 0u;
+        }
+        uint4 krow[kRef ? kVIters : 1];
+        if constexpr (kRef) {  // bf16 K rows, channel group g of key kk -> g * 2048 + kk * 16
+#pragma unroll
+          for (int it = 0; it < kVIters; ++it) {
+            const int e = pt + it * kLoadThreads;
+            const int kk = e / KCH, g = e % KCH;
+            krow[it] = make_uint4(0, 0, 0, 0);
+            if (kk < nk && g < dgroups)
+              krow[it] = __ldg(reinterpret_cast<const uint4*>(p.k + (tok0 + j0 + kk) * d + 8 * g));
+          }
+        }
+        float abuf[kAkIters];
+        uint4 vbuf[kDump ? 1 : kVIters];
+        if constexpr (!kDump) {  // the debug-scores variant gets no alpha_k / V
+#pragma unroll
+          for (int it = 0; it < kAkIters; ++it) {
+            const int kk = pt + it * kLoadThreads;
+            abuf[it] = (!kRef && kk < nk) ? p.ak[tok0 + j0 + kk] : 0.f;
+          }
+#pragma unroll
+          for (int it = 0; it < kVIters; ++it) {
+            const int e = pt + it * kLoadThreads;
+            const int kk = e / KCH, g = e % KCH;
+            vbuf[it] = make_uint4(0, 0, 0, 0);
+            if (kk < nk && g < dgroups)
+              vbuf[it] = __ldg(reinterpret_cast<const uint4*>(p.v + (tok0 + j0 + kk) * d + 8 * g));
+          }
+        }
+        uint32_t* kbs = reinterpret_cast<uint32_t*>(smem + L::kKb + s * kKeys * 16);
+#pragma unroll
+        for (int it = 0; it < kKbIters; ++it) {
+          const int e = pt + it * kLoadThreads;
+          if (e < kKeys * W) kbs[e] = kbuf[it];
+        }
+        if constexpr (kRef) {
+          uint8_t* ks = smem + L::kK + s * L::kTile;
+#pragma unroll
+          for (int it = 0; it < kVIters; ++it) {
+            const int e = pt + it * kLoadThreads;
+            if (e < kKeys * KCH) {
+              const int kk = e / KCH, g = e % KCH;
+              *reinterpret_cast<uint4*>(ks + g * 2048 + kk * 16) = krow[it];
+            }
+          }
+        }
+        if constexpr (!kDump) {
+          float* aks = reinterpret_cast<float*>(smem + L::kAk) + s * kKeys;
+#pragma unroll
+          for (int it = 0; it < kAkIters; ++it) {
+            const int kk = pt + it * kLoadThreads;
+            if (kk < kKeys) aks[kk] = abuf[it];
+          }
+          uint8_t* vs = smem + L::kV + s * L::kTile;
+#pragma unroll
+          for (int it = 0; it < kVIters; ++it) {
+            const int e = pt + it * kLoadThreads;
+            if (e < kKeys * KCH) {
+              const int kk = e / KCH, g = e % KCH;
+              *reinterpret_cast<uint4*>(vs + g * 2048 + kk * 16) = vbuf[it];
+            }
+          }
+        }
+        if constexpr (kTcQK && !kRef) {
+          asm volatile("bar.sync 1, %0;" ::"n"(kLoadThreads) : "memory");  // stores done
+          uint8_t* ks = smem + L::kK + s * L::kTile;
+#pragma unroll 4
+          for (int e = pt; e < kKeys * KCH; e += kLoadThreads) {
+            const int c = e / kKeys, kk = e % kKeys;  // consecutive threads: consecutive keys
+            uint4 val = make_uint4(0, 0, 0, 0);
+            if (8 * c < d) val = lut[(kbs[kk * W + (c >> 2)] >> (8 * (c & 3))) & 0xFFu];
+            *reinterpret_cast<uint4*>(ks + (kk >> 3) * (KDIM * 16) + c * 128 + (kk & 7) * 16) = val;
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&kv_full[s]);
+      }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -234,27 +503,33 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const Params p) {
       const uint32_t q_base = smem_u32(smem + L::kQ);
       const uint32_t k_base = smem_u32(smem + L::kK);
       const uint32_t v_base = smem_u32(smem + L::kV);
+      uint64_t* kready = kTma ? k_full : kv_full;  // "K operand stage s is ready"
       auto issue_qk = [&](int tt, int s) {
 #pragma unroll
         for (int ks = 0; ks < KDIM / 16; ++ks) {
-          const uint64_t a = smem_desc(q_base + tt * L::kTile + ks * 256, 128, KDIM * 16);
-          const uint64_t b = smem_desc(k_base + s * L::kTile + ks * 256, 128, KDIM * 16);
-          mma_ss(tmem + tt * 128, a, b, kIdescQK, ks > 0);
+          const uint64_t bdesc = smem_desc(k_base + s * L::kTile + ks * 2 * kKLbo, kKLbo, kKSbo);
+          if constexpr (kTma) {
+            mma_ts(tmem + tt * 128, tmem + 256 + 128 * tt + KDIM + ks * 8, bdesc, kIdescQK, ks > 0);
+          } else {
+            const uint64_t adesc = smem_desc(q_base + tt * L::kTile + ks * 256, 128, KDIM * 16);
+            mma_ss(tmem + tt * 128, adesc, bdesc, kIdescQK, ks > 0);
+          }
         }
         mma_commit(&s_full[tt]);
       };
       bool ok = true;
       if constexpr (kTcQK) {
-        ok = mbar_wait(&kv_full[0], 0, abort);
+        ok = mbar_wait(&kready[0], 0, abort);
         if (ok) {
           tc_fence_after();
           issue_qk(0, 0);
           issue_qk(1, 0);
+          if (kTma) mma_commit(&k_empty[0]);
         }
       }
       for (int j = 0; ok && j < ntiles; ++j) {
         const int s = j % kStages;
-        if (!kTcQK) {
+        if (!kDump && (kTma || !kTcQK)) {  // V ready (load mode TC: implied by kready)
           if (!(ok = mbar_wait(&kv_full[s], (j / kStages) & 1, abort))) break;
           tc_fence_after();
         }
@@ -264,18 +539,19 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const Params p) {
           if constexpr (!kDump) {
 #pragma unroll
             for (int ks = 0; ks < kKeys / 16; ++ks) {
-              const uint64_t b = smem_desc(v_base + s * L::kTile + ks * 256, 128, 2048);
-              mma_ts(tmem + 256 + tt * 128, tmem + tt * 128 + ks * 8, b, kIdescPV, (j > 0 || ks > 0));
+              const uint64_t bdesc = smem_desc(v_base + s * L::kTile + ks * 256, 128, 2048);
+              mma_ts(tmem + 256 + tt * 128, tmem + tt * 128 + ks * 8, bdesc, kIdescPV, (j > 0 || ks > 0));
             }
             mma_commit(&o_done[tt]);
           }
           if (kTcQK && j + 1 < ntiles) {
             const int s1 = (j + 1) % kStages;
             if (tt == 0) {
-              if (!(ok = mbar_wait(&kv_full[s1], ((j + 1) / kStages) & 1, abort))) break;
+              if (!(ok = mbar_wait(&kready[s1], ((j + 1) / kStages) & 1, abort))) break;
               tc_fence_after();
             }
             issue_qk(tt, s1);
+            if (kTma && tt == 1) mma_commit(&k_empty[s1]);
           }
         }
         mma_commit(&kv_empty[s]);
@@ -284,11 +560,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const Params p) {
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- softmax
-    const float ci = (!kDump && row_valid) ? p.scale * p.aq[tok0 + row] : 0.f;
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    // per-row factor of the logit: scale * alpha_q (binary) or scale (reference)
+    const float ci = kRef ? p.scale : ((!kDump && row_valid) ? p.scale * p.aq[tok0 + row] : 0.f);
     const uint32_t s_col = tmem + lane_base + t * 128;
     const uint32_t o_col = tmem + lane_base + 256 + t * 128;
-    const uint16_t* brow = kBias && row_valid ? p.bias + (static_cast<size_t>(h) * N + row) * N : nullptr;
+    const uint16_t* brow =
+        (kBias && !kTma && row_valid) ? p.bias + (static_cast<size_t>(h) * N + row) * N : nullptr;
     const bool bias_vec = (N % 8) == 0;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
@@ -298,9 +575,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const Params p) {
     };
     for (int j = 0; j < ntiles; ++j) {
       const int s = j % kStages;
+      const uint32_t ph = (j / kStages) & 1;
       const int j0 = j * kKeys;
-      float x[kKeys];
-      if (!(ok = wait_all(&kv_full[s], (j / kStages) & 1))) break;
+      float2 xs[kKeys / 2];  // this row's 128 scores, then logits (8-byte aligned storage)
+      float* x = reinterpret_cast<float*>(xs);
+      if (!kRef && (!kDump || !kTma)) {  // alpha_k (and in load mode sign words) of stage s
+        if (!(ok = wait_all(&kv_full[s], ph))) break;
+      }
       if constexpr (kTcQK) {
         if (!(ok = wait_all(&s_full[t], j & 1))) break;
         tc_fence_after();
@@ -308,15 +589,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const Params p) {
         for (int c = 0; c < kKeys; c += 32) tmem_ld32(s_col + c, reinterpret_cast<uint32_t*>(x + c));
         tmem_ld_wait();
       } else {
-        const uint32_t* kbs = reinterpret_cast<const uint32_t*>(smem + L::kKb) + s * kKeys * 4;
+        if (kTma && !(ok = wait_all(&kb_full[s], ph))) break;
+        const uint32_t* kbs = reinterpret_cast<const uint32_t*>(smem + L::kKb + s * kKeys * 16);
 #pragma unroll
         for (int c = 0; c < kKeys; ++c)
-          x[c] = static_cast<float>(binary_score<W>(qw, kbs + c * 4, d));
+          x[c] = static_cast<float>(binary_score<W>(qw, kbs + c * W, d));
       }
       if constexpr (kDump) {
         if (row_valid) {
           int32_t* srow = p.S + (tok0 + row) * N + j0;
-#pragma unroll 8
+#pragma unroll
           for (int c = 0; c < kKeys; ++c)
             if (j0 + c < N) srow[c] = static_cast<int32_t>(x[c]);
         }
@@ -324,47 +606,86 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const Params p) {
         mbar_arrive(&p_full[t]);
         continue;
       }
-      // logits = S * alpha_k * (scale * alpha_q) + bias, keys >= N masked
+      // logits = S * alpha_k * (scale * alpha_q) + bias (packed fp32 pairs)
       const float* aks = reinterpret_cast<const float*>(smem + L::kAk) + s * kKeys;
-      const bool tail = j0 + kKeys > N;
-      float mx = -INFINITY;
+      const uint8_t* bsm = smem + L::kBias + (s * 2 + t) * L::kBiasTile + r * 128;
+      if (kBias && kTma) {
+        if (!(ok = wait_all(&b_full[s * 2 + t], ph))) break;
+      }
+      float2* x2 = xs;
+      const float2 ci2 = make_float2(ci, ci);
 #pragma unroll
       for (int c0 = 0; c0 < kKeys; c0 += 8) {
-        float bv[8];
+        float2 bv[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) bv[e] = 0.f;
-        if (kBias && row_valid) {
-          if (bias_vec && !tail) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(brow + j0 + c0);
+        for (int e = 0; e < 4; ++e) bv[e] = make_float2(0.f, 0.f);
+        if constexpr (kBias) {
+          uint4 raw = make_uint4(0, 0, 0, 0);
+          bool have = false;
+          if constexpr (kTma) {
+            const int chunk = (c0 & 63) >> 3;
+            raw = *reinterpret_cast<const uint4*>(bsm + (c0 >> 6) * (L::kBiasTile / 2) +
+                                                  ((chunk ^ (r & 7)) << 4));
+            have = true;
+          } else if (row_valid) {
+            if (bias_vec && j0 + c0 + 8 <= N) {
+              raw = *reinterpret_cast<const uint4*>(brow + j0 + c0);
+              have = true;
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                if (j0 + c0 + 2 * e < N) bv[e].x = bf16_bits_to_float(brow[j0 + c0 + 2 * e]);
+                if (j0 + c0 + 2 * e + 1 < N) bv[e].y = bf16_bits_to_float(brow[j0 + c0 + 2 * e + 1]);
+              }
+            }
+          }
+          if (have) {
             const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              bv[2 * e] = __uint_as_float(rw[e] << 16);
-              bv[2 * e + 1] = __uint_as_float(rw[e] & 0xFFFF0000u);
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              if (j0 + c0 + e < N) bv[e] = bf16_bits_to_float(brow[j0 + c0 + e]);
+            for (int e = 0; e < 4; ++e)
+              bv[e] = make_float2(__uint_as_float(rw[e] << 16), __uint_as_float(rw[e] & 0xFFFF0000u));
           }
         }
+        if constexpr (kRef) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int c = c0 + e;
-          float lg = fmaf(x[c] * aks[c], ci, bv[e]);
-          if (tail && j0 + c >= N) lg = -INFINITY;
-          x[c] = lg;
-          mx = fmaxf(mx, lg);
+          for (int e = 0; e < 4; ++e) x2[c0 / 2 + e] = __ffma2_rn(x2[c0 / 2 + e], ci2, bv[e]);
+        } else {
+          const float4 a0 = *reinterpret_cast<const float4*>(aks + c0);
+          const float4 a1 = *reinterpret_cast<const float4*>(aks + c0 + 4);
+          const float2 av[4] = {make_float2(a0.x, a0.y), make_float2(a0.z, a0.w),
+                                make_float2(a1.x, a1.y), make_float2(a1.z, a1.w)};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            x2[c0 / 2 + e] = __ffma2_rn(__fmul2_rn(x2[c0 / 2 + e], av[e]), ci2, bv[e]);
         }
       }
-      const float m_new = fmaxf(m, mx);
-      const float corr = ex2((m - m_new) * kLog2e);  // 0 on the first tile
+      if (kBias && kTma) mbar_arrive(&b_empty[s * 2 + t]);
+      if (j0 + kKeys > N) {  // last tile: keys >= N take no part (warp-uniform branch)
+#pragma unroll
+        for (int c = 0; c < kKeys; ++c)
+          if (j0 + c >= N) x[c] = -INFINITY;
+      }
+      // row max of the tile: four independent 3-input max chains
+      float mx4[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+      for (int c = 4; c < kKeys; c += 8) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mx4[e] = max3f(mx4[e], x[c + e], x[c + 4 + e < kKeys ? c + 4 + e : c + e]);
+      }
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      // Lazy rescale: the running max m only moves when the tile max exceeds it
+      // by more than kRescale (natural-log units, = 8 in log2 units). Until then
+      // every p = exp(logit - m) <= 2^8, exact enough in fp32 and bf16, and the
+      // final division by l (summed against the same m) cancels the offset.
+      const bool grow = mx > m + kRescale;
+      const float m_new = grow ? mx : m;
+      const float corr = grow ? ex2((m - m_new) * kLog2e) : 1.f;  // 0 on the first tile
       if (j > 0) {
-        // O_t must hold PV of tile j-1 before it is rescaled (and before P_t
-        // is overwritten, which the MMA ordering already guarantees).
+        // O_t holds PV of tile j-1 once QK of tile j completed (in-order tensor
+        // pipe); the wait makes that visible before O_t is rescaled.
         if (!(ok = wait_all(&o_done[t], (j - 1) & 1))) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, corr != 1.f)) {
+        if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
           for (int c = 0; c < KDIM; c += 16) {
             uint32_t ov[16];
@@ -378,17 +699,24 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const Params p) {
       }
       l *= corr;
       m = m_new;
-      const float nm = -m * kLog2e;
-      uint32_t pk[kKeys / 2];
+      // P = exp(logit - m) as bf16 pairs into TMEM over S_t, 32 keys at a time
+      const float2 l2e2 = make_float2(kLog2e, kLog2e);
+      const float2 nm2 = make_float2(-m * kLog2e, -m * kLog2e);
+      float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < kKeys; c += 2) {
-        const float p0 = ex2(fmaf(x[c], kLog2e, nm));
-        const float p1 = ex2(fmaf(x[c + 1], kLog2e, nm));
-        l += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
+      for (int c0 = 0; c0 < kKeys; c0 += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float2 a = __ffma2_rn(x2[c0 / 2 + e], l2e2, nm2);
+          const float2 pp = make_float2(ex2(a.x), ex2(a.y));
+          ls[e & 3] = __fadd2_rn(ls[e & 3], pp);
+          pk[e] = pack_bf16x2(pp.x, pp.y);
+        }
+        tmem_st16(s_col + c0 / 2, pk);
       }
-      tmem_st32(s_col, pk);
-      tmem_st32(s_col + 32, pk + 32);
+      l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y) + (ls[2].x + ls[2].y) + (ls[3].x + ls[3].y);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
@@ -440,18 +768,95 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_kernel(const Params p) {
   }
 }
 
-template <int KDIM, bool kTcQK, bool kBias, bool kDump>
-inline int launch_tc(const Params& prm, int B, int H, int N, cudaStream_t st, std::string* msg) {
-  auto kern = fwd_tc_kernel<KDIM, kTcQK, kBias, kDump>;
-  const int smem = Layout<KDIM>::kLaunchBytes;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) {
-    *msg = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);
-    return BINATTN_ERR_CUDA;
+// ------------------------------------------------------------------- host
+using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+struct TensorMaps {
+  CUtensorMap v, ak, bias, k;
+};
+
+// One [BH][N][d] bf16 tensor as boxes of 8 channels x 128 keys: each box is one
+// column of 16-byte chunks of the no-swizzle operand layouts above.
+inline bool make_rows_map(EncodeTiledFn enc, CUtensorMap* tm, const uint16_t* base, cuuint64_t BH,
+                          cuuint64_t N, cuuint64_t d, const char* what, std::string* msg) {
+  const cuuint32_t es[3] = {1, 1, 1};
+  const cuuint64_t dims[3] = {d, N, BH};
+  const cuuint64_t strides[2] = {d * 2, N * d * 2};
+  const cuuint32_t box[3] = {8, kKeys, 1};
+  CUresult rc = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(base), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (rc != CUDA_SUCCESS) {
+    *msg = std::string("tensor map (") + what + ") rejected: " + std::to_string(rc);
+    return false;
   }
-  dim3 grid((N + 2 * kRows - 1) / (2 * kRows), B * H);
-  kern<<<grid, kThreads, smem, st>>>(prm);
-  e = cudaGetLastError();
+  return true;
+}
+
+// Tensor maps of one call. Returns false (with a message) if the driver rejects one.
+inline bool make_maps(const Params& p, bool with_bias, bool ref, TensorMaps* tm, std::string* msg) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) {
+    *msg = "cuTensorMapEncodeTiled entry point unavailable";
+    return false;
+  }
+  const cuuint32_t es[3] = {1, 1, 1};
+  const cuuint64_t BH = static_cast<cuuint64_t>(p.B) * p.H, N = p.N, d = p.d;
+  if (!make_rows_map(enc, &tm->v, p.v, BH, N, d, "V", msg)) return false;
+  if (ref) {
+    if (!make_rows_map(enc, &tm->k, p.k, BH, N, d, "K", msg)) return false;
+  } else {  // alpha_k [BH][N] fp32: box 128 keys
+    const cuuint64_t dims[2] = {N, BH};
+    const cuuint64_t strides[1] = {N * 4};
+    const cuuint32_t box[2] = {kKeys, 1};
+    CUresult rc = enc(&tm->ak, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p.ak), dims,
+                      strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                      CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (rc != CUDA_SUCCESS) { *msg = "tensor map (alpha_k) rejected: " + std::to_string(rc); return false; }
+  }
+  if (with_bias) {  // bias [H][N rows][N keys] bf16: box 64 keys x 128 rows, 128B swizzle
+    const cuuint64_t dims[3] = {N, N, static_cast<cuuint64_t>(p.H)};
+    const cuuint64_t strides[2] = {N * 2, N * N * 2};
+    const cuuint32_t box[3] = {64, kRows, 1};
+    CUresult rc = enc(&tm->bias, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(p.bias),
+                      dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (rc != CUDA_SUCCESS) { *msg = "tensor map (bias) rejected: " + std::to_string(rc); return false; }
+  }
+  return true;
+}
+
+template <int KDIM, bool kTma, int kQK, bool kBias, bool kDump>
+inline int launch_tc(const Params& prm, const TensorMaps& tm, cudaStream_t st, std::string* msg) {
+  auto kern = fwd_tc_kernel<KDIM, kTma, kQK, kBias, kDump>;
+  constexpr int smem = Layout<KDIM, kTma>::kLaunchBytes;
+  static_assert(smem <= 227 * 1024, "shared memory over the sm_100 per-CTA limit");
+  static bool configured = false;  // attribute set once per instantiation
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) {
+      *msg = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);
+      return BINATTN_ERR_CUDA;
+    }
+    configured = true;
+  }
+  dim3 grid(static_cast<unsigned>(prm.B * ((prm.N + 2 * kRows - 1) / (2 * kRows))), prm.H);
+  kern<<<grid, kThreads, smem, st>>>(prm, tm.v, tm.ak, tm.bias, tm.k);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     *msg = std::string("fwd_tc_kernel launch: ") + cudaGetErrorString(e);
     return BINATTN_ERR_CUDA;
@@ -459,18 +864,32 @@ inline int launch_tc(const Params& prm, int B, int H, int N, cudaStream_t st, st
   return BINATTN_OK;
 }
 
-template <bool kTcQK, bool kBias, bool kDump>
-inline int dispatch_kdim(const Params& prm, int B, int H, int N, int d, cudaStream_t st,
-                         std::string* msg) {
-  switch ((d + 15) / 16) {
-    case 1: return launch_tc<16, kTcQK, kBias, kDump>(prm, B, H, N, st, msg);
-    case 2: return launch_tc<32, kTcQK, kBias, kDump>(prm, B, H, N, st, msg);
-    case 3: return launch_tc<48, kTcQK, kBias, kDump>(prm, B, H, N, st, msg);
-    case 4: return launch_tc<64, kTcQK, kBias, kDump>(prm, B, H, N, st, msg);
-    case 5: return launch_tc<80, kTcQK, kBias, kDump>(prm, B, H, N, st, msg);
-    case 6: return launch_tc<96, kTcQK, kBias, kDump>(prm, B, H, N, st, msg);
-    case 7: return launch_tc<112, kTcQK, kBias, kDump>(prm, B, H, N, st, msg);
-    default: return launch_tc<128, kTcQK, kBias, kDump>(prm, B, H, N, st, msg);
+template <int KDIM, int kQK, bool kBias, bool kDump>
+inline int launch_mode(const Params& prm, cudaStream_t st, std::string* msg) {
+  TensorMaps tm;
+  std::memset(&tm, 0, sizeof tm);
+  if constexpr (tma_mode_kdim(KDIM)) {
+    if (prm.N % 8 == 0) {
+      std::string why;
+      if (make_maps(prm, kBias, kQK == kQkRef, &tm, &why))
+        return launch_tc<KDIM, true, kQK, kBias, kDump>(prm, tm, st, msg);
+      std::memset(&tm, 0, sizeof tm);  // the driver refused a map: use the load mode
+    }
+  }
+  return launch_tc<KDIM, false, kQK, kBias, kDump>(prm, tm, st, msg);
+}
+
+template <int kQK, bool kBias, bool kDump>
+inline int dispatch_kdim(const Params& prm, cudaStream_t st, std::string* msg) {
+  switch ((prm.d + 15) / 16) {
+    case 1: return launch_mode<16, kQK, kBias, kDump>(prm, st, msg);
+    case 2: return launch_mode<32, kQK, kBias, kDump>(prm, st, msg);
+    case 3: return launch_mode<48, kQK, kBias, kDump>(prm, st, msg);
+    case 4: return launch_mode<64, kQK, kBias, kDump>(prm, st, msg);
+    case 5: return launch_mode<80, kQK, kBias, kDump>(prm, st, msg);
+    case 6: return launch_mode<96, kQK, kBias, kDump>(prm, st, msg);
+    case 7: return launch_mode<112, kQK, kBias, kDump>(prm, st, msg);
+    default: return launch_mode<128, kQK, kBias, kDump>(prm, st, msg);
   }
 }
 
@@ -479,24 +898,28 @@ inline int dispatch_kdim(const Params& prm, int B, int H, int N, int d, cudaStre
 inline int forward_tc(bool tc_qk, const uint32_t* qb, const uint32_t* kb, const float* aq,
                       const float* ak, const uint16_t* bias, const uint16_t* v, float scale,
                       int B, int H, int N, int d, uint16_t* out, cudaStream_t st, std::string* msg) {
-  tc::Params prm{qb, kb, aq, ak, bias, v, out, nullptr, scale, H, N, d};
+  tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d};
   if (tc_qk)
-    return bias ? tc::dispatch_kdim<true, true, false>(prm, B, H, N, d, st, msg)
-                : tc::dispatch_kdim<true, false, false>(prm, B, H, N, d, st, msg);
-  return bias ? tc::dispatch_kdim<false, true, false>(prm, B, H, N, d, st, msg)
-              : tc::dispatch_kdim<false, false, false>(prm, B, H, N, d, st, msg);
+    return bias ? tc::dispatch_kdim<tc::kQkTc, true, false>(prm, st, msg)
+                : tc::dispatch_kdim<tc::kQkTc, false, false>(prm, st, msg);
+  return bias ? tc::dispatch_kdim<tc::kQkPopc, true, false>(prm, st, msg)
+              : tc::dispatch_kdim<tc::kQkPopc, false, false>(prm, st, msg);
 }
 
 inline int scores_tc(const uint32_t* qb, const uint32_t* kb, int B, int H, int N, int d, int32_t* S,
                      cudaStream_t st, std::string* msg) {
-  tc::Params prm{qb, kb, nullptr, nullptr, nullptr, nullptr, nullptr, S, 0.f, H, N, d};
-  return tc::dispatch_kdim<true, false, true>(prm, B, H, N, d, st, msg);
+  tc::Params prm{qb, kb, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S, 0.f, B, H, N, d};
+  return tc::dispatch_kdim<tc::kQkTc, false, true>(prm, st, msg);
 }
 
-inline int forward_ref_bf16(const uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*, float,
-                            int, int, int, int, uint16_t*, cudaStream_t, std::string* msg) {
-  *msg = "bf16 reference not built yet";
-  return BINATTN_ERR_UNSUPPORTED;
+// Full-precision softmax attention on the same tile pipeline (the speed
+// reference): S = Q K^T as a bf16 tcgen05.mma, logit = scale * S + bias.
+inline int forward_ref_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* bias,
+                            const uint16_t* v, float scale, int B, int H, int N, int d, uint16_t* out,
+                            cudaStream_t st, std::string* msg) {
+  tc::Params prm{nullptr, nullptr, q, k, nullptr, nullptr, bias, v, out, nullptr, scale, B, H, N, d};
+  return bias ? tc::dispatch_kdim<tc::kQkRef, true, false>(prm, st, msg)
+              : tc::dispatch_kdim<tc::kQkRef, false, false>(prm, st, msg);
 }
 
 }  // namespace binattn
