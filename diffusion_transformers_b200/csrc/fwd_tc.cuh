@@ -1,5 +1,5 @@
-// fwd_tc.cuh — tensor-core engines of binattn_forward (TC and POPC_TC) and the
-// debug-scores kernel of the TC engine.
+// fwd_tc.cuh — tensor-core engines of binattn_forward (TC and POPC_TC), the
+// debug-scores kernel of the TC engine, and the bf16 reference attention.
 //
 // Source: "BinaryAttention: One-Bit QK-Attention for Vision and Diffusion
 // Transformers", §2 methodology: scaled binary Q/K, XNOR/popcount similarity,
@@ -7,20 +7,25 @@
 // hardware-aware implementation bullet. The tiling here is new for sm_100a.
 //
 // One CTA (12 warps, one per SM) owns 256 query rows of one (b, h) as two
-// 128-row tiles t = 0, 1, and streams all keys in tiles of 128:
+// 128-row tiles t = 0, 1 and streams the keys in tiles of 64:
 //   warps 0-7   softmax: warpgroup t (warps 4t..4t+3), thread = one query row.
 //   warp 8      MMA issuer (one thread): tcgen05.mma, tcgen05.commit.
 //   warps 9-11  loaders, in one of two modes:
 //     TMA mode (KDIM <= 80, N % 8 == 0): warp 9 issues TMA / bulk copies of V
-//       and alpha_k (and the sign words for POPC_TC); warp 10 issues the bias
-//       tiles, each as soon as its stage is free; warp 11 loads the key sign
-//       words and expands them to +-1 bf16 operand tiles (TC engine). Q_t lives
-//       in tensor memory next to O_t.
+//       and alpha_k (and of the sign words for POPC_TC, of K for the reference);
+//       warp 10 issues the bias tiles, each as soon as its stage is free;
+//       warp 11 loads the key sign words and expands them to +-1 bf16 operand
+//       tiles (TC engine). Q_t lives in tensor memory next to O_t.
 //     load mode (other shapes): warps 9-11 load the same data with batched
 //       plain loads; Q_t lives in shared memory; softmax threads read the bias.
-// Tensor memory (512 columns): S_t at 128t (fp32, 128 keys); P_t written back
-// over the first 64 columns of S_t as bf16 pairs; O_t at 256 + 128t (KDIM
-// columns); in TMA mode Q_t at 256 + 128t + KDIM (KDIM/2 columns of bf16 pairs).
+//
+// Tensor memory, 256 columns per warpgroup t (base 256t): two score buffers
+// S_t^0, S_t^1 (64 fp32 columns each), O_t (KDIM columns) at +128 and, in TMA
+// mode, Q_t (KDIM/2 columns of bf16 pairs) at +128+KDIM. P_t of key tile kt is
+// written back as bf16 pairs over the first 32 columns of S_t^(kt%2). With two
+// score buffers the MMA warp issues S_t(kt+2) = Q_t K(kt+2)^T right after
+// O_t += P_t(kt) V(kt), so the scores of the next tile are ready while the
+// softmax threads still work on the current one.
 //
 // TC engine: S_t = Q_t K^T on the tensor core with +-1 bf16 operands. Pad
 // channels of Q are 0, so every product is +-1 or 0 and the fp32 accumulator
@@ -29,9 +34,10 @@
 // words (binary_score); the tensor core does P.V only.
 //
 // Softmax (per row, fp32, online over key tiles): logit = (S * alpha_k) *
-// (scale * alpha_q) + bias; running max m and sum l; O_t in TMEM is rescaled by
-// exp(m_old - m_new) when m grows; P = exp(logit - m) rounded to bf16 for the
-// P.V MMA; the epilogue divides by l and writes bf16.
+// (scale * alpha_q) + bias; running max m and sum l; O_t in TMEM is rescaled
+// only when the tile max exceeds m by more than 8 (log2 units); P =
+// exp(logit - m) rounded to bf16 for the P.V MMA; the epilogue divides by l and
+// writes bf16.
 //
 // Every mbarrier wait is bounded (sm100::mbar_wait); on a timeout the CTA
 // records a device status code, leaves its loops, waits for its own MMAs and
@@ -56,8 +62,9 @@ namespace tc {
 using namespace sm100;
 
 constexpr int kRows = 128;       // query rows per softmax warpgroup (MMA M)
-constexpr int kKeys = 128;       // keys per tile (QK MMA N, PV MMA K)
-constexpr int kStages = 2;
+constexpr int kKeys = 64;        // keys per tile (QK MMA N, PV MMA K)
+constexpr int kKS = 4;           // stages of the K / V / alpha_k / sign-word ring
+constexpr int kBS = 3;           // stages of the bias ring (per warpgroup)
 constexpr int kWarps = 12;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMmaWarp = 8;
@@ -70,38 +77,41 @@ constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 5.545177444479562f;  // 8 * ln 2: rescale O only past 2^8
 
+__host__ __device__ constexpr bool tma_mode_kdim(int kdim) { return kdim <= 80; }
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float m;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
   return m;
 }
 
-__host__ __device__ constexpr bool tma_mode_kdim(int kdim) { return kdim <= 80; }
-
-// Shared-memory map (byte offsets). An operand tile is 128 rows x KDIM bf16.
-//  Q_t, K_s  (K-major, no swizzle): 16-byte chunk (row r, channel group c) at
-//            (r / 8) * (KDIM * 16) + c * 128 + (r % 8) * 16
-//            -> descriptor LBO = 128 (next channel group), SBO = KDIM * 16 (next 8 rows).
-//  V_s       (MN-major, no swizzle): chunk (key j, d group g) at g * 2048 + j * 16
-//            -> descriptor LBO = 128 (next 8 keys), SBO = 2048 (next 8 d values).
-//            In TMA mode each d group is one TMA box of 8 x 128 elements.
-//  bias_s,t  (TMA mode) 128 rows x 128 keys bf16 as two 128B-swizzled boxes of
-//            64 keys: key k of row r at (k / 64) * 16384 + r * 128 +
-//            (((k % 64) / 8) ^ (r % 8)) * 16 + (k % 8) * 2.
-//  kb_s      sign words of the tile's keys, contiguous: key j word w at j * W + w.
+// Shared-memory map (byte offsets).
+//  Q_t (load mode) 128 rows x KDIM bf16, K-major, no swizzle: 16-byte chunk
+//           (row r, channel group c) at (r / 8) * (KDIM * 16) + c * 128 + (r % 8) * 16
+//           -> descriptor LBO = 128 (next channel group), SBO = KDIM * 16 (next 8 rows).
+//  K_s     64 keys x KDIM bf16. Binary: the same layout as Q_t. Reference:
+//           chunk (key j, channel group c) at c * 1024 + j * 16 (one TMA box of
+//           8 channels x 64 keys per group) -> LBO = 1024, SBO = 128.
+//  V_s     64 keys x KDIM bf16, MN-major, no swizzle: chunk (key j, d group g)
+//           at g * 1024 + j * 16 (one TMA box per group)
+//           -> LBO = 128 (next 8 keys), SBO = 1024 (next 8 d values).
+//  bias    (TMA mode) per stage and warpgroup: 128 rows x 64 keys bf16 as one
+//           128B-swizzled box: key k of row r at r * 128 + ((k / 8) ^ (r % 8)) * 16 + (k % 8) * 2.
+//  kb_s    sign words of the tile's keys, contiguous: key j word w at j * W + w.
 template <int KDIM, bool kTma>
 struct Layout {
-  static constexpr int kTile = kKeys * KDIM * 2;
-  static constexpr int kBiasTile = kRows * kKeys * 2;            // 32 KB
+  static constexpr int kQTile = kRows * KDIM * 2;
+  static constexpr int kKTile = kKeys * KDIM * 2;
+  static constexpr int kBiasTile = kRows * kKeys * 2;            // 16 KB
   static constexpr int kLut = 0;                                 // 256 x 16 B
-  static constexpr int kQ = 4096;                                // load mode: 2 tiles
-  static constexpr int kK = kQ + (kTma ? 0 : 2 * kTile);         // kStages tiles
-  static constexpr int kV = kK + kStages * kTile;                // kStages tiles
-  static constexpr int kBias = (kV + kStages * kTile + 1023) / 1024 * 1024;  // TMA: [kStages][2]
-  static constexpr int kAk = kBias + (kTma ? kStages * 2 * kBiasTile : 0);  // kStages x 128 fp32
-  static constexpr int kKb = kAk + kStages * kKeys * 4;          // kStages x 128 x 4 words
-  static constexpr int kBar = kKb + kStages * kKeys * 16;
-  static constexpr int kNumBars = 32;
+  static constexpr int kQ = 4096;                                // load mode: 2 Q tiles
+  static constexpr int kK = kQ + (kTma ? 0 : 2 * kQTile);        // kKS tiles
+  static constexpr int kV = kK + kKS * kKTile;                   // kKS tiles
+  static constexpr int kBias = (kV + kKS * kKTile + 1023) / 1024 * 1024;  // TMA: [kBS][2]
+  static constexpr int kAk = kBias + (kTma ? kBS * 2 * kBiasTile : 0);   // kKS x 64 fp32
+  static constexpr int kKb = kAk + kKS * kKeys * 4;              // kKS x 64 x 4 words
+  static constexpr int kBar = kKb + kKS * kKeys * 16;
+  static constexpr int kNumBars = 64;
   static constexpr int kMisc = kBar + 8 * kNumBars;              // tmem base, abort flag
   static constexpr int kBytes = kMisc + 16;
   // at least this much, so that one CTA occupies an SM (each CTA allocates all
@@ -150,10 +160,7 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
               const __grid_constant__ CUtensorMap tm_k) {
   constexpr bool kTcQK = kQK != kQkPopc;  // QK^T on the tensor core
   constexpr bool kRef = kQK == kQkRef;
-  // K operand layout (K-major, no swizzle): binary = rows of KDIM*16 bytes per
-  // 8 keys (LBO 128, SBO KDIM*16); reference = one TMA box of 8 channels x 128
-  // keys per channel group (LBO 2048, SBO 128).
-  constexpr uint32_t kKLbo = kRef ? 2048 : 128;
+  constexpr uint32_t kKLbo = kRef ? 1024 : 128;
   constexpr uint32_t kKSbo = kRef ? 128 : KDIM * 16;
   using L = Layout<KDIM, kTma>;
   constexpr int W = (KDIM + 31) / 32;  // packed words per token (= ceil(d / 32))
@@ -166,17 +173,21 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
   extern __shared__ __align__(1024) uint8_t smem[];
   uint4* lut = reinterpret_cast<uint4*>(smem + L::kLut);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* kv_full = bars + 0;    // [2] load mode: loaders -> all;  TMA mode: V + alpha_k tx
-  uint64_t* kv_empty = bars + 2;   // [2] MMA commit after PV of the stage
-  uint64_t* kb_full = bars + 4;    // [2] TMA mode: sign-word bulk copy tx
-  uint64_t* k_full = bars + 6;     // [2] TMA mode: expanders -> MMA
-  uint64_t* k_empty = bars + 8;    // [2] TMA mode: MMA commit after QK of the stage
-  uint64_t* b_full = bars + 10;    // [2][2] TMA mode: bias tile tx (stage, t)
-  uint64_t* b_empty = bars + 14;   // [2][2] TMA mode: softmax t done with bias tile
-  uint64_t* s_full = bars + 18;    // [2] QK commit -> softmax t
-  uint64_t* p_full = bars + 20;    // [2] softmax t (128 arrivals) -> MMA
-  uint64_t* o_done = bars + 22;    // [2] PV commit -> softmax t
-  uint64_t* drain = bars + 24;     // error path only
+  uint64_t* kv_full = bars + 0;     // [kKS] V + alpha_k (+ load mode: K, sign words)
+  uint64_t* kv_empty = bars + 4;    // [kKS] MMA commit after the stage's P.V
+  uint64_t* kb_full = bars + 8;     // [kKS] TMA mode POPC_TC: sign-word bulk copy
+  uint64_t* k_full = bars + 12;     // [kKS] TMA mode: K operand ready
+  uint64_t* k_empty = bars + 16;    // [kKS] TMA mode: MMA commit after the stage's QK
+  uint64_t* b_full = bars + 20;     // [kBS * 2] bias tile landed (stage, t)
+  uint64_t* b_empty = bars + 26;    // [kBS * 2] warpgroup t done with the bias tile
+  uint64_t* s_full = bars + 32;     // [2 t][2 buf] QK commit -> softmax t
+  uint64_t* p_full = bars + 36;     // [2 t][2 buf] softmax t (128 arrivals) -> MMA
+  // [2 t][2 buf] PV commit -> softmax t. Two barriers per warpgroup (by tile
+  // parity) so that every wait has at most one phase in flight: with double-
+  // buffered scores the softmax can be two tiles ahead of P.V, and a single
+  // barrier's parity would then be ambiguous.
+  uint64_t* o_done = bars + 40;
+  uint64_t* drain = bars + 44;      // error path only
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -190,7 +201,7 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
   const int N = p.N, d = p.d;
   const size_t tok0 = static_cast<size_t>(bh) * N;
   const int q0 = qt * 2 * kRows;
-  const int ntiles = (N + kKeys - 1) / kKeys;
+  const int nkt = (N + kKeys - 1) / kKeys;
   const int dgroups = d / 8;
 
   // ---------------------------------------------------------------- setup
@@ -206,35 +217,34 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
     lut[i] = make_uint4(w[0], w[1], w[2], w[3]);
   }
   if constexpr (kTma && !kDump) {
-    // V pad groups (g >= d / 8) are never written by TMA: zero them once (and
-    // the K pad groups of the reference kernel, which would otherwise hold
-    // whatever shared memory held before).
+    // Pad groups (g >= d / 8) of V (and of the reference K) are never written
+    // by TMA: zero them once so that no stale shared memory enters an MMA.
     const int npad = (KCH - dgroups) * kKeys;
-    for (int e = threadIdx.x; e < kStages * npad; e += kThreads) {
+    for (int e = threadIdx.x; e < kKS * npad; e += kThreads) {
       const int s = e / npad, rem = e % npad;
       const int g = dgroups + rem / kKeys, kk = rem % kKeys;
-      *reinterpret_cast<uint4*>(smem + L::kV + s * L::kTile + g * 2048 + kk * 16) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(smem + L::kV + s * L::kKTile + g * 1024 + kk * 16) = make_uint4(0, 0, 0, 0);
       if (kRef)
-        *reinterpret_cast<uint4*>(smem + L::kK + s * L::kTile + g * 2048 + kk * 16) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(smem + L::kK + s * L::kKTile + g * 1024 + kk * 16) = make_uint4(0, 0, 0, 0);
     }
   }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKS; ++s) {
       mbar_init(&kv_full[s], kTma ? 1 : kLoadThreads);
       mbar_init(&kv_empty[s], 1);
       mbar_init(&kb_full[s], 1);
       mbar_init(&k_full[s], kRef ? 1 : kExpandThreads);
       mbar_init(&k_empty[s], 1);
-      for (int t = 0; t < 2; ++t) {
-        mbar_init(&b_full[s * 2 + t], 1);
-        mbar_init(&b_empty[s * 2 + t], kRows);
-      }
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], kRows);
-      mbar_init(&o_done[t], 1);
+    for (int i = 0; i < kBS * 2; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], kRows);
     }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], kRows);
+    }
+    for (int i = 0; i < 4; ++i) mbar_init(&o_done[i], 1);
     mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
@@ -248,7 +258,7 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Softmax threads: this thread's query row and its +-1 row of Q_t.
+  // Softmax threads: this thread's query row and its operand row of Q_t.
   const int t = warp >> 2;                      // warpgroup (valid for warps 0-7)
   const int r = ((warp & 3) << 5) | lane;       // row within the tile = TMEM lane
   const int row = q0 + t * kRows + r;
@@ -271,9 +281,9 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
   };
   if (kTcQK && warp < 8) {
     if constexpr (kTma) {
-      // Q_t row in TMEM at column 256 + 128t + KDIM: column c2 holds channels
-      // 2*c2 (low half) and 2*c2 + 1, as bf16 +-1 (0 for pad channels).
-      const uint32_t qcol = tmem + lane_base + 256 + 128 * t + KDIM;
+      // Q_t row in TMEM at column 256t + 128 + KDIM: column c2 holds channels
+      // 2*c2 (low half) and 2*c2 + 1.
+      const uint32_t qcol = tmem + lane_base + 256 * t + 128 + KDIM;
 #pragma unroll
       for (int c = 0; c < KCH; c += 2) {
         uint32_t wv[8];
@@ -290,7 +300,7 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
       tmem_st_wait();
       tc_fence_before();
     } else {
-      uint8_t* qs = smem + L::kQ + t * L::kTile;
+      uint8_t* qs = smem + L::kQ + t * L::kQTile;
 #pragma unroll
       for (int c = 0; c < KCH; ++c)
         *reinterpret_cast<uint4*>(qs + (r >> 3) * (KDIM * 16) + c * 128 + (r & 7) * 16) = q_group(c);
@@ -303,36 +313,36 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
   if (warp >= kLoadWarp0) {
     if constexpr (kTma) {
       if (warp == kLoadWarp0) {
-        // ------------------------------------------------ TMA issuer (one thread)
+        // --------------------------------- V / alpha_k (/ K, sign words) issuer
         if (lane == 0) {
-          for (int j = 0; j < ntiles; ++j) {
-            const int s = j % kStages;
-            const uint32_t ph_prev = ((j / kStages) - 1) & 1;
-            const int j0 = j * kKeys;
+          for (int kt = 0; kt < nkt; ++kt) {
+            const int s = kt % kKS;
+            const uint32_t ph_prev = ((kt / kKS) - 1) & 1;
+            const int j0 = kt * kKeys;
             const int nk = min(kKeys, N - j0);
-            // Stage s is free once tile j - kStages is done with it: its QK MMAs
-            // (TC: K operand and sign words) and its P.V MMAs (V, alpha_k, and
-            // for POPC_TC the sign words read by the softmax threads).
-            if (j >= kStages) {
+            // Stage s is free once tile kt - kKS is done with it: its QK MMAs
+            // (reference K) and its P.V MMAs (V, alpha_k, and for POPC_TC the
+            // sign words read by the softmax threads before P was published).
+            if (kt >= kKS) {
               if (kRef && !mbar_wait(&k_empty[s], ph_prev, abort)) break;
               if (!kDump && !mbar_wait(&kv_empty[s], ph_prev, abort)) break;
             }
-            if constexpr (kRef) {  // bf16 K: one box of 8 channels x 128 keys per group
-              mbar_arrive_expect_tx(&k_full[s], dgroups * 2048);
+            if constexpr (kRef) {  // bf16 K: one box of 8 channels x 64 keys per group
+              mbar_arrive_expect_tx(&k_full[s], dgroups * 1024);
               for (int g = 0; g < dgroups; ++g)
-                tma_load_3d(smem + L::kK + s * L::kTile + g * 2048, &tm_k, 8 * g, j0, bh, &k_full[s]);
+                tma_load_3d(smem + L::kK + s * L::kKTile + g * 1024, &tm_k, 8 * g, j0, bh, &k_full[s]);
             } else if constexpr (!kTcQK) {
               // POPC_TC: sign words for the softmax threads, nk keys x W words,
               // contiguous and 16-byte aligned (N % 8 == 0). (For TC the
-              // expander warps load the words themselves.)
+              // expander warp loads the words itself.)
               const uint32_t nbytes = static_cast<uint32_t>(nk * W * 4);
               mbar_arrive_expect_tx(&kb_full[s], nbytes);
               bulk_load(smem + L::kKb + s * kKeys * 16, p.kb + (tok0 + j0) * W, nbytes, &kb_full[s]);
             }
             if constexpr (!kDump) {
-              mbar_arrive_expect_tx(&kv_full[s], dgroups * 2048 + (kRef ? 0 : kKeys * 4));
+              mbar_arrive_expect_tx(&kv_full[s], dgroups * 1024 + (kRef ? 0 : kKeys * 4));
               for (int g = 0; g < dgroups; ++g)
-                tma_load_3d(smem + L::kV + s * L::kTile + g * 2048, &tm_v, 8 * g, j0, bh, &kv_full[s]);
+                tma_load_3d(smem + L::kV + s * L::kKTile + g * 1024, &tm_v, 8 * g, j0, bh, &kv_full[s]);
               if (!kRef) tma_load_2d(smem + L::kAk + s * kKeys * 4, &tm_ak, j0, bh, &kv_full[s]);
             }
           }
@@ -340,48 +350,46 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
         __syncwarp();
       } else if (warp == kBiasWarp) {
         // ------------------------------------------------ bias issuer (one thread)
-        // The bias tile (128 rows x 128 keys of warpgroup t) is the largest
+        // The bias tile (128 rows x 64 keys of warpgroup t) is the largest
         // stream; each is requested as soon as warpgroup t released the stage.
         if (kBias && !kDump && lane == 0) {
-          for (int j = 0; j < ntiles; ++j) {
-            const int s = j % kStages;
-            const int j0 = j * kKeys;
+          for (int kt = 0; kt < nkt; ++kt) {
+            const int bs = kt % kBS;
             bool ok = true;
             for (int tt = 0; tt < 2; ++tt) {
-              uint64_t* bf = &b_full[s * 2 + tt];
-              if (j >= kStages && !(ok = mbar_wait(&b_empty[s * 2 + tt], ((j / kStages) - 1) & 1, abort)))
+              uint64_t* bf = &b_full[bs * 2 + tt];
+              if (kt >= kBS && !(ok = mbar_wait(&b_empty[bs * 2 + tt], ((kt / kBS) - 1) & 1, abort)))
                 break;
-              uint8_t* dst = smem + L::kBias + (s * 2 + tt) * L::kBiasTile;
               mbar_arrive_expect_tx(bf, L::kBiasTile);
-              tma_load_3d(dst, &tm_bias, j0, q0 + tt * kRows, h, bf);
-              tma_load_3d(dst + L::kBiasTile / 2, &tm_bias, j0 + 64, q0 + tt * kRows, h, bf);
+              tma_load_3d(smem + L::kBias + (bs * 2 + tt) * L::kBiasTile, &tm_bias, kt * kKeys,
+                          q0 + tt * kRows, h, bf);
             }
             if (!ok) break;
           }
         }
         __syncwarp();
       } else if (kTcQK && !kRef) {
-        // ------------------------------------------------ sign expanders
-        // Thread et owns keys et + 32u of every tile: it loads their sign words
-        // itself (the next tile's words are in flight while it waits for the
-        // stage) and writes their +-1 rows; consecutive threads write
+        // ------------------------------------------------ sign expander warp
+        // Thread et owns keys et and et + 32 of every tile: it loads their sign
+        // words itself (the next tile's words are in flight while it waits for
+        // the stage) and writes their +-1 rows; consecutive threads write
         // consecutive keys, which keeps the 16-byte stores conflict-free.
         constexpr int kPer = kKeys / kExpandThreads;
         const int et = threadIdx.x - kExpandWarp0 * 32;
         uint32_t wd[kPer][W];
-        auto load_words = [&](int j) {
+        auto load_words = [&](int kt) {
 #pragma unroll
           for (int u = 0; u < kPer; ++u) {
-            const int key = j * kKeys + et + u * kExpandThreads;
+            const int key = kt * kKeys + et + u * kExpandThreads;
 #pragma unroll
             for (int w = 0; w < W; ++w) wd[u][w] = key < N ? p.kb[(tok0 + key) * W + w] : 0u;
           }
         };
         load_words(0);
-        for (int j = 0; j < ntiles; ++j) {
-          const int s = j % kStages;
-          if (j >= kStages && !mbar_wait(&k_empty[s], ((j / kStages) - 1) & 1, abort)) break;
-          uint8_t* ks = smem + L::kK + s * L::kTile;
+        for (int kt = 0; kt < nkt; ++kt) {
+          const int s = kt % kKS;
+          if (kt >= kKS && !mbar_wait(&k_empty[s], ((kt / kKS) - 1) & 1, abort)) break;
+          uint8_t* ks = smem + L::kK + s * L::kKTile;
 #pragma unroll
           for (int u = 0; u < kPer; ++u) {
             const int kk = et + u * kExpandThreads;
@@ -394,25 +402,25 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
           }
           fence_proxy_async_smem();
           mbar_arrive(&k_full[s]);
-          if (j + 1 < ntiles) load_words(j + 1);
+          if (kt + 1 < nkt) load_words(kt + 1);
         }
       }
     } else {
       // -------------------------------------------- loaders (load mode)
       // Per key tile: (A) issue every global load of the tile at once (sign
-      // words, alpha_k, V), (B) store them into the stage, (C, TC) once all
-      // loaders have stored, expand the sign words to +-1 bf16.
+      // words, alpha_k, V, reference K), (B) store them into the stage, (C, TC)
+      // once all loaders have stored, expand the sign words to +-1 bf16.
       const int pt = threadIdx.x - kLoadWarp0 * 32;
       constexpr int kKbIters = (kKeys * W + kLoadThreads - 1) / kLoadThreads;
       constexpr int kAkIters = (kKeys + kLoadThreads - 1) / kLoadThreads;
       constexpr int kVIters = (kKeys * KCH + kLoadThreads - 1) / kLoadThreads;
-      for (int j = 0; j < ntiles; ++j) {
-        const int s = j % kStages;
+      for (int kt = 0; kt < nkt; ++kt) {
+        const int s = kt % kKS;
         // All 96 loaders agree (barrier with AND reduction) so that either all
         // reach the named barrier below or all leave the loop.
-        const bool ok = j < kStages || mbar_wait(&kv_empty[s], ((j / kStages) - 1) & 1, abort);
+        const bool ok = kt < kKS || mbar_wait(&kv_empty[s], ((kt / kKS) - 1) & 1, abort);
         if (!loaders_all(ok)) break;
-        const int j0 = j * kKeys;
+        const int j0 = kt * kKeys;
         const int nk = min(kKeys, N - j0);
         uint32_t kbuf[kKbIters];
 #pragma unroll
@@ -420,19 +428,9 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
           const int e = pt + it * kLoadThreads;
           kbuf[it] = (!kRef && e < nk * W) ? p.kb[(tok0 + j0) * W + e] : 0u;
         }
-        uint4 krow[kRef ? kVIters : 1];
-        if constexpr (kRef) {  // bf16 K rows, channel group g of key kk -> g * 2048 + kk * 16
-#pragma unroll
-          for (int it = 0; it < kVIters; ++it) {
-            const int e = pt + it * kLoadThreads;
-            const int kk = e / KCH, g = e % KCH;
-            krow[it] = make_uint4(0, 0, 0, 0);
-            if (kk < nk && g < dgroups)
-              krow[it] = __ldg(reinterpret_cast<const uint4*>(p.k + (tok0 + j0 + kk) * d + 8 * g));
-          }
-        }
         float abuf[kAkIters];
         uint4 vbuf[kDump ? 1 : kVIters];
+        uint4 krow[kRef ? kVIters : 1];
         if constexpr (!kDump) {  // the debug-scores variant gets no alpha_k / V
 #pragma unroll
           for (int it = 0; it < kAkIters; ++it) {
@@ -448,22 +446,21 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
               vbuf[it] = __ldg(reinterpret_cast<const uint4*>(p.v + (tok0 + j0 + kk) * d + 8 * g));
           }
         }
+        if constexpr (kRef) {
+#pragma unroll
+          for (int it = 0; it < kVIters; ++it) {
+            const int e = pt + it * kLoadThreads;
+            const int kk = e / KCH, g = e % KCH;
+            krow[it] = make_uint4(0, 0, 0, 0);
+            if (kk < nk && g < dgroups)
+              krow[it] = __ldg(reinterpret_cast<const uint4*>(p.k + (tok0 + j0 + kk) * d + 8 * g));
+          }
+        }
         uint32_t* kbs = reinterpret_cast<uint32_t*>(smem + L::kKb + s * kKeys * 16);
 #pragma unroll
         for (int it = 0; it < kKbIters; ++it) {
           const int e = pt + it * kLoadThreads;
           if (e < kKeys * W) kbs[e] = kbuf[it];
-        }
-        if constexpr (kRef) {
-          uint8_t* ks = smem + L::kK + s * L::kTile;
-#pragma unroll
-          for (int it = 0; it < kVIters; ++it) {
-            const int e = pt + it * kLoadThreads;
-            if (e < kKeys * KCH) {
-              const int kk = e / KCH, g = e % KCH;
-              *reinterpret_cast<uint4*>(ks + g * 2048 + kk * 16) = krow[it];
-            }
-          }
         }
         if constexpr (!kDump) {
           float* aks = reinterpret_cast<float*>(smem + L::kAk) + s * kKeys;
@@ -472,19 +469,30 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
             const int kk = pt + it * kLoadThreads;
             if (kk < kKeys) aks[kk] = abuf[it];
           }
-          uint8_t* vs = smem + L::kV + s * L::kTile;
+          uint8_t* vs = smem + L::kV + s * L::kKTile;
 #pragma unroll
           for (int it = 0; it < kVIters; ++it) {
             const int e = pt + it * kLoadThreads;
             if (e < kKeys * KCH) {
               const int kk = e / KCH, g = e % KCH;
-              *reinterpret_cast<uint4*>(vs + g * 2048 + kk * 16) = vbuf[it];
+              *reinterpret_cast<uint4*>(vs + g * 1024 + kk * 16) = vbuf[it];
+            }
+          }
+        }
+        if constexpr (kRef) {
+          uint8_t* ks = smem + L::kK + s * L::kKTile;
+#pragma unroll
+          for (int it = 0; it < kVIters; ++it) {
+            const int e = pt + it * kLoadThreads;
+            if (e < kKeys * KCH) {
+              const int kk = e / KCH, g = e % KCH;
+              *reinterpret_cast<uint4*>(ks + g * 1024 + kk * 16) = krow[it];
             }
           }
         }
         if constexpr (kTcQK && !kRef) {
-          asm volatile("bar.sync 1, %0;" ::"n"(kLoadThreads) : "memory");  // stores done
-          uint8_t* ks = smem + L::kK + s * L::kTile;
+          asm volatile("bar.sync 1, %0;" ::"n"(kLoadThreads) : "memory");  // stores of (B) done
+          uint8_t* ks = smem + L::kK + s * L::kKTile;
 #pragma unroll 4
           for (int e = pt; e < kKeys * KCH; e += kLoadThreads) {
             const int c = e / kKeys, kk = e % kKeys;  // consecutive threads: consecutive keys
@@ -503,55 +511,61 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
       const uint32_t q_base = smem_u32(smem + L::kQ);
       const uint32_t k_base = smem_u32(smem + L::kK);
       const uint32_t v_base = smem_u32(smem + L::kV);
-      uint64_t* kready = kTma ? k_full : kv_full;  // "K operand stage s is ready"
-      auto issue_qk = [&](int tt, int s) {
+      uint64_t* kready = kTma ? k_full : kv_full;  // "K operand of stage s is ready"
+      // S_t^(kt%2) = Q_t K(kt)^T
+      auto issue_qk = [&](int tt, int kt) {
+        const int s = kt % kKS;
+        const uint32_t s_tmem = tmem + 256 * tt + 64 * (kt & 1);
 #pragma unroll
         for (int ks = 0; ks < KDIM / 16; ++ks) {
-          const uint64_t bdesc = smem_desc(k_base + s * L::kTile + ks * 2 * kKLbo, kKLbo, kKSbo);
+          const uint64_t bdesc = smem_desc(k_base + s * L::kKTile + ks * 2 * kKLbo, kKLbo, kKSbo);
           if constexpr (kTma) {
-            mma_ts(tmem + tt * 128, tmem + 256 + 128 * tt + KDIM + ks * 8, bdesc, kIdescQK, ks > 0);
+            mma_ts(s_tmem, tmem + 256 * tt + 128 + KDIM + ks * 8, bdesc, kIdescQK, ks > 0);
           } else {
-            const uint64_t adesc = smem_desc(q_base + tt * L::kTile + ks * 256, 128, KDIM * 16);
-            mma_ss(tmem + tt * 128, adesc, bdesc, kIdescQK, ks > 0);
+            const uint64_t adesc = smem_desc(q_base + tt * L::kQTile + ks * 256, 128, KDIM * 16);
+            mma_ss(s_tmem, adesc, bdesc, kIdescQK, ks > 0);
           }
         }
-        mma_commit(&s_full[tt]);
+        mma_commit(&s_full[tt * 2 + (kt & 1)]);
       };
       bool ok = true;
       if constexpr (kTcQK) {
-        ok = mbar_wait(&kready[0], 0, abort);
-        if (ok) {
+        for (int kt = 0; ok && kt < 2 && kt < nkt; ++kt) {
+          if (!(ok = mbar_wait(&kready[kt % kKS], (kt / kKS) & 1, abort))) break;
           tc_fence_after();
-          issue_qk(0, 0);
-          issue_qk(1, 0);
-          if (kTma) mma_commit(&k_empty[0]);
+          issue_qk(0, kt);
+          issue_qk(1, kt);
+          if (kTma) mma_commit(&k_empty[kt % kKS]);
         }
       }
-      for (int j = 0; ok && j < ntiles; ++j) {
-        const int s = j % kStages;
+      for (int kt = 0; ok && kt < nkt; ++kt) {
+        const int s = kt % kKS;
         if (!kDump && (kTma || !kTcQK)) {  // V ready (load mode TC: implied by kready)
-          if (!(ok = mbar_wait(&kv_full[s], (j / kStages) & 1, abort))) break;
+          if (!(ok = mbar_wait(&kv_full[s], (kt / kKS) & 1, abort))) break;
           tc_fence_after();
         }
         for (int tt = 0; tt < 2; ++tt) {
-          if (!(ok = mbar_wait(&p_full[tt], j & 1, abort))) break;
+          if (!(ok = mbar_wait(&p_full[tt * 2 + (kt & 1)], (kt >> 1) & 1, abort))) break;
           tc_fence_after();
           if constexpr (!kDump) {
+            // O_t += P_t(kt) V(kt): A = P from TMEM (32 columns of bf16 pairs)
 #pragma unroll
             for (int ks = 0; ks < kKeys / 16; ++ks) {
-              const uint64_t bdesc = smem_desc(v_base + s * L::kTile + ks * 256, 128, 2048);
-              mma_ts(tmem + 256 + tt * 128, tmem + tt * 128 + ks * 8, bdesc, kIdescPV, (j > 0 || ks > 0));
+              const uint64_t bdesc = smem_desc(v_base + s * L::kKTile + ks * 256, 128, 1024);
+              mma_ts(tmem + 256 * tt + 128, tmem + 256 * tt + 64 * (kt & 1) + ks * 8, bdesc, kIdescPV,
+                     (kt > 0 || ks > 0));
             }
-            mma_commit(&o_done[tt]);
+            mma_commit(&o_done[tt * 2 + (kt & 1)]);
           }
-          if (kTcQK && j + 1 < ntiles) {
-            const int s1 = (j + 1) % kStages;
+          if (kTcQK && kt + 2 < nkt) {
+            // S_t^(kt%2) is free again: P_t(kt) was consumed by the MMA just
+            // issued (the tensor pipe executes in issue order).
             if (tt == 0) {
-              if (!(ok = mbar_wait(&kready[s1], ((j + 1) / kStages) & 1, abort))) break;
+              if (!(ok = mbar_wait(&kready[(kt + 2) % kKS], ((kt + 2) / kKS) & 1, abort))) break;
               tc_fence_after();
             }
-            issue_qk(tt, s1);
-            if (kTma && tt == 1) mma_commit(&k_empty[s1]);
+            issue_qk(tt, kt + 2);
+            if (kTma && tt == 1) mma_commit(&k_empty[(kt + 2) % kKS]);
           }
         }
         mma_commit(&kv_empty[s]);
@@ -562,8 +576,7 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
     // ---------------------------------------------------------------- softmax
     // per-row factor of the logit: scale * alpha_q (binary) or scale (reference)
     const float ci = kRef ? p.scale : ((!kDump && row_valid) ? p.scale * p.aq[tok0 + row] : 0.f);
-    const uint32_t s_col = tmem + lane_base + t * 128;
-    const uint32_t o_col = tmem + lane_base + 256 + t * 128;
+    const uint32_t o_col = tmem + lane_base + 256 * t + 128;
     const uint16_t* brow =
         (kBias && !kTma && row_valid) ? p.bias + (static_cast<size_t>(h) * N + row) * N : nullptr;
     const bool bias_vec = (N % 8) == 0;
@@ -573,23 +586,24 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
     };
-    for (int j = 0; j < ntiles; ++j) {
-      const int s = j % kStages;
-      const uint32_t ph = (j / kStages) & 1;
-      const int j0 = j * kKeys;
-      float2 xs[kKeys / 2];  // this row's 128 scores, then logits (8-byte aligned storage)
+    for (int kt = 0; kt < nkt; ++kt) {
+      const int s = kt % kKS;
+      const int buf = kt & 1;
+      const int j0 = kt * kKeys;
+      const uint32_t s_col = tmem + lane_base + 256 * t + 64 * buf;
+      float2 xs[kKeys / 2];  // this row's 64 scores, then logits (8-byte aligned storage)
       float* x = reinterpret_cast<float*>(xs);
       if (!kRef && (!kDump || !kTma)) {  // alpha_k (and in load mode sign words) of stage s
-        if (!(ok = wait_all(&kv_full[s], ph))) break;
+        if (!(ok = wait_all(&kv_full[s], (kt / kKS) & 1))) break;
       }
       if constexpr (kTcQK) {
-        if (!(ok = wait_all(&s_full[t], j & 1))) break;
+        if (!(ok = wait_all(&s_full[t * 2 + buf], (kt >> 1) & 1))) break;
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < kKeys; c += 32) tmem_ld32(s_col + c, reinterpret_cast<uint32_t*>(x + c));
+        tmem_ld32(s_col, reinterpret_cast<uint32_t*>(x));
+        tmem_ld32(s_col + 32, reinterpret_cast<uint32_t*>(x + 32));
         tmem_ld_wait();
       } else {
-        if (kTma && !(ok = wait_all(&kb_full[s], ph))) break;
+        if (kTma && !(ok = wait_all(&kb_full[s], (kt / kKS) & 1))) break;
         const uint32_t* kbs = reinterpret_cast<const uint32_t*>(smem + L::kKb + s * kKeys * 16);
 #pragma unroll
         for (int c = 0; c < kKeys; ++c)
@@ -603,16 +617,16 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
             if (j0 + c < N) srow[c] = static_cast<int32_t>(x[c]);
         }
         tc_fence_before();
-        mbar_arrive(&p_full[t]);
+        mbar_arrive(&p_full[t * 2 + buf]);
         continue;
       }
       // logits = S * alpha_k * (scale * alpha_q) + bias (packed fp32 pairs)
       const float* aks = reinterpret_cast<const float*>(smem + L::kAk) + s * kKeys;
-      const uint8_t* bsm = smem + L::kBias + (s * 2 + t) * L::kBiasTile + r * 128;
+      const int bs = kt % kBS;
+      const uint8_t* bsm = smem + L::kBias + (bs * 2 + t) * L::kBiasTile + r * 128;
       if (kBias && kTma) {
-        if (!(ok = wait_all(&b_full[s * 2 + t], ph))) break;
+        if (!(ok = wait_all(&b_full[bs * 2 + t], (kt / kBS) & 1))) break;
       }
-      float2* x2 = xs;
       const float2 ci2 = make_float2(ci, ci);
 #pragma unroll
       for (int c0 = 0; c0 < kKeys; c0 += 8) {
@@ -623,9 +637,7 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
           uint4 raw = make_uint4(0, 0, 0, 0);
           bool have = false;
           if constexpr (kTma) {
-            const int chunk = (c0 & 63) >> 3;
-            raw = *reinterpret_cast<const uint4*>(bsm + (c0 >> 6) * (L::kBiasTile / 2) +
-                                                  ((chunk ^ (r & 7)) << 4));
+            raw = *reinterpret_cast<const uint4*>(bsm + (((c0 >> 3) ^ (r & 7)) << 4));
             have = true;
           } else if (row_valid) {
             if (bias_vec && j0 + c0 + 8 <= N) {
@@ -648,7 +660,7 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
         }
         if constexpr (kRef) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) x2[c0 / 2 + e] = __ffma2_rn(x2[c0 / 2 + e], ci2, bv[e]);
+          for (int e = 0; e < 4; ++e) xs[c0 / 2 + e] = __ffma2_rn(xs[c0 / 2 + e], ci2, bv[e]);
         } else {
           const float4 a0 = *reinterpret_cast<const float4*>(aks + c0);
           const float4 a1 = *reinterpret_cast<const float4*>(aks + c0 + 4);
@@ -656,10 +668,10 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
                                 make_float2(a1.x, a1.y), make_float2(a1.z, a1.w)};
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            x2[c0 / 2 + e] = __ffma2_rn(__fmul2_rn(x2[c0 / 2 + e], av[e]), ci2, bv[e]);
+            xs[c0 / 2 + e] = __ffma2_rn(__fmul2_rn(xs[c0 / 2 + e], av[e]), ci2, bv[e]);
         }
       }
-      if (kBias && kTma) mbar_arrive(&b_empty[s * 2 + t]);
+      if (kBias && kTma) mbar_arrive(&b_empty[bs * 2 + t]);
       if (j0 + kKeys > N) {  // last tile: keys >= N take no part (warp-uniform branch)
 #pragma unroll
         for (int c = 0; c < kKeys; ++c)
@@ -670,7 +682,8 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
 #pragma unroll
       for (int c = 4; c < kKeys; c += 8) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) mx4[e] = max3f(mx4[e], x[c + e], x[c + 4 + e < kKeys ? c + 4 + e : c + e]);
+        for (int e = 0; e < 4; ++e)
+          mx4[e] = max3f(mx4[e], x[c + e], x[c + 4 + e < kKeys ? c + 4 + e : c + e]);
       }
       const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       // Lazy rescale: the running max m only moves when the tile max exceeds it
@@ -680,26 +693,36 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
       const bool grow = mx > m + kRescale;
       const float m_new = grow ? mx : m;
       const float corr = grow ? ex2((m - m_new) * kLog2e) : 1.f;  // 0 on the first tile
-      if (j > 0) {
-        // O_t holds PV of tile j-1 once QK of tile j completed (in-order tensor
-        // pipe); the wait makes that visible before O_t is rescaled.
-        if (!(ok = wait_all(&o_done[t], (j - 1) & 1))) break;
+      // P.V of tile kt-1 done: needed before O_t is rescaled, and (POPC_TC)
+      // before P_t(kt) overwrites the buffer that P.V of tile kt-2 read. (For
+      // TC the tensor pipe order already guarantees the latter: S_t(kt) was
+      // written after P.V of tile kt-2.) Completion of the previous phase of the
+      // same barrier (tile kt-3) is known here, so the parity is unambiguous.
+      auto wait_pv_prev = [&]() {
+        return wait_all(&o_done[t * 2 + ((kt - 1) & 1)], ((kt - 1) >> 1) & 1);
+      };
+      if (!kTcQK && kt >= 2) {
+        if (!(ok = wait_pv_prev())) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, grow)) {
+      }
+      if (kt > 0 && __any_sync(0xffffffffu, grow)) {
+        // O_t must hold P.V of tile kt-1 before it is rescaled; P.V of tile kt
+        // cannot start before this warpgroup publishes P_t(kt).
+        if (!(ok = wait_pv_prev())) break;
+        tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < KDIM; c += 16) {
-            uint32_t ov[16];
-            tmem_ld16(o_col + c, ov);
-            tmem_ld_wait();
+        for (int c = 0; c < KDIM; c += 16) {
+          uint32_t ov[16];
+          tmem_ld16(o_col + c, ov);
+          tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-            tmem_st16(o_col + c, ov);
-          }
+          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+          tmem_st16(o_col + c, ov);
         }
       }
       l *= corr;
       m = m_new;
-      // P = exp(logit - m) as bf16 pairs into TMEM over S_t, 32 keys at a time
+      // P = exp(logit - m) as bf16 pairs into TMEM over S_t^buf
       const float2 l2e2 = make_float2(kLog2e, kLog2e);
       const float2 nm2 = make_float2(-m * kLog2e, -m * kLog2e);
       float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
@@ -709,7 +732,7 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float2 a = __ffma2_rn(x2[c0 / 2 + e], l2e2, nm2);
+          const float2 a = __ffma2_rn(xs[c0 / 2 + e], l2e2, nm2);
           const float2 pp = make_float2(ex2(a.x), ex2(a.y));
           ls[e & 3] = __fadd2_rn(ls[e & 3], pp);
           pk[e] = pack_bf16x2(pp.x, pp.y);
@@ -719,10 +742,10 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
       l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y) + (ls[2].x + ls[2].y) + (ls[3].x + ls[3].y);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      mbar_arrive(&p_full[t * 2 + buf]);
     }
     if constexpr (!kDump) {
-      if (ok && wait_all(&o_done[t], (ntiles - 1) & 1)) {
+      if (ok && wait_all(&o_done[t * 2 + ((nkt - 1) & 1)], ((nkt - 1) >> 1) & 1)) {
         tc_fence_after();
         const float inv = 1.f / l;
         uint16_t* orow = p.out + (tok0 + row) * d;
@@ -788,7 +811,7 @@ struct TensorMaps {
   CUtensorMap v, ak, bias, k;
 };
 
-// One [BH][N][d] bf16 tensor as boxes of 8 channels x 128 keys: each box is one
+// One [BH][N][d] bf16 tensor as boxes of 8 channels x 64 keys: each box is one
 // column of 16-byte chunks of the no-swizzle operand layouts above.
 inline bool make_rows_map(EncodeTiledFn enc, CUtensorMap* tm, const uint16_t* base, cuuint64_t BH,
                           cuuint64_t N, cuuint64_t d, const char* what, std::string* msg) {
@@ -818,7 +841,7 @@ inline bool make_maps(const Params& p, bool with_bias, bool ref, TensorMaps* tm,
   if (!make_rows_map(enc, &tm->v, p.v, BH, N, d, "V", msg)) return false;
   if (ref) {
     if (!make_rows_map(enc, &tm->k, p.k, BH, N, d, "K", msg)) return false;
-  } else {  // alpha_k [BH][N] fp32: box 128 keys
+  } else {  // alpha_k [BH][N] fp32: box 64 keys
     const cuuint64_t dims[2] = {N, BH};
     const cuuint64_t strides[1] = {N * 4};
     const cuuint32_t box[2] = {kKeys, 1};
@@ -830,7 +853,7 @@ inline bool make_maps(const Params& p, bool with_bias, bool ref, TensorMaps* tm,
   if (with_bias) {  // bias [H][N rows][N keys] bf16: box 64 keys x 128 rows, 128B swizzle
     const cuuint64_t dims[3] = {N, N, static_cast<cuuint64_t>(p.H)};
     const cuuint64_t strides[2] = {N * 2, N * N * 2};
-    const cuuint32_t box[3] = {64, kRows, 1};
+    const cuuint32_t box[3] = {kKeys, kRows, 1};
     CUresult rc = enc(&tm->bias, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(p.bias),
                       dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

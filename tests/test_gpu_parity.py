@@ -19,6 +19,9 @@ ENGINES = ["simt", "popc_tc", "tc"]
 SMALL_SHAPES = [  # (B, H, N, d): several tiles and a ragged tail
     (1, 2, 256, 64), (2, 3, 129, 72), (1, 2, 197, 64), (1, 1, 1, 64), (2, 1, 7, 32),
     (1, 2, 127, 96), (1, 1, 300, 128), (2, 2, 257, 8), (1, 1, 130, 72),
+    # N % 8 == 0 with d <= 80 runs the TMA-fed pipeline: with and without a
+    # ragged last key tile, several query tiles, two key tiles in flight
+    (1, 2, 304, 64), (2, 2, 512, 72), (1, 1, 72, 16), (1, 3, 1000, 72),
 ]
 ODD_D_SHAPES = [(1, 2, 65, 33), (1, 1, 40, 1), (2, 1, 33, 100), (1, 1, 31, 127)]
 
