@@ -83,6 +83,35 @@ def algorithmic(w, with_bias=True):
                 eff_flops=4 * d * pairs, bytes=bytes_, pack_bytes=pack_bytes)
 
 
+# DRAM traffic of the forward kernel from one ncu capture (dram__bytes_read.sum
+# + dram__bytes_write.sum, one launch at dit_xl_1024 with bias; the summary is
+# profiles/fwd_tc_dit_xl_1024_bias.md), valid only for the kernel sources it was
+# taken on: any change to them turns the reported traffic back into null.
+NCU_TRAFFIC = {
+    "sources_sha256": "2055e52fc6818acb71eec426bef90febdbd3ce79d52ec30d006f4839c9cbedb4",
+    "bytes_per_launch": {"dit_xl_1024/bias": 582_176_768},
+}
+
+
+def kernel_sources_digest():
+    import hashlib
+    csrc = os.path.join(ROOT, "diffusion_transformers_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    with open(os.path.join(ROOT, "include", "binattn.h"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(key):
+    if kernel_sources_digest() != NCU_TRAFFIC["sources_sha256"]:
+        return None
+    return NCU_TRAFFIC["bytes_per_launch"].get(key)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -360,7 +389,9 @@ def run_gpu(args, w, rank, world, local_rank):
                     "effective_tflops": round(a0["eff_flops"] / fwd0_s / 1e12, 2)},
         "bf16_reference": ref,
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4),
+                     "traffic": ncu_traffic(f"{w.name}/bias"), "traffic_unit": "bytes per launch",
+                     "algorithmic_bytes": a["bytes"],
                      "kernel": "binattn forward (with bias)",
                      "peak_source": peaks["source"] + " (burst)",
                      "t_mem_us": round(t_mem * 1e6, 2), "t_tensor_us": round(t_tensor * 1e6, 2)},
