@@ -210,6 +210,31 @@ def cpu_oracle_sample(w, with_bias, target_s, inp=None):
                        f"{b3 * 1e3:.3f} ms per row), extrapolated to all rows as prep + rows x per-row")
 
 
+# ------------------------------------------------------------------ ranks
+def rank_seed(w, rank):
+    """Every rank draws its own batch of the workload (weak scaling): rank 0
+    uses the workload's seed, rank r the seed + 1000 r."""
+    return w.seed + 1000 * rank
+
+
+def max_over_ranks_of(x, world, device):
+    """Max of a per-rank scalar over all ranks (the step time of the job is
+    that of its slowest rank). Every rank must call it, in the same order."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_units(units_per_rank, world):
+    """Units processed by the whole job in one step: every rank processes its
+    own full batch, no data-path collective."""
+    return units_per_rank * world
+
+
 def run_reference(args, w, rank):
     if rank != 0:
         return
@@ -236,7 +261,7 @@ def run_gpu(args, w, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     peaks = measured_peaks()
 
-    inp = make_inputs(w, with_bias=True, seed=w.seed + 1000 * rank)
+    inp = make_inputs(w, with_bias=True, seed=rank_seed(w, rank))
 
     def to_dev(x):
         if x.dtype == np.uint16:
@@ -280,11 +305,7 @@ def run_gpu(args, w, rank, world, local_rank):
         torch.cuda.synchronize()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks_of(x, world, dev)
 
     if args.profile_once:
         for _ in range(args.warmup):
@@ -384,6 +405,7 @@ def run_gpu(args, w, rank, world, local_rank):
         "forward_ms_median": round(results["bias"]["fwd_ms_median"], 5),
         "pack_ms": round(results["bias"]["step_ms"] - results["bias"]["fwd_ms"], 5),
         "effective_tflops": round(eff_tflops, 2),
+        "job_effective_tflops": round(job_units(a["eff_flops"], world) / fwd_s / 1e12, 2),
         "no_bias": {"ms_per_step": round(results["no_bias"]["step_ms"], 5),
                     "forward_ms": round(results["no_bias"]["fwd_ms"], 5),
                     "effective_tflops": round(a0["eff_flops"] / fwd0_s / 1e12, 2)},

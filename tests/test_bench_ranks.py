@@ -1,0 +1,75 @@
+"""Host logic of bench.py's multi-rank path, on CPU with gloo, world size 2.
+
+Each rank draws its own batch (weak scaling) and the reported time is the max
+over ranks; no collective touches the data path.
+"""
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import bench
+    from diffusion_transformers_b200.synthetic import WORKLOADS, make_inputs
+
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        w = WORKLOADS["tiny"]
+        # per-rank time: the job's time is the slowest rank's
+        t = bench.max_over_ranks_of(1.0 + rank * 0.25, world, torch.device("cpu"))
+        # and the same call order on every rank keeps the collectives matched
+        t2 = bench.max_over_ranks_of(5.0 - rank, world, torch.device("cpu"))
+        seed = bench.rank_seed(w, rank)
+        q = make_inputs(w, with_bias=False, seed=seed)["q"]
+        out[rank] = (t, t2, seed, float(abs(q).sum()), bench.job_units(10, world))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_max_time_and_distinct_batches():
+    world = 2
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True,
+                       start_method="spawn")
+    r0, r1 = out[0], out[1]
+    assert r0[0] == r1[0] == 1.25
+    assert r0[1] == r1[1] == 5.0
+    assert r0[2] != r1[2]          # every rank its own batch
+    assert r0[3] != r1[3]
+    assert r0[4] == r1[4] == 20    # units of the whole job
+
+
+def test_single_rank_needs_no_process_group():
+    import bench
+    assert bench.max_over_ranks_of(3.5, 1, None) == 3.5
+    assert bench.job_units(7, 1) == 7
+
+
+def test_reference_arm_other_ranks_do_no_work(capsys):
+    import argparse
+
+    import bench
+    from diffusion_transformers_b200.synthetic import WORKLOADS
+    args = argparse.Namespace(steps=1, warmup=0, gpus=2, cpu_seconds=0.1, workload="tiny")
+    bench.run_reference(args, WORKLOADS["tiny"], rank=1)
+    assert capsys.readouterr().out == ""
