@@ -13,6 +13,7 @@
 #include "pack.cuh"
 #include "fwd_simt.cuh"
 #include "fwd_tc.cuh"
+#include "fwd_tc2.cuh"
 
 namespace {
 
@@ -174,8 +175,12 @@ int binattn_forward_engine(const uint32_t* q_bits, const uint32_t* k_bits, const
       if (!binattn::tc_supported(d))
         return fail(BINATTN_ERR_UNSUPPORTED, "engine %d needs d %% 8 == 0 (d = %d)", engine, d);
       std::string msg;
-      int rc = binattn::forward_tc(engine == BINATTN_ENGINE_TC, q_bits, k_bits, alpha_q, alpha_k, bias,
-                                   v, softmax_scale, B, H, N, d, out, st, &msg);
+      // TC: the 128-key e4m3 pipeline where it applies, else the 64-key one
+      int rc = engine == BINATTN_ENGINE_TC && binattn::tc2::supported(d, N, bias != nullptr, false)
+                   ? binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N,
+                                          d, out, st, &msg)
+                   : binattn::forward_tc(engine == BINATTN_ENGINE_TC, q_bits, k_bits, alpha_q, alpha_k, bias,
+                                         v, softmax_scale, B, H, N, d, out, st, &msg);
       if (rc) return fail(rc, "%s", msg.c_str());
       return ok();
     }
@@ -213,7 +218,9 @@ int binattn_scores_debug(const uint32_t* q_bits, const uint32_t* k_bits, int B, 
       if (!binattn::tc_supported(d))
         return fail(BINATTN_ERR_UNSUPPORTED, "engine TC needs d %% 8 == 0 (d = %d)", d);
       std::string msg;
-      int rc = binattn::scores_tc(q_bits, k_bits, B, H, N, d, S, st, &msg);
+      int rc = binattn::tc2::supported(d, N, false, false)
+                   ? binattn::scores_tc2(q_bits, k_bits, B, H, N, d, S, st, &msg)
+                   : binattn::scores_tc(q_bits, k_bits, B, H, N, d, S, st, &msg);
       if (rc) return fail(rc, "%s", msg.c_str());
       return ok();
     }
@@ -235,8 +242,11 @@ int binattn_ref_bf16_forward(const uint16_t* q, const uint16_t* k, const uint16_
   if (!binattn::tc_supported(d))
     return fail(BINATTN_ERR_UNSUPPORTED, "the bf16 reference needs d %% 8 == 0 (d = %d)", d);
   std::string msg;
-  int rc = binattn::forward_ref_bf16(q, k, bias, v, softmax_scale, B, H, N, d, out,
-                                     static_cast<cudaStream_t>(stream), &msg);
+  int rc = binattn::tc2::supported(d, N, bias != nullptr, true)
+               ? binattn::forward_ref_tc2(q, k, bias, v, softmax_scale, B, H, N, d, out,
+                                          static_cast<cudaStream_t>(stream), &msg)
+               : binattn::forward_ref_bf16(q, k, bias, v, softmax_scale, B, H, N, d, out,
+                                           static_cast<cudaStream_t>(stream), &msg);
   if (rc) return fail(rc, "%s", msg.c_str());
   return ok();
 }

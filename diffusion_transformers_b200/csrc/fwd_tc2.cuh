@@ -1,0 +1,759 @@
+// fwd_tc2.cuh — the TMA-fed forward pipeline with e4m3 +-1 operands for the
+// binary QK^T: binary forward, its debug-scores variant, and the bf16
+// reference attention on the same pipeline.
+//
+// Source: "BinaryAttention: One-Bit QK-Attention for Vision and Diffusion
+// Transformers", §2 methodology (scaled binary Q/K, XNOR/popcount similarity,
+// additive learnable bias, softmax, P.V) and the hardware-aware implementation
+// bullet (FlashAttention2-style tiling). The tiling below is new for sm_100a.
+//
+// Shapes: d % 8 == 0, d <= 80; with a bias also N % 8 == 0 (the bias rows are
+// TMA rows). One CTA (12 warps, one per SM) owns 256 query rows of one (b, h)
+// as two 128-row tiles t = 0, 1 and streams the keys in tiles of 64:
+//   warps 0-7  softmax: warpgroup t (warps 4t..4t+3), thread = query row = TMEM lane.
+//   warp 8, 9  MMA issuers, one thread each: warp 8 + t issues for tile t.
+//   warp 10    TMA: V (and the bf16 K of the reference attention), bias tiles.
+//   warp 11    binary engines: expands the key sign words to e4m3 +-1 operand
+//              rows and stages alpha_k, loading both two tiles ahead.
+//
+// Tensor memory, 256 columns per warpgroup t (base 256t):
+//   S_t^b  columns [64b, 64b + 64), b = 0, 1: fp32 scores of key tile kt with
+//          kt % 2 == b; P_t(kt) is written back as bf16 pairs over the first
+//          32 columns of S_t^b;
+//   O_t    columns [128, 128 + DV): fp32 accumulator, DV = P.V MMA N >= d + 1;
+//   Q_t    binary: e4m3 bytes, 4 channels per column, columns [224, 224 + 8W);
+//          reference: bf16 pairs, columns [128 + DV, 128 + DV + DV/2).
+// Channel d of V is 1 in every key row (the stage's pad channels are written
+// once and never by TMA), so O_t column d accumulates the row sum l of the
+// bf16 P actually multiplied, and every rescale of O rescales l with it.
+//
+// Issuer t, per key tile kt: once P_t(kt) is published, O_t += P_t(kt) V(kt);
+// then S_t^b = Q_t K(kt+2)^T into the buffer just read (the tensor pipe runs
+// one thread's MMAs in issue order), committed to s_full[t][b]. So the scores
+// of tile kt+1 are ready while the softmax threads work on tile kt, and the
+// commit of QK^T(kt+2) also proves P.V(kt) complete.
+//
+// Binary scores: Q and K bits become e4m3 +1.0 (0x38) / -1.0 (0xB8), pad
+// channels of Q are 0, and the fp32 accumulator holds the exact integer
+// d - 2 popcount(q XOR k) (kind::f8f6f4, K = 32 channels per MMA).
+//
+// Softmax per row, fp32, in two 32-key chunks per tile: logit = (S alpha_k)
+// (scale alpha_q) + bias; the running max m moves only when a chunk max
+// exceeds it by more than 8 (log2 units), and then rescales O_t (and l) and
+// the chunk of P already written in this tile; P = exp(logit - m) rounded to
+// bf16. The epilogue divides O by l (column d) and writes bf16.
+//
+// Every mbarrier wait is bounded (sm100::mbar_wait); on a timeout the CTA
+// records a device status code, leaves its loops, waits for its own MMAs and
+// frees its tensor memory.
+#pragma once
+#include "fwd_tc.cuh"
+
+namespace binattn {
+namespace tc2 {
+
+using namespace sm100;
+
+constexpr int kRows = 128;    // query rows per warpgroup (MMA M)
+constexpr int kKeys = 64;     // keys per tile (QK MMA N, P.V K)
+constexpr int kChunk = 32;    // keys per softmax chunk
+constexpr int kWarps = 12;
+constexpr int kThreads = kWarps * 32;
+constexpr int kMmaWarp0 = 8;   // warps 8, 9: MMA issuers for t = 0, 1
+constexpr int kTmaWarp = 10;
+constexpr int kExpandWarp = 11;
+constexpr int kTmemCols = 512;
+constexpr int kQColBin = 224;  // binary Q operand columns (<= 24)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescale = 5.545177444479562f;  // 8 ln 2: rescale only past a 2^8 growth
+
+// Score sources.
+constexpr int kModeBin = 0;   // binary forward
+constexpr int kModeRef = 1;   // bf16 reference attention
+constexpr int kModeDump = 2;  // binary scores only (debug)
+
+// Shapes this pipeline takes (the caller falls back to the load-mode pipeline otherwise).
+inline bool supported(int d, int N, bool with_bias, bool ref) {
+  if (d % 8 != 0 || d > 80) return false;
+  if (with_bias && N % 8 != 0) return false;
+  if (ref && d > 72) return false;  // Q_t of the reference needs DV/2 more columns
+  return true;
+}
+// P.V N: a multiple of 16 with room for the ones channel d.
+inline int dv_for(int d) { return d < 32 ? 32 : d < 64 ? 64 : d < 80 ? 80 : 96; }
+
+// Shared-memory map (byte offsets).
+//  bias   [kBS][2 t] 128 rows x 64 keys bf16 as one 128B-swizzled box (16 KB):
+//         key k of row r at r * 128 + ((k / 8) ^ (r % 8)) * 16 + (k % 8) * 2.
+//  K      [kKS] binary: 64 keys x 32W e4m3, K-major, no swizzle: 16-byte chunk
+//         (key j, channel group c of 16) at (j / 8) * (8 * 32W) + c * 128 + (j % 8) * 16
+//         -> LBO = 128, SBO = 8 * 32W. Reference: 64 keys x DV bf16, one TMA
+//         box of 8 channels x 64 keys per group: chunk (key j, group c of 8)
+//         at c * 1024 + j * 16 -> LBO = 1024, SBO = 128.
+//  V      [kKS] 64 keys x DV bf16, MN-major: chunk (key j, group g of 8) at
+//         g * 1024 + j * 16 -> LBO = 128 (next 8 keys), SBO = 1024 (next 8 channels).
+//  ak     [kKS] 64 fp32.
+template <int DV, int kMode, bool kBias>
+struct Layout {
+  static constexpr int kKS = kBias ? 4 : 8;                      // K / V / alpha_k stages
+  static constexpr int kBS = 4;                                  // bias stages (per t)
+  static constexpr int kBiasTile = kRows * kKeys * 2;            // 16 KB
+  static constexpr int kKTile = kMode == kModeRef ? kKeys * DV * 2 : kKeys * 96;
+  static constexpr int kVTile = kMode == kModeDump ? 0 : kKeys * DV * 2;
+  static constexpr int kBiasOff = 0;
+  static constexpr int kK = kBiasOff + (kBias ? kBS * 2 * kBiasTile : 0);
+  static constexpr int kV = kK + kKS * kKTile;
+  static constexpr int kAk = kV + kKS * kVTile;
+  static constexpr int kBar = kAk + kKS * kKeys * 4;
+  static constexpr int kNumBars = 48;
+  static constexpr int kMisc = kBar + 8 * kNumBars;  // tmem base, abort flag
+  static constexpr int kBytes = kMisc + 16;
+  // at least this much, so that one CTA occupies an SM (each CTA allocates all
+  // 512 TMEM columns)
+  static constexpr int kLaunchBytes = kBytes > 120 * 1024 ? kBytes : 120 * 1024;
+};
+
+// Instruction descriptor for kind::f8f6f4 with e4m3 A and B (format 0), fp32 D,
+// both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[tmem] * B[smem], 8-bit floating-point operands.
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
+}
+
+// Four e4m3 operand bytes from the low 4 bits of x, lowest bit first: +1.0
+// (0x38) for a set bit, -1.0 (0xB8) for a clear one. The multiply places bit
+// e of x at bit 8e (the shifted copies of x do not overlap, so no carries).
+__device__ __forceinline__ uint32_t e4m3_nibble(uint32_t x) {
+  const uint32_t spread = (x & 0xFu) * 0x00204081u;
+  return ((spread << 7) & 0x80808080u) ^ 0xB8B8B8B8u;
+}
+
+// Four e4m3 operand bytes from bits [j0, j0 + 4) of a sign word: +1 for a set
+// bit, -1 for a clear one; channels c >= d are 0 when zero_pad is set.
+__device__ __forceinline__ uint32_t e4m3_bytes(uint32_t word, int j0, int c0, int d, bool zero_pad) {
+  uint32_t v = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t byte = ((word >> (j0 + j)) & 1u) ? 0x38u : 0xB8u;
+    if (zero_pad && c0 + j >= d) byte = 0;
+    v |= byte << (8 * j);
+  }
+  return v;
+}
+
+template <int DV, int kMode, bool kBias>
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
+               const __grid_constant__ CUtensorMap tm_bias, const __grid_constant__ CUtensorMap tm_k) {
+  using L = Layout<DV, kMode, kBias>;
+  constexpr bool kRef = kMode == kModeRef;
+  constexpr bool kDump = kMode == kModeDump;
+  constexpr int kKS = L::kKS, kBS = L::kBS;
+  static_assert(DV % 16 == 0 && DV <= 96, "P.V N");
+  static_assert(!kRef || DV <= 80, "reference Q_t columns");
+  static_assert(kKS <= 8 && kBS <= 4, "barrier slots");
+
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* kv_full = bars + 0;    // [kKS] V (+ reference K) landed; binary: K expanded, alpha_k staged
+  uint64_t* kv_empty = bars + 8;   // [kKS] both issuers' commits after the tile's P.V
+  uint64_t* b_full = bars + 16;    // [kBS][2 t] bias tile landed
+  uint64_t* b_empty = bars + 24;   // [kBS][2 t] the 128 softmax threads of t are done with it
+  uint64_t* s_full = bars + 32;    // [2 t][2 b] QK^T commit + issuer arrive -> softmax t
+  uint64_t* p_full = bars + 36;    // [2 t][2 b] softmax t published P (128 arrivals) -> issuer t
+  uint64_t* o_done = bars + 40;    // [2 t][2 b] P.V commit of the last two tiles (no QK^T follows)
+  uint64_t* drain = bars + 44;     // [2 t] error path only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Batch entries sharing a bias tile (same h and query tile) are adjacent in
+  // launch order, so the bias tile is fetched from HBM once.
+  const int b = blockIdx.x % p.B;
+  const int qt = blockIdx.x / p.B;
+  const int h = blockIdx.y;
+  const int bh = b * p.H + h;
+  const int N = p.N, d = p.d;
+  const int W = (d + 31) / 32;                 // sign words per token (binary)
+  const size_t tok0 = static_cast<size_t>(bh) * N;
+  const int q0 = qt * 2 * kRows;
+  const int nkt = (N + kKeys - 1) / kKeys;
+  const int dgroups = d / 8;                   // 8-channel groups written by TMA
+  const int kq16 = (d + 15) / 16;              // reference QK^T MMAs (16 channels each)
+
+  // ---------------------------------------------------------------- setup
+  if constexpr (!kDump) {
+    // Channels >= d of every V stage (never written by TMA): channel d is 1.0
+    // (the row-sum column), the rest 0. Reference K: pad channels 0.
+    const int npad = (DV / 8 - dgroups) * kKeys;
+    for (int e = threadIdx.x; e < kKS * npad; e += kThreads) {
+      const int s = e / npad, rem = e % npad;
+      const int g = dgroups + rem / kKeys, kk = rem % kKeys;
+      *reinterpret_cast<uint4*>(smem + L::kV + s * L::kVTile + g * 1024 + kk * 16) =
+          make_uint4(g == dgroups ? 0x3F80u : 0u, 0u, 0u, 0u);
+    }
+    if constexpr (kRef) {
+      const int kpad = (2 * kq16 - dgroups) * kKeys;
+      for (int e = threadIdx.x; e < kKS * kpad; e += kThreads) {
+        const int s = e / kpad, rem = e % kpad;
+        const int g = dgroups + rem / kKeys, kk = rem % kKeys;
+        *reinterpret_cast<uint4*>(smem + L::kK + s * L::kKTile + g * 1024 + kk * 16) = make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kKS; ++s) {
+      mbar_init(&kv_full[s], kRef ? 1 : (kDump ? 32 : 33));
+      mbar_init(&kv_empty[s], 2);
+    }
+    for (int i = 0; i < kBS * 2; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], kRows);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&s_full[i], 2);  // the QK^T commit + the issuer's arrive (alpha_k, bias landed)
+      mbar_init(&p_full[i], kRows);
+      mbar_init(&o_done[i], 1);
+    }
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // Softmax threads: this thread's query row; Q_t operand row into TMEM.
+  const int t = warp >> 2;                   // warpgroup (warps 0-7)
+  const int r = ((warp & 3) << 5) | lane;    // row within the tile = TMEM lane
+  const int row = q0 + t * kRows + r;
+  const bool row_valid = warp < 8 && row < N;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  if (warp < 8) {
+    if constexpr (kRef) {
+      // bf16 pairs: column c2 holds channels 2 c2 (low half) and 2 c2 + 1
+      const uint32_t qcol = tmem + lane_base + 256 * t + 128 + DV;
+      for (int c = 0; c < 2 * kq16; c += 2) {
+        uint32_t wv[8];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint4 val = make_uint4(0, 0, 0, 0);
+          if (row_valid && 8 * (c + h2) < d)
+            val = *reinterpret_cast<const uint4*>(p.q + (tok0 + row) * d + 8 * (c + h2));
+          wv[4 * h2 + 0] = val.x;
+          wv[4 * h2 + 1] = val.y;
+          wv[4 * h2 + 2] = val.z;
+          wv[4 * h2 + 3] = val.w;
+        }
+        tmem_st8(qcol + 4 * c, wv);
+      }
+    } else {
+      // e4m3 bytes: column c4 holds channels 4 c4 .. 4 c4 + 3 (lowest byte first);
+      // pad channels (>= d) are 0 so they add nothing to the score.
+      const uint32_t qcol = tmem + lane_base + 256 * t + kQColBin;
+      for (int w = 0; w < W; ++w) {
+        const uint32_t word = row_valid ? p.qb[(tok0 + row) * W + w] : 0u;
+        uint32_t wv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) wv[j] = row_valid ? e4m3_bytes(word, 4 * j, 32 * w + 4 * j, d, true) : 0u;
+        tmem_st8(qcol + 8 * w, wv);
+      }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  tc_fence_after();
+
+  if (warp == kTmaWarp) {
+    // --------------------------- V (and reference K), bias: one thread issues
+    if (lane == 0 && (!kDump || kBias)) {
+      bool ok = true;
+      for (int kt = 0; ok && kt < nkt; ++kt) {
+        const int j0 = kt * kKeys;
+        if constexpr (!kDump) {
+          const int s = kt % kKS;
+          if (kt >= kKS && !(ok = mbar_wait(&kv_empty[s], ((kt / kKS) - 1) & 1, abort))) break;
+          mbar_arrive_expect_tx(&kv_full[s], static_cast<uint32_t>(dgroups * 1024 * (kRef ? 2 : 1)));
+          for (int g = 0; g < dgroups; ++g)
+            tma_load_3d(smem + L::kV + s * L::kVTile + g * 1024, &tm_v, 8 * g, j0, bh, &kv_full[s]);
+          if constexpr (kRef) {
+            for (int g = 0; g < dgroups; ++g)
+              tma_load_3d(smem + L::kK + s * L::kKTile + g * 1024, &tm_k, 8 * g, j0, bh, &kv_full[s]);
+          }
+        }
+        if constexpr (kBias) {
+          for (int t2 = 0; t2 < 2; ++t2) {
+            const int i = (kt % kBS) * 2 + t2;
+            if (kt >= kBS && !(ok = mbar_wait(&b_empty[i], ((kt / kBS) - 1) & 1, abort))) break;
+            mbar_arrive_expect_tx(&b_full[i], L::kBiasTile);
+            tma_load_3d(smem + L::kBiasOff + i * L::kBiasTile, &tm_bias, j0, q0 + t2 * kRows, h, &b_full[i]);
+          }
+        }
+      }
+    }
+  } else if (warp == kExpandWarp) {
+    // ------------------- binary: key sign words -> e4m3 +-1 rows, alpha_k
+    // The sign words and alpha_k of tile kt + 2 are loaded into registers
+    // before tile kt is expanded, so the global-load latency overlaps two tile
+    // periods instead of sitting between the stage's release and its refill.
+    if constexpr (!kRef) {
+      const int kb_row = 32 * W;  // operand bytes per key
+      struct TileRegs {
+        uint32_t wd[2][3];
+        float ak[2];
+      };
+      auto load_tile = [&](int kt, TileRegs& tr) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int key = kt * kKeys + lane + 32 * u;
+          const bool in = kt < nkt && key < N;
+#pragma unroll
+          for (int w = 0; w < 3; ++w) tr.wd[u][w] = (in && w < W) ? __ldg(p.kb + (tok0 + key) * W + w) : 0u;
+          tr.ak[u] = (!kDump && in) ? __ldg(p.ak + tok0 + key) : 0.f;
+        }
+      };
+      TileRegs cur, n1;
+      load_tile(0, cur);
+      load_tile(1, n1);
+      for (int kt = 0; kt < nkt; ++kt) {
+        TileRegs n2;
+        load_tile(kt + 2, n2);
+        const int s = kt % kKS;
+        const bool ok = kt < kKS || mbar_wait(&kv_empty[s], ((kt / kKS) - 1) & 1, abort);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        uint8_t* ks = smem + L::kK + s * L::kKTile;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int rr = lane + 32 * u;
+          uint8_t* dst = ks + (rr >> 3) * (8 * kb_row) + (rr & 7) * 16;
+#pragma unroll
+          for (int c = 0; c < 6; ++c) {
+            if (c < 2 * W) {
+              const uint32_t half = cur.wd[u][c >> 1] >> (16 * (c & 1));
+              *reinterpret_cast<uint4*>(dst + c * 128) =
+                  make_uint4(e4m3_nibble(half), e4m3_nibble(half >> 4), e4m3_nibble(half >> 8), e4m3_nibble(half >> 12));
+            }
+          }
+        }
+        if constexpr (!kDump) {
+          float* aks = reinterpret_cast<float*>(smem + L::kAk) + s * kKeys;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) aks[lane + 32 * u] = cur.ak[u];
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&kv_full[s]);
+        cur = n1;
+        n1 = n2;
+      }
+    }
+  } else if (warp >= kMmaWarp0) {
+    // ----------------------------------------------- MMA issuer of tile tt
+    const int tt = warp - kMmaWarp0;
+    if (lane == 0) {
+      constexpr uint32_t kIdQK = kRef ? idesc_bf16(kRows, kKeys, false) : idesc_e4m3(kRows, kKeys);
+      constexpr uint32_t kIdPV = idesc_bf16(kRows, DV, true);
+      const uint32_t kb_sbo = kRef ? 128u : static_cast<uint32_t>(8 * 32 * W);
+      const uint32_t base_t = tmem + 256 * tt;
+      // S_tt^(kt%2) = Q_tt K(kt)^T
+      auto issue_qk = [&](int kt) {
+        const uint32_t k_base = smem_u32(smem + L::kK + (kt % kKS) * L::kKTile);
+        const uint32_t d_col = base_t + 64 * (kt & 1);
+        if constexpr (kRef) {
+          for (int ks = 0; ks < kq16; ++ks)
+            mma_ts(d_col, base_t + 128 + DV + ks * 8, smem_desc(k_base + ks * 2048, 1024, kb_sbo), kIdQK, ks > 0);
+        } else {
+          for (int ks = 0; ks < W; ++ks)
+            mma_ts_f8(d_col, base_t + kQColBin + ks * 8, smem_desc(k_base + ks * 256, 128, kb_sbo), kIdQK, ks > 0);
+        }
+      };
+      bool ok = true;
+      // Tile kt's operands and softmax inputs are in shared memory: the K / V
+      // stage with alpha_k and, with a bias, this tile's bias box. The issuer
+      // waits for them and then arrives on s_full itself (release), so the
+      // softmax threads' single wait on s_full also covers alpha_k and the bias.
+      auto stage_ready = [&](int kt) {
+        if (!mbar_wait(&kv_full[kt % kKS], (kt / kKS) & 1, abort)) return false;
+        if (kBias && !mbar_wait(&b_full[(kt % kBS) * 2 + tt], (kt / kBS) & 1, abort)) return false;
+        mbar_arrive(&s_full[tt * 2 + (kt & 1)]);
+        tc_fence_after();
+        return true;
+      };
+      for (int kt = 0; ok && kt < 2 && kt < nkt; ++kt) {
+        if (!(ok = stage_ready(kt))) break;
+        issue_qk(kt);
+        mma_commit(&s_full[tt * 2 + (kt & 1)]);
+      }
+      for (int kt = 0; ok && kt < nkt; ++kt) {
+        const int s = kt % kKS;
+        const int bf = kt & 1;
+        if (!(ok = mbar_wait(&p_full[tt * 2 + bf], (kt >> 1) & 1, abort))) break;
+        tc_fence_after();
+        if constexpr (!kDump) {
+          // O_tt += P_tt(kt) V(kt): A = P (bf16 pairs, 8 columns per 16 keys)
+          const uint32_t v_base = smem_u32(smem + L::kV + s * L::kVTile);
+#pragma unroll
+          for (int ks = 0; ks < kKeys / 16; ++ks)
+            mma_ts(base_t + 128, base_t + 64 * bf + ks * 8, smem_desc(v_base + ks * 256, 128, 1024), kIdPV,
+                   (kt > 0 || ks > 0));
+        }
+        mma_commit(&kv_empty[s]);  // this issuer's last use of stage s
+        if (kt + 2 < nkt) {
+          if (!(ok = stage_ready(kt + 2))) break;
+          issue_qk(kt + 2);
+          mma_commit(&s_full[tt * 2 + bf]);
+        } else if constexpr (!kDump) {
+          mma_commit(&o_done[tt * 2 + bf]);
+        }
+      }
+      {  // wait (bounded) for every MMA of this thread before TMEM is freed
+        mma_commit(&drain[tt]);
+        volatile int never = 0;
+        mbar_wait(&drain[tt], 0, &never);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- softmax
+    // per-row factor of the logit: scale * alpha_q (binary) or scale (reference)
+    const float ci = kRef ? p.scale : ((!kDump && row_valid) ? p.scale * p.aq[tok0 + row] : 0.f);
+    const uint32_t o_col = tmem + lane_base + 256 * t + 128;
+    const int r7 = r & 7;
+    float m = -INFINITY;
+    bool ok = true;
+    // Waits are made warp-uniform: the tcgen05.ld/st below are warp-collective.
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+    };
+    // P.V of tile kt - 1 is complete once QK^T(kt + 1) (issued after it by the
+    // same thread) is, or, for the last tile, once its own commit lands.
+    auto wait_pv_prev = [&](int kt) {
+      const bool r1 = kt + 1 < nkt ? wait_all(&s_full[t * 2 + ((kt + 1) & 1)], ((kt + 1) >> 1) & 1)
+                                   : wait_all(&o_done[t * 2 + ((kt - 1) & 1)], 0);
+      tc_fence_after();
+      return r1;
+    };
+    // logits of chunk c (32 keys, in place): S * alpha_k * (scale * alpha_q) + bias
+    auto logits = [&](uint32_t* xr, int c, int kt, const uint8_t* bsm, const float* aks) {
+      float2* xs = reinterpret_cast<float2*>(xr);
+      float* x = reinterpret_cast<float*>(xr);
+      const float2 ci2 = make_float2(ci, ci);
+#pragma unroll
+      for (int q = 0; q < kChunk / 8; ++q) {
+        float2 bv[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+        if constexpr (kBias) {
+          const int u = 4 * c + q;  // 16-byte unit of the row in the 64-key box
+          const uint4 raw = *reinterpret_cast<const uint4*>(bsm + ((u ^ r7) << 4));
+          const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            bv[e] = make_float2(__uint_as_float(rw[e] << 16), __uint_as_float(rw[e] & 0xFFFF0000u));
+        }
+        if constexpr (kRef) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) xs[4 * q + e] = __ffma2_rn(xs[4 * q + e], ci2, bv[e]);
+        } else {
+          const float4 a0 = *reinterpret_cast<const float4*>(aks + kChunk * c + 8 * q);
+          const float4 a1 = *reinterpret_cast<const float4*>(aks + kChunk * c + 8 * q + 4);
+          const float2 av[4] = {make_float2(a0.x, a0.y), make_float2(a0.z, a0.w), make_float2(a1.x, a1.y),
+                                make_float2(a1.z, a1.w)};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) xs[4 * q + e] = __ffma2_rn(__fmul2_rn(xs[4 * q + e], av[e]), ci2, bv[e]);
+        }
+      }
+      const int j0 = kt * kKeys;
+      if (j0 + kChunk * (c + 1) > N) {  // keys >= N take no part (warp-uniform branch)
+#pragma unroll
+        for (int e = 0; e < kChunk; ++e)
+          if (j0 + kChunk * c + e >= N) x[e] = -INFINITY;
+      }
+    };
+    // Chunk max and the lazy rescale: m moves only when a chunk max exceeds it
+    // by more than kRescale; until then every p = exp(logit - m) <= 2^8, and the
+    // final division by l (summed against the same m) cancels the offset. When
+    // m moves, O_t (with l in column d) and the P chunk already written for
+    // this tile are rescaled.
+    auto settle_max = [&](const uint32_t* xr, int c, int kt, uint32_t p_col) {
+      const float* x = reinterpret_cast<const float*>(xr);
+      float mc[4];
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        float a = max3f(x[k4], x[k4 + 4], x[k4 + 8]);
+        a = max3f(a, x[k4 + 12], x[k4 + 16]);
+        a = max3f(a, x[k4 + 20], x[k4 + 24]);
+        mc[k4] = fmaxf(a, x[k4 + 28]);
+      }
+      const float cmax = fmaxf(max3f(mc[0], mc[1], mc[2]), mc[3]);
+      const bool grow = cmax > m + kRescale;
+      bool good = true;
+      if (__any_sync(0xffffffffu, grow)) {
+        const float m_new = grow ? cmax : m;
+        const float corr = grow ? ex2((m - m_new) * kLog2e) : 1.f;  // 0 while m is -inf
+        if (kt > 0 && (good = wait_pv_prev(kt))) {
+#pragma unroll
+          for (int cc = 0; cc < DV; cc += 16) {
+            uint32_t ov[16];
+            tmem_ld16(o_col + cc, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+            tmem_st16(o_col + cc, ov);
+          }
+        }
+        if (c > 0) {
+          tmem_st_wait();
+          uint32_t pv[16];
+          tmem_ld16(p_col, pv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float lo = __uint_as_float(pv[e] << 16) * corr;
+            const float hi = __uint_as_float(pv[e] & 0xFFFF0000u) * corr;
+            pv[e] = pack_bf16x2(lo, hi);
+          }
+          tmem_st16(p_col, pv);
+        }
+        m = m_new;
+      }
+      return good;
+    };
+    // P = exp(logit - m) of a chunk as bf16 pairs into 16 TMEM columns
+    auto exps = [&](const uint32_t* xr, uint32_t p_col) {
+      const float2* xs = reinterpret_cast<const float2*>(xr);
+      const float2 l2e2 = make_float2(kLog2e, kLog2e);
+      const float2 nm2 = make_float2(-m * kLog2e, -m * kLog2e);
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float2 a = __ffma2_rn(xs[e], l2e2, nm2);
+        pk[e] = pack_bf16x2(ex2(a.x), ex2(a.y));
+      }
+      tmem_st16(p_col, pk);
+    };
+
+    for (int kt = 0; kt < nkt; ++kt) {
+      const int s = kt % kKS;
+      const int bf = kt & 1;
+      const int bs = kt % kBS;
+      // scores, alpha_k and the bias tile of kt (see the issuer's stage_ready)
+      if (!(ok = wait_all(&s_full[t * 2 + bf], (kt >> 1) & 1))) break;
+      tc_fence_after();
+      const uint32_t s_col = tmem + lane_base + 256 * t + 64 * bf;
+      const uint8_t* bsm = smem + L::kBiasOff + (bs * 2 + t) * L::kBiasTile + r * 128;
+      const float* aks = reinterpret_cast<const float*>(smem + L::kAk) + s * kKeys;
+      uint32_t xa[kChunk], xb[kChunk];
+      tmem_ld32(s_col, xa);
+      tmem_ld32(s_col + kChunk, xb);
+      tmem_ld_wait();
+      if constexpr (kDump) {
+        if (row_valid) {
+          int32_t* srow = p.S + (tok0 + row) * N + kt * kKeys;
+#pragma unroll
+          for (int e = 0; e < kChunk; ++e) {
+            if (kt * kKeys + e < N) srow[e] = static_cast<int32_t>(__uint_as_float(xa[e]));
+            if (kt * kKeys + kChunk + e < N) srow[kChunk + e] = static_cast<int32_t>(__uint_as_float(xb[e]));
+          }
+        }
+      } else {
+        // chunk 1's logits are issued in the same straight-line block as chunk 0's exps
+        logits(xa, 0, kt, bsm, aks);
+        ok = settle_max(xa, 0, kt, s_col);
+        logits(xb, 1, kt, bsm, aks);
+        exps(xa, s_col);
+        ok = settle_max(xb, 1, kt, s_col) && ok;
+        exps(xb, s_col + 16);
+        if (kBias) mbar_arrive(&b_empty[bs * 2 + t]);
+        if (!__all_sync(0xffffffffu, ok)) break;
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[t * 2 + bf]);
+    }
+    if constexpr (!kDump) {
+      if (ok && wait_all(&o_done[t * 2 + ((nkt - 1) & 1)], 0)) {
+        tc_fence_after();
+        uint32_t lbits;  // l = O_t column d
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(lbits) : "r"(o_col + d));
+        tmem_ld_wait();
+        const float inv = 1.f / __uint_as_float(lbits);
+        uint16_t* orow = p.out + (tok0 + row) * d;
+#pragma unroll
+        for (int cc = 0; cc < DV; cc += 16) {
+          if (cc < d) {  // warp-uniform: d is the same for every thread
+            uint32_t ov[16];
+            tmem_ld16(o_col + cc, ov);
+            tmem_ld_wait();
+            if (row_valid) {
+#pragma unroll
+              for (int e = 0; e < 16; e += 8) {
+                if (cc + e < d) {
+                  uint4 o4;
+                  o4.x = pack_bf16x2(__uint_as_float(ov[e + 0]) * inv, __uint_as_float(ov[e + 1]) * inv);
+                  o4.y = pack_bf16x2(__uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
+                  o4.z = pack_bf16x2(__uint_as_float(ov[e + 4]) * inv, __uint_as_float(ov[e + 5]) * inv);
+                  o4.w = pack_bf16x2(__uint_as_float(ov[e + 6]) * inv, __uint_as_float(ov[e + 7]) * inv);
+                  *reinterpret_cast<uint4*>(orow + cc + e) = o4;
+                }
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------- teardown
+  // Both issuers waited for their own MMAs; every TMEM access of the softmax
+  // threads is complete (wait::ld / wait::st) before this barrier.
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------- host
+// One [BH][N][d] bf16 tensor as boxes of 8 channels x 64 keys: each box is one
+// column of 16-byte chunks of the no-swizzle operand layouts above. Keys >= N
+// of the last tile are outside the box's (b, h) plane and read as 0.
+inline bool make_rows_map(CUtensorMap* tm, const uint16_t* base, cuuint64_t BH, cuuint64_t N,
+                          cuuint64_t d, const char* what, std::string* msg) {
+  tc::EncodeTiledFn enc = tc::encode_fn();
+  if (!enc) {
+    *msg = "cuTensorMapEncodeTiled entry point unavailable";
+    return false;
+  }
+  const cuuint32_t es[3] = {1, 1, 1};
+  const cuuint64_t dims[3] = {d, N, BH};
+  const cuuint64_t strides[2] = {d * 2, N * d * 2};
+  const cuuint32_t box[3] = {8, kKeys, 1};
+  CUresult rc = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(base), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (rc != CUDA_SUCCESS) {
+    *msg = std::string("tensor map (") + what + ") rejected: " + std::to_string(rc);
+    return false;
+  }
+  return true;
+}
+
+// bias [H][N rows][N keys] bf16 as boxes of 64 keys x 128 rows, 128B swizzle.
+inline bool make_bias_map(CUtensorMap* tm, const uint16_t* bias, cuuint64_t H, cuuint64_t N,
+                          std::string* msg) {
+  tc::EncodeTiledFn enc = tc::encode_fn();
+  if (!enc) {
+    *msg = "cuTensorMapEncodeTiled entry point unavailable";
+    return false;
+  }
+  const cuuint32_t es[3] = {1, 1, 1};
+  const cuuint64_t dims[3] = {N, N, H};
+  const cuuint64_t strides[2] = {N * 2, N * N * 2};
+  const cuuint32_t box[3] = {64, kRows, 1};
+  CUresult rc = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(bias), dims, strides, box,
+                    es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (rc != CUDA_SUCCESS) {
+    *msg = "tensor map (bias) rejected: " + std::to_string(rc);
+    return false;
+  }
+  return true;
+}
+
+template <int DV, int kMode, bool kBias>
+inline int launch(const tc::Params& prm, cudaStream_t st, std::string* msg) {
+  CUtensorMap tm_v, tm_bias, tm_k;
+  std::memset(&tm_v, 0, sizeof tm_v);
+  std::memset(&tm_bias, 0, sizeof tm_bias);
+  std::memset(&tm_k, 0, sizeof tm_k);
+  const cuuint64_t BH = static_cast<cuuint64_t>(prm.B) * prm.H;
+  if (kMode != kModeDump && !make_rows_map(&tm_v, prm.v, BH, prm.N, prm.d, "V", msg)) return BINATTN_ERR_CUDA;
+  if (kMode == kModeRef && !make_rows_map(&tm_k, prm.k, BH, prm.N, prm.d, "K", msg)) return BINATTN_ERR_CUDA;
+  if (kBias && !make_bias_map(&tm_bias, prm.bias, prm.H, prm.N, msg)) return BINATTN_ERR_CUDA;
+  auto kern = fwd_tc2_kernel<DV, kMode, kBias>;
+  constexpr int smem = Layout<DV, kMode, kBias>::kLaunchBytes;
+  static_assert(smem <= 227 * 1024, "shared memory over the sm_100 per-CTA limit");
+  static bool configured = false;  // attribute set once per instantiation
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) {
+      *msg = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);
+      return BINATTN_ERR_CUDA;
+    }
+    configured = true;
+  }
+  dim3 grid(static_cast<unsigned>(prm.B * ((prm.N + 2 * kRows - 1) / (2 * kRows))), prm.H);
+  kern<<<grid, kThreads, smem, st>>>(prm, tm_v, tm_bias, tm_k);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    *msg = std::string("fwd_tc2_kernel launch: ") + cudaGetErrorString(e);
+    return BINATTN_ERR_CUDA;
+  }
+  return BINATTN_OK;
+}
+
+template <int kMode, bool kBias>
+inline int dispatch_dv(const tc::Params& prm, cudaStream_t st, std::string* msg) {
+  switch (dv_for(prm.d)) {
+    case 32: return launch<32, kMode, kBias>(prm, st, msg);
+    case 64: return launch<64, kMode, kBias>(prm, st, msg);
+    case 80: return launch<80, kMode, kBias>(prm, st, msg);
+    default:
+      if constexpr (kMode == kModeRef) {
+        *msg = "reference attention on the 128-key pipeline needs d <= 72";
+        return BINATTN_ERR_UNSUPPORTED;
+      } else {
+        return launch<96, kMode, kBias>(prm, st, msg);
+      }
+  }
+}
+
+}  // namespace tc2
+
+inline int forward_tc2(const uint32_t* qb, const uint32_t* kb, const float* aq, const float* ak,
+                       const uint16_t* bias, const uint16_t* v, float scale, int B, int H, int N, int d,
+                       uint16_t* out, cudaStream_t st, std::string* msg) {
+  tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d};
+  return bias ? tc2::dispatch_dv<tc2::kModeBin, true>(prm, st, msg)
+              : tc2::dispatch_dv<tc2::kModeBin, false>(prm, st, msg);
+}
+
+inline int scores_tc2(const uint32_t* qb, const uint32_t* kb, int B, int H, int N, int d, int32_t* S,
+                      cudaStream_t st, std::string* msg) {
+  tc::Params prm{qb, kb, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S, 0.f, B, H, N, d};
+  return tc2::launch<32, tc2::kModeDump, false>(prm, st, msg);
+}
+
+inline int forward_ref_tc2(const uint16_t* q, const uint16_t* k, const uint16_t* bias, const uint16_t* v,
+                           float scale, int B, int H, int N, int d, uint16_t* out, cudaStream_t st,
+                           std::string* msg) {
+  tc::Params prm{nullptr, nullptr, q, k, nullptr, nullptr, bias, v, out, nullptr, scale, B, H, N, d};
+  return bias ? tc2::dispatch_dv<tc2::kModeRef, true>(prm, st, msg)
+              : tc2::dispatch_dv<tc2::kModeRef, false>(prm, st, msg);
+}
+
+}  // namespace binattn

@@ -70,7 +70,9 @@ typedef enum {
  *               Needs d % 8 == 0.
  *   TC        — S by a tcgen05 MMA on +-1 operands expanded from the sign bits in
  *               shared memory (exact integer scores in an fp32 accumulator);
- *               P.V as a bf16 tcgen05 MMA. Needs d % 8 == 0.
+ *               P.V as a bf16 tcgen05 MMA. Needs d % 8 == 0. For d <= 80 (and,
+ *               with a bias, N % 8 == 0) the operands are e4m3 +-1.0 and the
+ *               inputs arrive by TMA; other shapes use bf16 +-1 operands.
  * (A warp-level mma.sync .b1 XOR-popc engine was measured on sm_100a and runs
  *  below __popc throughput; it is not built.)
  */
