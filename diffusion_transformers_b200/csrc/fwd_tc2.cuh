@@ -8,13 +8,13 @@
 // bullet (FlashAttention2-style tiling). The tiling below is new for sm_100a.
 //
 // Shapes: d % 8 == 0, d <= 80; with a bias also N % 8 == 0 (the bias rows are
-// TMA rows). One CTA (20 warps, one per SM) owns 256 query rows of one (b, h)
+// TMA rows). One CTA (12 warps, one per SM) owns 256 query rows of one (b, h)
 // as two 128-row tiles t = 0, 1 and streams the keys in tiles of 64:
-//   warps 0-15 softmax: warps 8t..8t+7 for tile t, two threads per query row
-//              (TMEM lane), each taking one 32-key half of every key tile.
-//   warp 16,17 MMA issuers, one thread each: warp 16 + t issues for tile t.
-//   warp 18    TMA: V (and the bf16 K of the reference attention), bias tiles.
-//   warp 19    binary engines: expands the key sign words to e4m3 +-1 operand
+//   warps 0-7  softmax: warps 4t..4t+3 for tile t, one thread per query row
+//              (TMEM lane).
+//   warp 8, 9  MMA issuers, one thread each: warp 8 + t issues for tile t.
+//   warp 10    TMA: V (and the bf16 K of the reference attention), bias tiles.
+//   warp 11    binary engines: expands the key sign words to e4m3 +-1 operand
 //              rows and stages alpha_k, loading both two tiles ahead.
 //
 // Tensor memory, 256 columns per warpgroup t (base 256t):
@@ -38,12 +38,13 @@
 // channels of Q are 0, and the fp32 accumulator holds the exact integer
 // d - 2 popcount(q XOR k) (kind::f8f6f4, K = 32 channels per MMA).
 //
-// Softmax per row, fp32, two threads per row (one per 32-key half): logit =
-// (S alpha_k) (scale alpha_q) + bias; the halves exchange their maxima through
-// shared memory, so the tile max is known before any exp; the running max m
-// moves only when the tile max exceeds it by more than 8 (log2 units), and then
-// each thread rescales its half of O_t (with l); P = exp(logit - m) rounded to
-// bf16. The epilogue divides O by l (column d) and writes bf16.
+// Softmax per row, fp32, one thread per row: logit = (S alpha_k)
+// (scale alpha_q) + bias; the tile's max is settled before any exp; the
+// running max m moves only when the tile max exceeds it by more than 8 (log2
+// units), and then O_t (with l) is rescaled; P = exp(logit - m) rounded to
+// bf16. The two 128-row tiles take turns on their exp phases (named barriers),
+// so one tile's exps overlap the other's logits. The epilogue divides O by l
+// (column d) and writes bf16.
 //
 // Every mbarrier wait is bounded (sm100::mbar_wait); on a timeout the CTA
 // records a device status code, leaves its loops, waits for its own MMAs and
@@ -59,13 +60,13 @@ using namespace sm100;
 constexpr int kRows = 128;    // query rows per warpgroup (MMA M)
 constexpr int kKeys = 64;     // keys per tile (QK MMA N, P.V K)
 constexpr int kChunk = 32;    // keys per softmax chunk
-constexpr int kSoftmaxWarps = 16;  // 8 per 128-row tile: 2 threads per row
-constexpr int kSoftmaxPerTile = 256;  // softmax threads per 128-row tile
-constexpr int kWarps = 20;
+constexpr int kSoftmaxWarps = 8;     // 4 per 128-row tile: one thread per row
+constexpr int kSoftmaxPerTile = 128;  // softmax threads per 128-row tile
+constexpr int kWarps = 12;
 constexpr int kThreads = kWarps * 32;
-constexpr int kMmaWarp0 = 16;  // warps 16, 17: MMA issuers for t = 0, 1
-constexpr int kTmaWarp = 18;
-constexpr int kExpandWarp = 19;
+constexpr int kMmaWarp0 = 8;  // warps 8, 9: MMA issuers for t = 0, 1
+constexpr int kTmaWarp = 10;
+constexpr int kExpandWarp = 11;
 constexpr int kTmemCols = 512;
 constexpr int kQColBin = 224;  // binary Q operand columns (<= 24)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -108,8 +109,7 @@ struct Layout {
   static constexpr int kK = kBiasOff + (kBias ? kBS * 2 * kBiasTile : 0);
   static constexpr int kV = kK + kKS * kKTile;
   static constexpr int kAk = kV + kKS * kVTile;
-  static constexpr int kXmax = kAk + kKS * kKeys * 4;           // [2 parity][2 t][2 half][128] fp32
-  static constexpr int kBar = kXmax + 2 * 2 * 2 * kRows * 4;
+  static constexpr int kBar = kAk + kKS * kKeys * 4;
   static constexpr int kNumBars = 48;
   static constexpr int kMisc = kBar + 8 * kNumBars;  // tmem base, abort flag
   static constexpr int kBytes = kMisc + 16;
@@ -267,15 +267,14 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   const uint32_t tmem = *tmem_slot;
 
   // Softmax threads: this thread's query row; Q_t operand row into TMEM.
-  // Softmax warp w < 16: tile t = w / 8, rows 32 (w % 4) .. + 31 (the warp's
-  // TMEM lane quadrant), key half kh = (w / 4) % 2 of every 64-key tile.
-  const int t = warp >> 3;
-  const int kh = (warp >> 2) & 1;
+  // Softmax warp w < 8: tile t = w / 4, rows 32 (w % 4) .. + 31 (the warp's
+  // TMEM lane quadrant), one thread per row.
+  const int t = warp >> 2;
   const int r = ((warp & 3) << 5) | lane;    // row within the tile = TMEM lane
   const int row = q0 + t * kRows + r;
   const bool row_valid = warp < kSoftmaxWarps && row < N;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  if (warp < kSoftmaxWarps && kh == 0) {
+  if (warp < kSoftmaxWarps) {
     if constexpr (kRef) {
       // bf16 pairs: column c2 holds channels 2 c2 (low half) and 2 c2 + 1
       const uint32_t qcol = tmem + lane_base + 256 * t + 128 + DV;
@@ -466,9 +465,6 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
     const float ci = kRef ? p.scale : ((!kDump && row_valid) ? p.scale * p.aq[tok0 + row] : 0.f);
     const uint32_t o_col = tmem + lane_base + 256 * t + 128;
     const int r7 = r & 7;
-    const int kc = kh * kChunk;  // this thread's first key within a key tile
-    // chunk maxima of the two halves of each row: [parity][t][half][row]
-    float* xmax = reinterpret_cast<float*>(smem + L::kXmax);
     float m = -INFINITY;
     bool ok = true;
     // Waits are made warp-uniform: the tcgen05.ld/st below are warp-collective.
@@ -483,6 +479,48 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       tc_fence_after();
       return r1;
     };
+    // logits of chunk c (32 keys, in place): S * alpha_k * (scale * alpha_q) + bias
+    auto logits = [&](uint32_t* xr, int c, const uint8_t* bsm, const float* aks) {
+      float2* xs = reinterpret_cast<float2*>(xr);
+      const float2 ci2 = make_float2(ci, ci);
+#pragma unroll
+      for (int q = 0; q < kChunk / 8; ++q) {
+        float2 bv[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+        if constexpr (kBias) {
+          const int u = 4 * c + q;  // 16-byte unit of the row in the 64-key box
+          const uint4 raw = *reinterpret_cast<const uint4*>(bsm + ((u ^ r7) << 4));
+          const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            bv[e] = make_float2(__uint_as_float(rw[e] << 16), __uint_as_float(rw[e] & 0xFFFF0000u));
+        }
+        if constexpr (kRef) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) xs[4 * q + e] = __ffma2_rn(xs[4 * q + e], ci2, bv[e]);
+        } else {
+          const float4 a0 = *reinterpret_cast<const float4*>(aks + kChunk * c + 8 * q);
+          const float4 a1 = *reinterpret_cast<const float4*>(aks + kChunk * c + 8 * q + 4);
+          const float2 av[4] = {make_float2(a0.x, a0.y), make_float2(a0.z, a0.w), make_float2(a1.x, a1.y),
+                                make_float2(a1.z, a1.w)};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) xs[4 * q + e] = __ffma2_rn(__fmul2_rn(xs[4 * q + e], av[e]), ci2, bv[e]);
+        }
+      }
+    };
+    // P = exp(logit - m) of a chunk as bf16 pairs into 16 TMEM columns
+    auto exps = [&](const uint32_t* xr, uint32_t p_col) {
+      const float2* xs = reinterpret_cast<const float2*>(xr);
+      const float2 l2e2 = make_float2(kLog2e, kLog2e);
+      const float2 nm2 = make_float2(-m * kLog2e, -m * kLog2e);
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float2 a = __ffma2_rn(xs[e], l2e2, nm2);
+        pk[e] = pack_bf16x2(ex2(a.x), ex2(a.y));
+      }
+      tmem_st16(p_col, pk);
+    };
 
     // The loop runs every key tile even after an error (with the work
     // skipped), so that each thread takes its part in every named barrier.
@@ -495,93 +533,67 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       if (ok) ok = wait_all(&s_full[t * 2 + bf], (kt >> 1) & 1);
       tc_fence_after();
       const uint32_t s_col = tmem + lane_base + 256 * t + 64 * bf;
-      uint32_t xr[kChunk];
+      uint32_t xa[kChunk], xb[kChunk];
       if (ok) {
-        tmem_ld32(s_col + kc, xr);
+        tmem_ld32(s_col, xa);
+        tmem_ld32(s_col + kChunk, xb);
         tmem_ld_wait();
       }
       if constexpr (kDump) {
         if (ok && row_valid) {
-          int32_t* srow = p.S + (tok0 + row) * N + kt * kKeys + kc;
+          int32_t* srow = p.S + (tok0 + row) * N + kt * kKeys;
 #pragma unroll
-          for (int e = 0; e < kChunk; ++e)
-            if (kt * kKeys + kc + e < N) srow[e] = static_cast<int32_t>(__uint_as_float(xr[e]));
+          for (int e = 0; e < kChunk; ++e) {
+            if (kt * kKeys + e < N) srow[e] = static_cast<int32_t>(__uint_as_float(xa[e]));
+            if (kt * kKeys + kChunk + e < N) srow[kChunk + e] = static_cast<int32_t>(__uint_as_float(xb[e]));
+          }
         }
       } else {
-        float* x = reinterpret_cast<float*>(xr);
-        float2* xs = reinterpret_cast<float2*>(xr);
-        float cmax = -INFINITY;
         if (ok) {
-          // logits = S * alpha_k * (scale * alpha_q) + bias, 8 keys per step
           const uint8_t* bsm = smem + L::kBiasOff + (bs * 2 + t) * L::kBiasTile + r * 128;
-          const float* aks = reinterpret_cast<const float*>(smem + L::kAk) + s * kKeys + kc;
-          const float2 ci2 = make_float2(ci, ci);
+          const float* aks = reinterpret_cast<const float*>(smem + L::kAk) + s * kKeys;
+          logits(xa, 0, bsm, aks);
+          logits(xb, 1, bsm, aks);
+          float* x0 = reinterpret_cast<float*>(xa);
+          float* x1 = reinterpret_cast<float*>(xb);
+          if (kt * kKeys + kKeys > N) {  // keys >= N take no part (warp-uniform branch)
 #pragma unroll
-          for (int q = 0; q < kChunk / 8; ++q) {
-            float2 bv[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                            make_float2(0.f, 0.f)};
-            if constexpr (kBias) {
-              const int u = 4 * kh + q;  // 16-byte unit of the row in the 64-key box
-              const uint4 raw = *reinterpret_cast<const uint4*>(bsm + ((u ^ r7) << 4));
-              const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                bv[e] = make_float2(__uint_as_float(rw[e] << 16), __uint_as_float(rw[e] & 0xFFFF0000u));
-            }
-            if constexpr (kRef) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) xs[4 * q + e] = __ffma2_rn(xs[4 * q + e], ci2, bv[e]);
-            } else {
-              const float4 a0 = *reinterpret_cast<const float4*>(aks + 8 * q);
-              const float4 a1 = *reinterpret_cast<const float4*>(aks + 8 * q + 4);
-              const float2 av[4] = {make_float2(a0.x, a0.y), make_float2(a0.z, a0.w), make_float2(a1.x, a1.y),
-                                    make_float2(a1.z, a1.w)};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) xs[4 * q + e] = __ffma2_rn(__fmul2_rn(xs[4 * q + e], av[e]), ci2, bv[e]);
+            for (int e = 0; e < kChunk; ++e) {
+              if (kt * kKeys + e >= N) x0[e] = -INFINITY;
+              if (kt * kKeys + kChunk + e >= N) x1[e] = -INFINITY;
             }
           }
-          if (kt * kKeys + kc + kChunk > N) {  // keys >= N take no part (warp-uniform branch)
-#pragma unroll
-            for (int e = 0; e < kChunk; ++e)
-              if (kt * kKeys + kc + e >= N) x[e] = -INFINITY;
-          }
+          // tile max: four independent 3-input max chains over both chunks
           float mc[4];
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4) {
-            float a = max3f(x[k4], x[k4 + 4], x[k4 + 8]);
-            a = max3f(a, x[k4 + 12], x[k4 + 16]);
-            a = max3f(a, x[k4 + 20], x[k4 + 24]);
-            mc[k4] = fmaxf(a, x[k4 + 28]);
+            float a = max3f(x0[k4], x0[k4 + 4], x0[k4 + 8]);
+            a = max3f(a, x0[k4 + 12], x0[k4 + 16]);
+            a = max3f(a, x0[k4 + 20], x0[k4 + 24]);
+            a = max3f(a, x0[k4 + 28], x1[k4]);
+            a = max3f(a, x1[k4 + 4], x1[k4 + 8]);
+            a = max3f(a, x1[k4 + 12], x1[k4 + 16]);
+            a = max3f(a, x1[k4 + 20], x1[k4 + 24]);
+            mc[k4] = fmaxf(a, x1[k4 + 28]);
           }
-          cmax = fmaxf(max3f(mc[0], mc[1], mc[2]), mc[3]);
-        }
-        // Row max of the tile: exchange the half maxima through shared memory
-        // (one slot per tile parity, so a slot is rewritten only after both
-        // halves have passed the next barrier).
-        float* slot = xmax + (bf * 2 + t) * 2 * kRows;
-        slot[kh * kRows + r] = cmax;
-        named_sync(1 + t, kSoftmaxPerTile);
-        const float tmax = fmaxf(cmax, slot[(kh ^ 1) * kRows + r]);
-        if (ok) {
+          const float tmax = fmaxf(max3f(mc[0], mc[1], mc[2]), mc[3]);
           // Lazy rescale: m moves only when the tile max exceeds it by more
           // than kRescale; until then every p = exp(logit - m) <= 2^8, and the
           // final division by l (summed against the same m) cancels the
-          // offset. Both threads of a row see the same tmax and take the same
-          // decision; each rescales its half of O_t (l lives in column d).
+          // offset. O_t holds l in column d, so one rescale covers both.
           const bool grow = tmax > m + kRescale;
           if (__any_sync(0xffffffffu, grow)) {
             const float m_new = grow ? tmax : m;
             const float corr = grow ? ex2((m - m_new) * kLog2e) : 1.f;  // 0 while m is -inf
             if (kt > 0 && (ok = wait_pv_prev(kt))) {
-              constexpr int kHalf = DV / 2;
 #pragma unroll
-              for (int cc = 0; cc < kHalf; cc += 8) {
-                uint32_t ov[8];
-                tmem_ld8(o_col + kh * kHalf + cc, ov);
+              for (int cc = 0; cc < DV; cc += 16) {
+                uint32_t ov[16];
+                tmem_ld16(o_col + cc, ov);
                 tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 8; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-                tmem_st8(o_col + kh * kHalf + cc, ov);
+                for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+                tmem_st16(o_col + cc, ov);
               }
             }
             m = m_new;
@@ -592,16 +604,8 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         // while the other computes its logits.
         named_sync(3 + t, 2 * kSoftmaxPerTile);
         if (ok) {
-          // P = exp(logit - m) as bf16 pairs into columns [16 kh, 16 kh + 16) of S_t^bf
-          const float2 l2e2 = make_float2(kLog2e, kLog2e);
-          const float2 nm2 = make_float2(-m * kLog2e, -m * kLog2e);
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float2 a = __ffma2_rn(xs[e], l2e2, nm2);
-            pk[e] = pack_bf16x2(ex2(a.x), ex2(a.y));
-          }
-          tmem_st16(s_col + 16 * kh, pk);
+          exps(xa, s_col);
+          exps(xb, s_col + 16);
           if (kBias) mbar_arrive(&b_empty[bs * 2 + t]);
         }
         if (!(t == 1 && kt == nkt - 1)) named_arrive(4 - t, 2 * kSoftmaxPerTile);  // pass the token on
@@ -621,10 +625,9 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         tmem_ld_wait();
         const float inv = 1.f / __uint_as_float(lbits);
         uint16_t* orow = p.out + (tok0 + row) * d;
-        // the two threads of a row store alternate 16-channel blocks
 #pragma unroll
         for (int cc = 0; cc < DV; cc += 16) {
-          if (((cc >> 4) & 1) == kh && cc < d) {  // warp-uniform
+          if (cc < d) {  // warp-uniform: d is the same for every thread
             uint32_t ov[16];
             tmem_ld16(o_col + cc, ov);
             tmem_ld_wait();
