@@ -150,6 +150,15 @@ int binattn_pack(const void* x, int dtype, int B, int H, int N, int d, uint32_t*
     const float* xf = static_cast<const float*>(x);
     if (vec) binattn::pack_kernel<float, true><<<grid, binattn::kPackThreads, smem, st>>>(xf, n_tokens, d, W, bits, alpha);
     else binattn::pack_kernel<float, false><<<grid, binattn::kPackThreads, 0, st>>>(xf, n_tokens, d, W, bits, alpha);
+  } else if (d % 8 == 0) {  // whole 16-byte chunks per token: one thread per token
+    const uint16_t* xb = static_cast<const uint16_t*>(x);
+    const unsigned rgrid = static_cast<unsigned>((n_tokens + binattn::kPackThreads - 1) / binattn::kPackThreads);
+    switch (W) {
+      case 1: binattn::pack_bf16_rows_kernel<1><<<rgrid, binattn::kPackThreads, 0, st>>>(xb, n_tokens, d, bits, alpha); break;
+      case 2: binattn::pack_bf16_rows_kernel<2><<<rgrid, binattn::kPackThreads, 0, st>>>(xb, n_tokens, d, bits, alpha); break;
+      case 3: binattn::pack_bf16_rows_kernel<3><<<rgrid, binattn::kPackThreads, 0, st>>>(xb, n_tokens, d, bits, alpha); break;
+      default: binattn::pack_bf16_rows_kernel<4><<<rgrid, binattn::kPackThreads, 0, st>>>(xb, n_tokens, d, bits, alpha); break;
+    }
   } else {
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     if (vec) binattn::pack_kernel<uint16_t, true><<<grid, binattn::kPackThreads, smem, st>>>(xb, n_tokens, d, W, bits, alpha);

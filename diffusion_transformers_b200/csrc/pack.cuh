@@ -63,6 +63,50 @@ pack_kernel(const T* __restrict__ x, long long n_tokens, int d, int W,
   }
 }
 
+
+// bf16 rows with d % 8 == 0 (every token a whole number of 16-byte chunks):
+// one thread per token. The thread issues all of its row's 16-byte loads,
+// builds its sign words with x >= 0 compares (8 channels per chunk, 4 chunks
+// per word), and sums |x| in eight partial sums (one per position in a chunk)
+// combined by a tree, so each alpha is a sum of depth <= d/8 + 2 in fp32.
+template <int W>
+__global__ void __launch_bounds__(kPackThreads)
+pack_bf16_rows_kernel(const uint16_t* __restrict__ x, long long n_tokens, int d,
+                      uint32_t* __restrict__ bits, float* __restrict__ alpha) {
+  const long long t = static_cast<long long>(blockIdx.x) * kPackThreads + threadIdx.x;
+  if (t >= n_tokens) return;
+  const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
+  const int ng = d / 8;  // 16-byte chunks per token
+  uint4 v[4 * W];
+#pragma unroll
+  for (int g = 0; g < 4 * W; ++g) v[g] = g < ng ? __ldg(src + g) : make_uint4(0, 0, 0, 0);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int g = 4 * w + j;
+      if (g < ng) {
+        const uint32_t pr[4] = {v[g].x, v[g].y, v[g].z, v[g].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          // channel 8g + 2k in the low half, 8g + 2k + 1 in the high half
+          const float lo = __uint_as_float(pr[k] << 16);
+          const float hi = __uint_as_float(pr[k] & 0xFFFF0000u);
+          word |= (lo >= 0.f ? 1u : 0u) << (8 * j + 2 * k);
+          word |= (hi >= 0.f ? 1u : 0u) << (8 * j + 2 * k + 1);
+          acc[2 * k] += fabsf(lo);
+          acc[2 * k + 1] += fabsf(hi);
+        }
+      }
+    }
+    bits[t * W + w] = word;
+  }
+  const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+  alpha[t] = sum / static_cast<float>(d);
+}
+
 inline size_t pack_smem_bytes(int d, int esize, bool vec) {
   return vec ? static_cast<size_t>(kPackTokens) * d * esize : 0;
 }
