@@ -251,6 +251,58 @@ def run_reference(args, w, rank):
 
 
 # ------------------------------------------------------------------- GPU
+def time_configs(names, args, rank, world, dev, stream, peaks, flush, max_over_ranks):
+    """Forward (with the dense bias) and whole-step times of other workloads:
+    each one seeded and synthetic, timed over min(steps, 10) steps with a cold
+    L2, max over ranks. Every rank runs the same list in the same order."""
+    import torch
+    from diffusion_transformers_b200 import binattn
+
+    def to_dev(x):
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(x).to(dev)
+
+    rows = []
+    steps = max(1, min(args.steps, 10))
+    for name in names:
+        w = WORKLOADS[name]
+        inp = make_inputs(w, with_bias=True, seed=rank_seed(w, rank))
+        q, k, v, bias = to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"]), to_dev(inp["bias"])
+        scale = inp["softmax_scale"]
+        qb, aq = binattn.pack(q, stream=stream)
+        kb, ak = binattn.pack(k, stream=stream)
+        out = torch.empty_like(v)
+        for _ in range(3):
+            binattn.pack(q, qb, aq, stream)
+            binattn.pack(k, kb, ak, stream)
+            binattn.forward(qb, kb, aq, ak, bias, v, scale, out=out, engine=args.engine, stream=stream)
+        torch.cuda.synchronize()
+        ev = []
+        for _ in range(steps):
+            flush.fill_(1)
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record(stream)
+            binattn.pack(q, qb, aq, stream)
+            binattn.pack(k, kb, ak, stream)
+            e[1].record(stream)
+            binattn.forward(qb, kb, aq, ak, bias, v, scale, out=out, engine=args.engine, stream=stream)
+            e[2].record(stream)
+            ev.append(e)
+        torch.cuda.synchronize()
+        binattn.device_status(stream)
+        step_ms = max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in ev) / steps)
+        fwd_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / steps)
+        a = algorithmic(w, True)
+        t_roof = max(a["bytes"] / (peaks["hbm_gbs"] * 1e9), a["eff_flops"] / (peaks["bf16_tflops"] * 1e12))
+        rows.append({"workload": name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bias": True,
+                     "forward_ms": round(fwd_ms, 5), "step_ms": round(step_ms, 5),
+                     "effective_tflops": round(a["eff_flops"] / (fwd_ms * 1e-3) / 1e12, 2),
+                     "roofline_frac": round(t_roof / (fwd_ms * 1e-3), 4)})
+        del q, k, v, bias, qb, kb, aq, ak, out
+    return rows
+
+
 def run_gpu(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -376,6 +428,10 @@ def run_gpu(args, w, rank, world, local_rank):
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
 
+    # the other workloads of the parity suite, timed the same way (forward with bias)
+    others = time_configs([n for n in WORKLOADS if n != w.name], args, rank, world, dev, stream, peaks,
+                          flush, max_over_ranks)
+
     if rank != 0:
         return
     a = algorithmic(w, True)
@@ -410,6 +466,7 @@ def run_gpu(args, w, rank, world, local_rank):
                     "forward_ms": round(results["no_bias"]["fwd_ms"], 5),
                     "effective_tflops": round(a0["eff_flops"] / fwd0_s / 1e12, 2)},
         "bf16_reference": ref,
+        "other_workloads": others,
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
                      "frac": round(achieved / peak, 4),
                      "traffic": ncu_traffic(f"{w.name}/bias"), "traffic_unit": "bytes per launch",
