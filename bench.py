@@ -85,11 +85,11 @@ def algorithmic(w, with_bias=True):
 
 # DRAM traffic of the forward kernel from one ncu capture (dram__bytes_read.sum
 # + dram__bytes_write.sum, one launch at dit_xl_1024 with bias; the summary is
-# profiles/fwd_tc_dit_xl_1024_bias.md), valid only for the kernel sources it was
+# profiles/fwd_tc2_dit_xl_1024_bias.md), valid only for the kernel sources it was
 # taken on: any change to them turns the reported traffic back into null.
 NCU_TRAFFIC = {
-    "sources_sha256": "2055e52fc6818acb71eec426bef90febdbd3ce79d52ec30d006f4839c9cbedb4",
-    "bytes_per_launch": {"dit_xl_1024/bias": 582_176_768},
+    "sources_sha256": "ac3fb190eda82e7c0f4d67b20ac258f7b5f48cbd3adc475554d5e18470648457",
+    "bytes_per_launch": {"dit_xl_1024/bias": 584_370_432},
 }
 
 
