@@ -20,9 +20,9 @@ ENGINES = {"auto": ENGINE_AUTO, "simt": ENGINE_SIMT, "popc_tc": ENGINE_POPC_TC, 
 
 # Every symbol include/binattn.h declares.
 EXPORTS = (
-    "binattn_pack", "binattn_forward", "binattn_forward_engine", "binattn_scores_debug",
-    "binattn_ref_bf16_forward", "binattn_device_status", "binattn_strerror",
-    "binattn_last_error_message", "binattn_abi_version",
+    "binattn_pack", "binattn_forward", "binattn_forward_engine", "binattn_forward_workspace_bytes",
+    "binattn_forward_ws", "binattn_scores_debug", "binattn_ref_bf16_forward", "binattn_device_status",
+    "binattn_strerror", "binattn_last_error_message", "binattn_abi_version",
 )
 
 
@@ -52,13 +52,17 @@ def lib() -> ctypes.CDLL:
     L.binattn_pack.argtypes = [P, I, I, I, I, I, P, P, P]
     L.binattn_forward.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, P]
     L.binattn_forward_engine.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, I, P]
+    L.binattn_forward_workspace_bytes.argtypes = [I, I, I, I, I]
+    L.binattn_forward_workspace_bytes.restype = ctypes.c_size_t
+    L.binattn_forward_ws.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
     L.binattn_scores_debug.argtypes = [P, P, I, I, I, I, P, I, P]
     L.binattn_ref_bf16_forward.argtypes = [P, P, P, P, F, I, I, I, I, P, P]
     L.binattn_device_status.argtypes = [P]
     L.binattn_strerror.argtypes = [I]
     L.binattn_strerror.restype = ctypes.c_char_p
     L.binattn_last_error_message.restype = ctypes.c_char_p
-    for name in ("binattn_pack", "binattn_forward", "binattn_forward_engine", "binattn_scores_debug",
+    for name in ("binattn_pack", "binattn_forward", "binattn_forward_engine", "binattn_forward_ws",
+                 "binattn_scores_debug",
                  "binattn_ref_bf16_forward", "binattn_device_status", "binattn_abi_version"):
         getattr(L, name).restype = I
     _lib = L
@@ -135,6 +139,31 @@ def scores_debug(q_bits: torch.Tensor, k_bits: torch.Tensor, d: int,
     _check(lib().binattn_scores_debug(_ptr(q_bits), _ptr(k_bits), B, H, N, d, _ptr(S), int(engine),
                                       _stream(stream)), "binattn_scores_debug")
     return S
+
+
+def workspace_bytes(B: int, H: int, N: int, d: int, has_bias: bool) -> int:
+    """Device workspace bytes forward_ws needs (0: forward already takes the fast path)."""
+    return int(lib().binattn_forward_workspace_bytes(B, H, N, d, int(bool(has_bias))))
+
+
+def forward_ws(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor,
+               alpha_k: torch.Tensor, bias: torch.Tensor | None, v: torch.Tensor,
+               softmax_scale: float, workspace: torch.Tensor | None = None,
+               out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """forward (engine AUTO) with a caller-owned workspace (uint8 CUDA tensor of at
+    least workspace_bytes(...) bytes; allocated here when None)."""
+    B, H, N, d = v.shape
+    need = workspace_bytes(B, H, N, d, bias is not None)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=v.device)
+    size = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().binattn_forward_ws(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k), _ptr(bias),
+                                    _ptr(v), float(softmax_scale), B, H, N, d, _ptr(out), _ptr(workspace),
+                                    ctypes.c_size_t(size), _stream(stream)),
+           "binattn_forward_ws")
+    return out
 
 
 def ref_bf16_forward(q: torch.Tensor, k: torch.Tensor, bias: torch.Tensor | None, v: torch.Tensor,

@@ -205,6 +205,49 @@ int binattn_forward(const uint32_t* q_bits, const uint32_t* k_bits, const float*
                                 d, out, BINATTN_ENGINE_AUTO, stream);
 }
 
+namespace {
+// Padded bias rows for the TMA-fed pipeline: the workspace holds [H][N][ld]
+// bf16, ld = N rounded up to a multiple of 8.
+int padded_bias_ld(int N) { return (N + 7) / 8 * 8; }
+bool needs_padded_bias(int d, int N, bool has_bias) {
+  return has_bias && N % 8 != 0 && binattn::tc2::supported(d, N, true, false, padded_bias_ld(N));
+}
+}  // namespace
+
+size_t binattn_forward_workspace_bytes(int B, int H, int N, int d, int has_bias) {
+  if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
+  if (!needs_padded_bias(d, N, has_bias != 0)) return 0;
+  return static_cast<size_t>(H) * N * padded_bias_ld(N) * 2;
+}
+
+int binattn_forward_ws(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
+                       const float* alpha_k, const uint16_t* bias, const uint16_t* v,
+                       float softmax_scale, int B, int H, int N, int d, uint16_t* out,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (int rc = check_forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out))
+    return rc;
+  if (!needs_padded_bias(d, N, bias != nullptr))
+    return binattn_forward_engine(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out,
+                                  BINATTN_ENGINE_AUTO, stream);
+  const size_t need = binattn_forward_workspace_bytes(B, H, N, d, 1);
+  BINATTN_CHECK_PTR(workspace);
+  if (!aligned16(workspace)) return fail(BINATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  if (workspace_bytes < need)
+    return fail(BINATTN_ERR_ARG, "workspace of %zu bytes is below the %zu this shape needs", workspace_bytes, need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int ld = padded_bias_ld(N);
+  uint16_t* padded = static_cast<uint16_t*>(workspace);
+  const long long rows = static_cast<long long>(H) * N;
+  const unsigned grid = static_cast<unsigned>((rows * ld + 255) / 256);
+  binattn::tc2::pad_bias_rows_kernel<<<grid, 256, 0, st>>>(bias, rows, N, ld, padded);
+  if (int rc = launch_status("pad_bias_rows_kernel")) return rc;
+  std::string msg;
+  int rc = binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, padded, v, softmax_scale, B, H, N, d, out, st,
+                                &msg, ld);
+  if (rc) return fail(rc, "%s", msg.c_str());
+  return ok();
+}
+
 int binattn_scores_debug(const uint32_t* q_bits, const uint32_t* k_bits, int B, int H, int N,
                          int d, int32_t* S, int engine, void* stream) {
   BINATTN_CHECK_PTR(q_bits);

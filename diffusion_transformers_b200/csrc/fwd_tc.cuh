@@ -132,6 +132,7 @@ struct Params {
   int32_t* S;  // debug scores (dump mode)
   float scale;
   int B, H, N, d;
+  int bias_ld;  // elements between bias rows (N, or the padded row length); 0 means N
 };
 
 // Named barrier 1 over the load-mode loader warps with an AND reduction.

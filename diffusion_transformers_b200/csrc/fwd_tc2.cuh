@@ -78,9 +78,10 @@ constexpr int kModeRef = 1;   // bf16 reference attention
 constexpr int kModeDump = 2;  // binary scores only (debug)
 
 // Shapes this pipeline takes (the caller falls back to the load-mode pipeline otherwise).
-inline bool supported(int d, int N, bool with_bias, bool ref) {
+// bias_ld: elements between bias rows (N, or a padded length; TMA needs % 8 == 0).
+inline bool supported(int d, int N, bool with_bias, bool ref, int bias_ld = 0) {
   if (d % 8 != 0 || d > 80) return false;
-  if (with_bias && N % 8 != 0) return false;
+  if (with_bias && (bias_ld > 0 ? bias_ld : N) % 8 != 0) return false;
   if (ref && d > 72) return false;  // Q_t of the reference needs DV/2 more columns
   return true;
 }
@@ -661,6 +662,18 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   }
 }
 
+// Bias rows padded to ld elements (ld % 8 == 0, pad 0), so that they are TMA
+// rows: out[(h * N + i) * ld + j] = j < N ? bias[(h * N + i) * N + j] : 0.
+__global__ void __launch_bounds__(256) pad_bias_rows_kernel(const uint16_t* __restrict__ bias,
+                                                            long long rows, int N, int ld,
+                                                            uint16_t* __restrict__ out) {
+  const long long e = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  if (e >= rows * ld) return;
+  const long long row = e / ld;
+  const int j = static_cast<int>(e - row * ld);
+  out[e] = j < N ? bias[row * N + j] : static_cast<uint16_t>(0);
+}
+
 // ------------------------------------------------------------------- host
 // One [BH][N][d] bf16 tensor as boxes of 8 channels x 64 keys: each box is one
 // column of 16-byte chunks of the no-swizzle operand layouts above. Keys >= N
@@ -686,9 +699,10 @@ inline bool make_rows_map(CUtensorMap* tm, const uint16_t* base, cuuint64_t BH, 
   return true;
 }
 
-// bias [H][N rows][N keys] bf16 as boxes of 64 keys x 128 rows, 128B swizzle.
+// bias [H][N rows][N keys] bf16, rows ld elements apart (ld % 8 == 0), as boxes of
+// 64 keys x 128 rows, 128B swizzle.
 inline bool make_bias_map(CUtensorMap* tm, const uint16_t* bias, cuuint64_t H, cuuint64_t N,
-                          std::string* msg) {
+                          cuuint64_t ld, std::string* msg) {
   tc::EncodeTiledFn enc = tc::encode_fn();
   if (!enc) {
     *msg = "cuTensorMapEncodeTiled entry point unavailable";
@@ -696,7 +710,7 @@ inline bool make_bias_map(CUtensorMap* tm, const uint16_t* bias, cuuint64_t H, c
   }
   const cuuint32_t es[3] = {1, 1, 1};
   const cuuint64_t dims[3] = {N, N, H};
-  const cuuint64_t strides[2] = {N * 2, N * N * 2};
+  const cuuint64_t strides[2] = {ld * 2, N * ld * 2};
   const cuuint32_t box[3] = {64, kRows, 1};
   CUresult rc = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(bias), dims, strides, box,
                     es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -717,7 +731,8 @@ inline int launch(const tc::Params& prm, cudaStream_t st, std::string* msg) {
   const cuuint64_t BH = static_cast<cuuint64_t>(prm.B) * prm.H;
   if (kMode != kModeDump && !make_rows_map(&tm_v, prm.v, BH, prm.N, prm.d, "V", msg)) return BINATTN_ERR_CUDA;
   if (kMode == kModeRef && !make_rows_map(&tm_k, prm.k, BH, prm.N, prm.d, "K", msg)) return BINATTN_ERR_CUDA;
-  if (kBias && !make_bias_map(&tm_bias, prm.bias, prm.H, prm.N, msg)) return BINATTN_ERR_CUDA;
+  if (kBias && !make_bias_map(&tm_bias, prm.bias, prm.H, prm.N, prm.bias_ld > 0 ? prm.bias_ld : prm.N, msg))
+    return BINATTN_ERR_CUDA;
   auto kern = fwd_tc2_kernel<DV, kMode, kBias>;
   constexpr int smem = Layout<DV, kMode, kBias>::kLaunchBytes;
   static_assert(smem <= 227 * 1024, "shared memory over the sm_100 per-CTA limit");
@@ -760,8 +775,8 @@ inline int dispatch_dv(const tc::Params& prm, cudaStream_t st, std::string* msg)
 
 inline int forward_tc2(const uint32_t* qb, const uint32_t* kb, const float* aq, const float* ak,
                        const uint16_t* bias, const uint16_t* v, float scale, int B, int H, int N, int d,
-                       uint16_t* out, cudaStream_t st, std::string* msg) {
-  tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d};
+                       uint16_t* out, cudaStream_t st, std::string* msg, int bias_ld = 0) {
+  tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d, bias_ld};
   return bias ? tc2::dispatch_dv<tc2::kModeBin, true>(prm, st, msg)
               : tc2::dispatch_dv<tc2::kModeBin, false>(prm, st, msg);
 }

@@ -34,6 +34,7 @@
 #ifndef BINATTN_H
 #define BINATTN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -124,6 +125,34 @@ int binattn_forward(const uint32_t *q_bits, const uint32_t *k_bits,
                     const float *alpha_q, const float *alpha_k,
                     const uint16_t *bias, const uint16_t *v, float softmax_scale,
                     int B, int H, int N, int d, uint16_t *out, void *stream);
+
+/*
+ * binattn_forward_workspace_bytes — device workspace that binattn_forward_ws
+ * needs for this shape: 0 when binattn_forward already takes the TMA-fed
+ * pipeline, else H * N * roundup(N, 8) * 2 bytes (a bias whose rows are not a
+ * multiple of 8 elements, with 8 <= d <= 80 and d % 8 == 0). Never fails.
+ */
+size_t binattn_forward_workspace_bytes(int B, int H, int N, int d, int has_bias);
+
+/*
+ * binattn_forward_ws — binattn_forward (engine AUTO) with a caller-owned
+ * device workspace, for biases whose row length N is not a multiple of 8: the
+ * bias is first copied into the workspace with each row padded to
+ * roundup(N, 8) elements (pad 0), so that its rows are TMA rows, and the
+ * forward then runs on the TMA-fed pipeline. Same result as binattn_forward.
+ *   workspace        device, 16-byte aligned, at least
+ *                    binattn_forward_workspace_bytes(...) bytes, overwritten;
+ *                    may be NULL when that size is 0.
+ *   workspace_bytes  its size.
+ * Errors: BINATTN_ERR_NULL / ERR_ALIGN for the workspace, BINATTN_ERR_ARG when
+ * it is smaller than needed; otherwise as binattn_forward. Asynchronous on
+ * `stream`; the workspace must not be reused before the call completes.
+ */
+int binattn_forward_ws(const uint32_t *q_bits, const uint32_t *k_bits,
+                       const float *alpha_q, const float *alpha_k,
+                       const uint16_t *bias, const uint16_t *v, float softmax_scale,
+                       int B, int H, int N, int d, uint16_t *out,
+                       void *workspace, size_t workspace_bytes, void *stream);
 
 /* binattn_forward with an explicit score engine (binattn_engine). Returns
  * BINATTN_ERR_UNSUPPORTED when the engine cannot serve the shape. */

@@ -92,3 +92,29 @@ def test_scores_and_ref_host_validation(L):
 def test_last_error_message_is_specific(L):
     assert _fwd(L, v=A + 8) == 4
     assert b"v is not 16-byte aligned" in L.binattn_last_error_message()
+
+
+def test_workspace_bytes(L):
+    # a bias whose rows are not a multiple of 8 elements: [H][N][roundup(N, 8)] bf16
+    assert L.binattn_forward_workspace_bytes(64, 12, 197, 64, 1) == 12 * 197 * 200 * 2
+    assert L.binattn_forward_workspace_bytes(32, 16, 577, 64, 1) == 16 * 577 * 584 * 2
+    # rows already TMA rows, no bias, or a shape the TMA-fed pipeline does not take
+    assert L.binattn_forward_workspace_bytes(2, 16, 4096, 72, 1) == 0
+    assert L.binattn_forward_workspace_bytes(64, 12, 197, 64, 0) == 0
+    assert L.binattn_forward_workspace_bytes(1, 1, 197, 128, 1) == 0
+    assert L.binattn_forward_workspace_bytes(1, 1, 197, 33, 1) == 0
+    assert L.binattn_forward_workspace_bytes(0, 1, 197, 64, 1) == 0
+
+
+def test_forward_ws_host_validation(L):
+    def fws(ws=A, size=1 << 30, bias=A, N=197, d=64):
+        return L.binattn_forward_ws(P(A), P(A), P(A), P(A), P(bias) if bias else None, P(A),
+                                    ctypes.c_float(0.125), 1, 2, N, d, P(A),
+                                    P(ws) if ws else None, ctypes.c_size_t(size), None)
+    need = L.binattn_forward_workspace_bytes(1, 2, 197, 64, 1)
+    assert fws(ws=0) == 1
+    assert fws(ws=A + 8) == 4
+    assert fws(size=need - 1) == 8
+    assert b"workspace" in L.binattn_last_error_message()
+    assert fws(bias=A + 2) == 4
+    assert fws(N=0) == 2

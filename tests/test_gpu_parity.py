@@ -152,3 +152,46 @@ def test_device_errors_are_reported():
                         ctypes.c_void_p(bits.data_ptr()), ctypes.c_void_p(alpha.data_ptr()), None)
     assert rc == 4
     binattn.device_status()
+
+
+# ------------------------------------------- forward with a workspace (padded bias rows)
+# Bias rows of N % 8 != 0 elements are not TMA rows; binattn_forward_ws pads
+# them into the workspace and runs the TMA-fed pipeline. Same bar as forward.
+WS_SHAPES = [(2, 3, 129, 72), (1, 2, 197, 64), (1, 1, 130, 72), (2, 2, 65, 16), (1, 1, 1, 64),
+             (1, 3, 1001, 40), (1, 2, 300, 8)]
+
+
+def _run_ws(inp, with_bias=True):
+    q, k, v = dev(inp["q"]), dev(inp["k"]), dev(inp["v"])
+    bias = dev(inp["bias"]) if with_bias else None
+    qb, aq = binattn.pack(q)
+    kb, ak = binattn.pack(k)
+    B, H, N, d = v.shape
+    need = binattn.workspace_bytes(B, H, N, d, with_bias)
+    ws = torch.full((max(need, 16),), 0xA5, dtype=torch.uint8, device="cuda")  # stale bytes on purpose
+    out = binattn.forward_ws(qb, kb, aq, ak, bias, v, inp["softmax_scale"], workspace=ws)
+    torch.cuda.synchronize()
+    binattn.device_status()
+    return out, need
+
+
+@pytest.mark.parametrize("shape", WS_SHAPES)
+def test_forward_ws_small(orc, shape):
+    B, H, N, d = shape
+    c = make_custom(B, H, N, d, seed=5 * N + d, with_bias=True, bias_std=0.5)
+    ref = orc.forward(c["q"], c["k"], c["bias"], c["v"], c["softmax_scale"])
+    out, need = _run_ws(c)
+    assert need == (H * N * ((N + 7) // 8 * 8) * 2 if N % 8 else 0)
+    check_o(bf16_to_f64(out), ref, f"ws {shape}")
+
+
+@pytest.mark.parametrize("name", ["deit_b", "vit_l384"])
+def test_forward_ws_full_size_sampled(orc, name):
+    inp = make_inputs(name, with_bias=True)
+    B, H, N, d = inp["B"], inp["H"], inp["N"], inp["d"]
+    rows = sample_rows(B, H, N, 96, seed=7)
+    ref = orc.forward_rows(inp["q"], inp["k"], inp["bias"], inp["v"], inp["softmax_scale"], rows)
+    out, need = _run_ws(inp)
+    assert need > 0
+    got = out.view(B * H * N, d)[torch.from_numpy(rows).cuda()]
+    check_o(bf16_to_f64(got), ref, f"ws {name}")
