@@ -21,8 +21,9 @@ ENGINES = {"auto": ENGINE_AUTO, "simt": ENGINE_SIMT, "popc_tc": ENGINE_POPC_TC, 
 # Every symbol include/binattn.h declares.
 EXPORTS = (
     "binattn_pack", "binattn_forward", "binattn_forward_engine", "binattn_forward_workspace_bytes",
-    "binattn_forward_ws", "binattn_scores_debug", "binattn_ref_bf16_forward", "binattn_device_status",
-    "binattn_strerror", "binattn_last_error_message", "binattn_abi_version",
+    "binattn_forward_ws", "binattn_forward_static_ws", "binattn_scores_debug",
+    "binattn_ref_bf16_forward", "binattn_device_status", "binattn_strerror",
+    "binattn_last_error_message", "binattn_abi_version",
 )
 
 
@@ -55,6 +56,7 @@ def lib() -> ctypes.CDLL:
     L.binattn_forward_workspace_bytes.argtypes = [I, I, I, I, I]
     L.binattn_forward_workspace_bytes.restype = ctypes.c_size_t
     L.binattn_forward_ws.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
+    L.binattn_forward_static_ws.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, P]
     L.binattn_scores_debug.argtypes = [P, P, I, I, I, I, P, I, P]
     L.binattn_ref_bf16_forward.argtypes = [P, P, P, P, F, I, I, I, I, P, P]
     L.binattn_device_status.argtypes = [P]
@@ -62,6 +64,7 @@ def lib() -> ctypes.CDLL:
     L.binattn_strerror.restype = ctypes.c_char_p
     L.binattn_last_error_message.restype = ctypes.c_char_p
     for name in ("binattn_pack", "binattn_forward", "binattn_forward_engine", "binattn_forward_ws",
+                 "binattn_forward_static_ws",
                  "binattn_scores_debug",
                  "binattn_ref_bf16_forward", "binattn_device_status", "binattn_abi_version"):
         getattr(L, name).restype = I
@@ -163,6 +166,19 @@ def forward_ws(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor
                                     _ptr(v), float(softmax_scale), B, H, N, d, _ptr(out), _ptr(workspace),
                                     ctypes.c_size_t(size), _stream(stream)),
            "binattn_forward_ws")
+    return out
+
+
+def forward_static_ws(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor,
+                      alpha_k: torch.Tensor, bias: torch.Tensor | None, v: torch.Tensor,
+                      softmax_scale: float, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """forward_ws on the library's static workspace: the call allocates no device memory."""
+    B, H, N, d = v.shape
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=v.device)
+    _check(lib().binattn_forward_static_ws(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k), _ptr(bias),
+                                           _ptr(v), float(softmax_scale), B, H, N, d, _ptr(out), _stream(stream)),
+           "binattn_forward_static_ws")
     return out
 
 

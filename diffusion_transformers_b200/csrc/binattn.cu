@@ -248,6 +248,32 @@ int binattn_forward_ws(const uint32_t* q_bits, const uint32_t* k_bits, const flo
   return ok();
 }
 
+namespace {
+// Static workspace of binattn_forward_static_ws: part of the loaded module, so
+// the call itself allocates no device memory.
+constexpr size_t kStaticWorkspaceBytes = size_t(32) << 20;
+__device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+}  // namespace
+
+int binattn_forward_static_ws(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
+                              const float* alpha_k, const uint16_t* bias, const uint16_t* v,
+                              float softmax_scale, int B, int H, int N, int d, uint16_t* out,
+                              void* stream) {
+  if (int rc = check_forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out))
+    return rc;
+  const size_t need = binattn_forward_workspace_bytes(B, H, N, d, bias != nullptr);
+  if (need > kStaticWorkspaceBytes)
+    return fail(BINATTN_ERR_UNSUPPORTED, "this shape needs %zu bytes of workspace; the static one holds %zu",
+                need, kStaticWorkspaceBytes);
+  void* ws = nullptr;
+  if (need) {
+    cudaError_t e = cudaGetSymbolAddress(&ws, g_static_workspace);
+    if (e != cudaSuccess) return fail(BINATTN_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+  }
+  return binattn_forward_ws(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out, ws,
+                            need ? kStaticWorkspaceBytes : 0, stream);
+}
+
 int binattn_scores_debug(const uint32_t* q_bits, const uint32_t* k_bits, int B, int H, int N,
                          int d, int32_t* S, int engine, void* stream) {
   BINATTN_CHECK_PTR(q_bits);

@@ -154,6 +154,19 @@ int binattn_forward_ws(const uint32_t *q_bits, const uint32_t *k_bits,
                        int B, int H, int N, int d, uint16_t *out,
                        void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * binattn_forward_static_ws — binattn_forward_ws with the library's own static
+ * device workspace (32 MiB, part of the loaded module) instead of a caller's:
+ * the call allocates no device memory. Returns BINATTN_ERR_UNSUPPORTED when
+ * the shape needs more workspace than that (binattn_forward_workspace_bytes).
+ * The workspace is shared by every call in the process: calls that need it
+ * must not run concurrently (use one stream, or synchronise between them).
+ */
+int binattn_forward_static_ws(const uint32_t *q_bits, const uint32_t *k_bits,
+                              const float *alpha_q, const float *alpha_k,
+                              const uint16_t *bias, const uint16_t *v, float softmax_scale,
+                              int B, int H, int N, int d, uint16_t *out, void *stream);
+
 /* binattn_forward with an explicit score engine (binattn_engine). Returns
  * BINATTN_ERR_UNSUPPORTED when the engine cannot serve the shape. */
 int binattn_forward_engine(const uint32_t *q_bits, const uint32_t *k_bits,
