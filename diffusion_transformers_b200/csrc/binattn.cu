@@ -206,18 +206,24 @@ int binattn_forward(const uint32_t* q_bits, const uint32_t* k_bits, const float*
 }
 
 namespace {
-// Padded bias rows for the TMA-fed pipeline: the workspace holds [H][N][ld]
-// bf16, ld = N rounded up to a multiple of 8.
+// Workspace of binattn_forward_ws, for calls that run on the TMA-fed pipeline:
+//  [0, pad)          the bias with rows padded to ld = roundup(N, 8) elements,
+//                    when N % 8 != 0 (bias rows must be TMA rows);
+//  [pad, pad + part) partial results of the split tail pairs (tc2::split_plan).
+// pad is rounded up to 256 bytes.
 int padded_bias_ld(int N) { return (N + 7) / 8 * 8; }
-bool needs_padded_bias(int d, int N, bool has_bias) {
-  return has_bias && N % 8 != 0 && binattn::tc2::supported(d, N, true, false, padded_bias_ld(N));
+bool ws_path(int d, int N, bool has_bias) {
+  return binattn::tc2::supported(d, N, has_bias, false, has_bias ? padded_bias_ld(N) : 0);
+}
+size_t ws_pad_bytes(int H, int N, bool has_bias) {
+  if (!has_bias || N % 8 == 0) return 0;
+  return (static_cast<size_t>(H) * N * padded_bias_ld(N) * 2 + 255) / 256 * 256;
 }
 }  // namespace
 
 size_t binattn_forward_workspace_bytes(int B, int H, int N, int d, int has_bias) {
-  if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
-  if (!needs_padded_bias(d, N, has_bias != 0)) return 0;
-  return static_cast<size_t>(H) * N * padded_bias_ld(N) * 2;
+  if (B < 1 || H < 1 || N < 1 || d < 1 || !ws_path(d, N, has_bias != 0)) return 0;
+  return ws_pad_bytes(H, N, has_bias != 0) + binattn::tc2::split_part_bytes(B, H, N, d);
 }
 
 int binattn_forward_ws(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
@@ -226,24 +232,30 @@ int binattn_forward_ws(const uint32_t* q_bits, const uint32_t* k_bits, const flo
                        void* workspace, size_t workspace_bytes, void* stream) {
   if (int rc = check_forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out))
     return rc;
-  if (!needs_padded_bias(d, N, bias != nullptr))
+  const size_t need = binattn_forward_workspace_bytes(B, H, N, d, bias != nullptr);
+  if (need == 0)
     return binattn_forward_engine(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out,
                                   BINATTN_ENGINE_AUTO, stream);
-  const size_t need = binattn_forward_workspace_bytes(B, H, N, d, 1);
   BINATTN_CHECK_PTR(workspace);
-  if (!aligned16(workspace)) return fail(BINATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
   if (workspace_bytes < need)
     return fail(BINATTN_ERR_ARG, "workspace of %zu bytes is below the %zu this shape needs", workspace_bytes, need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int ld = padded_bias_ld(N);
-  uint16_t* padded = static_cast<uint16_t*>(workspace);
-  const long long rows = static_cast<long long>(H) * N;
-  const unsigned grid = static_cast<unsigned>((rows * ld + 255) / 256);
-  binattn::tc2::pad_bias_rows_kernel<<<grid, 256, 0, st>>>(bias, rows, N, ld, padded);
-  if (int rc = launch_status("pad_bias_rows_kernel")) return rc;
+  const size_t pad = ws_pad_bytes(H, N, bias != nullptr);
+  const uint16_t* fbias = bias;
+  int ld = 0;
+  if (pad) {
+    ld = padded_bias_ld(N);
+    uint16_t* padded = static_cast<uint16_t*>(workspace);
+    const long long rows = static_cast<long long>(H) * N;
+    const unsigned grid = static_cast<unsigned>((rows * ld + 255) / 256);
+    binattn::tc2::pad_bias_rows_kernel<<<grid, 256, 0, st>>>(bias, rows, N, ld, padded);
+    if (int rc = launch_status("pad_bias_rows_kernel")) return rc;
+    fbias = padded;
+  }
+  float* part = need > pad ? reinterpret_cast<float*>(static_cast<char*>(workspace) + pad) : nullptr;
   std::string msg;
-  int rc = binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, padded, v, softmax_scale, B, H, N, d, out, st,
-                                &msg, ld);
+  int rc = binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, fbias, v, softmax_scale, B, H, N, d, out, st,
+                                &msg, ld, part);
   if (rc) return fail(rc, "%s", msg.c_str());
   return ok();
 }

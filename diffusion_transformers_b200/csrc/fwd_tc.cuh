@@ -133,6 +133,12 @@ struct Params {
   float scale;
   int B, H, N, d;
   int bias_ld;  // elements between bias rows (N, or the padded row length); 0 means N
+  // 128-key-tile pipeline only: CTAs cover 256-row pairs pair_base + blockIdx.x
+  // (split == 0), or, with split == 1, CTA 2i + h covers key half h of pair
+  // pair_base + i and writes partial results to `part`.
+  int pair_base;
+  int split;
+  float* part;
 };
 
 // Named barrier 1 over the load-mode loader warps with an AND reduction.
@@ -922,7 +928,7 @@ inline int dispatch_kdim(const Params& prm, cudaStream_t st, std::string* msg) {
 inline int forward_tc(bool tc_qk, const uint32_t* qb, const uint32_t* kb, const float* aq,
                       const float* ak, const uint16_t* bias, const uint16_t* v, float scale,
                       int B, int H, int N, int d, uint16_t* out, cudaStream_t st, std::string* msg) {
-  tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d};
+  tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d, 0, 0, 0, nullptr};
   if (tc_qk)
     return bias ? tc::dispatch_kdim<tc::kQkTc, true, false>(prm, st, msg)
                 : tc::dispatch_kdim<tc::kQkTc, false, false>(prm, st, msg);
@@ -932,7 +938,8 @@ inline int forward_tc(bool tc_qk, const uint32_t* qb, const uint32_t* kb, const 
 
 inline int scores_tc(const uint32_t* qb, const uint32_t* kb, int B, int H, int N, int d, int32_t* S,
                      cudaStream_t st, std::string* msg) {
-  tc::Params prm{qb, kb, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S, 0.f, B, H, N, d};
+  tc::Params prm{qb,      kb,      nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S,
+                 0.f,     B,       H,       N,       d,       0,       0,       0,       nullptr};
   return tc::dispatch_kdim<tc::kQkTc, false, true>(prm, st, msg);
 }
 
@@ -941,7 +948,7 @@ inline int scores_tc(const uint32_t* qb, const uint32_t* kb, int B, int H, int N
 inline int forward_ref_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* bias,
                             const uint16_t* v, float scale, int B, int H, int N, int d, uint16_t* out,
                             cudaStream_t st, std::string* msg) {
-  tc::Params prm{nullptr, nullptr, q, k, nullptr, nullptr, bias, v, out, nullptr, scale, B, H, N, d};
+  tc::Params prm{nullptr, nullptr, q, k, nullptr, nullptr, bias, v, out, nullptr, scale, B, H, N, d, 0, 0, 0, nullptr};
   return bias ? tc::dispatch_kdim<tc::kQkRef, true, false>(prm, st, msg)
               : tc::dispatch_kdim<tc::kQkRef, false, false>(prm, st, msg);
 }

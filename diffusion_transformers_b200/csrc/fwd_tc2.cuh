@@ -207,15 +207,23 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Batch entries sharing a bias tile (same h and query tile) are adjacent in
   // launch order, so the bias tile is fetched from HBM once.
-  const int b = blockIdx.x % p.B;
-  const int qt = blockIdx.x / p.B;
-  const int h = blockIdx.y;
+  // 256-row pair of this CTA (b fastest, then the query tile, then h), and
+  // with split, which half of the key tiles it takes.
+  const int nq = (p.N + 2 * kRows - 1) / (2 * kRows);
+  const int pidx = p.pair_base + (p.split ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x));
+  const int half = p.split ? static_cast<int>(blockIdx.x & 1) : 0;
+  const int b = pidx % p.B;
+  const int qt = (pidx / p.B) % nq;
+  const int h = pidx / (p.B * nq);
   const int bh = b * p.H + h;
   const int N = p.N, d = p.d;
   const int W = (d + 31) / 32;                 // sign words per token (binary)
   const size_t tok0 = static_cast<size_t>(bh) * N;
   const int q0 = qt * 2 * kRows;
-  const int nkt = (N + kKeys - 1) / kKeys;
+  const int nkt_all = (N + kKeys - 1) / kKeys;
+  const int kt_begin = p.split && half ? nkt_all / 2 : 0;
+  const int nkt = p.split ? (half ? nkt_all - nkt_all / 2 : nkt_all / 2) : nkt_all;  // tiles of this CTA
+  const int key0 = kt_begin * kKeys;  // first key of this CTA
   const int dgroups = d / 8;                   // 8-channel groups written by TMA
   const int kq16 = (d + 15) / 16;              // reference QK^T MMAs (16 channels each)
 
@@ -317,7 +325,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
     if (lane == 0 && (!kDump || kBias)) {
       bool ok = true;
       for (int kt = 0; ok && kt < nkt; ++kt) {
-        const int j0 = kt * kKeys;
+        const int j0 = key0 + kt * kKeys;
         if constexpr (!kDump) {
           const int s = kt % kKS;
           if (kt >= kKS && !(ok = mbar_wait(&kv_empty[s], ((kt / kKS) - 1) & 1, abort))) break;
@@ -353,7 +361,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       auto load_tile = [&](int kt, TileRegs& tr) {
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          const int key = kt * kKeys + lane + 32 * u;
+          const int key = key0 + kt * kKeys + lane + 32 * u;
           const bool in = kt < nkt && key < N;
 #pragma unroll
           for (int w = 0; w < 3; ++w) tr.wd[u][w] = (in && w < W) ? __ldg(p.kb + (tok0 + key) * W + w) : 0u;
@@ -542,11 +550,11 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       }
       if constexpr (kDump) {
         if (ok && row_valid) {
-          int32_t* srow = p.S + (tok0 + row) * N + kt * kKeys;
+          int32_t* srow = p.S + (tok0 + row) * N + key0 + kt * kKeys;
 #pragma unroll
           for (int e = 0; e < kChunk; ++e) {
-            if (kt * kKeys + e < N) srow[e] = static_cast<int32_t>(__uint_as_float(xa[e]));
-            if (kt * kKeys + kChunk + e < N) srow[kChunk + e] = static_cast<int32_t>(__uint_as_float(xb[e]));
+            if (key0 + kt * kKeys + e < N) srow[e] = static_cast<int32_t>(__uint_as_float(xa[e]));
+            if (key0 + kt * kKeys + kChunk + e < N) srow[kChunk + e] = static_cast<int32_t>(__uint_as_float(xb[e]));
           }
         }
       } else {
@@ -557,11 +565,12 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
           logits(xb, 1, bsm, aks);
           float* x0 = reinterpret_cast<float*>(xa);
           float* x1 = reinterpret_cast<float*>(xb);
-          if (kt * kKeys + kKeys > N) {  // keys >= N take no part (warp-uniform branch)
+          const int jt = key0 + kt * kKeys;
+          if (jt + kKeys > N) {  // keys >= N take no part (warp-uniform branch)
 #pragma unroll
             for (int e = 0; e < kChunk; ++e) {
-              if (kt * kKeys + e >= N) x0[e] = -INFINITY;
-              if (kt * kKeys + kChunk + e >= N) x1[e] = -INFINITY;
+              if (jt + e >= N) x0[e] = -INFINITY;
+              if (jt + kChunk + e >= N) x1[e] = -INFINITY;
             }
           }
           // tile max: four independent 3-input max chains over both chunks
@@ -624,6 +633,27 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         uint32_t lbits;  // l = O_t column d
         asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(lbits) : "r"(o_col + d));
         tmem_ld_wait();
+        if (p.split) {
+          // Partial result of this key half: unnormalised O (d fp32), then m, then l.
+          // channel-major: value c of row r256 of (pair slot, half) at
+          // ((slot * 2 + half) * (d + 2) + c) * 256 + r256, so that a warp's 32
+          // rows store (and the combine kernel loads) 128 contiguous bytes
+          const int r256 = t * kRows + r;
+          float* dst = p.part + static_cast<size_t>((pidx - p.pair_base) * 2 + half) * (d + 2) * (2 * kRows) + r256;
+          for (int cc = 0; cc < d; cc += 8) {  // warp-uniform trip count: the loads are collective
+            uint32_t ov[8];
+            tmem_ld8(o_col + cc, ov);
+            tmem_ld_wait();
+            if (row_valid) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) dst[(cc + e) * (2 * kRows)] = __uint_as_float(ov[e]);
+            }
+          }
+          if (row_valid) {
+            dst[d * (2 * kRows)] = m;
+            dst[(d + 1) * (2 * kRows)] = __uint_as_float(lbits);
+          }
+        } else {
         const float inv = 1.f / __uint_as_float(lbits);
         uint16_t* orow = p.out + (tok0 + row) * d;
 #pragma unroll
@@ -646,6 +676,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
               }
             }
           }
+        }
         }
       }
     }
@@ -672,6 +703,39 @@ __global__ void __launch_bounds__(256) pad_bias_rows_kernel(const uint16_t* __re
   const long long row = e / ld;
   const int j = static_cast<int>(e - row * ld);
   out[e] = j < N ? bias[row * N + j] : static_cast<uint16_t>(0);
+}
+
+// Joins the two key halves of split pairs: for row i with partials (O_h, m_h,
+// l_h), M = max(m_0, m_1), w_h = exp(m_h - M), O = (w_0 O_0 + w_1 O_1) /
+// (w_0 l_0 + w_1 l_1), rounded to bf16. One thread per row of the split pairs.
+__global__ void __launch_bounds__(256) combine_halves_kernel(const float* __restrict__ part, int pair_base,
+                                                             int npairs, int B, int H, int N, int d,
+                                                             uint16_t* __restrict__ out) {
+  const int i = blockIdx.x * 256 + threadIdx.x;  // row of the split pairs
+  if (i >= npairs * 2 * kRows) return;
+  const int pidx = pair_base + i / (2 * kRows);
+  const int rr = i % (2 * kRows);
+  const int nq = (N + 2 * kRows - 1) / (2 * kRows);
+  const int b = pidx % B, qt = (pidx / B) % nq, h = pidx / (B * nq);
+  const int row = qt * 2 * kRows + rr;
+  if (row >= N) return;
+  // channel-major partials (see the split epilogue): value c of half h at p_h[c * 256]
+  constexpr int kS = 2 * kRows;
+  const float* p0 = part + static_cast<size_t>(i / kS) * 2 * (d + 2) * kS + rr;
+  const float* p1 = p0 + static_cast<size_t>(d + 2) * kS;
+  const float m0 = p0[d * kS], m1 = p1[d * kS];
+  const float M = fmaxf(m0, m1);
+  const float w0 = ex2((m0 - M) * kLog2e), w1 = ex2((m1 - M) * kLog2e);
+  const float inv = 1.f / (w0 * p0[(d + 1) * kS] + w1 * p1[(d + 1) * kS]);
+  uint16_t* orow = out + ((static_cast<size_t>(b) * H + h) * N + row) * d;
+  for (int c = 0; c < d; c += 8) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      w[e] = pack_bf16x2((w0 * p0[(c + 2 * e) * kS] + w1 * p1[(c + 2 * e) * kS]) * inv,
+                         (w0 * p0[(c + 2 * e + 1) * kS] + w1 * p1[(c + 2 * e + 1) * kS]) * inv);
+    *reinterpret_cast<uint4*>(orow + c) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
 }
 
 // ------------------------------------------------------------------- host
@@ -723,7 +787,7 @@ inline bool make_bias_map(CUtensorMap* tm, const uint16_t* bias, cuuint64_t H, c
 }
 
 template <int DV, int kMode, bool kBias>
-inline int launch(const tc::Params& prm, cudaStream_t st, std::string* msg) {
+inline int launch(const tc::Params& prm, int ctas, cudaStream_t st, std::string* msg) {
   CUtensorMap tm_v, tm_bias, tm_k;
   std::memset(&tm_v, 0, sizeof tm_v);
   std::memset(&tm_bias, 0, sizeof tm_bias);
@@ -745,8 +809,7 @@ inline int launch(const tc::Params& prm, cudaStream_t st, std::string* msg) {
     }
     configured = true;
   }
-  dim3 grid(static_cast<unsigned>(prm.B * ((prm.N + 2 * kRows - 1) / (2 * kRows))), prm.H);
-  kern<<<grid, kThreads, smem, st>>>(prm, tm_v, tm_bias, tm_k);
+  kern<<<static_cast<unsigned>(ctas), kThreads, smem, st>>>(prm, tm_v, tm_bias, tm_k);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     *msg = std::string("fwd_tc2_kernel launch: ") + cudaGetErrorString(e);
@@ -756,43 +819,101 @@ inline int launch(const tc::Params& prm, cudaStream_t st, std::string* msg) {
 }
 
 template <int kMode, bool kBias>
-inline int dispatch_dv(const tc::Params& prm, cudaStream_t st, std::string* msg) {
+inline int dispatch_dv(const tc::Params& prm, int ctas, cudaStream_t st, std::string* msg) {
   switch (dv_for(prm.d)) {
-    case 32: return launch<32, kMode, kBias>(prm, st, msg);
-    case 64: return launch<64, kMode, kBias>(prm, st, msg);
-    case 80: return launch<80, kMode, kBias>(prm, st, msg);
+    case 32: return launch<32, kMode, kBias>(prm, ctas, st, msg);
+    case 64: return launch<64, kMode, kBias>(prm, ctas, st, msg);
+    case 80: return launch<80, kMode, kBias>(prm, ctas, st, msg);
     default:
       if constexpr (kMode == kModeRef) {
         *msg = "reference attention on the 128-key pipeline needs d <= 72";
         return BINATTN_ERR_UNSUPPORTED;
       } else {
-        return launch<96, kMode, kBias>(prm, st, msg);
+        return launch<96, kMode, kBias>(prm, ctas, st, msg);
       }
   }
 }
 
+// 256-row pairs of a call (one CTA each without a split).
+inline int total_pairs(int B, int H, int N) { return B * H * ((N + 2 * kRows - 1) / (2 * kRows)); }
+
+// Tail split: with P pairs on S SMs, the first floor(P / S) * S pairs run as
+// whole CTAs; when that is at least one wave, the remaining R pairs fill at
+// most one wave twice over (2R <= S) and there are at least 32 key tiles (a
+// measured threshold: with 16 or fewer the split costs more than it saves), each
+// of the R pairs runs as two CTAs that take one half of the key tiles each,
+// and a combine kernel joins the halves. Without a device to ask, no split.
+struct SplitPlan {
+  int full, tail;
+};
+inline SplitPlan split_plan(int B, int H, int N) {
+  const int P = total_pairs(B, H, N);
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      nsm <= 0) {
+    cudaGetLastError();
+    return {P, 0};
+  }
+  const int full = P / nsm * nsm, tail = P - full;
+  // worth it only behind at least one whole wave and with enough key tiles
+  // that half of them outweighs the extra launch and the combine
+  if (full == 0 || tail == 0 || 2 * tail > nsm || (N + kKeys - 1) / kKeys < 32) return {P, 0};
+  return {full, tail};
+}
+// Bytes of the partial results of the split pairs (fp32 O, m, l per row and half).
+inline size_t split_part_bytes(int B, int H, int N, int d) {
+  const SplitPlan pl = split_plan(B, H, N);
+  return static_cast<size_t>(pl.tail) * 2 * kRows * 2 * (d + 2) * 4;
+}
+
 }  // namespace tc2
 
+// part: workspace for the tail split (tc2::split_part_bytes), or null for no split.
 inline int forward_tc2(const uint32_t* qb, const uint32_t* kb, const float* aq, const float* ak,
                        const uint16_t* bias, const uint16_t* v, float scale, int B, int H, int N, int d,
-                       uint16_t* out, cudaStream_t st, std::string* msg, int bias_ld = 0) {
-  tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d, bias_ld};
-  return bias ? tc2::dispatch_dv<tc2::kModeBin, true>(prm, st, msg)
-              : tc2::dispatch_dv<tc2::kModeBin, false>(prm, st, msg);
+                       uint16_t* out, cudaStream_t st, std::string* msg, int bias_ld = 0,
+                       float* part = nullptr) {
+  tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d, bias_ld, 0, 0,
+                 nullptr};
+  const tc2::SplitPlan plan = part ? tc2::split_plan(B, H, N) : tc2::SplitPlan{tc2::total_pairs(B, H, N), 0};
+  auto run = [&](int ctas) {
+    return bias ? tc2::dispatch_dv<tc2::kModeBin, true>(prm, ctas, st, msg)
+                : tc2::dispatch_dv<tc2::kModeBin, false>(prm, ctas, st, msg);
+  };
+  if (plan.full > 0) {
+    if (int rc = run(plan.full)) return rc;
+  }
+  if (plan.tail > 0) {
+    prm.pair_base = plan.full;
+    prm.split = 1;
+    prm.part = part;
+    if (int rc = run(2 * plan.tail)) return rc;
+    const int rows = plan.tail * 2 * tc2::kRows;
+    tc2::combine_halves_kernel<<<(rows + 255) / 256, 256, 0, st>>>(part, plan.full, plan.tail, B, H, N, d, out);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      *msg = std::string("combine_halves_kernel launch: ") + cudaGetErrorString(e);
+      return BINATTN_ERR_CUDA;
+    }
+  }
+  return BINATTN_OK;
 }
 
 inline int scores_tc2(const uint32_t* qb, const uint32_t* kb, int B, int H, int N, int d, int32_t* S,
                       cudaStream_t st, std::string* msg) {
-  tc::Params prm{qb, kb, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S, 0.f, B, H, N, d};
-  return tc2::launch<32, tc2::kModeDump, false>(prm, st, msg);
+  tc::Params prm{qb, kb, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S, 0.f, B, H, N, d, 0, 0, 0,
+                 nullptr};
+  return tc2::launch<32, tc2::kModeDump, false>(prm, tc2::total_pairs(B, H, N), st, msg);
 }
 
 inline int forward_ref_tc2(const uint16_t* q, const uint16_t* k, const uint16_t* bias, const uint16_t* v,
                            float scale, int B, int H, int N, int d, uint16_t* out, cudaStream_t st,
                            std::string* msg) {
-  tc::Params prm{nullptr, nullptr, q, k, nullptr, nullptr, bias, v, out, nullptr, scale, B, H, N, d};
-  return bias ? tc2::dispatch_dv<tc2::kModeRef, true>(prm, st, msg)
-              : tc2::dispatch_dv<tc2::kModeRef, false>(prm, st, msg);
+  tc::Params prm{nullptr, nullptr, q, k, nullptr, nullptr, bias, v, out, nullptr, scale, B, H, N, d, 0, 0, 0,
+                 nullptr};
+  const int ctas = tc2::total_pairs(B, H, N);
+  return bias ? tc2::dispatch_dv<tc2::kModeRef, true>(prm, ctas, st, msg)
+              : tc2::dispatch_dv<tc2::kModeRef, false>(prm, ctas, st, msg);
 }
 
 }  // namespace binattn

@@ -128,18 +128,25 @@ int binattn_forward(const uint32_t *q_bits, const uint32_t *k_bits,
 
 /*
  * binattn_forward_workspace_bytes — device workspace that binattn_forward_ws
- * needs for this shape: 0 when binattn_forward already takes the TMA-fed
- * pipeline, else H * N * roundup(N, 8) * 2 bytes (a bias whose rows are not a
- * multiple of 8 elements, with 8 <= d <= 80 and d % 8 == 0). Never fails.
+ * needs for this shape on the current device; 0 when binattn_forward_ws would
+ * simply run binattn_forward. For the TMA-fed pipeline (d % 8 == 0, d <= 80)
+ * it holds (a) a copy of the bias with rows padded to roundup(N, 8) elements
+ * when N % 8 != 0 (H * N * roundup(N, 8) * 2 bytes, rounded up to 256), and
+ * (b) when the 256-row pairs of the call leave a last wave at most half full
+ * of the device's SMs, fp32 partial results of those R pairs, whose key tiles
+ * are then split over two CTAs each (R * 512 * 2 * (d + 2) * 4 bytes). Never
+ * fails; a call with no CUDA device to query gets no part (b).
  */
 size_t binattn_forward_workspace_bytes(int B, int H, int N, int d, int has_bias);
 
 /*
  * binattn_forward_ws — binattn_forward (engine AUTO) with a caller-owned
- * device workspace, for biases whose row length N is not a multiple of 8: the
- * bias is first copied into the workspace with each row padded to
- * roundup(N, 8) elements (pad 0), so that its rows are TMA rows, and the
- * forward then runs on the TMA-fed pipeline. Same result as binattn_forward.
+ * device workspace of binattn_forward_workspace_bytes(...) bytes: biases with
+ * N % 8 != 0 run on the TMA-fed pipeline from a padded copy, and a short last
+ * wave of row pairs is split by key halves (each half writes unnormalised O,
+ * its row max m and row sum l; a combine kernel joins them: O = (w0 O0 +
+ * w1 O1) / (w0 l0 + w1 l1), w_h = exp(m_h - max(m0, m1))). Same result as
+ * binattn_forward up to fp32 rounding.
  *   workspace        device, 16-byte aligned, at least
  *                    binattn_forward_workspace_bytes(...) bytes, overwritten;
  *                    may be NULL when that size is 0.

@@ -94,13 +94,29 @@ def test_last_error_message_is_specific(L):
     assert b"v is not 16-byte aligned" in L.binattn_last_error_message()
 
 
+def _expected_ws(B, H, N, d, has_bias):
+    """Padded bias (rounded to 256 bytes) + split-tail partials (only with a device to ask)."""
+    pad = 0
+    if has_bias and N % 8:
+        pad = -(-H * N * (-(-N // 8) * 8) * 2 // 256) * 256
+    split = 0
+    import torch
+    if torch.cuda.is_available():
+        nsm = torch.cuda.get_device_properties(0).multi_processor_count
+        P = B * H * (-(-N // 256))
+        tail = P - P // nsm * nsm
+        if P // nsm and tail and 2 * tail <= nsm and -(-N // 64) >= 32:
+            split = tail * 512 * 2 * (d + 2) * 4
+    return pad + split
+
+
 def test_workspace_bytes(L):
     # a bias whose rows are not a multiple of 8 elements: [H][N][roundup(N, 8)] bf16
-    assert L.binattn_forward_workspace_bytes(64, 12, 197, 64, 1) == 12 * 197 * 200 * 2
-    assert L.binattn_forward_workspace_bytes(32, 16, 577, 64, 1) == 16 * 577 * 584 * 2
-    # rows already TMA rows, no bias, or a shape the TMA-fed pipeline does not take
-    assert L.binattn_forward_workspace_bytes(2, 16, 4096, 72, 1) == 0
-    assert L.binattn_forward_workspace_bytes(64, 12, 197, 64, 0) == 0
+    for shape in [(64, 12, 197, 64), (32, 16, 577, 64), (2, 16, 4096, 72), (1, 2, 300, 8)]:
+        assert L.binattn_forward_workspace_bytes(*shape, 1) == _expected_ws(*shape, True), shape
+    assert L.binattn_forward_workspace_bytes(64, 12, 197, 64, 1) >= 12 * 197 * 200 * 2
+    # no bias, or a shape the TMA-fed pipeline does not take
+    assert L.binattn_forward_workspace_bytes(64, 12, 197, 64, 0) == _expected_ws(64, 12, 197, 64, False)
     assert L.binattn_forward_workspace_bytes(1, 1, 197, 128, 1) == 0
     assert L.binattn_forward_workspace_bytes(1, 1, 197, 33, 1) == 0
     assert L.binattn_forward_workspace_bytes(0, 1, 197, 64, 1) == 0

@@ -154,9 +154,11 @@ def test_device_errors_are_reported():
     binattn.device_status()
 
 
-# ------------------------------------------- forward with a workspace (padded bias rows)
+# ------------------------------------------- forward with a workspace
 # Bias rows of N % 8 != 0 elements are not TMA rows; binattn_forward_ws pads
-# them into the workspace and runs the TMA-fed pipeline. Same bar as forward.
+# them into the workspace and runs the TMA-fed pipeline, and splits a short
+# last wave of row pairs by key halves (partials joined by a combine kernel).
+# Same bar as forward.
 WS_SHAPES = [(2, 3, 129, 72), (1, 2, 197, 64), (1, 1, 130, 72), (2, 2, 65, 16), (1, 1, 1, 64),
              (1, 3, 1001, 40), (1, 2, 300, 8)]
 
@@ -181,7 +183,8 @@ def test_forward_ws_small(orc, shape):
     c = make_custom(B, H, N, d, seed=5 * N + d, with_bias=True, bias_std=0.5)
     ref = orc.forward(c["q"], c["k"], c["bias"], c["v"], c["softmax_scale"])
     out, need = _run_ws(c)
-    assert need == (H * N * ((N + 7) // 8 * 8) * 2 if N % 8 else 0)
+    if N % 8:
+        assert need >= H * N * ((N + 7) // 8 * 8) * 2
     check_o(bf16_to_f64(out), ref, f"ws {shape}")
 
 
@@ -195,3 +198,30 @@ def test_forward_ws_full_size_sampled(orc, name):
     assert need > 0
     got = out.view(B * H * N, d)[torch.from_numpy(rows).cuda()]
     check_o(bf16_to_f64(got), ref, f"ws {name}")
+
+
+# Shapes whose 256-row pairs leave a short last wave behind at least one full
+# wave, with >= 32 key tiles: the tail pairs run split by key halves. Checked on
+# every row of the split pairs (the last pairs in launch order) plus random rows.
+SPLIT_SHAPES = [(1, 19, 2048, 72, True), (2, 10, 2100, 40, False)]
+
+
+@pytest.mark.parametrize("shape", SPLIT_SHAPES)
+def test_forward_ws_split_tail(orc, shape):
+    B, H, N, d, with_bias = shape
+    c = make_custom(B, H, N, d, seed=7 * N + d, with_bias=with_bias, bias_std=0.5)
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    nq = (N + 255) // 256
+    pairs = B * H * nq
+    tail = pairs % nsm
+    assert pairs // nsm and tail and 2 * tail <= nsm  # the split runs
+    rows = []
+    for pidx in range(pairs - tail, pairs):  # pair -> (b, query tile, h), b fastest
+        b, qt, h = pidx % B, (pidx // B) % nq, pidx // (B * nq)
+        rows += [(b * H + h) * N + i for i in range(qt * 256, min(N, qt * 256 + 256))]
+    rows = np.unique(np.concatenate([np.array(rows, dtype=np.int64), sample_rows(B, H, N, 64, seed=3)]))
+    ref = orc.forward_rows(c["q"], c["k"], c["bias"] if with_bias else None, c["v"], c["softmax_scale"], rows)
+    out, need = _run_ws(c, with_bias=with_bias)
+    assert need > 0
+    got = out.view(B * H * N, d)[torch.from_numpy(rows).cuda()]
+    check_o(bf16_to_f64(got), ref, f"split {shape}")
