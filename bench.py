@@ -83,13 +83,15 @@ def algorithmic(w, with_bias=True):
                 eff_flops=4 * d * pairs, bytes=bytes_, pack_bytes=pack_bytes)
 
 
-# DRAM traffic of the forward kernel from one ncu capture (dram__bytes_read.sum
-# + dram__bytes_write.sum, one launch at dit_xl_1024 with bias; the summary is
-# profiles/fwd_tc2_dit_xl_1024_bias.md), valid only for the kernel sources it was
-# taken on: any change to them turns the reported traffic back into null.
+# DRAM traffic of one forward call from one ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum summed over the launches the call makes at dit_xl_1024
+# with bias: the full-wave launch, the key-split tail launch and the combine; the
+# summary is profiles/fwd_tc2_dit_xl_1024_bias.md), valid only for the kernel
+# sources it was taken on: any change to them turns the reported traffic back
+# into null.
 NCU_TRAFFIC = {
-    "sources_sha256": "ac3fb190eda82e7c0f4d67b20ac258f7b5f48cbd3adc475554d5e18470648457",
-    "bytes_per_launch": {"dit_xl_1024/bias": 584_370_432},
+    "sources_sha256": "3458a310fa957c45a925d761ca55f1ae84acd8dfc0160ffac7f1b9444b69e2ca",
+    "bytes_per_call": {"dit_xl_1024/bias": 591_615_232},
 }
 
 
@@ -109,7 +111,7 @@ def kernel_sources_digest():
 def ncu_traffic(key):
     if kernel_sources_digest() != NCU_TRAFFIC["sources_sha256"]:
         return None
-    return NCU_TRAFFIC["bytes_per_launch"].get(key)
+    return NCU_TRAFFIC["bytes_per_call"].get(key)
 
 
 def measured_peaks():
@@ -515,7 +517,8 @@ def run_gpu(args, w, rank, world, local_rank):
         "other_workloads": others,
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
                      "frac": round(achieved / peak, 4),
-                     "traffic": ncu_traffic(f"{w.name}/bias"), "traffic_unit": "bytes per launch",
+                     "traffic": ncu_traffic(f"{w.name}/bias"),
+                     "traffic_unit": "bytes per forward call (its 3 launches)",
                      "algorithmic_bytes": a["bytes"],
                      "kernel": "binattn forward (with bias)",
                      "peak_source": peaks["source"] + " (burst)",
