@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "binattn.h"
@@ -261,12 +262,40 @@ int binattn_forward_ws(const uint32_t* q_bits, const uint32_t* k_bits, const flo
 }
 
 namespace {
-// Static workspace of binattn_forward_static_ws: part of the loaded module, so
-// the call itself allocates no device memory.
+// Scratch of binattn_forward_static_ws: a file-scope device array, so the call
+// needs no allocation. Every device that loads the library holds it until the
+// process exits. Host code cannot pass the array's name to a kernel (on the
+// host it names a stand-in, not device memory): the device address is looked
+// up once per device, with that device current, and kept in g_static_addr.
 constexpr size_t kStaticWorkspaceBytes = size_t(32) << 20;
 __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+constexpr int kStaticMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_addr[kStaticMaxDevices];  // null until the device's first call
+
+// Device address of g_static_workspace on the current device.
+int static_workspace_addr(void** addr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(BINATTN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kStaticMaxDevices)
+    return fail(BINATTN_ERR_UNSUPPORTED, "device %d is beyond the %d the static workspace tracks", dev,
+                kStaticMaxDevices);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess) return fail(BINATTN_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    g_static_addr[dev] = p;
+  }
+  *addr = g_static_addr[dev];
+  return BINATTN_OK;
+}
 }  // namespace
 
+// Nothing in the workspace has to start at zero: every byte a call reads from
+// it (the padded bias copy, the partials of split pairs) is written earlier in
+// the same call, so the previous call's contents never leak into a result.
 int binattn_forward_static_ws(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
                               const float* alpha_k, const uint16_t* bias, const uint16_t* v,
                               float softmax_scale, int B, int H, int N, int d, uint16_t* out,
@@ -278,12 +307,9 @@ int binattn_forward_static_ws(const uint32_t* q_bits, const uint32_t* k_bits, co
     return fail(BINATTN_ERR_UNSUPPORTED, "this shape needs %zu bytes of workspace; the static one holds %zu",
                 need, kStaticWorkspaceBytes);
   void* ws = nullptr;
-  if (need) {
-    cudaError_t e = cudaGetSymbolAddress(&ws, g_static_workspace);
-    if (e != cudaSuccess) return fail(BINATTN_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
-  }
+  if (int rc = static_workspace_addr(&ws)) return rc;
   return binattn_forward_ws(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out, ws,
-                            need ? kStaticWorkspaceBytes : 0, stream);
+                            kStaticWorkspaceBytes, stream);
 }
 
 int binattn_scores_debug(const uint32_t* q_bits, const uint32_t* k_bits, int B, int H, int N,

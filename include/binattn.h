@@ -162,12 +162,30 @@ int binattn_forward_ws(const uint32_t *q_bits, const uint32_t *k_bits,
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * binattn_forward_static_ws — binattn_forward_ws with the library's own static
- * device workspace (32 MiB, part of the loaded module) instead of a caller's:
- * the call allocates no device memory. Returns BINATTN_ERR_UNSUPPORTED when
- * the shape needs more workspace than that (binattn_forward_workspace_bytes).
- * The workspace is shared by every call in the process: calls that need it
- * must not run concurrently (use one stream, or synchronise between them).
+ * binattn_forward_static_ws — binattn_forward_ws for callers that cannot
+ * allocate device memory: a plug-in or hook that is handed its buffers by a
+ * host framework whose caching allocator owns the device's memory, or a
+ * latency-bound loop where a cudaMalloc, which can synchronise the device,
+ * is not allowed. The paper has no counterpart of this call; it is a
+ * convenience of this library.
+ *
+ * The scratch is a file-scope __device__ array of 32 MiB (256-byte aligned)
+ * inside the library, which every GPU that loads the library holds until the
+ * process exits. The caller still passes every input and the output, as for
+ * binattn_forward_ws. The call allocates and frees nothing, through CUDA or
+ * any library.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ *    first call before any stream capture that includes this call.
+ *  - Shapes whose binattn_forward_workspace_bytes exceeds 32 MiB return
+ *    BINATTN_ERR_UNSUPPORTED before anything is launched (for example a bias
+ *    with N % 8 != 0 and H * N * roundup(N, 8) * 2 > 32 MiB).
+ *  - Every call in the process shares the one array, which keeps the last
+ *    call's contents. Nothing in it needs to start at zero (each call writes
+ *    what it reads), but calls whose kernels overlap on the GPU (other
+ *    streams, other host threads) race on it and corrupt each other's
+ *    results: serialise them (one stream, or synchronise between calls).
+ * Other errors are those of binattn_forward_ws.
  */
 int binattn_forward_static_ws(const uint32_t *q_bits, const uint32_t *k_bits,
                               const float *alpha_q, const float *alpha_k,
