@@ -15,6 +15,7 @@
 #include "fwd_simt.cuh"
 #include "fwd_tc.cuh"
 #include "fwd_tc2.cuh"
+#include "fwd_tc3.cuh"
 
 namespace {
 
@@ -185,12 +186,19 @@ int binattn_forward_engine(const uint32_t* q_bits, const uint32_t* k_bits, const
       if (!binattn::tc_supported(d))
         return fail(BINATTN_ERR_UNSUPPORTED, "engine %d needs d %% 8 == 0 (d = %d)", engine, d);
       std::string msg;
-      // TC: the 128-key e4m3 pipeline where it applies, else the 64-key one
-      int rc = engine == BINATTN_ENGINE_TC && binattn::tc2::supported(d, N, bias != nullptr, false)
-                   ? binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N,
-                                          d, out, st, &msg)
-                   : binattn::forward_tc(engine == BINATTN_ENGINE_TC, q_bits, k_bits, alpha_q, alpha_k, bias,
-                                         v, softmax_scale, B, H, N, d, out, st, &msg);
+      // TC: e4m3 +-1 operands where the shape allows, on the pipeline that
+      // measured fastest for it (128-key tiles without a bias, 64-key tiles
+      // with one); other shapes use bf16 +-1 operands
+      int rc;
+      if (engine == BINATTN_ENGINE_TC && !bias && binattn::tc3::supported(d, N, false))
+        rc = binattn::forward_tc3(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out, st,
+                                  &msg);
+      else if (engine == BINATTN_ENGINE_TC && binattn::tc2::supported(d, N, bias != nullptr, false))
+        rc = binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out, st,
+                                  &msg);
+      else
+        rc = binattn::forward_tc(engine == BINATTN_ENGINE_TC, q_bits, k_bits, alpha_q, alpha_k, bias, v,
+                                 softmax_scale, B, H, N, d, out, st, &msg);
       if (rc) return fail(rc, "%s", msg.c_str());
       return ok();
     }
@@ -214,7 +222,7 @@ namespace {
 // pad is rounded up to 256 bytes.
 int padded_bias_ld(int N) { return (N + 7) / 8 * 8; }
 bool ws_path(int d, int N, bool has_bias) {
-  return binattn::tc2::supported(d, N, has_bias, false, has_bias ? padded_bias_ld(N) : 0);
+  return binattn::tc3::supported(d, N, has_bias, has_bias ? padded_bias_ld(N) : 0);
 }
 size_t ws_pad_bytes(int H, int N, bool has_bias) {
   if (!has_bias || N % 8 == 0) return 0;
@@ -255,8 +263,10 @@ int binattn_forward_ws(const uint32_t* q_bits, const uint32_t* k_bits, const flo
   }
   float* part = need > pad ? reinterpret_cast<float*>(static_cast<char*>(workspace) + pad) : nullptr;
   std::string msg;
-  int rc = binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, fbias, v, softmax_scale, B, H, N, d, out, st,
-                                &msg, ld, part);
+  int rc = fbias ? binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, fbias, v, softmax_scale, B, H, N, d,
+                                        out, st, &msg, ld, part)
+                 : binattn::forward_tc3(q_bits, k_bits, alpha_q, alpha_k, fbias, v, softmax_scale, B, H, N, d,
+                                        out, st, &msg, ld, part);
   if (rc) return fail(rc, "%s", msg.c_str());
   return ok();
 }
