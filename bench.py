@@ -437,6 +437,35 @@ def run_gpu(args, w, rank, world, local_rank):
     clocks = sampler.stop()
     binattn.device_status(stream)
 
+    # the same step with Q binarised inside the forward (binattn_forward_fused_ws):
+    # pack(K) + the fused forward; its own timed region, same protocol
+    fused = {}
+    if args.engine == "auto":
+        for name, b in (("bias", bias), ("no_bias", None)):
+            need = binattn.fused_workspace_bytes(B, H, N, d, q.dtype, b is not None)
+            fws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+
+            def fstep():
+                binattn.pack(k, kb, ak, stream)
+                binattn.forward_fused_ws(q, kb, ak, b, v, scale, workspace=fws, out=out, stream=stream)
+
+            fstep()
+            torch.cuda.synchronize()
+            barrier()
+            ev = []
+            for _ in range(args.steps):
+                flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fstep()
+                e1.record(stream)
+                ev.append((e0, e1))
+            torch.cuda.synchronize()
+            barrier()
+            fused[name] = {"ms_per_step": round(max_over_ranks(sum(a.elapsed_time(c) for a, c in ev) / len(ev)), 5)}
+            del fws
+        binattn.device_status(stream)
+
     # in-build bf16 attention on the same shapes (speed reference)
     ref = None
     try:
@@ -510,6 +539,7 @@ def run_gpu(args, w, rank, world, local_rank):
         "pack_ms": round(results["bias"]["step_ms"] - results["bias"]["fwd_ms"], 5),
         "effective_tflops": round(eff_tflops, 2),
         "job_effective_tflops": round(job_units(a["eff_flops"], world) / fwd_s / 1e12, 2),
+        "fused_q_step": dict(fused, step="pack(K) + binattn_forward_fused_ws (Q binarised in the forward)"),
         "no_bias": {"ms_per_step": round(results["no_bias"]["step_ms"], 5),
                     "forward_ms": round(results["no_bias"]["fwd_ms"], 5),
                     "effective_tflops": round(a0["eff_flops"] / fwd0_s / 1e12, 2)},

@@ -21,7 +21,8 @@ ENGINES = {"auto": ENGINE_AUTO, "simt": ENGINE_SIMT, "popc_tc": ENGINE_POPC_TC, 
 # Every symbol include/binattn.h declares.
 EXPORTS = (
     "binattn_pack", "binattn_forward", "binattn_forward_engine", "binattn_forward_workspace_bytes",
-    "binattn_forward_ws", "binattn_forward_static_ws", "binattn_scores_debug",
+    "binattn_forward_ws", "binattn_forward_static_ws", "binattn_forward_fused_workspace_bytes",
+    "binattn_forward_fused_ws", "binattn_scores_debug",
     "binattn_ref_bf16_forward", "binattn_device_status", "binattn_strerror",
     "binattn_last_error_message", "binattn_abi_version",
 )
@@ -57,6 +58,9 @@ def lib() -> ctypes.CDLL:
     L.binattn_forward_workspace_bytes.restype = ctypes.c_size_t
     L.binattn_forward_ws.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
     L.binattn_forward_static_ws.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, P]
+    L.binattn_forward_fused_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    L.binattn_forward_fused_workspace_bytes.restype = ctypes.c_size_t
+    L.binattn_forward_fused_ws.argtypes = [P, I, P, P, P, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
     L.binattn_scores_debug.argtypes = [P, P, I, I, I, I, P, I, P]
     L.binattn_ref_bf16_forward.argtypes = [P, P, P, P, F, I, I, I, I, P, P]
     L.binattn_device_status.argtypes = [P]
@@ -64,7 +68,7 @@ def lib() -> ctypes.CDLL:
     L.binattn_strerror.restype = ctypes.c_char_p
     L.binattn_last_error_message.restype = ctypes.c_char_p
     for name in ("binattn_pack", "binattn_forward", "binattn_forward_engine", "binattn_forward_ws",
-                 "binattn_forward_static_ws",
+                 "binattn_forward_static_ws", "binattn_forward_fused_ws",
                  "binattn_scores_debug",
                  "binattn_ref_bf16_forward", "binattn_device_status", "binattn_abi_version"):
         getattr(L, name).restype = I
@@ -179,6 +183,34 @@ def forward_static_ws(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch
     _check(lib().binattn_forward_static_ws(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k), _ptr(bias),
                                            _ptr(v), float(softmax_scale), B, H, N, d, _ptr(out), _stream(stream)),
            "binattn_forward_static_ws")
+    return out
+
+
+def fused_workspace_bytes(B: int, H: int, N: int, d: int, q_dtype: torch.dtype, has_bias: bool) -> int:
+    """Device workspace bytes forward_fused_ws needs."""
+    dt = {torch.float32: F32, torch.bfloat16: BF16}[q_dtype]
+    return int(lib().binattn_forward_fused_workspace_bytes(B, H, N, d, dt, int(bool(has_bias))))
+
+
+def forward_fused_ws(q: torch.Tensor, k_bits: torch.Tensor, alpha_k: torch.Tensor, bias: torch.Tensor | None,
+                     v: torch.Tensor, softmax_scale: float, workspace: torch.Tensor | None = None,
+                     out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """pack(Q) + forward_ws in one call; the forward kernel binarises bf16 Q itself
+    where the shape allows (same result as pack followed by forward_ws)."""
+    B, H, N, d = v.shape
+    dt = {torch.float32: F32, torch.bfloat16: BF16}.get(q.dtype)
+    if dt is None:
+        raise TypeError(f"q must be float32 or bfloat16, got {q.dtype}")
+    need = fused_workspace_bytes(B, H, N, d, q.dtype, bias is not None)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=v.device)
+    size = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().binattn_forward_fused_ws(_ptr(q), dt, _ptr(k_bits), _ptr(alpha_k), _ptr(bias), _ptr(v),
+                                          float(softmax_scale), B, H, N, d, _ptr(out), _ptr(workspace),
+                                          ctypes.c_size_t(size), _stream(stream)),
+           "binattn_forward_fused_ws")
     return out
 
 

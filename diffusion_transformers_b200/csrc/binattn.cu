@@ -235,20 +235,13 @@ size_t binattn_forward_workspace_bytes(int B, int H, int N, int d, int has_bias)
   return ws_pad_bytes(H, N, has_bias != 0) + binattn::tc2::split_part_bytes(B, H, N, d);
 }
 
-int binattn_forward_ws(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
-                       const float* alpha_k, const uint16_t* bias, const uint16_t* v,
-                       float softmax_scale, int B, int H, int N, int d, uint16_t* out,
-                       void* workspace, size_t workspace_bytes, void* stream) {
-  if (int rc = check_forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out))
-    return rc;
-  const size_t need = binattn_forward_workspace_bytes(B, H, N, d, bias != nullptr);
-  if (need == 0)
-    return binattn_forward_engine(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out,
-                                  BINATTN_ENGINE_AUTO, stream);
-  BINATTN_CHECK_PTR(workspace);
-  if (workspace_bytes < need)
-    return fail(BINATTN_ERR_ARG, "workspace of %zu bytes is below the %zu this shape needs", workspace_bytes, need);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+namespace {
+// The TMA-fed forward with a workspace (ws_path(d, N, bias) holds): bias rows
+// padded into the workspace when N % 8 != 0, a short last wave split by key
+// halves, and with qh set, Q binarised inside the kernel.
+int forward_tma_ws(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q, const float* alpha_k,
+                   const uint16_t* bias, const uint16_t* v, float softmax_scale, int B, int H, int N, int d,
+                   uint16_t* out, void* workspace, size_t need, const uint16_t* qh, cudaStream_t st) {
   const size_t pad = ws_pad_bytes(H, N, bias != nullptr);
   const uint16_t* fbias = bias;
   int ld = 0;
@@ -264,11 +257,73 @@ int binattn_forward_ws(const uint32_t* q_bits, const uint32_t* k_bits, const flo
   float* part = need > pad ? reinterpret_cast<float*>(static_cast<char*>(workspace) + pad) : nullptr;
   std::string msg;
   int rc = fbias ? binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, fbias, v, softmax_scale, B, H, N, d,
-                                        out, st, &msg, ld, part)
+                                        out, st, &msg, ld, part, qh)
                  : binattn::forward_tc3(q_bits, k_bits, alpha_q, alpha_k, fbias, v, softmax_scale, B, H, N, d,
-                                        out, st, &msg, ld, part);
+                                        out, st, &msg, ld, part, qh);
   if (rc) return fail(rc, "%s", msg.c_str());
   return ok();
+}
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Whether binattn_forward_fused_ws binarises Q inside the forward kernel.
+bool fused_path(int q_dtype, int d, int N, bool has_bias) { return q_dtype == BINATTN_BF16 && ws_path(d, N, has_bias); }
+}  // namespace
+
+int binattn_forward_ws(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
+                       const float* alpha_k, const uint16_t* bias, const uint16_t* v,
+                       float softmax_scale, int B, int H, int N, int d, uint16_t* out,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (int rc = check_forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out))
+    return rc;
+  const size_t need = binattn_forward_workspace_bytes(B, H, N, d, bias != nullptr);
+  if (need == 0)
+    return binattn_forward_engine(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out,
+                                  BINATTN_ENGINE_AUTO, stream);
+  BINATTN_CHECK_PTR(workspace);
+  if (workspace_bytes < need)
+    return fail(BINATTN_ERR_ARG, "workspace of %zu bytes is below the %zu this shape needs", workspace_bytes, need);
+  return forward_tma_ws(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out, workspace, need,
+                        nullptr, static_cast<cudaStream_t>(stream));
+}
+
+size_t binattn_forward_fused_workspace_bytes(int B, int H, int N, int d, int q_dtype, int has_bias) {
+  if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
+  const size_t fw = binattn_forward_workspace_bytes(B, H, N, d, has_bias);
+  if (fused_path(q_dtype, d, N, has_bias != 0)) return fw;
+  const size_t tokens = static_cast<size_t>(B) * H * N;
+  return round256(fw) + round256(tokens * binattn::words_for(d) * 4) + round256(tokens * 4);
+}
+
+int binattn_forward_fused_ws(const void* q, int q_dtype, const uint32_t* k_bits, const float* alpha_k,
+                             const uint16_t* bias, const uint16_t* v, float softmax_scale, int B, int H, int N,
+                             int d, uint16_t* out, void* workspace, size_t workspace_bytes, void* stream) {
+  BINATTN_CHECK_PTR(q);
+  if (q_dtype != BINATTN_F32 && q_dtype != BINATTN_BF16)
+    return fail(BINATTN_ERR_DTYPE, "q_dtype %d is neither BINATTN_F32 nor BINATTN_BF16", q_dtype);
+  // k_bits stands in for the absent q_bits / alpha_q in the common checks
+  if (int rc = check_forward_args(k_bits, k_bits, alpha_k, alpha_k, bias, v, softmax_scale, B, H, N, d, out))
+    return rc;
+  const size_t need = binattn_forward_fused_workspace_bytes(B, H, N, d, q_dtype, bias != nullptr);
+  if (need) {
+    BINATTN_CHECK_PTR(workspace);
+    if (workspace_bytes < need)
+      return fail(BINATTN_ERR_ARG, "workspace of %zu bytes is below the %zu this shape needs", workspace_bytes,
+                  need);
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t fw = binattn_forward_workspace_bytes(B, H, N, d, bias != nullptr);
+  if (fused_path(q_dtype, d, N, bias != nullptr))
+    return forward_tma_ws(nullptr, k_bits, nullptr, alpha_k, bias, v, softmax_scale, B, H, N, d, out, workspace, fw,
+                          static_cast<const uint16_t*>(q), st);
+  // Other shapes and fp32 Q: binattn_pack into the workspace, then the forward.
+  char* ws = static_cast<char*>(workspace);
+  const size_t tokens = static_cast<size_t>(B) * H * N;
+  uint32_t* q_bits = reinterpret_cast<uint32_t*>(ws + round256(fw));
+  float* alpha_q = reinterpret_cast<float*>(ws + round256(fw) + round256(tokens * binattn::words_for(d) * 4));
+  if (int rc = binattn_pack(q, q_dtype, B, H, N, d, q_bits, alpha_q, stream)) return rc;
+  return binattn_forward_ws(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out,
+                            fw ? workspace : nullptr, fw, stream);
 }
 
 namespace {

@@ -139,6 +139,10 @@ struct Params {
   int pair_base;
   int split;
   float* part;
+  // bf16 Q [B,H,N,d] for a forward that binarises Q itself (TMA-fed pipelines
+  // only): each row's sign words and alpha_q come from pack_row_bf16 in the
+  // kernel, and qb / aq are not read. Null: qb / aq from binattn_pack.
+  const uint16_t* qh = nullptr;
 };
 
 // Named barrier 1 over the load-mode loader warps with an AND reduction.

@@ -51,6 +51,7 @@
 // frees its tensor memory.
 #pragma once
 #include "fwd_tc.cuh"
+#include "pack.cuh"
 
 namespace binattn {
 namespace tc2 {
@@ -283,6 +284,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   const int row = q0 + t * kRows + r;
   const bool row_valid = warp < kSoftmaxWarps && row < N;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  float aq_row = 0.f;  // alpha_q of this thread's row (binary forward)
   if (warp < kSoftmaxWarps) {
     if constexpr (kRef) {
       // bf16 pairs: column c2 holds channels 2 c2 (low half) and 2 c2 + 1
@@ -305,8 +307,19 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       // e4m3 bytes: column c4 holds channels 4 c4 .. 4 c4 + 3 (lowest byte first);
       // pad channels (>= d) are 0 so they add nothing to the score.
       const uint32_t qcol = tmem + lane_base + 256 * t + kQColBin;
+      uint32_t qw[3] = {0u, 0u, 0u};
+      if (row_valid && !kDump) {
+        if (p.qh) {
+          pack_row_bf16_w(p.qh + (tok0 + row) * d, d, W, qw, aq_row);  // Q binarised here
+        } else {
+          for (int w = 0; w < W; ++w) qw[w] = p.qb[(tok0 + row) * W + w];
+          aq_row = p.aq[tok0 + row];
+        }
+      } else if (row_valid) {
+        for (int w = 0; w < W; ++w) qw[w] = p.qb[(tok0 + row) * W + w];
+      }
       for (int w = 0; w < W; ++w) {
-        const uint32_t word = row_valid ? p.qb[(tok0 + row) * W + w] : 0u;
+        const uint32_t word = w == 0 ? qw[0] : w == 1 ? qw[1] : qw[2];
         uint32_t wv[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) wv[j] = row_valid ? e4m3_bytes(word, 4 * j, 32 * w + 4 * j, d, true) : 0u;
@@ -471,7 +484,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   } else {
     // ---------------------------------------------------------------- softmax
     // per-row factor of the logit: scale * alpha_q (binary) or scale (reference)
-    const float ci = kRef ? p.scale : ((!kDump && row_valid) ? p.scale * p.aq[tok0 + row] : 0.f);
+    const float ci = kRef ? p.scale : ((!kDump && row_valid) ? p.scale * aq_row : 0.f);
     const uint32_t o_col = tmem + lane_base + 256 * t + 128;
     const int r7 = r & 7;
     float m = -INFINITY;
@@ -869,12 +882,13 @@ inline size_t split_part_bytes(int B, int H, int N, int d) {
 }  // namespace tc2
 
 // part: workspace for the tail split (tc2::split_part_bytes), or null for no split.
+// qh: bf16 Q for a forward that binarises Q itself (qb, aq then unused), or null.
 inline int forward_tc2(const uint32_t* qb, const uint32_t* kb, const float* aq, const float* ak,
                        const uint16_t* bias, const uint16_t* v, float scale, int B, int H, int N, int d,
                        uint16_t* out, cudaStream_t st, std::string* msg, int bias_ld = 0,
-                       float* part = nullptr) {
+                       float* part = nullptr, const uint16_t* qh = nullptr) {
   tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d, bias_ld, 0, 0,
-                 nullptr};
+                 nullptr, qh};
   const tc2::SplitPlan plan = part ? tc2::split_plan(B, H, N) : tc2::SplitPlan{tc2::total_pairs(B, H, N), 0};
   auto run = [&](int ctas) {
     return bias ? tc2::dispatch_dv<tc2::kModeBin, true>(prm, ctas, st, msg)

@@ -271,13 +271,23 @@ fwd_tc3_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   const int row = q0 + t * kRows + r;
   const bool row_valid = warp < kSoftmaxWarps && row < N;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  float aq_row = 0.f;  // alpha_q of this thread's row
   if (warp < kSoftmaxWarps) {
     // Q_t operand row r in shared memory, e4m3 +-1 with pad channels (>= d)
     // 0, K-major like K: 16-byte chunk (row r, channel group c of 16) at
     // (r / 8) * (8 * 32W) + c * 128 + (r % 8) * 16.
     uint8_t* qrow = smem + L::kQ + t * L::kQTile + (r >> 3) * (8 * 32 * W) + (r & 7) * 16;
+    uint32_t qw[3] = {0u, 0u, 0u};
+    if (row_valid) {
+      if (p.qh) {
+        pack_row_bf16_w(p.qh + (tok0 + row) * d, d, W, qw, aq_row);  // Q binarised here
+      } else {
+        for (int w = 0; w < W; ++w) qw[w] = p.qb[(tok0 + row) * W + w];
+        aq_row = p.aq[tok0 + row];
+      }
+    }
     for (int w = 0; w < W; ++w) {
-      const uint32_t word = row_valid ? p.qb[(tok0 + row) * W + w] : 0u;
+      const uint32_t word = w == 0 ? qw[0] : w == 1 ? qw[1] : qw[2];
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         uint4 v4;
@@ -454,7 +464,7 @@ fwd_tc3_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     // ---------------------------------------------------------------- softmax
     constexpr int KA = L::kKA;
-    const float ci = row_valid ? p.scale * p.aq[tok0 + row] : 0.f;
+    const float ci = row_valid ? p.scale * aq_row : 0.f;
     const uint32_t s_col = tmem + lane_base + 256 * t;
     const uint32_t o_col = s_col + 128;
     const int r7 = r & 7;
@@ -737,12 +747,13 @@ inline int dispatch_dv(const tc::Params& prm, int ctas, cudaStream_t st, std::st
 // Binary forward on the 128-key pipeline. part: workspace for the tail split
 // (tc2::split_part_bytes), or null for no split. The split plan, the partial
 // layout and the combine kernel are those of the 64-key pipeline.
+// qh: bf16 Q for a forward that binarises Q itself (qb, aq then unused), or null.
 inline int forward_tc3(const uint32_t* qb, const uint32_t* kb, const float* aq, const float* ak,
                        const uint16_t* bias, const uint16_t* v, float scale, int B, int H, int N, int d,
                        uint16_t* out, cudaStream_t st, std::string* msg, int bias_ld = 0,
-                       float* part = nullptr) {
+                       float* part = nullptr, const uint16_t* qh = nullptr) {
   tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d, bias_ld, 0, 0,
-                 nullptr};
+                 nullptr, qh};
   const tc2::SplitPlan plan = part ? tc2::split_plan(B, H, N) : tc2::SplitPlan{tc2::total_pairs(B, H, N), 0};
   auto run = [&](int ctas) {
     return bias ? tc3::dispatch_dv<tc3::kModeBin, true>(prm, ctas, st, msg)

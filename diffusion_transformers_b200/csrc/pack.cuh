@@ -64,18 +64,17 @@ pack_kernel(const T* __restrict__ x, long long n_tokens, int d, int W,
 }
 
 
-// bf16 rows with d % 8 == 0 (every token a whole number of 16-byte chunks):
-// one thread per token. The thread issues all of its row's 16-byte loads,
-// builds its sign words with x >= 0 compares (8 channels per chunk, 4 chunks
-// per word), and sums |x| in eight partial sums (one per position in a chunk)
-// combined by a tree, so each alpha is a sum of depth <= d/8 + 2 in fp32.
+// Sign words and alpha of one bf16 row with d % 8 == 0 (a whole number of
+// 16-byte chunks, 16-byte aligned): all of the row's 16-byte loads are issued
+// at once, the sign words come from x >= 0 compares (8 channels per chunk, 4
+// chunks per word), and |x| is summed in eight partial sums (one per position
+// in a chunk) combined by a tree, so alpha is a sum of depth <= d/8 + 2 in
+// fp32. binattn_pack and the forward that binarises Q itself both call this,
+// so their bits and alpha are identical.
 template <int W>
-__global__ void __launch_bounds__(kPackThreads)
-pack_bf16_rows_kernel(const uint16_t* __restrict__ x, long long n_tokens, int d,
-                      uint32_t* __restrict__ bits, float* __restrict__ alpha) {
-  const long long t = static_cast<long long>(blockIdx.x) * kPackThreads + threadIdx.x;
-  if (t >= n_tokens) return;
-  const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
+__device__ __forceinline__ void pack_row_bf16(const uint16_t* __restrict__ row, int d, uint32_t* words,
+                                              float& alpha) {
+  const uint4* src = reinterpret_cast<const uint4*>(row);
   const int ng = d / 8;  // 16-byte chunks per token
   uint4 v[4 * W];
 #pragma unroll
@@ -101,10 +100,36 @@ pack_bf16_rows_kernel(const uint16_t* __restrict__ x, long long n_tokens, int d,
         }
       }
     }
-    bits[t * W + w] = word;
+    words[w] = word;
   }
   const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-  alpha[t] = sum / static_cast<float>(d);
+  alpha = sum / static_cast<float>(d);
+}
+
+// The same for a row with W = ceil(d / 32) <= 3 known only at run time.
+__device__ __forceinline__ void pack_row_bf16_w(const uint16_t* __restrict__ row, int d, int W, uint32_t* words,
+                                                float& alpha) {
+  switch (W) {
+    case 1: pack_row_bf16<1>(row, d, words, alpha); break;
+    case 2: pack_row_bf16<2>(row, d, words, alpha); break;
+    default: pack_row_bf16<3>(row, d, words, alpha); break;
+  }
+}
+
+// bf16 rows with d % 8 == 0 (every token a whole number of 16-byte chunks):
+// one thread per token (pack_row_bf16).
+template <int W>
+__global__ void __launch_bounds__(kPackThreads)
+pack_bf16_rows_kernel(const uint16_t* __restrict__ x, long long n_tokens, int d,
+                      uint32_t* __restrict__ bits, float* __restrict__ alpha) {
+  const long long t = static_cast<long long>(blockIdx.x) * kPackThreads + threadIdx.x;
+  if (t >= n_tokens) return;
+  uint32_t words[W];
+  float a;
+  pack_row_bf16<W>(x + t * d, d, words, a);
+#pragma unroll
+  for (int w = 0; w < W; ++w) bits[t * W + w] = words[w];
+  alpha[t] = a;
 }
 
 inline size_t pack_smem_bytes(int d, int esize, bool vec) {

@@ -192,6 +192,42 @@ int binattn_forward_static_ws(const uint32_t *q_bits, const uint32_t *k_bits,
                               const uint16_t *bias, const uint16_t *v, float softmax_scale,
                               int B, int H, int N, int d, uint16_t *out, void *stream);
 
+/*
+ * binattn_forward_fused_workspace_bytes — device workspace that
+ * binattn_forward_fused_ws needs for this shape and Q dtype on the current
+ * device (0 when it needs none). For bf16 Q on the TMA-fed pipeline (d % 8 == 0,
+ * d <= 80) it equals binattn_forward_workspace_bytes; otherwise it adds room for
+ * Q's sign words and alpha_q (each part rounded up to 256 bytes).
+ */
+size_t binattn_forward_fused_workspace_bytes(int B, int H, int N, int d, int q_dtype, int has_bias);
+
+/*
+ * binattn_forward_fused_ws — binattn_pack of Q and binattn_forward_ws in one
+ * call, with Q's binarisation done by the forward kernel itself where it can.
+ *
+ * Source: §2 (scaled binary representations; the forward as for
+ * binattn_forward). The result is the same computation: for bf16 Q with
+ * d % 8 == 0 and d <= 80, the forward kernel derives each query row's sign
+ * words and alpha_q with the same device code and summation order as
+ * binattn_pack, so O is bit-identical to binattn_pack followed by
+ * binattn_forward_ws. Other shapes and fp32 Q run binattn_pack into the
+ * workspace, then binattn_forward_ws.
+ *
+ *   q                 [B, H, N, d] dtype `q_dtype` (BINATTN_F32 or BINATTN_BF16),
+ *                     device, read.
+ *   k_bits, alpha_k   from binattn_pack of K, device, read.
+ *   bias, v, softmax_scale, out: as binattn_forward.
+ *   workspace         device, 16-byte aligned, at least
+ *                     binattn_forward_fused_workspace_bytes(...) bytes,
+ *                     overwritten; may be NULL when that size is 0.
+ *   workspace_bytes   its size.
+ * Errors: as binattn_forward_ws, and BINATTN_ERR_DTYPE for an unknown q_dtype.
+ */
+int binattn_forward_fused_ws(const void *q, int q_dtype, const uint32_t *k_bits, const float *alpha_k,
+                             const uint16_t *bias, const uint16_t *v, float softmax_scale,
+                             int B, int H, int N, int d, uint16_t *out,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
 /* binattn_forward with an explicit score engine (binattn_engine). Returns
  * BINATTN_ERR_UNSUPPORTED when the engine cannot serve the shape. */
 int binattn_forward_engine(const uint32_t *q_bits, const uint32_t *k_bits,

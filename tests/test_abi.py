@@ -134,3 +134,34 @@ def test_forward_ws_host_validation(L):
     assert b"workspace" in L.binattn_last_error_message()
     assert fws(bias=A + 2) == 4
     assert fws(N=0) == 2
+
+
+def test_fused_workspace_bytes(L):
+    # bf16 Q on the TMA-fed pipeline: the forward's own workspace only
+    for shape in [(64, 12, 197, 64), (2, 16, 4096, 72), (1, 2, 300, 8)]:
+        assert L.binattn_forward_fused_workspace_bytes(*shape, 1, 1) == L.binattn_forward_workspace_bytes(*shape, 1)
+    # fp32 Q or a shape the TMA-fed pipeline does not take: room for Q's sign words and alpha_q
+    B, H, N, d = 1, 2, 197, 33
+    tok = B * H * N
+    r256 = lambda x: -(-x // 256) * 256
+    assert L.binattn_forward_fused_workspace_bytes(B, H, N, d, 1, 1) == r256(tok * 2 * 4) + r256(tok * 4)
+    fw = L.binattn_forward_workspace_bytes(1, 2, 197, 64, 1)
+    assert L.binattn_forward_fused_workspace_bytes(1, 2, 197, 64, 0, 1) == r256(fw) + r256(394 * 2 * 4) + r256(394 * 4)
+    assert L.binattn_forward_fused_workspace_bytes(0, 2, 197, 64, 1, 1) == 0
+
+
+def test_forward_fused_host_validation(L):
+    def ffs(q=A, dt=1, ws=A, size=1 << 30, bias=A, N=197, d=64, out=A):
+        return L.binattn_forward_fused_ws(P(q) if q else None, dt, P(A), P(A), P(bias) if bias else None, P(A),
+                                          ctypes.c_float(0.125), 1, 2, N, d, P(out) if out else None,
+                                          P(ws) if ws else None, ctypes.c_size_t(size), None)
+    need = L.binattn_forward_fused_workspace_bytes(1, 2, 197, 64, 1, 1)
+    assert need > 0
+    assert ffs(q=0) == 1
+    assert ffs(q=A + 4) == 4
+    assert ffs(dt=5) == 3
+    assert ffs(out=0) == 1
+    assert ffs(ws=0) == 1
+    assert ffs(size=need - 1) == 8
+    assert ffs(N=0) == 2
+    assert ffs(bias=A + 2) == 4

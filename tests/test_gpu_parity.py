@@ -225,3 +225,54 @@ def test_forward_ws_split_tail(orc, shape):
     assert need > 0
     got = out.view(B * H * N, d)[torch.from_numpy(rows).cuda()]
     check_o(bf16_to_f64(got), ref, f"split {shape}")
+
+
+# ------------------------------- forward that binarises Q itself (fused a1/a2)
+# bf16 Q on the TMA-fed pipelines is binarised inside the forward kernel with
+# the same device code as binattn_pack, so O must equal pack + forward_ws bit
+# for bit; fp32 Q and other shapes go through pack into the workspace.
+FUSED_SHAPES = [(2, 3, 129, 72, True), (1, 2, 197, 64, True), (2, 2, 300, 64, False), (1, 2, 256, 40, False),
+                (1, 1, 65, 16, True), (1, 2, 100, 36, True), (1, 19, 2048, 72, True), (2, 10, 2100, 40, False)]
+
+
+@pytest.mark.parametrize("shape", FUSED_SHAPES)
+def test_forward_fused_equals_pack_then_forward(orc, shape):
+    B, H, N, d, with_bias = shape
+    c = make_custom(B, H, N, d, seed=11 * N + d, with_bias=with_bias, bias_std=0.5)
+    q, k, v = dev(c["q"]), dev(c["k"]), dev(c["v"])
+    bias = dev(c["bias"]) if with_bias else None
+    qb, aq = binattn.pack(q)
+    kb, ak = binattn.pack(k)
+    want = binattn.forward_ws(qb, kb, aq, ak, bias, v, c["softmax_scale"])
+    got = binattn.forward_fused_ws(q, kb, ak, bias, v, c["softmax_scale"])
+    torch.cuda.synchronize()
+    binattn.device_status()
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16)), f"fused {shape}"
+    if B * H * N <= 4096:
+        ref = orc.forward(c["q"], c["k"], c["bias"] if with_bias else None, c["v"], c["softmax_scale"])
+        check_o(bf16_to_f64(got), ref, f"fused {shape}")
+
+
+def test_forward_fused_fp32_q_and_full_size():
+    # fp32 Q (the tiny config) takes the pack-into-workspace route
+    inp = make_inputs("tiny", with_bias=True)
+    q, k, v, bias = dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), dev(inp["bias"])
+    qb, aq = binattn.pack(q)
+    kb, ak = binattn.pack(k)
+    want = binattn.forward_ws(qb, kb, aq, ak, bias, v, inp["softmax_scale"])
+    got = binattn.forward_fused_ws(q, kb, ak, bias, v, inp["softmax_scale"])
+    torch.cuda.synchronize()
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+    # DiT-XL/2 1024 px, both bias cases, whole output
+    for with_bias in (True, False):
+        inp = make_inputs("dit_xl_1024", with_bias=with_bias)
+        q, k, v = dev(inp["q"]), dev(inp["k"]), dev(inp["v"])
+        bias = dev(inp["bias"]) if with_bias else None
+        qb, aq = binattn.pack(q)
+        kb, ak = binattn.pack(k)
+        want = binattn.forward_ws(qb, kb, aq, ak, bias, v, inp["softmax_scale"])
+        got = binattn.forward_fused_ws(q, kb, ak, bias, v, inp["softmax_scale"])
+        torch.cuda.synchronize()
+        binattn.device_status()
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16)), f"dit_xl_1024 bias={with_bias}"
+        del q, k, v, bias, qb, kb, aq, ak, want, got
