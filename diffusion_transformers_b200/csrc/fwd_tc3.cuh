@@ -1,46 +1,56 @@
-// fwd_tc3.cuh — the forward pipeline with 128-key tiles: binary forward (e4m3
-// +-1 operands for QK^T) and the bf16 reference attention on the same pipeline.
+// fwd_tc3.cuh — the binary forward with 128-key tiles (e4m3 +-1 operands for
+// QK^T). It serves the forward without a bias, where it measured as fast as
+// the 64-key pipeline of fwd_tc2.cuh or a little faster.
 //
 // Source: "BinaryAttention: One-Bit QK-Attention for Vision and Diffusion
 // Transformers", §2 methodology (scaled binary Q/K, XNOR/popcount similarity,
 // additive learnable bias, softmax, P.V) and the hardware-aware implementation
 // bullet (FlashAttention2-style tiling). The tiling below is new for sm_100a.
 //
-// Shapes: d % 8 == 0, d <= 80 (reference: d <= 72); with a bias the row stride
-// of the bias is a multiple of 8 elements (the bias rows are TMA rows). One CTA
-// (12 warps, one per SM) owns 256 query rows of one (b, h) as two 128-row tiles
-// t = 0, 1 and streams the keys in tiles of 128:
+// Shapes: d % 8 == 0, d <= 80; with a bias the row stride of the bias is a
+// multiple of 8 elements (the bias rows are TMA rows). One CTA (12 warps, one
+// per SM) owns 256 query rows of one (b, h) as two 128-row tiles t = 0, 1 and
+// streams the keys in tiles of 128:
 //   warps 0-7  softmax: warps 4t..4t+3 for tile t, one thread per query row
 //              (TMEM lane).
 //   warp 8, 9  MMA issuers, one thread each: warp 8 + t issues for tile t.
-//   warp 10    TMA: V (and the bf16 K of the reference), the bias boxes.
-//   warp 11    binary: expands the key sign words to e4m3 +-1 operand rows and
-//              stages alpha_k, with the loads two tiles ahead.
+//   warp 10    TMA: V and the bias boxes (two 64-key boxes per tile), and L2
+//              prefetches of the bias two key tiles ahead.
+//   warp 11    expands the key sign words to e4m3 +-1 operand rows and stages
+//              alpha_k, with the loads two tiles ahead.
+// A warpgroup register split (setmaxnreg) gives the softmax warps 216
+// registers, enough for the 128 fp32 logits of a row.
+//
+// Shared memory holds Q_t as an e4m3 +-1 operand (pad channels 0), written
+// once by the softmax threads; with Params::qh set they binarise bf16 Q
+// themselves (pack_row_bf16, the same code and order as binattn_pack).
 //
 // Tensor memory, 256 columns per tile t (base 256 t):
-//   S_t  [0, 128)        fp32 scores of the current key tile; P_t (bf16 pairs,
-//                         key 2c and 2c + 1 in column c) overwrites [0, 64);
+//   S_t  [0, 128)        fp32 scores of the current key tile; part A of P_t
+//                         (bf16 pairs, keys 2c and 2c + 1 in column c, the
+//                         first KA keys) overwrites its first KA / 2 columns;
 //   O_t  [128, 128 + DV) fp32 accumulator, DV >= d + 1 (column d holds l);
-//   Q_t  binary: e4m3 bytes, 4 channels per column, [224, 224 + 8W);
-//        reference: bf16 pairs, [128 + DV, 128 + DV + DV / 2).
+//   P_B  [128 + DV, 256) part B of P_t: the remaining KB keys (96 for d <= 72).
 //
-// One score buffer per tile: the issuer of tile t runs, per key tile kt,
-//   O_t += P_t(kt) V(kt)    as two halves of 64 keys, each as soon as the
-//                           softmax threads publish that half of P;
-//   S_t  = Q_t K(kt + 1)^T  into the buffer P_t(kt) was just read from
-//                           (one thread's MMAs run in issue order).
-// While tile t waits for its next scores, tile 1 - t computes: the two tiles
-// keep the exp unit busy between them. Because QK^T(kt) is issued after
-// P.V(kt - 1) by the same thread, the scores' commit also proves that P.V
-// complete, so the softmax threads may rescale O_t as soon as S_t(kt) lands.
+// One score buffer per tile. The issuer of tile t runs, per key tile kt:
+//   1. waits for the operands of tile kt + 1;
+//   2. O_t += P_A V once part A is published;
+//   3. S_t = Q_t K(kt + 1)^T into S_t right behind it (one thread's MMAs run
+//      in issue order, and part B is not in S_t);
+//   4. O_t += P_B V once part B is published.
+// So the turnaround from P to the next scores overlaps the exps of part B.
+// Because QK^T(kt) is issued after P.V part A of kt - 1, the scores' commit
+// proves that part complete; part B's own commit (pb_free) covers the rest
+// before O_t is rescaled or P_B is rewritten.
 //
-// Softmax per row, fp32, one thread per row: logit = (S alpha_k)(scale
-// alpha_q) + bias; the tile max is settled before any exp; the running max m
-// moves only when the tile max exceeds it by more than 8 ln 2, and then O_t
-// (with l in column d) is rescaled; P = exp(logit - m) rounded to bf16. Channel
-// d of every V stage is 1.0, so O_t column d sums the bf16 P actually
-// multiplied. The epilogue divides O by l and writes bf16 (or, for a split key
-// half, the unnormalised partials that combine_halves_kernel joins).
+// Softmax per row, fp32: logit = (S alpha_k)(scale alpha_q) + bias; the tile
+// max is settled before any exp; the running max m moves only when the tile max
+// exceeds it by more than 8 ln 2, and then O_t (with l in column d) is
+// rescaled; P = exp(logit - m) rounded to bf16. The two tiles take turns on
+// their part-A exp phases through named barriers 3 and 4. Channel d of every V
+// stage is 1.0, so O_t column d sums the bf16 P actually multiplied. The
+// epilogue divides O by l and writes bf16 (or, for a split key half, the
+// unnormalised partials that combine_halves_kernel joins).
 //
 // Every mbarrier wait is bounded (sm100::mbar_wait); on a timeout the CTA
 // records a device status code, leaves its loops, waits for its own MMAs and
@@ -62,7 +72,7 @@ using tc2::tmem_ld8;
 
 constexpr int kRows = 128;    // query rows per tile (MMA M)
 constexpr int kKeys = 128;    // keys per tile (QK MMA N, P.V K)
-constexpr int kHalf = 64;     // keys per published half of P
+constexpr int kHalf = 64;     // keys per bias box (a 128B-swizzled box spans 64 bf16 keys)
 constexpr int kSoftmaxPerTile = 128;
 constexpr int kWarps = 12;
 constexpr int kThreads = kWarps * 32;

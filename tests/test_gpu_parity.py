@@ -134,6 +134,28 @@ def test_forward_special_cases(orc, engine):
         check_o(bf16_to_f64(r["out"]), ref, f"{kw} {engine}")
 
 
+# Keys whose scale alpha_k grows with the key index: every later key tile has
+# larger logits, so the running max grows tile after tile and O (with l) is
+# rescaled again and again, in both pipelines (no bias: 128-key tiles; bias:
+# 64-key tiles), on a ragged N.
+@pytest.mark.parametrize("with_bias", [False, True])
+@pytest.mark.parametrize("d", [64, 72])
+def test_forward_growing_max(orc, with_bias, d):
+    from diffusion_transformers_b200.synthetic import f32_to_bf16_bits
+    B, H, N = 1, 2, 700
+    c = make_custom(B, H, N, d, seed=91 + d, with_bias=with_bias, bias_std=0.5)
+    grow = (1.0 + np.arange(N, dtype=np.float32) / 24.0)[None, None, :, None]
+    c["k"] = f32_to_bf16_bits(bf16_to_f64_np(c["k"]) * grow)
+    ref = orc.forward(c["q"], c["k"], c["bias"] if with_bias else None, c["v"], c["softmax_scale"])
+    r = run_path(c, with_bias=with_bias)
+    check_o(bf16_to_f64(r["out"]), ref, f"growing max d={d} bias={with_bias}")
+
+
+def bf16_to_f64_np(bits):
+    from diffusion_transformers_b200.synthetic import bf16_bits_to_f32
+    return bf16_bits_to_f32(bits).astype(np.float32)
+
+
 @pytest.mark.parametrize("engine", ENGINES)
 def test_forward_deterministic(engine):
     c = make_custom(2, 2, 300, 72, seed=9)
