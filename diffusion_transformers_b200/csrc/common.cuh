@@ -1,6 +1,7 @@
 // common.cuh — shared internals of libbinattn (one translation unit).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -30,6 +31,22 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
 }
 
 __host__ __device__ constexpr int words_for(int d) { return (d + 31) / 32; }
+
+// One-time set-up of a kernel (function attributes) is per device: `done`
+// holds one bit per device ordinal below 64. needs_setup is true while the
+// current device's bit is clear (always, for ordinals it cannot track);
+// mark_setup sets it once the set-up has succeeded. Two host threads may both
+// run the set-up for one device; it is idempotent.
+inline bool needs_setup(const std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return true;
+  return !(done.load(std::memory_order_acquire) & (1ull << dev));
+}
+inline void mark_setup(std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64)
+    done.fetch_or(1ull << dev, std::memory_order_release);
+}
 
 // The binary score of one (query, key) pair from packed sign bits:
 // S = d - 2 * popcount(q XOR k) over W words. Pad bits (channels >= d) are 0

@@ -879,14 +879,14 @@ inline int launch_tc(const Params& prm, const TensorMaps& tm, cudaStream_t st, s
   auto kern = fwd_tc_kernel<KDIM, kTma, kQK, kBias, kDump>;
   constexpr int smem = Layout<KDIM, kTma>::kLaunchBytes;
   static_assert(smem <= 227 * 1024, "shared memory over the sm_100 per-CTA limit");
-  static bool configured = false;  // attribute set once per instantiation
-  if (!configured) {
+  static std::atomic<uint64_t> configured{0};  // attribute set once per device and instantiation
+  if (needs_setup(configured)) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) {
       *msg = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);
       return BINATTN_ERR_CUDA;
     }
-    configured = true;
+    mark_setup(configured);
   }
   dim3 grid(static_cast<unsigned>(prm.B * ((prm.N + 2 * kRows - 1) / (2 * kRows))), prm.H);
   kern<<<grid, kThreads, smem, st>>>(prm, tm.v, tm.ak, tm.bias, tm.k);

@@ -813,14 +813,14 @@ inline int launch(const tc::Params& prm, int ctas, cudaStream_t st, std::string*
   auto kern = fwd_tc2_kernel<DV, kMode, kBias>;
   constexpr int smem = Layout<DV, kMode, kBias>::kLaunchBytes;
   static_assert(smem <= 227 * 1024, "shared memory over the sm_100 per-CTA limit");
-  static bool configured = false;  // attribute set once per instantiation
-  if (!configured) {
+  static std::atomic<uint64_t> configured{0};  // attribute set once per device and instantiation
+  if (needs_setup(configured)) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) {
       *msg = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);
       return BINATTN_ERR_CUDA;
     }
-    configured = true;
+    mark_setup(configured);
   }
   kern<<<static_cast<unsigned>(ctas), kThreads, smem, st>>>(prm, tm_v, tm_bias, tm_k);
   cudaError_t e = cudaGetLastError();

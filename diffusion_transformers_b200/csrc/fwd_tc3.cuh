@@ -711,8 +711,8 @@ inline int launch(const tc::Params& prm, int ctas, cudaStream_t st, std::string*
   auto kern = fwd_tc3_kernel<DV, kMode, kBias>;
   constexpr int smem = Layout<DV, kMode, kBias>::kLaunchBytes;
   static_assert(smem <= 227 * 1024, "shared memory over the sm_100 per-CTA limit");
-  static bool configured = false;
-  if (!configured) {
+  static std::atomic<uint64_t> configured{0};  // set-up once per device
+  if (needs_setup(configured)) {
     // The register split assumes the launch gives kLaunchRegs per thread: with
     // fewer, the softmax warpgroups' setmaxnreg.inc could not be satisfied.
     cudaFuncAttributes fa;
@@ -731,7 +731,7 @@ inline int launch(const tc::Params& prm, int ctas, cudaStream_t st, std::string*
       *msg = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);
       return BINATTN_ERR_CUDA;
     }
-    configured = true;
+    mark_setup(configured);
   }
   kern<<<static_cast<unsigned>(ctas), kThreads, smem, st>>>(prm, tm_v, tm_bias);
   cudaError_t e = cudaGetLastError();
