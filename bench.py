@@ -24,6 +24,7 @@ import argparse
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -87,24 +88,32 @@ def algorithmic(w, with_bias=True):
 # dram__bytes_write.sum summed over the launches the call makes at dit_xl_1024
 # with bias: the full-wave launch, the key-split tail launch and the combine; the
 # summary is profiles/fwd_tc2_dit_xl_1024_bias.md), valid only for the kernel
-# sources it was taken on: any change to them turns the reported traffic back
-# into null.
+# sources it was taken on: any change to their code turns the reported traffic
+# back into null. The digest covers the code only (comments removed, runs of
+# white space collapsed), so an edit of a comment keeps the capture valid.
 NCU_TRAFFIC = {
-    "sources_sha256": "d538588d20e22a3900db4c7f6bdb0dd6ed7b1ede9ff6bea5859c1a41b1bbf2bb",
+    "sources_sha256": "583f2e64017821cf280786dffad1769301b411b431bdb25bf90831377d9331e6",
     "bytes_per_call": {"dit_xl_1024/bias": 590_076_672},
 }
 
+_C_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'|//[^\n]*|/\*.*?\*/', re.S)
 
-def kernel_sources_digest():
+
+def code_only(text):
+    """C/C++/CUDA source with comments removed and white space collapsed."""
+    kept = _C_TOKENS.sub(lambda m: " " if m.group(0)[0] == "/" else m.group(0), text)
+    return " ".join(kept.split())
+
+
+def kernel_sources_digest(root=ROOT):
     import hashlib
-    csrc = os.path.join(ROOT, "diffusion_transformers_b200", "csrc")
+    csrc = os.path.join(root, "diffusion_transformers_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
-    with open(os.path.join(ROOT, "include", "binattn.h"), "rb") as f:
-        h.update(f.read())
+    paths = [os.path.join(csrc, n) for n in sorted(os.listdir(csrc)) if n.endswith((".cu", ".cuh", ".h"))]
+    paths.append(os.path.join(root, "include", "binattn.h"))
+    for path in paths:
+        with open(path, encoding="utf-8") as f:
+            h.update(os.path.basename(path).encode() + b"\0" + code_only(f.read()).encode())
     return h.hexdigest()
 
 

@@ -27,7 +27,7 @@
  *    before anything is launched; on any error nothing is launched and the
  *    outputs are untouched. No exception or abort crosses the ABI.
  *    binattn_last_error_message() gives a one-line detail for the calling thread.
- *  - Sizes: B, H, N >= 1; 1 <= d <= 128; B*H <= 2^20; N <= 65536.
+ *  - Sizes: B, H, N >= 1; 1 <= d <= 128; B*H <= 65535; N <= 65535.
  *    All pointers must be 16-byte aligned.
  *  - Inputs containing NaN or Inf are outside the contract.
  */

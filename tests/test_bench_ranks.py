@@ -73,3 +73,13 @@ def test_reference_arm_other_ranks_do_no_work(capsys):
     args = argparse.Namespace(steps=1, warmup=0, gpus=2, cpu_seconds=0.1, workload="tiny")
     bench.run_reference(args, WORKLOADS["tiny"], rank=1)
     assert capsys.readouterr().out == ""
+
+
+def test_traffic_digest_ignores_comments_only():
+    import bench
+
+    src = 'int f(int x) { // doubles\n  return 2 * x; /* multi\n line */ }\nconst char* s = "a//b /*c*/";\n'
+    same = '/* header */ int f(int x) {\n\n return 2*x; }   const char* s = "a//b /*c*/";'
+    assert bench.code_only(src) == bench.code_only(same.replace("2*x", "2 * x"))
+    assert '"a//b /*c*/"' in bench.code_only(src)
+    assert bench.code_only(src) != bench.code_only(src.replace("2 * x", "3 * x"))
