@@ -3,6 +3,8 @@
 Argument marshalling only: every step of the computation runs in the CUDA
 kernels of libbinattn.so. torch is used for device memory and streams. There is
 no CPU fallback: if the library is missing, importing a function raises.
+Each call first checks the shapes, dtypes and device of its tensors, which the
+ABI cannot see behind its pointers, and runs with that device current.
 """
 from __future__ import annotations
 
@@ -91,9 +93,36 @@ def _ptr(t: torch.Tensor | None):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream) -> ctypes.c_void_p:
+_BITS = (torch.int32, getattr(torch, "uint32", torch.int32))
+
+
+def _expect(t: torch.Tensor | None, name: str, shape, dtypes) -> None:
+    """Shape and dtype of one argument; the C ABI sees only pointers, so a
+    tensor smaller than the sizes passed with it would be read out of bounds."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {tuple(str(d) for d in dtypes)}")
+
+
+def _device(*tensors: torch.Tensor | None) -> torch.device:
+    """The one CUDA device that holds every given tensor."""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"all tensors must be on one CUDA device, got {sorted(str(d) for d in devs)}")
+    dev = devs.pop()
+    if dev.type != "cuda":
+        raise ValueError(f"libbinattn takes CUDA tensors, got {dev}")
+    return dev
+
+
+def _stream(stream, dev: torch.device) -> ctypes.c_void_p:
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(dev)
+    elif stream.device != dev:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {dev}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -108,13 +137,30 @@ def pack(x: torch.Tensor, bits: torch.Tensor | None = None, alpha: torch.Tensor 
     dt = {torch.float32: F32, torch.bfloat16: BF16}.get(x.dtype)
     if dt is None:
         raise TypeError(f"pack takes float32 or bfloat16, got {x.dtype}")
+    _expect(bits, "bits", (B, H, N, _words(d)), _BITS)
+    _expect(alpha, "alpha", (B, H, N), (torch.float32,))
+    dev = _device(x, bits, alpha)
     if bits is None:
-        bits = torch.empty((B, H, N, _words(d)), dtype=torch.int32, device=x.device)
+        bits = torch.empty((B, H, N, _words(d)), dtype=torch.int32, device=dev)
     if alpha is None:
-        alpha = torch.empty((B, H, N), dtype=torch.float32, device=x.device)
-    _check(lib().binattn_pack(_ptr(x), dt, B, H, N, d, _ptr(bits), _ptr(alpha), _stream(stream)),
-           "binattn_pack")
+        alpha = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().binattn_pack(_ptr(x), dt, B, H, N, d, _ptr(bits), _ptr(alpha), _stream(stream, dev)),
+               "binattn_pack")
     return bits, alpha
+
+
+def _forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, out) -> torch.device:
+    """Checks shared by the forward calls; V [B,H,N,d] fixes the sizes."""
+    B, H, N, d = v.shape
+    _expect(v, "v", (B, H, N, d), (torch.bfloat16,))
+    _expect(q_bits, "q_bits", (B, H, N, _words(d)), _BITS)
+    _expect(k_bits, "k_bits", (B, H, N, _words(d)), _BITS)
+    _expect(alpha_q, "alpha_q", (B, H, N), (torch.float32,))
+    _expect(alpha_k, "alpha_k", (B, H, N), (torch.float32,))
+    _expect(bias, "bias", (H, N, N), (torch.bfloat16,))
+    _expect(out, "out", (B, H, N, d), (torch.bfloat16,))
+    return _device(q_bits, k_bits, alpha_q, alpha_k, bias, v, out)
 
 
 def forward(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor,
@@ -125,12 +171,14 @@ def forward(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor,
     B, H, N, d = v.shape
     if isinstance(engine, str):
         engine = ENGINES[engine]
+    dev = _forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, out)
     if out is None:
-        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=v.device)
-    _check(lib().binattn_forward_engine(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k),
-                                        _ptr(bias), _ptr(v), float(softmax_scale), B, H, N, d,
-                                        _ptr(out), int(engine), _stream(stream)),
-           "binattn_forward_engine")
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().binattn_forward_engine(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k),
+                                            _ptr(bias), _ptr(v), float(softmax_scale), B, H, N, d,
+                                            _ptr(out), int(engine), _stream(stream, dev)),
+               "binattn_forward_engine")
     return out
 
 
@@ -141,10 +189,15 @@ def scores_debug(q_bits: torch.Tensor, k_bits: torch.Tensor, d: int,
     B, H, N, _ = q_bits.shape
     if isinstance(engine, str):
         engine = ENGINES[engine]
+    _expect(q_bits, "q_bits", (B, H, N, _words(d)), _BITS)
+    _expect(k_bits, "k_bits", (B, H, N, _words(d)), _BITS)
+    _expect(S, "S", (B, H, N, N), (torch.int32,))
+    dev = _device(q_bits, k_bits, S)
     if S is None:
-        S = torch.empty((B, H, N, N), dtype=torch.int32, device=q_bits.device)
-    _check(lib().binattn_scores_debug(_ptr(q_bits), _ptr(k_bits), B, H, N, d, _ptr(S), int(engine),
-                                      _stream(stream)), "binattn_scores_debug")
+        S = torch.empty((B, H, N, N), dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().binattn_scores_debug(_ptr(q_bits), _ptr(k_bits), B, H, N, d, _ptr(S), int(engine),
+                                          _stream(stream, dev)), "binattn_scores_debug")
     return S
 
 
@@ -160,16 +213,20 @@ def forward_ws(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor
     """forward (engine AUTO) with a caller-owned workspace (uint8 CUDA tensor of at
     least workspace_bytes(...) bytes; allocated here when None)."""
     B, H, N, d = v.shape
+    dev = _forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, out)
+    if workspace is not None:
+        _device(workspace, v)
     need = workspace_bytes(B, H, N, d, bias is not None)
     if workspace is None and need:
-        workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     if out is None:
-        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=v.device)
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
     size = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().binattn_forward_ws(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k), _ptr(bias),
-                                    _ptr(v), float(softmax_scale), B, H, N, d, _ptr(out), _ptr(workspace),
-                                    ctypes.c_size_t(size), _stream(stream)),
-           "binattn_forward_ws")
+    with torch.cuda.device(dev):
+        _check(lib().binattn_forward_ws(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k), _ptr(bias),
+                                        _ptr(v), float(softmax_scale), B, H, N, d, _ptr(out), _ptr(workspace),
+                                        ctypes.c_size_t(size), _stream(stream, dev)),
+               "binattn_forward_ws")
     return out
 
 
@@ -178,11 +235,14 @@ def forward_static_ws(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch
                       softmax_scale: float, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """forward_ws on the library's static workspace: the call allocates no device memory."""
     B, H, N, d = v.shape
+    dev = _forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, out)
     if out is None:
-        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=v.device)
-    _check(lib().binattn_forward_static_ws(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k), _ptr(bias),
-                                           _ptr(v), float(softmax_scale), B, H, N, d, _ptr(out), _stream(stream)),
-           "binattn_forward_static_ws")
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().binattn_forward_static_ws(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k),
+                                               _ptr(bias), _ptr(v), float(softmax_scale), B, H, N, d, _ptr(out),
+                                               _stream(stream, dev)),
+               "binattn_forward_static_ws")
     return out
 
 
@@ -201,16 +261,20 @@ def forward_fused_ws(q: torch.Tensor, k_bits: torch.Tensor, alpha_k: torch.Tenso
     dt = {torch.float32: F32, torch.bfloat16: BF16}.get(q.dtype)
     if dt is None:
         raise TypeError(f"q must be float32 or bfloat16, got {q.dtype}")
+    _expect(q, "q", (B, H, N, d), (q.dtype,))
+    dev = _forward_args(None, k_bits, None, alpha_k, bias, v, out)
+    _device(q, v, workspace)
     need = fused_workspace_bytes(B, H, N, d, q.dtype, bias is not None)
     if workspace is None and need:
-        workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     if out is None:
-        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=v.device)
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
     size = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().binattn_forward_fused_ws(_ptr(q), dt, _ptr(k_bits), _ptr(alpha_k), _ptr(bias), _ptr(v),
-                                          float(softmax_scale), B, H, N, d, _ptr(out), _ptr(workspace),
-                                          ctypes.c_size_t(size), _stream(stream)),
-           "binattn_forward_fused_ws")
+    with torch.cuda.device(dev):
+        _check(lib().binattn_forward_fused_ws(_ptr(q), dt, _ptr(k_bits), _ptr(alpha_k), _ptr(bias), _ptr(v),
+                                              float(softmax_scale), B, H, N, d, _ptr(out), _ptr(workspace),
+                                              ctypes.c_size_t(size), _stream(stream, dev)),
+               "binattn_forward_fused_ws")
     return out
 
 
@@ -219,17 +283,25 @@ def ref_bf16_forward(q: torch.Tensor, k: torch.Tensor, bias: torch.Tensor | None
                      stream=None) -> torch.Tensor:
     """Full-precision bf16 softmax attention on the same shapes (speed reference)."""
     B, H, N, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        _expect(t, name, (B, H, N, d), (torch.bfloat16,))
+    _expect(bias, "bias", (H, N, N), (torch.bfloat16,))
+    dev = _device(q, k, bias, v, out)
     if out is None:
-        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
-    _check(lib().binattn_ref_bf16_forward(_ptr(q), _ptr(k), _ptr(bias), _ptr(v), float(softmax_scale),
-                                          B, H, N, d, _ptr(out), _stream(stream)),
-           "binattn_ref_bf16_forward")
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().binattn_ref_bf16_forward(_ptr(q), _ptr(k), _ptr(bias), _ptr(v), float(softmax_scale),
+                                              B, H, N, d, _ptr(out), _stream(stream, dev)),
+               "binattn_ref_bf16_forward")
     return out
 
 
 def device_status(stream=None) -> None:
-    """Synchronize and raise if a kernel abandoned a bounded wait."""
-    _check(lib().binattn_device_status(_stream(stream)), "binattn_device_status")
+    """Synchronize and raise if a kernel abandoned a bounded wait (current device,
+    or the device of `stream`)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if stream is None else stream.device
+    with torch.cuda.device(dev):
+        _check(lib().binattn_device_status(_stream(stream, dev)), "binattn_device_status")
 
 
 def abi_version() -> int:

@@ -165,3 +165,111 @@ def test_forward_fused_host_validation(L):
     assert ffs(size=need - 1) == 8
     assert ffs(N=0) == 2
     assert ffs(bias=A + 2) == 4
+
+
+def test_binding_checks_shapes_dtypes_and_device():
+    # The binding checks sizes, dtypes and the device before any call into the
+    # library: the ABI sees bare pointers and would read a short tensor out of
+    # bounds. CPU tensors of the right shapes reach the device check.
+    import torch
+
+    B, H, N, d = 2, 3, 37, 72
+    W = 3
+    bf = dict(dtype=torch.bfloat16)
+    q, k, v = torch.zeros(B, H, N, d, **bf), torch.zeros(B, H, N, d, **bf), torch.zeros(B, H, N, d, **bf)
+    bias = torch.zeros(H, N, N, **bf)
+    qb, kb = torch.zeros(B, H, N, W, dtype=torch.int32), torch.zeros(B, H, N, W, dtype=torch.int32)
+    aq, ak = torch.zeros(B, H, N), torch.zeros(B, H, N)
+    cpu = "libbinattn takes CUDA tensors"
+
+    def raises(exc, match, fn, *a, **kw):
+        with pytest.raises(exc, match=match):
+            fn(*a, **kw)
+
+    # valid shapes: only the device is wrong
+    raises(ValueError, cpu, binattn.pack, q)
+    raises(ValueError, cpu, binattn.pack, q, qb, aq)
+    raises(ValueError, cpu, binattn.forward, qb, kb, aq, ak, bias, v, 0.1)
+    raises(ValueError, cpu, binattn.forward, qb, kb, aq, ak, None, v, 0.1, out=torch.zeros_like(v))
+    raises(ValueError, cpu, binattn.forward_static_ws, qb, kb, aq, ak, bias, v, 0.1)
+    raises(ValueError, cpu, binattn.scores_debug, qb, kb, d)
+    raises(ValueError, cpu, binattn.ref_bf16_forward, q, k, bias, v, 0.1)
+    raises(ValueError, cpu, binattn.forward_ws, qb, kb, aq, ak, bias, v, 0.1,
+           workspace=torch.zeros(64, dtype=torch.uint8))
+    raises(ValueError, cpu, binattn.forward_fused_ws, q.float(), kb, ak, None, v, 0.1)
+    # wrong shapes and dtypes
+    raises(ValueError, "bits has shape", binattn.pack, q, qb[..., :2], aq)
+    raises(ValueError, "alpha has shape", binattn.pack, q, qb, aq[:, :, :5])
+    raises(TypeError, "bits has dtype", binattn.pack, q, qb.float(), aq)
+    raises(ValueError, "k_bits has shape", binattn.forward, qb, kb[:, :, :5], aq, ak, bias, v, 0.1)
+    raises(ValueError, "q_bits has shape", binattn.forward, qb[..., :2], kb, aq, ak, bias, v, 0.1)
+    raises(ValueError, "bias has shape", binattn.forward, qb, kb, aq, ak, bias[:, :5], v, 0.1)
+    raises(ValueError, "bias has shape", binattn.forward_ws, qb, kb, aq, ak, bias[:1], v, 0.1)
+    raises(TypeError, "bias has dtype", binattn.forward, qb, kb, aq, ak, bias.float(), v, 0.1)
+    raises(TypeError, "v has dtype", binattn.forward, qb, kb, aq, ak, bias, v.float(), 0.1)
+    raises(ValueError, "alpha_q has shape", binattn.forward_static_ws, qb, kb, aq[:1], ak, bias, v, 0.1)
+    raises(ValueError, "out has shape", binattn.forward, qb, kb, aq, ak, bias, v, 0.1, out=v[:1])
+    raises(ValueError, "alpha_k has shape", binattn.forward_fused_ws, q, kb, ak[:1], bias, v, 0.1)
+    raises(ValueError, "q has shape", binattn.forward_fused_ws, q[:1], kb, ak, bias, v, 0.1)
+    raises(ValueError, "S has shape", binattn.scores_debug, qb, kb, d, S=torch.zeros(1, dtype=torch.int32))
+    raises(ValueError, "k has shape", binattn.ref_bf16_forward, q, k[:1], bias, v, 0.1)
+    # the words per token follow d
+    raises(ValueError, "q_bits has shape", binattn.scores_debug, qb, kb, 64)
+
+
+def test_binding_marshals_every_call(monkeypatch):
+    # Each binding function, with its device handling stubbed out, hands the
+    # library exactly the arguments the ABI declares: the count of the real
+    # argtypes, the sizes of the tensors and the pointers of the tensors.
+    import contextlib
+    import types
+
+    import torch
+
+    real = binattn.lib()
+    calls = []
+
+    class FakeLib:
+        def __getattr__(self, name):
+            fn = getattr(real, name)
+
+            def call(*args):
+                if fn.argtypes is not None:
+                    assert len(args) == len(fn.argtypes), name
+                calls.append((name, args))
+                return 0 if name != "binattn_forward_workspace_bytes" else 4096
+            return call
+
+    cpu = torch.device("cpu")
+    monkeypatch.setattr(binattn, "lib", lambda: FakeLib())
+    monkeypatch.setattr(binattn, "_device", lambda *t: cpu)
+    monkeypatch.setattr(torch.cuda, "device", lambda dev: contextlib.nullcontext())
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda dev=None: types.SimpleNamespace(cuda_stream=0, device=cpu))
+
+    B, H, N, d = 1, 2, 33, 40
+    bf = dict(dtype=torch.bfloat16)
+    q, v = torch.zeros(B, H, N, d, **bf), torch.zeros(B, H, N, d, **bf)
+    bias = torch.zeros(H, N, N, **bf)
+    qb, aq = binattn.pack(q)
+    assert qb.shape == (B, H, N, 2) and qb.dtype == torch.int32 and aq.shape == (B, H, N)
+    name, args = calls[-1]
+    assert name == "binattn_pack" and args[1:6] == (binattn.BF16, B, H, N, d)
+    assert args[0].value == q.data_ptr() and args[6].value == qb.data_ptr()
+    out = binattn.forward(qb, qb, aq, aq, bias, v, 0.25, engine="tc")
+    name, args = calls[-1]
+    assert name == "binattn_forward_engine" and args[7:11] == (B, H, N, d) and args[12] == binattn.ENGINE_TC
+    assert args[4].value == bias.data_ptr() and args[11].value == out.data_ptr() and args[6] == 0.25
+    binattn.forward(qb, qb, aq, aq, None, v, 0.25)
+    assert calls[-1][1][4] is None
+    binattn.forward_ws(qb, qb, aq, aq, bias, v, 0.25)
+    name, args = calls[-1]
+    assert name == "binattn_forward_ws" and args[13].value == 4096
+    binattn.forward_static_ws(qb, qb, aq, aq, bias, v, 0.25)
+    assert calls[-1][0] == "binattn_forward_static_ws"
+    binattn.forward_fused_ws(q, qb, aq, bias, v, 0.25)
+    name, args = calls[-1]
+    assert name == "binattn_forward_fused_ws" and args[1] == binattn.BF16 and args[7:11] == (B, H, N, d)
+    S = binattn.scores_debug(qb, qb, d)
+    assert S.shape == (B, H, N, N) and calls[-1][1][2:6] == (B, H, N, d)
+    binattn.ref_bf16_forward(q, q, None, v, 0.25)
+    assert calls[-1][0] == "binattn_ref_bf16_forward" and calls[-1][1][5:9] == (B, H, N, d)
