@@ -296,6 +296,47 @@ def pin_worked_example(orc):
     assert np.allclose(O, want, rtol=1e-14, atol=1e-15)
 
 
+# ------------------------------------------------- statistics of the inputs
+def pin_alpha_half_normal_mean(orc):
+    """For x ~ N(0, sigma^2) the mean of |x| is sqrt(2/pi) * sigma (the
+    half-normal mean), so the average alpha over many tokens of each synthetic
+    workload is sqrt(2/pi) times its mean channel scale: 1 for N(0,1), E[U(0.5,2)]
+    = 1.25 for per-token stds, (61 + 3 * 8) / 64 with three x8 outlier channels.
+    Checks the generators' recipes together with the oracle's alpha (5 standard
+    errors)."""
+    from diffusion_transformers_b200.synthetic import make_inputs
+
+    c = math.sqrt(2.0 / math.pi)
+    for name, scale in (("dit_xl_512", 1.0), ("deit_b", 1.25), ("vit_l384", (61 + 3 * 8) / 64)):
+        inp = make_inputs(name, with_bias=False, B=1)
+        for key in ("q", "k"):
+            _, a = orc.pack(inp[key])
+            a = a.reshape(-1)
+            se = a.std() / math.sqrt(a.size)
+            assert abs(a.mean() - c * scale) <= 5 * se + 2e-3 * c * scale, \
+                f"{name} {key}: mean alpha {a.mean():.5f} vs sqrt(2/pi)*{scale:.4f} = {c * scale:.5f}"
+
+
+def pin_sign_correlation_arcsin(orc):
+    """For a bivariate normal pair with correlation rho, E[sign x * sign y] =
+    (2/pi) * arcsin(rho) (the orthant-probability identity). Q and K drawn
+    with channel-wise correlation rho give mean S_ii / d at that value; pairs of
+    independent tokens give 0. d = 72 also exercises the pad bits."""
+    rng = np.random.default_rng(21)
+    H, N, d = 4, 256, 72
+    for rho in (-0.7, 0.0, 0.3, 0.9):
+        q = rng.standard_normal((1, H, N, d))
+        k = rho * q + math.sqrt(1.0 - rho * rho) * rng.standard_normal((1, H, N, d))
+        S = orc.scores(q.astype(np.float32), k.astype(np.float32)).astype(np.float64) / d
+        diag = np.diagonal(S, axis1=2, axis2=3)
+        want = 2.0 / math.pi * math.asin(rho)
+        se = math.sqrt(max(1.0 - want * want, 1e-3) / (diag.size * d))
+        assert abs(diag.mean() - want) <= 5 * se, f"rho={rho}: mean S/d {diag.mean():.4f} vs {want:.4f}"
+        off = S.sum(axis=(2, 3)) - diag.sum(axis=2)
+        n_off = H * N * (N - 1)
+        assert abs(off.sum() / n_off) <= 5 / math.sqrt(n_off * d), f"rho={rho}: independent tokens correlate"
+
+
 ALL_PINS = [
     pin_sign_predicate_exhaustive,
     pin_pack_layout_packbits,
@@ -312,4 +353,6 @@ ALL_PINS = [
     pin_convex_hull,
     pin_bruteforce_matrix_form,
     pin_worked_example,
+    pin_alpha_half_normal_mean,
+    pin_sign_correlation_arcsin,
 ]
