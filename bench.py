@@ -123,6 +123,15 @@ def ncu_traffic(key):
     return NCU_TRAFFIC["bytes_per_call"].get(key)
 
 
+def percentile(xs, q):
+    """Linearly interpolated q-quantile (0 <= q <= 1) of a non-empty sequence."""
+    s = sorted(xs)
+    pos = q * (len(s) - 1)
+    lo = int(math.floor(pos))
+    hi = min(lo + 1, len(s) - 1)
+    return s[lo] + (s[hi] - s[lo]) * (pos - lo)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -442,6 +451,8 @@ def run_gpu(args, w, rank, world, local_rank):
         results[name] = dict(step_ms=max_over_ranks(sum(step_ms) / len(step_ms)),
                              fwd_ms=max_over_ranks(sum(fwd_ms) / len(fwd_ms)),
                              fwd_ms_median=statistics.median(fwd_ms),
+                             fwd_ms_p10=percentile(fwd_ms, 0.1),
+                             fwd_ms_p90=percentile(fwd_ms, 0.9),
                              fwd_ms_min=min(fwd_ms))
     clocks = sampler.stop()
     binattn.device_status(stream)
@@ -545,6 +556,8 @@ def run_gpu(args, w, rank, world, local_rank):
                                               else "binattn_forward"},
         "forward_ms": round(results["bias"]["fwd_ms"], 5),
         "forward_ms_median": round(results["bias"]["fwd_ms_median"], 5),
+        "forward_ms_p10": round(results["bias"]["fwd_ms_p10"], 5),
+        "forward_ms_p90": round(results["bias"]["fwd_ms_p90"], 5),
         "pack_ms": round(results["bias"]["step_ms"] - results["bias"]["fwd_ms"], 5),
         "effective_tflops": round(eff_tflops, 2),
         "job_effective_tflops": round(job_units(a["eff_flops"], world) / fwd_s / 1e12, 2),

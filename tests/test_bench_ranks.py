@@ -83,3 +83,15 @@ def test_traffic_digest_ignores_comments_only():
     assert bench.code_only(src) == bench.code_only(same.replace("2*x", "2 * x"))
     assert '"a//b /*c*/"' in bench.code_only(src)
     assert bench.code_only(src) != bench.code_only(src.replace("2 * x", "3 * x"))
+
+
+def test_percentile_matches_numpy():
+    import numpy as np
+
+    import bench
+
+    rng = np.random.default_rng(4)
+    for n in (1, 2, 5, 20, 101):
+        xs = rng.random(n).tolist()
+        for q in (0.0, 0.1, 0.5, 0.9, 1.0):
+            assert abs(bench.percentile(xs, q) - float(np.percentile(xs, 100 * q))) < 1e-12
