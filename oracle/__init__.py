@@ -77,6 +77,24 @@ class Oracle:
         raise TypeError(f"oracle takes float32 or bf16-as-uint16, got {x.dtype}")
 
     @staticmethod
+    def _bf16(a, name: str, shape) -> np.ndarray | None:
+        """bf16 bit patterns (uint16) of the given shape, C-contiguous; None stays None."""
+        if a is None:
+            return None
+        if a.dtype != np.uint16:
+            raise TypeError(f"{name} must hold bf16 bit patterns (uint16), got {a.dtype}")
+        if tuple(a.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(a.shape)}, expected {tuple(shape)}")
+        return np.ascontiguousarray(a)
+
+    @staticmethod
+    def _qk(q, k) -> tuple[np.ndarray, np.ndarray]:
+        """Q and K of one shape and one dtype, C-contiguous."""
+        if q.shape != k.shape or q.dtype != k.dtype:
+            raise ValueError(f"q {q.shape} {q.dtype} and k {k.shape} {k.dtype} differ")
+        return np.ascontiguousarray(q), np.ascontiguousarray(k)
+
+    @staticmethod
     def _rows(rows) -> np.ndarray:
         r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
         return r
@@ -106,7 +124,7 @@ class Oracle:
         B, H, N, d = q.shape
         r = self._rows(rows)
         S = np.zeros((r.size, N), dtype=np.int32)
-        q = np.ascontiguousarray(q); k = np.ascontiguousarray(k)
+        q, k = self._qk(q, k)
         rc = self.lib.oracle_scores_rows(_ptr(q), _ptr(k), self._dtype_code(q), B, H, N, d,
                                          r.size, r.ctypes.data_as(_i64p), _ptr(S))
         if rc:
@@ -122,8 +140,8 @@ class Oracle:
         B, H, N, d = q.shape
         r = self._rows(rows)
         P = np.zeros((r.size, N), dtype=np.float64)
-        q = np.ascontiguousarray(q); k = np.ascontiguousarray(k)
-        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16)
+        q, k = self._qk(q, k)
+        b = self._bf16(bias, "bias", (H, N, N))
         rc = self.lib.oracle_probs_rows(_ptr(q), _ptr(k), self._dtype_code(q), _ptr(b),
                                         float(softmax_scale), B, H, N, d,
                                         r.size, r.ctypes.data_as(_i64p), _ptr(P))
@@ -136,9 +154,9 @@ class Oracle:
         B, H, N, d = q.shape
         r = self._rows(rows)
         O = np.zeros((r.size, d), dtype=np.float64)
-        q = np.ascontiguousarray(q); k = np.ascontiguousarray(k)
-        v = np.ascontiguousarray(v, dtype=np.uint16)
-        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16)
+        q, k = self._qk(q, k)
+        v = self._bf16(v, "v", (B, H, N, d))
+        b = self._bf16(bias, "bias", (H, N, N))
         rc = self.lib.oracle_forward_rows(_ptr(q), _ptr(k), self._dtype_code(q), _ptr(b),
                                           _ptr(v), float(softmax_scale), B, H, N, d,
                                           r.size, r.ctypes.data_as(_i64p), _ptr(O))
@@ -150,9 +168,9 @@ class Oracle:
         """O fp64 [B,H,N,d] for every row."""
         B, H, N, d = q.shape
         O = np.zeros((B, H, N, d), dtype=np.float64)
-        q = np.ascontiguousarray(q); k = np.ascontiguousarray(k)
-        v = np.ascontiguousarray(v, dtype=np.uint16)
-        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16)
+        q, k = self._qk(q, k)
+        v = self._bf16(v, "v", (B, H, N, d))
+        b = self._bf16(bias, "bias", (H, N, N))
         rc = self.lib.oracle_forward(_ptr(q), _ptr(k), self._dtype_code(q), _ptr(b), _ptr(v),
                                      float(softmax_scale), B, H, N, d, _ptr(O))
         if rc:
