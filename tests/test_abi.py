@@ -273,3 +273,21 @@ def test_binding_marshals_every_call(monkeypatch):
     assert S.shape == (B, H, N, N) and calls[-1][1][2:6] == (B, H, N, d)
     binattn.ref_bf16_forward(q, q, None, v, 0.25)
     assert calls[-1][0] == "binattn_ref_bf16_forward" and calls[-1][1][5:9] == (B, H, N, d)
+
+
+@pytest.mark.parametrize("lang,std", [("c", "c99"), ("c++", "c++11")])
+def test_header_is_plain_c(tmp_path, lang, std):
+    # The boundary header needs no CUDA or torch include: it compiles as plain
+    # C99 and C++11, and a C program can take the address of every entry point.
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    inc = os.path.dirname(HEADER)
+    src = tmp_path / ("use.c" if lang == "c" else "use.cpp")
+    names = declared_functions()
+    src.write_text('#include "binattn.h"\nvoid* const table[] = {\n' +
+                   ",\n".join(f"  (void*){n}" for n in names) + "\n};\n")
+    subprocess.run([cc, f"-std={std}", "-Wall", "-Werror", "-fsyntax-only", "-I", inc, str(src)], check=True)
