@@ -5,9 +5,11 @@ Tolerance on O (bf16 output, fp32 accumulation): max |O_gpu - O_ref| <= 2e-2
 and ||O_gpu - O_ref||_2 / ||O_ref||_2 <= 5e-3, with O_ref the oracle's
 unrounded fp64 result. Where |O_ref| >= 8 the bf16 half-ulp alone (>= 2^-5)
 exceeds 2e-2; there the element bound becomes 2e-2 + half an ulp of bf16 at
-|O_ref|, reported separately.
+|O_ref|, and a warning names every case that needed it.
 """
 from __future__ import annotations
+
+import warnings
 
 import numpy as np
 import torch
@@ -55,11 +57,16 @@ def check_o(o_gpu: np.ndarray, o_ref: np.ndarray, what: str = "") -> dict:
     big = np.abs(o_ref) >= 8.0
     small_max = float(err[~big].max()) if (~big).any() else 0.0
     assert small_max <= MAX_ABS, f"{what}: max-abs {small_max:.3e} > {MAX_ABS}"
+    fallback = False
     if big.any():
         bound = MAX_ABS + bf16_half_ulp(o_ref[big])
         assert np.all(err[big] <= bound), f"{what}: large-|O| elements beyond 2e-2 + half ulp"
+        fallback = bool((err[big] > MAX_ABS).any())
+        if fallback:  # flagged, not silent: the plain 2e-2 bar did not hold there
+            warnings.warn(f"{what}: {int((err[big] > MAX_ABS).sum())} elements with |O_ref| >= 8 "
+                          f"passed only under 2e-2 + half a bf16 ulp (max-abs {float(err.max()):.3e})")
     assert rel_rms <= REL_RMS, f"{what}: rel-RMS {rel_rms:.3e} > {REL_RMS}"
-    return dict(max_abs=float(err.max()), rel_rms=rel_rms)
+    return dict(max_abs=float(err.max()), rel_rms=rel_rms, half_ulp_fallback=fallback)
 
 
 def sample_rows(B: int, H: int, N: int, n: int, seed: int = 0) -> np.ndarray:
