@@ -23,6 +23,9 @@
  *  - bf16 tensors are passed as uint16_t bit patterns.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream). Work is
  *    enqueued asynchronously; results are valid after the stream is synchronized.
+ *  - Kernels launch on the calling thread's current device (cudaSetDevice).
+ *    Every pointer and the stream must belong to that device; one-time kernel
+ *    set-up is done once per device.
  *  - Every call returns a binattn_status. Arguments are validated on the host
  *    before anything is launched; on any error nothing is launched and the
  *    outputs are untouched. No exception or abort crosses the ABI.
