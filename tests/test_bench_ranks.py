@@ -95,3 +95,26 @@ def test_percentile_matches_numpy():
         xs = rng.random(n).tolist()
         for q in (0.0, 0.1, 0.5, 0.9, 1.0):
             assert abs(bench.percentile(xs, q) - float(np.percentile(xs, 100 * q))) < 1e-12
+
+
+def test_algorithmic_work_matches_the_hand_figures():
+    # Bytes (bits + alphas + V + O + bias once) and work per forward call,
+    # against the figures worked out by hand for the five workloads:
+    # MB to 0.1, pairs to 3 digits, P.V GFLOP to 3 digits.
+    import bench
+    from diffusion_transformers_b200.synthetic import WORKLOADS
+
+    want = {  # name: (MB with bias, pairs, P.V GFLOP)
+        "tiny": (0.41, 1.31e5, 0.0168),
+        "deit_b": (43.3, 2.98e7, 3.81),
+        "vit_l384": (93.4, 1.70e8, 21.8),
+        "dit_xl_512": (75.5, 1.34e8, 19.3),
+        "dit_xl_1024": (578.8, 5.37e8, 77.3),
+    }
+    for name, (mb, pairs, gflop) in want.items():
+        a = bench.algorithmic(WORKLOADS[name], True)
+        assert round(a["bytes"] / 1e6, 1 if mb >= 1 else 2) == mb, name
+        assert abs(a["pairs"] / pairs - 1) < 5e-3, name
+        assert abs(a["pv_flops"] / 1e9 / gflop - 1) < 5e-3, name
+        assert a["eff_flops"] == 2 * a["pv_flops"] == a["pv_flops"] + a["qk_ops"]
+    assert round(bench.algorithmic(WORKLOADS["dit_xl_1024"], False)["bytes"] / 1e6, 1) == 41.9
