@@ -1,7 +1,11 @@
-"""Host logic of bench.py's multi-rank path, on CPU with gloo, world size 2.
+"""Host logic of bench.py, on CPU.
 
-Each rank draws its own batch (weak scaling) and the reported time is the max
-over ranks; no collective touches the data path.
+- The multi-rank path with gloo, world size 2: each rank draws its own batch
+  (weak scaling) and the reported time is the max over ranks; no collective
+  touches the data path.
+- The source digest that keeps the ncu traffic figure tied to the kernels.
+- The percentiles of the timed steps.
+- The algorithmic bytes and work behind the roofline.
 """
 import os
 import socket
