@@ -60,10 +60,11 @@ class Oracle:
         lib.oracle_probs_rows.argtypes = [V, V, I, V, D, L, L, L, L, L, _i64p, V]
         lib.oracle_forward_rows.argtypes = [V, V, I, V, V, D, L, L, L, L, L, _i64p, V]
         lib.oracle_forward.argtypes = [V, V, I, V, V, D, L, L, L, L, V]
+        lib.oracle_forward_spread.argtypes = [V, V, I, V, V, D, L, L, L, L, V, V]
         lib.oracle_num_threads.restype = I
         lib.oracle_set_num_threads.argtypes = [I]
         for f in ("oracle_pack", "oracle_scores_rows", "oracle_probs_rows",
-                  "oracle_forward_rows", "oracle_forward"):
+                  "oracle_forward_rows", "oracle_forward", "oracle_forward_spread"):
             getattr(lib, f).restype = I
         self.lib = lib
 
@@ -176,6 +177,21 @@ class Oracle:
         if rc:
             raise RuntimeError(f"oracle_forward failed ({rc})")
         return O
+
+    def forward_spread(self, q, k, bias, v, softmax_scale):
+        """O and its spread E, both fp64 [B,H,N,d], for every row:
+        E[b,h,i,c] = sum_j P_ij |V_jc - O_ic| (the bf16-P error scale)."""
+        B, H, N, d = q.shape
+        O = np.zeros((B, H, N, d), dtype=np.float64)
+        E = np.zeros((B, H, N, d), dtype=np.float64)
+        q, k = self._qk(q, k)
+        v = self._bf16(v, "v", (B, H, N, d))
+        b = self._bf16(bias, "bias", (H, N, N))
+        rc = self.lib.oracle_forward_spread(_ptr(q), _ptr(k), self._dtype_code(q), _ptr(b), _ptr(v),
+                                            float(softmax_scale), B, H, N, d, _ptr(O), _ptr(E))
+        if rc:
+            raise RuntimeError(f"oracle_forward_spread failed ({rc})")
+        return O, E
 
 
 _default: Oracle | None = None

@@ -35,6 +35,13 @@
  * become the top half of a float). Rows are processed in parallel with OpenMP;
  * each row's arithmetic is sequential in the order written above.
  *
+ * Besides O, oracle_forward_spread(_rows) returns, for every output element,
+ * E_ic = sum_j P_ij * |V_jc - O_ic|: how far the values a row averages lie
+ * from their average. Rounding each P_ij to an 8-bit significand (relative
+ * 2^-9), with the row sum taken from the same rounded values, moves O_ic by at
+ * most about 2^-8 * E_ic; the GPU parity tests use it as that element's bound
+ * where it exceeds the fixed one. It is a plain definition, not a method step.
+ *
  * Parity pins for each function live in the CPU test suite (exhaustive sign
  * predicate, packbits layout, Hamming identity, closed forms, invariants and an
  * independent numpy formulation on small cases).
@@ -323,6 +330,69 @@ int oracle_forward(const void *q, const void *k, int qk_dtype,
         rows[t] = (int64_t)t;
     int rc = oracle_forward_rows(q, k, qk_dtype, bias, v, softmax_scale,
                                  B, H, N, d, (long)T, rows, O);
+    free(rows);
+    return rc;
+}
+
+/*
+ * O rows as oracle_forward_rows, plus the spread E_rows[r*d + c] =
+ * sum_j P_ij * |V_jc - O_ic| of each output element (fp64). O comes from
+ * oracle_forward_rows; the probabilities are evaluated a second time for E.
+ */
+int oracle_forward_spread_rows(const void *q, const void *k, int qk_dtype,
+                               const uint16_t *bias, const uint16_t *v,
+                               double softmax_scale, long B, long H, long N, long d,
+                               long nrows, const int64_t *rows, double *O_rows, double *E_rows)
+{
+    if (!E_rows)
+        return 1;
+    int rc = oracle_forward_rows(q, k, qk_dtype, bias, v, softmax_scale, B, H, N, d, nrows, rows, O_rows);
+    if (rc)
+        return rc;
+    prep_t p;
+    if (prep_init(&p, q, k, qk_dtype, B, H, N, d)) {
+        prep_free(&p);
+        return 3;
+    }
+    int err = 0;
+    long r;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (r = 0; r < nrows; r++) {
+        double *P = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!P) {
+#pragma omp atomic write
+            err = 3;
+            continue;
+        }
+        size_t qtok = (size_t)rows[r];
+        size_t vtok0 = qtok / (size_t)N * (size_t)N;  /* key 0 of this (b, h) */
+        probs_row(&p, qtok, bias, softmax_scale, P);
+        for (long c = 0; c < d; c++) {
+            const double oc = O_rows[(size_t)r * d + c];
+            double e = 0.0;
+            for (long j = 0; j < N; j++)
+                e += P[j] * fabs(load_elem(v, ORACLE_BF16, (vtok0 + (size_t)j) * d + c) - oc);
+            E_rows[(size_t)r * d + c] = e;
+        }
+        free(P);
+    }
+    prep_free(&p);
+    return err;
+}
+
+/* All rows: O and E [B, H, N, d] in fp64. */
+int oracle_forward_spread(const void *q, const void *k, int qk_dtype,
+                          const uint16_t *bias, const uint16_t *v, double softmax_scale,
+                          long B, long H, long N, long d, double *O, double *E)
+{
+    size_t T = (size_t)B * H * N;
+    int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (T + 1));
+    if (!rows)
+        return 3;
+    for (size_t t = 0; t < T; t++)
+        rows[t] = (int64_t)t;
+    int rc = oracle_forward_spread_rows(q, k, qk_dtype, bias, v, softmax_scale,
+                                        B, H, N, d, (long)T, rows, O, E);
     free(rows);
     return rc;
 }

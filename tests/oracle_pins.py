@@ -337,6 +337,42 @@ def pin_sign_correlation_arcsin(orc):
         assert abs(off.sum() / n_off) <= 5 / math.sqrt(n_off * d), f"rho={rho}: independent tokens correlate"
 
 
+# ------------------------------------- spread of an output (tolerance scale)
+def pin_spread_uniform_is_mean_abs_deviation(orc):
+    """Uniform P (every key row of a head identical, no bias): O_i = mean_j V_j
+    and E_ic = mean_j |V_jc - mean V_c|, the mean absolute deviation."""
+    B, H, N, d = 2, 2, 9, 40
+    rng = np.random.default_rng(41)
+    q = rng.standard_normal((B, H, N, d)).astype(np.float32)
+    k = np.ascontiguousarray(np.broadcast_to(rng.standard_normal((B, H, 1, d)).astype(np.float32), (B, H, N, d)))
+    v = f32_to_bf16_bits(rng.standard_normal((B, H, N, d)).astype(np.float32) * 3)
+    O, E = orc.forward_spread(q, k, None, v, 0.9)
+    vf = _f64(v)
+    mad = np.abs(vf - vf.mean(axis=2, keepdims=True)).mean(axis=2, keepdims=True)
+    assert np.array_equal(O, orc.forward(q, k, None, v, 0.9))
+    assert np.allclose(E, np.broadcast_to(mad, E.shape), rtol=1e-12, atol=1e-14)
+
+
+def pin_spread_two_keys_closed_form(orc):
+    """N = 2, scale 0, bias row (b1, b2): P = (p, 1 - p) with
+    p = 1 / (1 + e^(b2 - b1)), and E_ic = 2 p (1 - p) |V_0c - V_1c|; a one-hot
+    bias (+40) gives E ~ 0 (at most 2 e^-40 max|V|)."""
+    B, H, N, d = 1, 3, 2, 16
+    rng = np.random.default_rng(42)
+    c = make_custom(B, H, N, d, seed=43, with_bias=False)
+    bias = f32_to_bf16_bits(rng.uniform(-2, 2, size=(H, N, N)).astype(np.float32))
+    O, E = orc.forward_spread(c["q"], c["k"], bias, c["v"], 0.0)
+    b, v = _f64(bias), _f64(c["v"])
+    for h in range(H):
+        for i in range(N):
+            p = 1.0 / (1.0 + math.exp(b[h, i, 1] - b[h, i, 0]))
+            assert np.allclose(E[0, h, i], 2 * p * (1 - p) * np.abs(v[0, h, 0] - v[0, h, 1]), rtol=1e-12, atol=1e-15)
+    onehot = np.zeros((H, N, N), dtype=np.float32)
+    onehot[:, :, 0] = 40.0
+    _, E1 = orc.forward_spread(c["q"], c["k"], f32_to_bf16_bits(onehot), c["v"], 0.0)
+    assert np.all(E1 <= 2 * math.exp(-40) * np.abs(v).max() * 2)
+
+
 ALL_PINS = [
     pin_sign_predicate_exhaustive,
     pin_pack_layout_packbits,
@@ -355,4 +391,6 @@ ALL_PINS = [
     pin_worked_example,
     pin_alpha_half_normal_mean,
     pin_sign_correlation_arcsin,
+    pin_spread_uniform_is_mean_abs_deviation,
+    pin_spread_two_keys_closed_form,
 ]

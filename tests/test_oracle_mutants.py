@@ -52,6 +52,10 @@ MUTANTS = [
      "o += P[j] * load_elem(v, ORACLE_BF16, qtok * d + c);"),
     ("last key dropped from P.V",
      "for (long j = 0; j < N; j++)\n                o +=", "for (long j = 0; j < N - 1; j++)\n                o +="),
+    ("spread without the absolute value",
+     "e += P[j] * fabs(load_elem(", "e += P[j] * (load_elem("),
+    ("spread not weighted by P",
+     "e += P[j] * fabs(", "e += fabs("),
 ]
 
 

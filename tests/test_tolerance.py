@@ -1,6 +1,7 @@
 """The O tolerance of the GPU parity tests, on CPU: max-abs 2e-2 and rel-RMS
 5e-3 against the fp64 oracle, with half a bf16 ulp more (and a warning) only
-where |O_ref| >= 8."""
+where |O_ref| >= 8, and the bf16-P spread bound (with a warning) only where
+a test passes the oracle's spread and that bound is the larger."""
 import numpy as np
 import pytest
 
@@ -18,7 +19,7 @@ def test_check_o_bars():
     rng = np.random.default_rng(0)
     ref = rng.standard_normal(4096)
     assert not check_o(ref + 1e-3, ref)["half_ulp_fallback"]
-    with pytest.raises(AssertionError, match="max-abs"):
+    with pytest.raises(AssertionError, match="beyond their bound"):
         check_o(ref + np.where(np.arange(4096) == 7, 0.021, 0.0), ref)
     ref3 = np.clip(ref, -3.0, 3.0)
     with pytest.raises(AssertionError, match="rel-RMS"):
@@ -32,5 +33,26 @@ def test_check_o_large_values_fallback_is_flagged():
     with pytest.warns(UserWarning, match="half a bf16 ulp"):
         assert check_o(got, ref)["half_ulp_fallback"]
     got[-1] = ref[-1] - 0.06
-    with pytest.raises(AssertionError, match="large-"):
+    with pytest.raises(AssertionError, match="beyond their bound"):
         check_o(got, ref)
+
+
+def test_check_o_spread_bound_is_flagged():
+    # |O| in [4, 8): half an ulp is 2^-6; with spread E = 6 the bf16-P bound
+    # is 2^-8 * 6 + 2^-6 + 1e-3 = 0.0402 (the outlier channels of ViT-L)
+    ref = np.concatenate([np.full(1000, 0.3), [5.0]])
+    spread = np.concatenate([np.full(1000, 0.5), [6.0]])
+    got = ref.copy()
+    got[-1] += 0.03
+    with pytest.raises(AssertionError, match="beyond their bound"):
+        check_o(got, ref)  # without the spread: the plain 2e-2 bar
+    with pytest.warns(UserWarning, match="spread bound"):
+        assert check_o(got, ref, spread=spread)["half_ulp_fallback"]
+    got[-1] = ref[-1] + 0.041
+    with pytest.raises(AssertionError, match="beyond their bound"):
+        check_o(got, ref, spread=spread)
+    # small spreads never loosen the 2e-2 bar
+    got = ref.copy()
+    got[3] += 0.021
+    with pytest.raises(AssertionError, match="beyond their bound"):
+        check_o(got, ref, spread=spread)
