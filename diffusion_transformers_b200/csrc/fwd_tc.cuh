@@ -143,6 +143,10 @@ struct Params {
   // only): each row's sign words and alpha_q come from pack_row_bf16 in the
   // kernel, and qb / aq are not read. Null: qb / aq from binattn_pack.
   const uint16_t* qh = nullptr;
+  // Test only (the entry point that makes a bounded wait run out): with
+  // stall_after >= 0 the TMA producer of the 64-key pipeline issues nothing
+  // from key tile stall_after on, so the stage's consumers time out.
+  int stall_after = -1;
 };
 
 // Named barrier 1 over the load-mode loader warps with an AND reduction.
@@ -744,9 +748,11 @@ fwd_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tm_v,
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float2 a = __ffma2_rn(xs[c0 / 2 + e], l2e2, nm2);
-          const float2 pp = make_float2(ex2(a.x), ex2(a.y));
-          ls[e & 3] = __fadd2_rn(ls[e & 3], pp);
-          pk[e] = pack_bf16x2(pp.x, pp.y);
+          pk[e] = pack_bf16x2(ex2(a.x), ex2(a.y));
+          // l sums the bf16 P the P.V MMA multiplies, so that the weights of
+          // O = (P V) / l sum to one exactly
+          ls[e & 3] = __fadd2_rn(ls[e & 3], make_float2(__uint_as_float(pk[e] << 16),
+                                                        __uint_as_float(pk[e] & 0xFFFF0000u)));
         }
         tmem_st16(s_col + c0 / 2, pk);
       }

@@ -298,3 +298,59 @@ def test_forward_fused_fp32_q_and_full_size():
         binattn.device_status()
         assert torch.equal(got.view(torch.int16), want.view(torch.int16)), f"dit_xl_1024 bias={with_bias}"
         del q, k, v, bias, qb, kb, aq, ak, want, got
+
+
+# ------------------------------------------- the benchmarked calls, every row
+# bench.py times binattn_forward_ws with a workspace of
+# binattn_forward_workspace_bytes: at DiT-XL/2 1024 px that is the full waves
+# of 256-row pairs, the key-split tail pairs and the combine kernel, with and
+# without the bias; on the other workloads the padded-bias route or the plain
+# forward. Each call is compared here with the oracle on every output row, at
+# the workload's own size and seed, together with binattn_forward (no
+# workspace) and binattn_forward_fused_ws on the same inputs.
+BENCHMARKED = [("dit_xl_1024", True), ("dit_xl_1024", False), ("dit_xl_512", True),
+               ("vit_l384", True), ("deit_b", True), ("tiny", True)]
+
+
+@pytest.mark.parametrize("name,with_bias", BENCHMARKED)
+def test_benchmarked_calls_every_row(orc, name, with_bias):
+    inp = make_inputs(name, with_bias=with_bias)
+    B, H, N, d = inp["B"], inp["H"], inp["N"], inp["d"]
+    ref, spread = orc.forward_spread(inp["q"], inp["k"], inp["bias"] if with_bias else None, inp["v"],
+                                     inp["softmax_scale"])
+    out, need = _run_ws(inp, with_bias=with_bias)
+    if name == "dit_xl_1024":
+        assert need > 0  # the split tail runs, as in the bench
+    check_o(bf16_to_f64(out), ref, f"forward_ws {name} bias={with_bias}", spread)
+    del out
+    r = run_path(inp, engine="auto", with_bias=with_bias)
+    check_o(bf16_to_f64(r["out"]), ref, f"forward {name} bias={with_bias}", spread)
+    if inp["q"].dtype == np.uint16:
+        got = binattn.forward_fused_ws(r["q"], r["kb"], r["ak"], r["bias"], r["v"], inp["softmax_scale"])
+        torch.cuda.synchronize()
+        binattn.device_status()
+        check_o(bf16_to_f64(got), ref, f"forward_fused_ws {name} bias={with_bias}", spread)
+
+
+# ------------------------------------------------- a bounded wait runs out
+# The TMA producer stops after two key tiles: every CTA's consumers give up
+# once their bounded waits run out (about 2 s), the CTA drains its own
+# tensor-core work, frees its tensor memory and returns, and the device status
+# reports the timeout. The context stays usable: the next call on it meets the
+# oracle.
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_bounded_wait_runs_out_and_context_survives(orc, with_bias):
+    c = make_custom(1, 2, 512, 72, seed=123, with_bias=with_bias, bias_std=0.5)
+    q, k, v = dev(c["q"]), dev(c["k"]), dev(c["v"])
+    bias = dev(c["bias"]) if with_bias else None
+    qb, aq = binattn.pack(q)
+    kb, ak = binattn.pack(k)
+    binattn.device_status()
+    binattn.test_wait_timeout(qb, kb, aq, ak, bias, v, c["softmax_scale"], stall_after=2)
+    with pytest.raises(binattn.BinattnError) as exc:
+        binattn.device_status()
+    assert exc.value.status == 7  # BINATTN_ERR_TIMEOUT
+    binattn.device_status()  # read and cleared
+    ref = orc.forward(c["q"], c["k"], c["bias"] if with_bias else None, c["v"], c["softmax_scale"])
+    r = run_path(c, engine="tc", with_bias=with_bias)
+    check_o(bf16_to_f64(r["out"]), ref, f"after timeout bias={with_bias}")
