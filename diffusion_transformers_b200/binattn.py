@@ -26,7 +26,7 @@ EXPORTS = (
     "binattn_forward_ws", "binattn_forward_static_ws", "binattn_forward_fused_workspace_bytes",
     "binattn_forward_fused_ws", "binattn_scores_debug",
     "binattn_ref_bf16_forward", "binattn_device_status", "binattn_strerror",
-    "binattn_last_error_message", "binattn_abi_version",
+    "binattn_last_error_message", "binattn_abi_version", "binattn_test_wait_timeout",
 )
 
 
@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
     L.binattn_forward_fused_ws.argtypes = [P, I, P, P, P, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
     L.binattn_scores_debug.argtypes = [P, P, I, I, I, I, P, I, P]
     L.binattn_ref_bf16_forward.argtypes = [P, P, P, P, F, I, I, I, I, P, P]
+    L.binattn_test_wait_timeout.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, I, P]
     L.binattn_device_status.argtypes = [P]
     L.binattn_strerror.argtypes = [I]
     L.binattn_strerror.restype = ctypes.c_char_p
@@ -72,7 +73,8 @@ def lib() -> ctypes.CDLL:
     for name in ("binattn_pack", "binattn_forward", "binattn_forward_engine", "binattn_forward_ws",
                  "binattn_forward_static_ws", "binattn_forward_fused_ws",
                  "binattn_scores_debug",
-                 "binattn_ref_bf16_forward", "binattn_device_status", "binattn_abi_version"):
+                 "binattn_ref_bf16_forward", "binattn_device_status", "binattn_abi_version",
+                 "binattn_test_wait_timeout"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -293,6 +295,25 @@ def ref_bf16_forward(q: torch.Tensor, k: torch.Tensor, bias: torch.Tensor | None
         _check(lib().binattn_ref_bf16_forward(_ptr(q), _ptr(k), _ptr(bias), _ptr(v), float(softmax_scale),
                                               B, H, N, d, _ptr(out), _stream(stream, dev)),
                "binattn_ref_bf16_forward")
+    return out
+
+
+def test_wait_timeout(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor,
+                      alpha_k: torch.Tensor, bias: torch.Tensor | None, v: torch.Tensor,
+                      softmax_scale: float, stall_after: int, out: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """Test only: the 64-key forward with its TMA producer stopped at key tile
+    stall_after, so that its bounded waits run out (binattn_test_wait_timeout).
+    `out` is undefined afterwards; the timeout shows in device_status()."""
+    B, H, N, d = v.shape
+    dev = _forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, out)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().binattn_test_wait_timeout(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k),
+                                               _ptr(bias), _ptr(v), float(softmax_scale), B, H, N, d,
+                                               _ptr(out), int(stall_after), _stream(stream, dev)),
+               "binattn_test_wait_timeout")
     return out
 
 

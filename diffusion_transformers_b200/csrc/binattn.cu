@@ -432,6 +432,22 @@ int binattn_ref_bf16_forward(const uint16_t* q, const uint16_t* k, const uint16_
   return ok();
 }
 
+int binattn_test_wait_timeout(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
+                              const float* alpha_k, const uint16_t* bias, const uint16_t* v,
+                              float softmax_scale, int B, int H, int N, int d, uint16_t* out,
+                              int stall_after, void* stream) {
+  if (int rc = check_forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out))
+    return rc;
+  if (!binattn::tc2::supported(d, N, bias != nullptr, false))
+    return fail(BINATTN_ERR_UNSUPPORTED, "the 64-key pipeline does not take d = %d, N = %d", d, N);
+  if (stall_after < 0) return fail(BINATTN_ERR_ARG, "stall_after must be >= 0");
+  std::string msg;
+  const int rc = binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out,
+                                      static_cast<cudaStream_t>(stream), &msg, 0, nullptr, nullptr, stall_after);
+  if (rc) return fail(rc, "%s", msg.c_str());
+  return ok();
+}
+
 int binattn_device_status(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(st);

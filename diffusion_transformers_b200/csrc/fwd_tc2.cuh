@@ -338,6 +338,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
     if (lane == 0 && (!kDump || kBias)) {
       bool ok = true;
       for (int kt = 0; ok && kt < nkt; ++kt) {
+        if (p.stall_after >= 0 && kt >= p.stall_after) break;  // test only
         const int j0 = key0 + kt * kKeys;
         if constexpr (!kDump) {
           const int s = kt % kKS;
@@ -886,9 +887,9 @@ inline size_t split_part_bytes(int B, int H, int N, int d) {
 inline int forward_tc2(const uint32_t* qb, const uint32_t* kb, const float* aq, const float* ak,
                        const uint16_t* bias, const uint16_t* v, float scale, int B, int H, int N, int d,
                        uint16_t* out, cudaStream_t st, std::string* msg, int bias_ld = 0,
-                       float* part = nullptr, const uint16_t* qh = nullptr) {
+                       float* part = nullptr, const uint16_t* qh = nullptr, int stall_after = -1) {
   tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d, bias_ld, 0, 0,
-                 nullptr, qh};
+                 nullptr, qh, stall_after};
   const tc2::SplitPlan plan = part ? tc2::split_plan(B, H, N) : tc2::SplitPlan{tc2::total_pairs(B, H, N), 0};
   auto run = [&](int ctas) {
     return bias ? tc2::dispatch_dv<tc2::kModeBin, true>(prm, ctas, st, msg)

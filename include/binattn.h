@@ -261,6 +261,24 @@ int binattn_ref_bf16_forward(const uint16_t *q, const uint16_t *k,
                              uint16_t *out, void *stream);
 
 /*
+ * binattn_test_wait_timeout — test only: the binary forward on the 64-key
+ * pipeline (d % 8 == 0, d <= 80; with a bias, N % 8 == 0), arguments as for
+ * binattn_forward, except that its TMA producer issues nothing from key tile
+ * stall_after (>= 0) on. The consumers of that stage then wait for data that
+ * never comes, until their bounded waits run out (about 2 s of SM clock):
+ * each CTA records BINATTN_ERR_TIMEOUT in the device status word, waits
+ * (bounded) for its own tensor-core work, frees its tensor memory and
+ * returns; `out` is undefined. binattn_device_status(stream) then returns
+ * BINATTN_ERR_TIMEOUT and the context stays usable. The pages have no
+ * counterpart of this call; it exists to test the failure path.
+ */
+int binattn_test_wait_timeout(const uint32_t *q_bits, const uint32_t *k_bits,
+                              const float *alpha_q, const float *alpha_k,
+                              const uint16_t *bias, const uint16_t *v, float softmax_scale,
+                              int B, int H, int N, int d, uint16_t *out,
+                              int stall_after, void *stream);
+
+/*
  * binattn_device_status — synchronizes `stream`, then reads and clears the
  * library's device status word. Returns BINATTN_OK, or BINATTN_ERR_TIMEOUT when
  * a kernel abandoned a bounded wait (its outputs are then undefined), or
