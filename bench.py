@@ -50,6 +50,10 @@ def parse():
     ap.add_argument("--impl", default="binattn", choices=["binattn", "reference"])
     ap.add_argument("--workload", default="dit_xl_1024", choices=sorted(WORKLOADS))
     ap.add_argument("--engine", default="auto")
+    ap.add_argument("--shard", default="none", choices=["none", "heads"],
+                    help="with N > 1: none = every rank runs its own batch (weak scaling); heads = one "
+                         "batch split by heads, rank r holding only its heads' Q, K, V and bias (strong "
+                         "scaling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the bounded oracle sample")
@@ -82,6 +86,53 @@ def algorithmic(w, with_bias=True):
     pack_bytes = 2 * (BH * N * d * 2 + BH * N * W * 4 + BH * N * 4)
     return dict(pairs=pairs, qk_ops=2 * d * pairs, pv_flops=2 * d * pairs,
                 eff_flops=4 * d * pairs, bytes=bytes_, pack_bytes=pack_bytes)
+
+
+# The binary QK^T runs on tcgen05.mma kind::f8f6f4 with e4m3 +-1 operands. Its
+# dense rate is twice the bf16 rate (NVIDIA's nominal 4.5 against 2.25 PFLOP/s
+# per GPU; on this part an e4m3 M=128 N=128 K=32 MMA and a bf16 M=128 N=128
+# K=16 MMA both take 64 cycles), so its peak is 2x the measured bf16 figure.
+E4M3_OVER_BF16 = 2.0
+MUFU_EXP_PER_CLK_PER_SM = 16  # ex2 throughput of the special-function unit
+
+
+def roofline_terms(w, with_bias, peaks, n_sm=148, sm_mhz=None):
+    """Roofline of one forward call: T_roof = max(T_mem, T_QK + T_PV), with
+    T_mem = algorithmic bytes / HBM peak, T_PV = P.V flops / bf16 peak and
+    T_QK = binary QK ops / e4m3 peak (the pipe the scores run on). The exp
+    floor (one ex2 per pair on the special-function unit) is reported beside
+    it; it is not part of T_roof."""
+    a = algorithmic(w, with_bias)
+    bf16 = peaks["bf16_tflops"] * 1e12
+    e4m3 = E4M3_OVER_BF16 * bf16
+    t_mem = a["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_pv = a["pv_flops"] / bf16
+    t_qk = a["qk_ops"] / e4m3
+    t_tensor = t_pv + t_qk
+    clk = (sm_mhz or peaks.get("sm_max_mhz") or 1965.0) * 1e6
+    t_mufu = a["pairs"] / (MUFU_EXP_PER_CLK_PER_SM * n_sm * clk)
+    return dict(t_mem=t_mem, t_pv=t_pv, t_qk=t_qk, t_tensor=t_tensor, t_roof=max(t_mem, t_tensor),
+                t_mufu=t_mufu, bound="hbm" if t_mem >= t_tensor else "tensor",
+                tensor_peak_tflops=(a["qk_ops"] + a["pv_flops"]) / t_tensor / 1e12, work=a)
+
+
+def roofline_line(w, with_bias, peaks, fwd_s, n_sm=148, sm_mhz=None):
+    """The bench line's roofline object for a forward call of fwd_s seconds:
+    frac = T_roof / fwd_s. Bound hbm: achieved = algorithmic bytes / time
+    against the HBM peak. Bound tensor: achieved = (QK ops + P.V flops) / time
+    against the blended peak (QK ops + P.V flops) / (T_QK + T_PV)."""
+    r = roofline_terms(w, with_bias, peaks, n_sm, sm_mhz)
+    a = r["work"]
+    if r["bound"] == "hbm":
+        achieved, peak, unit = a["bytes"] / fwd_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved, peak, unit = (a["qk_ops"] + a["pv_flops"]) / fwd_s / 1e12, r["tensor_peak_tflops"], "TFLOP/s"
+    return {"bound": r["bound"], "achieved": round(achieved, 2), "peak": round(peak, 2), "unit": unit,
+            "frac": round(r["t_roof"] / fwd_s, 4),
+            "t_roof_us": round(r["t_roof"] * 1e6, 2), "t_mem_us": round(r["t_mem"] * 1e6, 2),
+            "t_qk_us": round(r["t_qk"] * 1e6, 2), "t_pv_us": round(r["t_pv"] * 1e6, 2),
+            "t_exp_floor_us": round(r["t_mufu"] * 1e6, 2),
+            "exp_floor_frac": round(r["t_mufu"] / fwd_s, 4)}
 
 
 # DRAM traffic of one forward call from one ncu capture (dram__bytes_read.sum +
@@ -138,8 +189,10 @@ def measured_peaks():
         with open(path) as f:
             p = json.load(f)
         return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"],
-                    bf16_tflops_sustained=p.get("bf16_tflops_sustained"), source="measured")
-    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+                    bf16_tflops_sustained=p.get("bf16_tflops_sustained"),
+                    sm_max_mhz=p.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, sm_max_mhz=1965.0,
+                source="fallback")
 
 
 # ------------------------------------------------------------------ clocks
@@ -303,6 +356,7 @@ def time_configs(names, args, rank, world, dev, stream, peaks, flush, max_over_r
 
     rows = []
     steps = max(1, min(args.steps, 10))
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
     for name in names:
         w = WORKLOADS[name]
         inp = make_inputs(w, with_bias=True, seed=rank_seed(w, rank))
@@ -342,7 +396,7 @@ def time_configs(names, args, rank, world, dev, stream, peaks, flush, max_over_r
         step_ms = max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in ev) / steps)
         fwd_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / steps)
         a = algorithmic(w, True)
-        t_roof = max(a["bytes"] / (peaks["hbm_gbs"] * 1e9), a["eff_flops"] / (peaks["bf16_tflops"] * 1e12))
+        t_roof = roofline_terms(w, True, peaks, n_sm)["t_roof"]
         rows.append({"workload": name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bias": True,
                      "call": "binattn_forward_ws" if ws is not None else "binattn_forward",
                      "forward_ms": round(fwd_ms, 5), "step_ms": round(step_ms, 5),
@@ -352,7 +406,20 @@ def time_configs(names, args, rank, world, dev, stream, peaks, flush, max_over_r
     return rows
 
 
-def run_gpu(args, w, rank, world, local_rank):
+def rank_inputs(w, rank, world, shard_mode):
+    """This rank's workload and inputs. Replicas: the whole workload on its own
+    seed. Heads: one batch (the workload's seed on every rank) of which this
+    rank holds heads head_range(H, world, rank) only, bias slice included."""
+    import dataclasses
+
+    from diffusion_transformers_b200 import shard
+    if shard_mode == "heads" and world > 1:
+        inp = shard.shard_inputs(make_inputs(w, with_bias=True, seed=w.seed), world, rank)
+        return dataclasses.replace(w, H=inp["H"]), inp
+    return w, make_inputs(w, with_bias=True, seed=rank_seed(w, rank))
+
+
+def run_gpu(args, w_job, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     from diffusion_transformers_b200 import binattn
@@ -362,7 +429,8 @@ def run_gpu(args, w, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     peaks = measured_peaks()
 
-    inp = make_inputs(w, with_bias=True, seed=rank_seed(w, rank))
+    sharded = args.shard == "heads" and world > 1
+    w, inp = rank_inputs(w_job, rank, world, args.shard)
 
     def to_dev(x):
         if x.dtype == np.uint16:
@@ -524,8 +592,8 @@ def run_gpu(args, w, rank, world, local_rank):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
 
     # the other workloads of the parity suite, timed the same way (forward with bias)
-    others = time_configs([n for n in WORKLOADS if n != w.name], args, rank, world, dev, stream, peaks,
-                          flush, max_over_ranks)
+    others = [] if sharded else time_configs([n for n in WORKLOADS if n != w.name], args, rank, world, dev,
+                                             stream, peaks, flush, max_over_ranks)
 
     if rank != 0:
         return
@@ -534,24 +602,22 @@ def run_gpu(args, w, rank, world, local_rank):
     fwd_s = results["bias"]["fwd_ms"] * 1e-3
     eff_tflops = a["eff_flops"] / fwd_s / 1e12
     fwd0_s = results["no_bias"]["fwd_ms"] * 1e-3
-    peak_t = peaks["bf16_tflops"]
-    t_mem = a["bytes"] / (peaks["hbm_gbs"] * 1e9)
-    t_tensor = a["eff_flops"] / (peak_t * 1e12)
-    bound = "hbm" if t_mem > t_tensor else "tensor"
-    if bound == "hbm":
-        achieved, peak, unit = a["bytes"] / fwd_s / 1e9, peaks["hbm_gbs"], "GB/s"
-    else:
-        achieved, peak, unit = eff_tflops, peak_t, "TFLOP/s"
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    roof = roofline_line(w, True, peaks, fwd_s, n_sm)
+    roof0 = roofline_line(w, False, peaks, fwd0_s, n_sm)
     line = {
         "metric": METRIC,
         "value": round(results["bias"]["step_ms"], 5),
         "unit": "ms",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(results["bias"]["step_ms"], 5),
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": False, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
         "dtype": "bf16", "dtype_detail": "1-bit Q/K scores (exact int), fp32 softmax, bf16 P.V, fp32 accumulate",
         "data": "synthetic",
-        "config": workload_config(w, True) | {"engine": args.engine, "parallelism": f"replicas x{world}",
+        "config": workload_config(w_job, True) | {"engine": args.engine,
+                                                  "parallelism": (f"heads sharded x{world} ({w.H} per rank, "
+                                                                  "no data-path collective)") if sharded
+                                                  else f"replicas x{world}",
                                               "call": "binattn_forward_ws" if ws["bias"] is not None
                                               else "binattn_forward"},
         "forward_ms": round(results["bias"]["fwd_ms"], 5),
@@ -560,21 +626,24 @@ def run_gpu(args, w, rank, world, local_rank):
         "forward_ms_p90": round(results["bias"]["fwd_ms_p90"], 5),
         "pack_ms": round(results["bias"]["step_ms"] - results["bias"]["fwd_ms"], 5),
         "effective_tflops": round(eff_tflops, 2),
-        "job_effective_tflops": round(job_units(a["eff_flops"], world) / fwd_s / 1e12, 2),
+        "job_effective_tflops": round((algorithmic(w_job, True)["eff_flops"] if sharded
+                                       else job_units(a["eff_flops"], world)) / fwd_s / 1e12, 2),
         "fused_q_step": dict(fused, step="pack(K) + binattn_forward_fused_ws (Q binarised in the forward)"),
         "no_bias": {"ms_per_step": round(results["no_bias"]["step_ms"], 5),
                     "forward_ms": round(results["no_bias"]["fwd_ms"], 5),
-                    "effective_tflops": round(a0["eff_flops"] / fwd0_s / 1e12, 2)},
+                    "effective_tflops": round(a0["eff_flops"] / fwd0_s / 1e12, 2),
+                    "roofline": roof0},
         "bf16_reference": ref,
         "other_workloads": others,
-        "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-                     "frac": round(achieved / peak, 4),
-                     "traffic": ncu_traffic(f"{w.name}/bias"),
-                     "traffic_unit": "bytes per forward call (its 3 launches)",
-                     "algorithmic_bytes": a["bytes"],
-                     "kernel": "binattn forward (with bias)",
-                     "peak_source": peaks["source"] + " (burst)",
-                     "t_mem_us": round(t_mem * 1e6, 2), "t_tensor_us": round(t_tensor * 1e6, 2)},
+        "roofline": roof | {
+            "traffic": ncu_traffic(f"{w.name}/bias"),
+            "traffic_unit": "bytes per forward call (its 3 launches)",
+            "algorithmic_bytes": a["bytes"],
+            "kernel": "binattn forward (with bias)",
+            "peak_source": (peaks["source"] + " (burst): HBM copy GB/s; bf16 TFLOP/s for P.V, "
+                            f"x{E4M3_OVER_BF16:g} for the e4m3 QK pipe (nominal 4.5/2.25 PFLOP/s)"),
+            "t_exp_floor_basis": f"1 ex2 per pair at {MUFU_EXP_PER_CLK_PER_SM}/clk/SM, {n_sm} SMs, "
+                                 f"{peaks.get('sm_max_mhz', 1965.0):g} MHz"},
         "e2e": {"value": round(e2e_ms, 4), "unit": "ms",
                 "h2d_bytes_per_step": int(3 * B * H * N * d * 2),
                 "d2h_bytes_per_step": int(B * H * N * d * 2)},

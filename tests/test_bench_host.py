@@ -11,6 +11,7 @@ import os
 import socket
 import sys
 
+import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
@@ -122,3 +123,42 @@ def test_algorithmic_work_matches_the_hand_figures():
         assert abs(a["pv_flops"] / 1e9 / gflop - 1) < 5e-3, name
         assert a["eff_flops"] == 2 * a["pv_flops"] == a["pv_flops"] + a["qk_ops"]
     assert round(bench.algorithmic(WORKLOADS["dit_xl_1024"], False)["bytes"] / 1e6, 1) == 41.9
+
+
+def test_rank_inputs_heads_shard_one_batch():
+    # --shard heads: every rank slices the same batch (the workload's seed) and
+    # holds only its heads; replicas: every rank its own seed, all heads
+    import bench
+    from diffusion_transformers_b200.synthetic import WORKLOADS, make_inputs
+
+    w = WORKLOADS["tiny"]
+    full = make_inputs(w, with_bias=True, seed=w.seed)
+    parts = [bench.rank_inputs(w, r, 2, "heads") for r in range(2)]
+    assert [p[0].H for p in parts] == [1, 1]
+    q = np.concatenate([p[1]["q"] for p in parts], axis=1)
+    b = np.concatenate([p[1]["bias"] for p in parts], axis=0)
+    assert np.array_equal(q, full["q"]) and np.array_equal(b, full["bias"])
+    w1, inp1 = bench.rank_inputs(w, 1, 2, "none")
+    assert w1.H == w.H and not np.array_equal(inp1["q"], full["q"])
+    assert bench.rank_inputs(w, 0, 1, "heads")[0].H == w.H
+
+
+def test_roofline_prices_qk_at_the_e4m3_pipe():
+    # T_roof = max(T_mem, T_QK + T_PV), T_QK at twice the bf16 rate (the e4m3
+    # pipe the binary scores run on); frac = T_roof / time
+    import bench
+    from diffusion_transformers_b200.synthetic import WORKLOADS
+
+    peaks = dict(hbm_gbs=6540.8, bf16_tflops=1622.9, sm_max_mhz=1965.0)
+    w = WORKLOADS["dit_xl_1024"]
+    r = bench.roofline_terms(w, True, peaks)
+    assert abs(r["t_qk"] * 2 - r["t_pv"]) < 1e-15
+    assert abs(r["t_mem"] * 1e6 - 88.49) < 0.01 and abs(r["t_tensor"] * 1e6 - 71.45) < 0.01
+    assert r["bound"] == "hbm" and r["t_roof"] == r["t_mem"]
+    assert abs(r["t_mufu"] * 1e6 - 115.38) < 0.01
+    line = bench.roofline_line(w, True, peaks, 309e-6)
+    assert abs(line["frac"] - 0.2864) < 1e-4 and line["unit"] == "GB/s"
+    r0 = bench.roofline_terms(w, False, peaks)
+    assert r0["bound"] == "tensor"
+    line0 = bench.roofline_line(w, False, peaks, 2 * r0["t_tensor"])
+    assert line0["frac"] == 0.5 and abs(line0["achieved"] * 2 - line0["peak"]) < 0.02
