@@ -17,8 +17,9 @@ from . import build as _build
 
 OK = 0
 F32, BF16 = 0, 1
-ENGINE_AUTO, ENGINE_SIMT, ENGINE_POPC_TC, ENGINE_TC = 0, 1, 2, 3
-ENGINES = {"auto": ENGINE_AUTO, "simt": ENGINE_SIMT, "popc_tc": ENGINE_POPC_TC, "tc": ENGINE_TC}
+ENGINE_AUTO, ENGINE_SIMT, ENGINE_POPC_TC, ENGINE_TC, ENGINE_TC_BIASED = 0, 1, 2, 3, 4
+ENGINES = {"auto": ENGINE_AUTO, "simt": ENGINE_SIMT, "popc_tc": ENGINE_POPC_TC, "tc": ENGINE_TC,
+           "tc_biased": ENGINE_TC_BIASED}
 
 # Every symbol include/binattn.h declares.
 EXPORTS = (

@@ -154,12 +154,13 @@ int binattn_pack(const void* x, int dtype, int B, int H, int N, int d, uint32_t*
     else binattn::pack_kernel<float, false><<<grid, binattn::kPackThreads, 0, st>>>(xf, n_tokens, d, W, bits, alpha);
   } else if (d % 8 == 0) {  // whole 16-byte chunks per token: one thread per token
     const uint16_t* xb = static_cast<const uint16_t*>(x);
-    const unsigned rgrid = static_cast<unsigned>((n_tokens + binattn::kPackThreads - 1) / binattn::kPackThreads);
+    constexpr int kT = binattn::kRowsTokens;
+    const unsigned rgrid = static_cast<unsigned>((n_tokens + kT - 1) / kT);
     switch (W) {
-      case 1: binattn::pack_bf16_rows_kernel<1><<<rgrid, binattn::kPackThreads, 0, st>>>(xb, n_tokens, d, bits, alpha); break;
-      case 2: binattn::pack_bf16_rows_kernel<2><<<rgrid, binattn::kPackThreads, 0, st>>>(xb, n_tokens, d, bits, alpha); break;
-      case 3: binattn::pack_bf16_rows_kernel<3><<<rgrid, binattn::kPackThreads, 0, st>>>(xb, n_tokens, d, bits, alpha); break;
-      default: binattn::pack_bf16_rows_kernel<4><<<rgrid, binattn::kPackThreads, 0, st>>>(xb, n_tokens, d, bits, alpha); break;
+      case 1: binattn::pack_bf16_rows_kernel<1><<<rgrid, kT, 0, st>>>(xb, n_tokens, d, bits, alpha); break;
+      case 2: binattn::pack_bf16_rows_kernel<2><<<rgrid, kT, 0, st>>>(xb, n_tokens, d, bits, alpha); break;
+      case 3: binattn::pack_bf16_rows_kernel<3><<<rgrid, kT, 0, st>>>(xb, n_tokens, d, bits, alpha); break;
+      default: binattn::pack_bf16_rows_kernel<4><<<rgrid, kT, 0, st>>>(xb, n_tokens, d, bits, alpha); break;
     }
   } else {
     const uint16_t* xb = static_cast<const uint16_t*>(x);
@@ -395,13 +396,20 @@ int binattn_scores_debug(const uint32_t* q_bits, const uint32_t* k_bits, int B, 
         case 3: return launch_scores_popc<3>(q_bits, k_bits, B, H, N, d, S, st);
         default: return launch_scores_popc<4>(q_bits, k_bits, B, H, N, d, S, st);
       }
-    case BINATTN_ENGINE_TC: {
+    case BINATTN_ENGINE_TC:
+    case BINATTN_ENGINE_TC_BIASED: {
       if (!binattn::tc_supported(d))
         return fail(BINATTN_ERR_UNSUPPORTED, "engine TC needs d %% 8 == 0 (d = %d)", d);
+      // the kernel the TC forward runs for this shape: without a bias the
+      // 128-key pipeline, with one the 64-key pipeline, else the load-mode one
       std::string msg;
-      int rc = binattn::tc2::supported(d, N, false, false)
-                   ? binattn::scores_tc2(q_bits, k_bits, B, H, N, d, S, st, &msg)
-                   : binattn::scores_tc(q_bits, k_bits, B, H, N, d, S, st, &msg);
+      int rc;
+      if (engine == BINATTN_ENGINE_TC && binattn::tc3::supported(d, N, false))
+        rc = binattn::scores_tc3(q_bits, k_bits, B, H, N, d, S, st, &msg);
+      else if (binattn::tc2::supported(d, N, false, false))
+        rc = binattn::scores_tc2(q_bits, k_bits, B, H, N, d, S, st, &msg);
+      else
+        rc = binattn::scores_tc(q_bits, k_bits, B, H, N, d, S, st, &msg);
       if (rc) return fail(rc, "%s", msg.c_str());
       return ok();
     }

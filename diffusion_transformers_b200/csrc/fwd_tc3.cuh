@@ -88,7 +88,8 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchReg
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 5.545177444479562f;  // 8 ln 2
 
-constexpr int kModeBin = 0;  // binary forward (the only mode of this pipeline)
+constexpr int kModeBin = 0;   // binary forward
+constexpr int kModeDump = 2;  // binary scores only (debug): the same QK^T, S written to global memory
 
 inline bool supported(int d, int N, bool with_bias, int bias_ld = 0) {
   if (d % 8 != 0 || d > 80) return false;
@@ -196,7 +197,8 @@ fwd_tc3_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   using L = Layout<DV, kMode, kBias>;
   constexpr int kKS = L::kKS, kBS = L::kBS;
   static_assert(DV % 16 == 0 && DV <= 96, "P.V N");
-  static_assert(kMode == kModeBin, "binary forward only");
+  static_assert(kMode == kModeBin || kMode == kModeDump, "binary forward or its scores");
+  constexpr bool kDump = kMode == kModeDump;
   static_assert(L::kKA >= 16 && L::kKB >= 16, "both parts of P hold keys");
   static_assert(kKS >= 2 && kKS <= 4 && kBS <= 2, "stages / barrier slots");
 
@@ -249,7 +251,7 @@ fwd_tc3_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kKS; ++s) {
-      mbar_init(&kv_full[s], 33);
+      mbar_init(&kv_full[s], kDump ? 32 : 33);  // the expander's lanes (+ the V copy's arrive)
       mbar_init(&kv_empty[s], 2);
     }
     for (int i = 0; i < kBS * 2; ++i) {
@@ -293,7 +295,7 @@ fwd_tc3_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         pack_row_bf16_w(p.qh + (tok0 + row) * d, d, W, qw, aq_row);  // Q binarised here
       } else {
         for (int w = 0; w < W; ++w) qw[w] = p.qb[(tok0 + row) * W + w];
-        aq_row = p.aq[tok0 + row];
+        if (!kDump) aq_row = p.aq[tok0 + row];  // the score dump has no alphas
       }
     }
     for (int w = 0; w < W; ++w) {
@@ -323,7 +325,7 @@ fwd_tc3_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
    if (warp == kTmaWarp) {
     // ------------------------------------ V (and reference K), bias boxes
-    if (lane == 0) {
+    if (lane == 0 && !kDump) {
       bool ok = true;
       for (int kt = 0; ok && kt < nkt; ++kt) {
         const int j0 = key0 + kt * kKeys;
@@ -367,7 +369,7 @@ fwd_tc3_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
           const bool in = kt < nkt && key < N;
 #pragma unroll
           for (int w = 0; w < 3; ++w) tr.wd[u][w] = (in && w < W) ? __ldg(p.kb + (tok0 + key) * W + w) : 0u;
-          tr.ak[u] = in ? __ldg(p.ak + tok0 + key) : 0.f;
+          tr.ak[u] = (!kDump && in) ? __ldg(p.ak + tok0 + key) : 0.f;  // the score dump has no alphas
         }
       };
       TileRegs cur, n1;
@@ -444,8 +446,11 @@ fwd_tc3_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         // O_tt += P_A V(keys 0 .. KA): P part A over S columns [0, KA / 2)
         if (!(ok = mbar_wait(&pa_full[tt], kt & 1, abort))) break;
         tc_fence_after();
-        for (int ks = 0; ks < KA / 16; ++ks)
-          mma_ts(base_t + 128, base_t + ks * 8, smem_desc(v_base + ks * 256, 128, 2048), kIdPV, (kt > 0 || ks > 0));
+        if constexpr (!kDump) {
+          for (int ks = 0; ks < KA / 16; ++ks)
+            mma_ts(base_t + 128, base_t + ks * 8, smem_desc(v_base + ks * 256, 128, 2048), kIdPV,
+                   (kt > 0 || ks > 0));
+        }
         // then QK^T(kt + 1) over all of S: part A of P has been read (the
         // tensor pipe runs this thread's MMAs in order) and part B is elsewhere
         if (more) {
@@ -455,9 +460,11 @@ fwd_tc3_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         // O_tt += P_B V(keys KA .. 128): P part B in its own columns
         if (!(ok = mbar_wait(&pb_full[tt], kt & 1, abort))) break;
         tc_fence_after();
-        for (int ks = 0; ks < KB / 16; ++ks)
-          mma_ts(base_t + 128, base_t + L::kPB0 + ks * 8, smem_desc(v_base + (KA / 16 + ks) * 256, 128, 2048),
-                 kIdPV, 1u);
+        if constexpr (!kDump) {
+          for (int ks = 0; ks < KB / 16; ++ks)
+            mma_ts(base_t + 128, base_t + L::kPB0 + ks * 8, smem_desc(v_base + (KA / 16 + ks) * 256, 128, 2048),
+                   kIdPV, 1u);
+        }
         mma_commit(&kv_empty[s]);  // this issuer's last use of stage s
         mma_commit(&pb_free[tt]);
         if (!more) mma_commit(&o_done[tt]);
@@ -484,6 +491,34 @@ fwd_tc3_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
     };
 
+    if constexpr (kDump) {
+      // Scores only: every tile's S is loaded, written out as integers and
+      // both parts are handed back at once. As in the forward, part B of
+      // tile kt is handed on only after the issuer's part-B commit of tile
+      // kt - 1, so these threads never run two phases ahead of its waits.
+      for (int kt = 0; kt < nkt; ++kt) {
+        if (ok) ok = wait_all(&s_full[t], kt & 1);
+        tc_fence_after();
+        if (ok) {
+          uint32_t xr[kKeys];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(s_col + 32 * c, xr + 32 * c);
+          tmem_ld_wait();
+          tc_fence_before();
+          if (row_valid) {
+            const int jt = key0 + kt * kKeys;
+            int32_t* srow = p.S + (tok0 + row) * N + jt;
+#pragma unroll
+            for (int e = 0; e < kKeys; ++e)
+              if (jt + e < N) srow[e] = static_cast<int32_t>(__uint_as_float(xr[e]));
+          }
+          mbar_arrive(&pa_full[t]);
+          if (kt > 0) ok = wait_all(&pb_free[t], (kt - 1) & 1);
+          if (ok) mbar_arrive(&pb_full[t]);
+        }
+        ok = __all_sync(0xffffffffu, ok);
+      }
+    } else {
     // The loop runs every key tile even after an error (with the work
     // skipped), so that each thread takes its part in every named barrier.
     if (t == 1) named_arrive(3, 2 * kSoftmaxPerTile);  // tile 0 takes the first exp turn
@@ -663,6 +698,7 @@ fwd_tc3_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         }
       }
     }
+    }  // the forward (not kDump)
   }
 
   // ------------------------------------------------------------- teardown
@@ -705,7 +741,7 @@ inline int launch(const tc::Params& prm, int ctas, cudaStream_t st, std::string*
   std::memset(&tm_v, 0, sizeof tm_v);
   std::memset(&tm_bias, 0, sizeof tm_bias);
   const cuuint64_t BH = static_cast<cuuint64_t>(prm.B) * prm.H;
-  if (!make_rows_map(&tm_v, prm.v, BH, prm.N, prm.d, "V", msg)) return BINATTN_ERR_CUDA;
+  if (kMode != kModeDump && !make_rows_map(&tm_v, prm.v, BH, prm.N, prm.d, "V", msg)) return BINATTN_ERR_CUDA;
   if (kBias && !tc2::make_bias_map(&tm_bias, prm.bias, prm.H, prm.N, prm.bias_ld > 0 ? prm.bias_ld : prm.N, msg))
     return BINATTN_ERR_CUDA;
   auto kern = fwd_tc3_kernel<DV, kMode, kBias>;
@@ -753,6 +789,15 @@ inline int dispatch_dv(const tc::Params& prm, int ctas, cudaStream_t st, std::st
 }
 
 }  // namespace tc3
+
+// Integer scores S [B,H,N,N] as the 128-key pipeline computes them (its QK^T
+// with Q and K both e4m3 in shared memory), for d % 8 == 0, d <= 80.
+inline int scores_tc3(const uint32_t* qb, const uint32_t* kb, int B, int H, int N, int d, int32_t* S,
+                      cudaStream_t st, std::string* msg) {
+  tc::Params prm{qb, kb, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S, 0.f, B, H, N, d, 0, 0, 0,
+                 nullptr};
+  return tc3::launch<32, tc3::kModeDump, false>(prm, tc2::total_pairs(B, H, N), st, msg);
+}
 
 // Binary forward on the 128-key pipeline. part: workspace for the tail split
 // (tc2::split_part_bytes), or null for no split. The split plan, the partial

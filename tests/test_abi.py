@@ -81,6 +81,10 @@ def test_scores_and_ref_host_validation(L):
     assert L.binattn_scores_debug(P(A), P(0), 1, 1, 4, 64, P(A), 0, None) == 1
     assert L.binattn_scores_debug(P(A), P(A), 1, 1, 4, 200, P(A), 0, None) == 2
     assert L.binattn_scores_debug(P(A), P(A), 1, 1, 4, 64, P(A), 9, None) == 8
+    # both TC score kernels need d % 8 == 0; TC_BIASED is not a forward engine
+    assert L.binattn_scores_debug(P(A), P(A), 1, 1, 4, 33, P(A), binattn.ENGINE_TC_BIASED, None) == 5
+    assert L.binattn_scores_debug(P(A), P(A), 1, 1, 4, 33, P(A), binattn.ENGINE_TC, None) == 5
+    assert _fwd(L, engine=binattn.ENGINE_TC_BIASED) == 8
     assert L.binattn_ref_bf16_forward(P(A), P(A), None, P(A), ctypes.c_float(1.0), 1, 1, 4, 33,
                                       P(A), None) == 5
     assert L.binattn_ref_bf16_forward(P(A), P(A), None, P(A + 2), ctypes.c_float(1.0), 1, 1, 4, 64,

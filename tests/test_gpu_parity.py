@@ -54,8 +54,12 @@ def test_pack_exact_full_size(orc, name):
 
 # --------------------------------------------------------------- scores (a3, a8)
 # The POPC_TC forward uses the same __popc routine as SIMT (one debug kernel);
-# the TC engine has its own tensor-core score routine and needs d % 8 == 0.
-SCORE_CASES = [(s, e) for s in SMALL_SHAPES + ODD_D_SHAPES for e in ["simt"] + [x for x in ENGINES if x == "tc"]
+# the TC engine has its own tensor-core score routines and needs d % 8 == 0:
+# "tc" dumps from the kernel a forward without a bias runs (the 128-key
+# pipeline where it applies), "tc_biased" from the one a forward with a bias
+# runs (the 64-key pipeline).
+TC_SCORE_ENGINES = ["tc", "tc_biased"]
+SCORE_CASES = [(s, e) for s in SMALL_SHAPES + ODD_D_SHAPES for e in ["simt"] + TC_SCORE_ENGINES
                if e == "simt" or s[3] % 8 == 0]
 
 
@@ -76,7 +80,7 @@ def test_scores_exact_full_size_sampled(orc, name):
     qb, _ = binattn.pack(dev(inp["q"]))
     kb, _ = binattn.pack(dev(inp["k"]))
     rows = sample_rows(B, H, N, 48)
-    for engine in ["simt"] + [e for e in ENGINES if e != "simt"]:
+    for engine in ["simt", "popc_tc"] + TC_SCORE_ENGINES:
         S = binattn.scores_debug(qb, kb, d, engine=engine)
         got = S.view(B * H * N, N)[torch.from_numpy(rows).cuda()].cpu().numpy()
         del S
