@@ -64,21 +64,15 @@ pack_kernel(const T* __restrict__ x, long long n_tokens, int d, int W,
 }
 
 
-// Sign words and alpha of one bf16 row with d % 8 == 0 (a whole number of
-// 16-byte chunks, 16-byte aligned): all of the row's 16-byte loads are issued
-// at once, the sign words come from x >= 0 compares (8 channels per chunk, 4
-// chunks per word), and |x| is summed in eight partial sums (one per position
-// in a chunk) combined by a tree, so alpha is a sum of depth <= d/8 + 2 in
-// fp32. binattn_pack and the forward that binarises Q itself both call this,
-// so their bits and alpha are identical.
+// Sign words and alpha of one bf16 row with d % 8 == 0 from its 16-byte
+// chunks v[0 .. d/8) (chunks beyond d/8 are ignored): the sign words come from
+// x >= 0 compares (8 channels per chunk, 4 chunks per word), and |x| is summed
+// in eight partial sums (one per position in a chunk) combined by a tree, so
+// alpha is a sum of depth <= d/8 + 2 in fp32. binattn_pack and the forward that
+// binarises Q itself both call this, so their bits and alpha are identical.
 template <int W>
-__device__ __forceinline__ void pack_row_bf16(const uint16_t* __restrict__ row, int d, uint32_t* words,
-                                              float& alpha) {
-  const uint4* src = reinterpret_cast<const uint4*>(row);
+__device__ __forceinline__ void pack_row_chunks(const uint4 (&v)[4 * W], int d, uint32_t* words, float& alpha) {
   const int ng = d / 8;  // 16-byte chunks per token
-  uint4 v[4 * W];
-#pragma unroll
-  for (int g = 0; g < 4 * W; ++g) v[g] = g < ng ? __ldg(src + g) : make_uint4(0, 0, 0, 0);
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int w = 0; w < W; ++w) {
@@ -106,6 +100,19 @@ __device__ __forceinline__ void pack_row_bf16(const uint16_t* __restrict__ row, 
   alpha = sum / static_cast<float>(d);
 }
 
+// The same for a row read straight from global memory (16-byte aligned): all
+// of the row's 16-byte loads are issued at once.
+template <int W>
+__device__ __forceinline__ void pack_row_bf16(const uint16_t* __restrict__ row, int d, uint32_t* words,
+                                              float& alpha) {
+  const uint4* src = reinterpret_cast<const uint4*>(row);
+  const int ng = d / 8;
+  uint4 v[4 * W];
+#pragma unroll
+  for (int g = 0; g < 4 * W; ++g) v[g] = g < ng ? __ldg(src + g) : make_uint4(0, 0, 0, 0);
+  pack_row_chunks<W>(v, d, words, alpha);
+}
+
 // The same for a row with W = ceil(d / 32) <= 3 known only at run time.
 __device__ __forceinline__ void pack_row_bf16_w(const uint16_t* __restrict__ row, int d, int W, uint32_t* words,
                                                 float& alpha) {
@@ -117,16 +124,35 @@ __device__ __forceinline__ void pack_row_bf16_w(const uint16_t* __restrict__ row
 }
 
 // bf16 rows with d % 8 == 0 (every token a whole number of 16-byte chunks):
-// one thread per token (pack_row_bf16).
+// a block stages kRowsTokens consecutive tokens, one contiguous byte range,
+// into shared memory with coalesced 16-byte loads, token tk at chunk
+// tk * pitch (pitch = d/8 rounded up to odd, so that the 8 threads of a
+// shared-memory wavefront read 8 different bank groups); then each thread packs
+// one token from there with pack_row_chunks.
+constexpr int kRowsTokens = 128;
 template <int W>
-__global__ void __launch_bounds__(kPackThreads)
+__global__ void __launch_bounds__(kRowsTokens)
 pack_bf16_rows_kernel(const uint16_t* __restrict__ x, long long n_tokens, int d,
                       uint32_t* __restrict__ bits, float* __restrict__ alpha) {
-  const long long t = static_cast<long long>(blockIdx.x) * kPackThreads + threadIdx.x;
-  if (t >= n_tokens) return;
+  __shared__ uint4 stage[kRowsTokens * (4 * W + 1)];
+  const long long t0 = static_cast<long long>(blockIdx.x) * kRowsTokens;
+  const int ntok = static_cast<int>(min(static_cast<long long>(kRowsTokens), n_tokens - t0));
+  const int ng = d / 8;
+  const int pitch = ng | 1;
+  const uint4* src = reinterpret_cast<const uint4*>(x + t0 * d);
+  for (int c = threadIdx.x; c < ntok * ng; c += kRowsTokens) {
+    const int tk = c / ng;
+    stage[tk * pitch + (c - tk * ng)] = __ldg(src + c);
+  }
+  __syncthreads();
+  if (static_cast<int>(threadIdx.x) >= ntok) return;
+  uint4 v[4 * W];
+#pragma unroll
+  for (int g = 0; g < 4 * W; ++g) v[g] = g < ng ? stage[threadIdx.x * pitch + g] : make_uint4(0, 0, 0, 0);
   uint32_t words[W];
   float a;
-  pack_row_bf16<W>(x + t * d, d, words, a);
+  pack_row_chunks<W>(v, d, words, a);
+  const long long t = t0 + threadIdx.x;
 #pragma unroll
   for (int w = 0; w < W; ++w) bits[t * W + w] = words[w];
   alpha[t] = a;
