@@ -61,10 +61,14 @@ class Oracle:
         lib.oracle_forward_rows.argtypes = [V, V, I, V, V, D, L, L, L, L, L, _i64p, V]
         lib.oracle_forward.argtypes = [V, V, I, V, V, D, L, L, L, L, V]
         lib.oracle_forward_spread.argtypes = [V, V, I, V, V, D, L, L, L, L, V, V]
+        lib.oracle_quantize_v.argtypes = [V, L, L, L, L, V, V]
+        lib.oracle_forward_int8_rows.argtypes = [V, V, I, V, V, D, L, L, L, L, L, _i64p, V]
+        lib.oracle_forward_int8.argtypes = [V, V, I, V, V, D, L, L, L, L, V]
         lib.oracle_num_threads.restype = I
         lib.oracle_set_num_threads.argtypes = [I]
         for f in ("oracle_pack", "oracle_scores_rows", "oracle_probs_rows",
-                  "oracle_forward_rows", "oracle_forward", "oracle_forward_spread"):
+                  "oracle_forward_rows", "oracle_forward", "oracle_forward_spread",
+                  "oracle_quantize_v", "oracle_forward_int8_rows", "oracle_forward_int8"):
             getattr(lib, f).restype = I
         self.lib = lib
 
@@ -192,6 +196,47 @@ class Oracle:
         if rc:
             raise RuntimeError(f"oracle_forward_spread failed ({rc})")
         return O, E
+
+    # ------------------------------------------------- the 8-bit P.V variant
+    def quantize_v(self, v):
+        """Per-channel 8-bit code of V (bf16 bits [B,H,N,d]): vq int8 [B,H,N,d]
+        and the scale s fp32 [B,H,d], V ~ s * vq."""
+        B, H, N, d = v.shape
+        v = self._bf16(v, "v", (B, H, N, d))
+        vq = np.zeros((B, H, N, d), dtype=np.int8)
+        s = np.zeros((B, H, d), dtype=np.float32)
+        rc = self.lib.oracle_quantize_v(_ptr(v), B, H, N, d, _ptr(vq), _ptr(s))
+        if rc:
+            raise RuntimeError(f"oracle_quantize_v failed ({rc})")
+        return vq, s
+
+    def forward_int8_rows(self, q, k, bias, v, softmax_scale, rows) -> np.ndarray:
+        """O rows (fp64, unrounded) of the 8-bit P.V forward for flat query-row ids."""
+        B, H, N, d = q.shape
+        r = self._rows(rows)
+        O = np.zeros((r.size, d), dtype=np.float64)
+        q, k = self._qk(q, k)
+        v = self._bf16(v, "v", (B, H, N, d))
+        b = self._bf16(bias, "bias", (H, N, N))
+        rc = self.lib.oracle_forward_int8_rows(_ptr(q), _ptr(k), self._dtype_code(q), _ptr(b), _ptr(v),
+                                               float(softmax_scale), B, H, N, d,
+                                               r.size, r.ctypes.data_as(_i64p), _ptr(O))
+        if rc:
+            raise RuntimeError(f"oracle_forward_int8_rows failed ({rc})")
+        return O
+
+    def forward_int8(self, q, k, bias, v, softmax_scale) -> np.ndarray:
+        """O fp64 [B,H,N,d] of the 8-bit P.V forward, every row."""
+        B, H, N, d = q.shape
+        O = np.zeros((B, H, N, d), dtype=np.float64)
+        q, k = self._qk(q, k)
+        v = self._bf16(v, "v", (B, H, N, d))
+        b = self._bf16(bias, "bias", (H, N, N))
+        rc = self.lib.oracle_forward_int8(_ptr(q), _ptr(k), self._dtype_code(q), _ptr(b), _ptr(v),
+                                          float(softmax_scale), B, H, N, d, _ptr(O))
+        if rc:
+            raise RuntimeError(f"oracle_forward_int8 failed ({rc})")
+        return O
 
 
 _default: Oracle | None = None

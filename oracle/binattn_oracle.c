@@ -42,6 +42,19 @@
  * most about 2^-8 * E_ic; the GPU parity tests use it as that element's bound
  * where it exceeds the fixed one. It is a plain definition, not a method step.
  *
+ * The 8-bit P.V variant ([ES] §2 "Cuantización Híbrida": attention
+ * coefficients, range [0, 1], in a static unsigned 8-bit code; values in a
+ * per-channel 8-bit code; [KO] §2 나-3; [ES] §2 "Implementación en Hardware":
+ * mma.s32.u8.s8.s32) is oracle_forward_int8(_rows), read as:
+ *   7. per (b, h, channel c): s_c = max_j |V_jc| / 127 and
+ *      vq_jc = rint(V_jc / s_c) (round half to even, clamped to [-127, 127]),
+ *      both in fp32, the precision in which the GPU takes these integer
+ *      decisions; s_c = 0 gives vq = 0;
+ *   8. u_ij = rint(255 * exp(logit_ij - m_i)) with m_i = max_j logit_ij, so
+ *      every u is in [0, 255] and the row max gets 255;
+ *   9. O_ic = s_c * (sum_j u_ij vq_jc) / (sum_j u_ij), the row sum taken from
+ *      the same 8-bit weights.
+ *
  * Parity pins for each function live in the CPU test suite (exhaustive sign
  * predicate, packbits layout, Hamming identity, closed forms, invariants and an
  * independent numpy formulation on small cases).
@@ -219,9 +232,9 @@ int oracle_scores_rows(const void *q, const void *k, int qk_dtype,
     return 0;
 }
 
-/* Steps 3-5 for one query row: attention probabilities P[j], j < N. */
-static void probs_row(const prep_t *p, size_t qtok, const uint16_t *bias,
-                      double softmax_scale, double *P)
+/* Steps 3-5 up to the normalisation: P[j] = exp(logit_j - max_j logit_j). */
+static void expdiff_row(const prep_t *p, size_t qtok, const uint16_t *bias,
+                        double softmax_scale, double *P)
 {
     const long N = p->N, H = p->H;
     size_t bh = qtok / (size_t)N;
@@ -239,12 +252,19 @@ static void probs_row(const prep_t *p, size_t qtok, const uint16_t *bias,
         if (logit > m)
             m = logit;
     }
-    double z = 0.0;
-    for (long j = 0; j < N; j++) {
-        P[j] = exp(P[j] - m);
-        z += P[j];
-    }
     for (long j = 0; j < N; j++)
+        P[j] = exp(P[j] - m);
+}
+
+/* Steps 3-5 for one query row: attention probabilities P[j], j < N. */
+static void probs_row(const prep_t *p, size_t qtok, const uint16_t *bias,
+                      double softmax_scale, double *P)
+{
+    expdiff_row(p, qtok, bias, softmax_scale, P);
+    double z = 0.0;
+    for (long j = 0; j < p->N; j++)
+        z += P[j];
+    for (long j = 0; j < p->N; j++)
         P[j] /= z;
 }
 
@@ -393,6 +413,115 @@ int oracle_forward_spread(const void *q, const void *k, int qk_dtype,
         rows[t] = (int64_t)t;
     int rc = oracle_forward_spread_rows(q, k, qk_dtype, bias, v, softmax_scale,
                                         B, H, N, d, (long)T, rows, O, E);
+    free(rows);
+    return rc;
+}
+
+/*
+ * Step 7: per-channel 8-bit code of V (bf16 [B, H, N, d]): vq int8 [B, H, N, d]
+ * and s fp32 [B, H, d], in fp32 arithmetic.
+ */
+int oracle_quantize_v(const uint16_t *v, long B, long H, long N, long d, int8_t *vq, float *s)
+{
+    if (!v || !vq || !s || d < 1 || N < 1)
+        return 1;
+    long bh;
+#pragma omp parallel for schedule(static)
+    for (bh = 0; bh < B * H; bh++) {
+        for (long c = 0; c < d; c++) {
+            float mx = 0.0f;
+            for (long j = 0; j < N; j++) {
+                float a = fabsf((float)load_elem(v, ORACLE_BF16, ((size_t)bh * N + j) * d + c));
+                if (a > mx)
+                    mx = a;
+            }
+            const float sc = mx / 127.0f;
+            s[(size_t)bh * d + c] = sc;
+            for (long j = 0; j < N; j++) {
+                const size_t idx = ((size_t)bh * N + j) * d + c;
+                float q = 0.0f;
+                if (sc > 0.0f) {
+                    q = nearbyintf((float)load_elem(v, ORACLE_BF16, idx) / sc);
+                    if (q > 127.0f)
+                        q = 127.0f;
+                    if (q < -127.0f)
+                        q = -127.0f;
+                }
+                vq[idx] = (int8_t)q;
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Steps 1-5 and 7-9: the 8-bit P.V forward for selected rows, O_rows[r*d + c]
+ * (fp64, unrounded). V is bf16 [B, H, N, d]; bias is bf16 [H, N, N] or NULL.
+ */
+int oracle_forward_int8_rows(const void *q, const void *k, int qk_dtype,
+                             const uint16_t *bias, const uint16_t *v,
+                             double softmax_scale, long B, long H, long N, long d,
+                             long nrows, const int64_t *rows, double *O_rows)
+{
+    if (!q || !k || !v || !rows || !O_rows || d < 1 || N < 1)
+        return 1;
+    if (check_rows(nrows, rows, B, H, N))
+        return 2;
+    int8_t *vq = (int8_t *)malloc((size_t)B * H * N * d);
+    float *s = (float *)malloc(sizeof(float) * (size_t)B * H * d);
+    prep_t p;
+    if (!vq || !s || prep_init(&p, q, k, qk_dtype, B, H, N, d)) {
+        free(vq);
+        free(s);
+        if (vq && s)
+            prep_free(&p);
+        return 3;
+    }
+    oracle_quantize_v(v, B, H, N, d, vq, s);
+    int err = 0;
+    long r;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (r = 0; r < nrows; r++) {
+        double *U = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!U) {
+#pragma omp atomic write
+            err = 3;
+            continue;
+        }
+        size_t qtok = (size_t)rows[r];
+        size_t bh = qtok / (size_t)N;
+        expdiff_row(&p, qtok, bias, softmax_scale, U);
+        double usum = 0.0;
+        for (long j = 0; j < N; j++) {
+            U[j] = nearbyint(255.0 * U[j]);
+            usum += U[j];
+        }
+        for (long c = 0; c < d; c++) {
+            double acc = 0.0;
+            for (long j = 0; j < N; j++)
+                acc += U[j] * (double)vq[(bh * (size_t)N + (size_t)j) * d + c];
+            O_rows[(size_t)r * d + c] = (double)s[bh * (size_t)d + c] * acc / usum;
+        }
+        free(U);
+    }
+    prep_free(&p);
+    free(vq);
+    free(s);
+    return err;
+}
+
+/* All rows of the 8-bit P.V forward: O [B, H, N, d] in fp64. */
+int oracle_forward_int8(const void *q, const void *k, int qk_dtype,
+                        const uint16_t *bias, const uint16_t *v, double softmax_scale,
+                        long B, long H, long N, long d, double *O)
+{
+    size_t T = (size_t)B * H * N;
+    int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (T + 1));
+    if (!rows)
+        return 3;
+    for (size_t t = 0; t < T; t++)
+        rows[t] = (int64_t)t;
+    int rc = oracle_forward_int8_rows(q, k, qk_dtype, bias, v, softmax_scale, B, H, N, d, (long)T, rows, O);
     free(rows);
     return rc;
 }

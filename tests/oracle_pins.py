@@ -373,6 +373,74 @@ def pin_spread_two_keys_closed_form(orc):
     assert np.all(E1 <= 2 * math.exp(-40) * np.abs(v).max() * 2)
 
 
+# ------------------------------------------------- the 8-bit P.V variant
+def _exact_v(rng, B, H, N, d):
+    """bf16 V whose every channel of every (b, h) holds k * 2^-3 with integers
+    |k| <= 127 and some |k| = 127: the per-channel scale is exactly 2^-3 and
+    the 8-bit code is k itself."""
+    kk = rng.integers(-127, 128, size=(B, H, N, d))
+    kk[:, :, 0, :] = 127 * np.where(rng.random((B, H, d)) < 0.5, 1, -1)
+    return f32_to_bf16_bits((kk * 0.125).astype(np.float32)), kk
+
+
+def pin_quantize_v_closed_form(orc):
+    """Per-channel code: V = k * 2^-3 with max |k| = 127 gives s = 2^-3 and
+    vq = k exactly; an all-zero channel gives s = 0, vq = 0; ties round to
+    even (2.5 -> 2, 3.5 -> 4, -2.5 -> -2 at s = 1)."""
+    rng = np.random.default_rng(51)
+    v, kk = _exact_v(rng, 2, 3, 17, 12)
+    vb = v.copy()
+    vb[1, 2, :, 5] = 0  # an all-zero channel
+    vq, s = orc.quantize_v(vb)
+    want = kk.copy()
+    want[1, 2, :, 5] = 0
+    assert np.array_equal(vq, want.astype(np.int8))
+    ws = np.full(s.shape, 0.125, dtype=np.float32)
+    ws[1, 2, 5] = 0.0
+    assert np.array_equal(s, ws)
+    t = np.zeros((1, 1, 5, 1), dtype=np.float32)
+    t[0, 0, :, 0] = [127.0, 2.5, 3.5, -2.5, -126.5]
+    vq, s = orc.quantize_v(f32_to_bf16_bits(t))
+    assert s[0, 0, 0] == 1.0 and list(vq[0, 0, :, 0]) == [127, 2, 4, -2, -126]
+
+
+def pin_int8_uniform_scores(orc):
+    """Every key row of a head identical, no bias: every u is 255, and
+    O = s * mean_j vq_j = 2^-3 * mean_j k_j for the exact V above."""
+    B, H, N, d = 2, 2, 11, 24
+    rng = np.random.default_rng(52)
+    q = rng.standard_normal((B, H, N, d)).astype(np.float32)
+    k = np.ascontiguousarray(np.broadcast_to(rng.standard_normal((B, H, 1, d)).astype(np.float32), (B, H, N, d)))
+    v, kk = _exact_v(rng, B, H, N, d)
+    O = orc.forward_int8(q, k, None, v, 0.8)
+    want = np.broadcast_to(0.125 * kk.mean(axis=2, keepdims=True), O.shape)
+    assert np.allclose(O, want, rtol=1e-13, atol=1e-15)
+
+
+def pin_int8_two_keys_closed_form(orc):
+    """N = 2, scale 0, bias row (b0, b1): the larger logit gets u = 255, the
+    other u = rint(255 e^-|b0 - b1|), and O = 2^-3 (u0 k0 + u1 k1) / (u0 + u1);
+    a one-hot bias of 40 gives O = 2^-3 k of that key (u = 0 elsewhere)."""
+    B, H, N, d = 1, 4, 2, 8
+    rng = np.random.default_rng(53)
+    c = make_custom(B, H, N, d, seed=54, with_bias=False)
+    v, kk = _exact_v(rng, B, H, N, d)
+    bias = f32_to_bf16_bits(rng.uniform(-3, 3, size=(H, N, N)).astype(np.float32))
+    O = orc.forward_int8(c["q"], c["k"], bias, v, 0.0)
+    b = _f64(bias)
+    for h in range(H):
+        for i in range(N):
+            e = np.exp(b[h, i] - b[h, i].max())
+            u = np.array([255.0 if x == 1.0 else float(np.rint(255.0 * x)) for x in e])
+            want = 0.125 * (u[:, None] * kk[0, h]).sum(axis=0) / u.sum()
+            assert np.allclose(O[0, h, i], want, rtol=1e-13, atol=1e-15), (h, i)
+    onehot = np.zeros((H, N, N), dtype=np.float32)
+    onehot[:, 0, 1] = 40.0
+    onehot[:, 1, 0] = 40.0
+    O1 = orc.forward_int8(c["q"], c["k"], f32_to_bf16_bits(onehot), v, 0.0)
+    assert np.array_equal(O1[0, :, 0], 0.125 * kk[0, :, 1]) and np.array_equal(O1[0, :, 1], 0.125 * kk[0, :, 0])
+
+
 ALL_PINS = [
     pin_sign_predicate_exhaustive,
     pin_pack_layout_packbits,
@@ -393,4 +461,7 @@ ALL_PINS = [
     pin_sign_correlation_arcsin,
     pin_spread_uniform_is_mean_abs_deviation,
     pin_spread_two_keys_closed_form,
+    pin_quantize_v_closed_form,
+    pin_int8_uniform_scores,
+    pin_int8_two_keys_closed_form,
 ]

@@ -56,6 +56,18 @@ MUTANTS = [
      "e += P[j] * fabs(load_elem(", "e += P[j] * (load_elem("),
     ("spread not weighted by P",
      "e += P[j] * fabs(", "e += fabs("),
+    ("8-bit P on 256 levels",
+     "U[j] = nearbyint(255.0 * U[j]);", "U[j] = nearbyint(256.0 * U[j]);"),
+    ("8-bit P truncated",
+     "U[j] = nearbyint(255.0 * U[j]);", "U[j] = floor(255.0 * U[j]);"),
+    ("V code scale over 128",
+     "const float sc = mx / 127.0f;", "const float sc = mx / 128.0f;"),
+    ("V code truncated",
+     "q = nearbyintf((float)load_elem(v, ORACLE_BF16, idx) / sc);",
+     "q = truncf((float)load_elem(v, ORACLE_BF16, idx) / sc);"),
+    ("8-bit row sum dropped",
+     "O_rows[(size_t)r * d + c] = (double)s[bh * (size_t)d + c] * acc / usum;",
+     "O_rows[(size_t)r * d + c] = (double)s[bh * (size_t)d + c] * acc / 255.0;"),
 ]
 
 
