@@ -397,11 +397,37 @@ def time_configs(names, args, rank, world, dev, stream, peaks, flush, max_over_r
         fwd_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / steps)
         a = algorithmic(w, True)
         t_roof = roofline_terms(w, True, peaks, n_sm)["t_roof"]
-        rows.append({"workload": name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bias": True,
-                     "call": "binattn_forward_ws" if ws is not None else "binattn_forward",
-                     "forward_ms": round(fwd_ms, 5), "step_ms": round(step_ms, 5),
-                     "effective_tflops": round(a["eff_flops"] / (fwd_ms * 1e-3) / 1e12, 2),
-                     "roofline_frac": round(t_roof / (fwd_ms * 1e-3), 4)})
+        row = {"workload": name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bias": True,
+               "call": "binattn_forward_ws" if ws is not None else "binattn_forward",
+               "forward_ms": round(fwd_ms, 5), "step_ms": round(step_ms, 5),
+               "effective_tflops": round(a["eff_flops"] / (fwd_ms * 1e-3) / 1e12, 2),
+               "roofline_frac": round(t_roof / (fwd_ms * 1e-3), 4)}
+        # The bias is a learned parameter: stored once with padded rows, the call
+        # reads it as it is (binattn_forward_bias_ld_ws) instead of padding it.
+        if args.engine == "auto" and w.N % 8 and w.d % 8 == 0 and w.d <= 80:
+            stored = binattn.pad_bias(bias)
+            wsl = torch.empty(max(16, binattn.lib().binattn_forward_bias_ld_workspace_bytes(
+                w.B, w.H, w.N, w.d, stored.shape[2])), dtype=torch.uint8, device=dev)
+            fl = lambda: binattn.forward_bias_ld_ws(qb, kb, aq, ak, stored, v, scale, workspace=wsl, out=out,
+                                                    stream=stream)
+            for _ in range(3):
+                fl()
+            torch.cuda.synchronize()
+            evl = []
+            for _ in range(steps):
+                flush.fill_(1)
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                e[0].record(stream)
+                fl()
+                e[1].record(stream)
+                evl.append(e)
+            torch.cuda.synchronize()
+            binattn.device_status(stream)
+            fl_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evl) / steps)
+            row["stored_padded_bias"] = {"call": "binattn_forward_bias_ld_ws", "forward_ms": round(fl_ms, 5),
+                                         "roofline_frac": round(t_roof / (fl_ms * 1e-3), 4)}
+            del stored, wsl
+        rows.append(row)
         del q, k, v, bias, qb, kb, aq, ak, out, ws
     return rows
 
@@ -554,6 +580,37 @@ def run_gpu(args, w_job, rank, world, local_rank):
             del fws
         binattn.device_status(stream)
 
+    # the 8-bit P.V variant (binattn_forward_int8: V's 8-bit code, the row-max
+    # pass and the 8-bit pass), same step and protocol
+    int8 = {}
+    if args.engine == "auto" and d % 8 == 0 and d <= 80:
+        for name, b in (("bias", bias), ("no_bias", None)):
+            iws = torch.empty(max(16, binattn.int8_workspace_bytes(B, H, N, d, b is not None)), dtype=torch.uint8,
+                              device=dev)
+            f8 = lambda b=b, iws=iws: binattn.forward_int8(qb, kb, aq, ak, b, v, scale, workspace=iws, out=out,
+                                                           stream=stream)
+            step(b)
+            f8()
+            torch.cuda.synchronize()
+            barrier()
+            ev = []
+            for _ in range(args.steps):
+                flush.fill_(1)
+                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                e0.record(stream)
+                binattn.pack(q, qb, aq, stream)
+                binattn.pack(k, kb, ak, stream)
+                e1.record(stream)
+                f8()
+                e2.record(stream)
+                ev.append((e0, e1, e2))
+            torch.cuda.synchronize()
+            barrier()
+            int8[name] = {"ms_per_step": round(max_over_ranks(sum(a.elapsed_time(c) for a, _, c in ev) / len(ev)), 5),
+                          "forward_ms": round(max_over_ranks(sum(b_.elapsed_time(c) for _, b_, c in ev) / len(ev)), 5)}
+            del iws
+        binattn.device_status(stream)
+
     # in-build bf16 attention on the same shapes (speed reference)
     ref = None
     try:
@@ -634,6 +691,8 @@ def run_gpu(args, w_job, rank, world, local_rank):
                     "effective_tflops": round(a0["eff_flops"] / fwd0_s / 1e12, 2),
                     "roofline": roof0},
         "bf16_reference": ref,
+        "int8_pv": dict(int8, call="binattn_forward_int8 (V 8-bit code + row-max pass + 8-bit P.V pass)",
+                        step="pack(Q) + pack(K) + binattn_forward_int8"),
         "other_workloads": others,
         "roofline": roof | {
             "traffic": ncu_traffic(f"{w.name}/bias"),
@@ -648,6 +707,7 @@ def run_gpu(args, w_job, rank, world, local_rank):
                 "h2d_bytes_per_step": int(3 * B * H * N * d * 2),
                 "d2h_bytes_per_step": int(B * H * N * d * 2)},
         "gpu_launches": args.steps * (step_launches(w, True, args.engine) + step_launches(w, False, args.engine)),
+        "gpu_launches_counts": "kernels of the timed headline steps (with and without the bias)",
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

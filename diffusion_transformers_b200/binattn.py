@@ -28,6 +28,8 @@ EXPORTS = (
     "binattn_forward_fused_ws", "binattn_scores_debug",
     "binattn_ref_bf16_forward", "binattn_device_status", "binattn_strerror",
     "binattn_last_error_message", "binattn_abi_version", "binattn_test_wait_timeout",
+    "binattn_forward_bias_ld_workspace_bytes", "binattn_padded_bias_ld", "binattn_forward_bias_ld_ws",
+    "binattn_quantize_v", "binattn_forward_int8_workspace_bytes", "binattn_forward_int8",
 )
 
 
@@ -61,6 +63,18 @@ def lib() -> ctypes.CDLL:
     L.binattn_forward_workspace_bytes.restype = ctypes.c_size_t
     L.binattn_forward_ws.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
     L.binattn_forward_static_ws.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, P]
+    L.binattn_forward_bias_ld_workspace_bytes.argtypes = [I, I, I, I, I]
+    L.binattn_forward_bias_ld_workspace_bytes.restype = ctypes.c_size_t
+    L.binattn_padded_bias_ld.argtypes = [I]
+    L.binattn_padded_bias_ld.restype = I
+    L.binattn_forward_bias_ld_ws.argtypes = [P, P, P, P, P, I, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
+    L.binattn_forward_bias_ld_ws.restype = I
+    L.binattn_quantize_v.argtypes = [P, I, I, I, I, P, P, P]
+    L.binattn_quantize_v.restype = I
+    L.binattn_forward_int8_workspace_bytes.argtypes = [I, I, I, I, I]
+    L.binattn_forward_int8_workspace_bytes.restype = ctypes.c_size_t
+    L.binattn_forward_int8.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
+    L.binattn_forward_int8.restype = I
     L.binattn_forward_fused_workspace_bytes.argtypes = [I, I, I, I, I, I]
     L.binattn_forward_fused_workspace_bytes.restype = ctypes.c_size_t
     L.binattn_forward_fused_ws.argtypes = [P, I, P, P, P, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
@@ -230,6 +244,90 @@ def forward_ws(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor
                                         _ptr(v), float(softmax_scale), B, H, N, d, _ptr(out), _ptr(workspace),
                                         ctypes.c_size_t(size), _stream(stream, dev)),
                "binattn_forward_ws")
+    return out
+
+
+def padded_bias_ld(N: int) -> int:
+    """Row stride (elements) at which a stored bias is read by the TMA-fed
+    pipeline as it is: N rounded up to a multiple of 8."""
+    return int(lib().binattn_padded_bias_ld(int(N)))
+
+
+def pad_bias(bias: torch.Tensor) -> torch.Tensor:
+    """A learned bias [H, N, N] stored once as [H, N, padded_bias_ld(N)] (zero
+    pad), for forward_bias_ld_ws. Plain torch copy: it is done once, not per call."""
+    H, N, _ = bias.shape
+    out = torch.zeros((H, N, padded_bias_ld(N)), dtype=bias.dtype, device=bias.device)
+    out[:, :, :N] = bias
+    return out
+
+
+def forward_bias_ld_ws(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor,
+                       alpha_k: torch.Tensor, bias: torch.Tensor, v: torch.Tensor, softmax_scale: float,
+                       workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """forward_ws with a bias [H, N, ld] whose rows are ld >= N elements apart
+    (only its first N columns are read), e.g. from pad_bias()."""
+    B, H, N, d = v.shape
+    if bias.dim() != 3 or bias.shape[0] != H or bias.shape[1] != N or bias.shape[2] < N:
+        raise ValueError(f"bias must be [H={H}, N={N}, ld >= N], got {tuple(bias.shape)}")
+    if bias.dtype != torch.bfloat16 or not bias.is_contiguous():
+        raise TypeError("bias must be a contiguous bfloat16 tensor")
+    ld = bias.shape[2]
+    dev = _forward_args(q_bits, k_bits, alpha_q, alpha_k, None, v, out)
+    _device(bias, v)
+    if workspace is not None:
+        _device(workspace, v)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    need = int(lib().binattn_forward_bias_ld_workspace_bytes(B, H, N, d, ld))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    size = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        _check(lib().binattn_forward_bias_ld_ws(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k), _ptr(bias),
+                                                ld, _ptr(v), float(softmax_scale), B, H, N, d, _ptr(out),
+                                                _ptr(workspace), ctypes.c_size_t(size), _stream(stream, dev)),
+               "binattn_forward_bias_ld_ws")
+    return out
+
+
+def quantize_v(v: torch.Tensor, stream=None):
+    """V's per-channel 8-bit code: vq int8 [B,H,N,d] and scale fp32 [B,H,d]."""
+    B, H, N, d = v.shape
+    _expect(v, "v", (B, H, N, d), (torch.bfloat16,))
+    dev = _device(v)
+    vq = torch.empty((B, H, N, d), dtype=torch.int8, device=dev)
+    scale = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().binattn_quantize_v(_ptr(v), B, H, N, d, _ptr(vq), _ptr(scale), _stream(stream, dev)),
+               "binattn_quantize_v")
+    return vq, scale
+
+
+def int8_workspace_bytes(B: int, H: int, N: int, d: int, has_bias: bool) -> int:
+    return int(lib().binattn_forward_int8_workspace_bytes(B, H, N, d, int(has_bias)))
+
+
+def forward_int8(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor, alpha_k: torch.Tensor,
+                 bias: torch.Tensor | None, v: torch.Tensor, softmax_scale: float,
+                 workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """O [B,H,N,d] bfloat16 of the 8-bit P.V forward (binattn_forward_int8)."""
+    B, H, N, d = v.shape
+    dev = _forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, out)
+    if workspace is not None:
+        _device(workspace, v)
+    need = int8_workspace_bytes(B, H, N, d, bias is not None)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    size = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        _check(lib().binattn_forward_int8(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k), _ptr(bias),
+                                          _ptr(v), float(softmax_scale), B, H, N, d, _ptr(out), _ptr(workspace),
+                                          ctypes.c_size_t(size), _stream(stream, dev)), "binattn_forward_int8")
     return out
 
 

@@ -16,6 +16,7 @@
 #include "fwd_tc.cuh"
 #include "fwd_tc2.cuh"
 #include "fwd_tc3.cuh"
+#include "quantv.cuh"
 
 namespace {
 
@@ -225,33 +226,46 @@ int padded_bias_ld(int N) { return (N + 7) / 8 * 8; }
 bool ws_path(int d, int N, bool has_bias) {
   return binattn::tc3::supported(d, N, has_bias, has_bias ? padded_bias_ld(N) : 0);
 }
-size_t ws_pad_bytes(int H, int N, bool has_bias) {
-  if (!has_bias || N % 8 == 0) return 0;
+// Bytes of the padded bias copy: needed when the bias rows (bias_ld elements
+// apart) are not TMA rows.
+size_t ws_pad_bytes(int H, int N, bool has_bias, int bias_ld) {
+  if (!has_bias || bias_ld % 8 == 0) return 0;
   return (static_cast<size_t>(H) * N * padded_bias_ld(N) * 2 + 255) / 256 * 256;
+}
+size_t ws_bytes(int B, int H, int N, int d, bool has_bias, int bias_ld) {
+  if (B < 1 || H < 1 || N < 1 || d < 1 || !ws_path(d, N, has_bias)) return 0;
+  return ws_pad_bytes(H, N, has_bias, bias_ld) + binattn::tc2::split_part_bytes(B, H, N, d);
 }
 }  // namespace
 
 size_t binattn_forward_workspace_bytes(int B, int H, int N, int d, int has_bias) {
-  if (B < 1 || H < 1 || N < 1 || d < 1 || !ws_path(d, N, has_bias != 0)) return 0;
-  return ws_pad_bytes(H, N, has_bias != 0) + binattn::tc2::split_part_bytes(B, H, N, d);
+  return ws_bytes(B, H, N, d, has_bias != 0, N);
+}
+
+int binattn_padded_bias_ld(int N) { return N < 1 ? 0 : padded_bias_ld(N); }
+
+size_t binattn_forward_bias_ld_workspace_bytes(int B, int H, int N, int d, int bias_ld) {
+  if (bias_ld < N) return 0;
+  return ws_bytes(B, H, N, d, true, bias_ld);
 }
 
 namespace {
 // The TMA-fed forward with a workspace (ws_path(d, N, bias) holds): bias rows
 // padded into the workspace when N % 8 != 0, a short last wave split by key
 // halves, and with qh set, Q binarised inside the kernel.
+// bias_ld: elements between the caller's bias rows (>= N).
 int forward_tma_ws(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q, const float* alpha_k,
-                   const uint16_t* bias, const uint16_t* v, float softmax_scale, int B, int H, int N, int d,
-                   uint16_t* out, void* workspace, size_t need, const uint16_t* qh, cudaStream_t st) {
-  const size_t pad = ws_pad_bytes(H, N, bias != nullptr);
+                   const uint16_t* bias, int bias_ld, const uint16_t* v, float softmax_scale, int B, int H, int N,
+                   int d, uint16_t* out, void* workspace, size_t need, const uint16_t* qh, cudaStream_t st) {
+  const size_t pad = ws_pad_bytes(H, N, bias != nullptr, bias_ld);
   const uint16_t* fbias = bias;
-  int ld = 0;
+  int ld = bias_ld == N ? 0 : bias_ld;
   if (pad) {
     ld = padded_bias_ld(N);
     uint16_t* padded = static_cast<uint16_t*>(workspace);
     const long long rows = static_cast<long long>(H) * N;
     const unsigned grid = static_cast<unsigned>((rows * ld + 255) / 256);
-    binattn::tc2::pad_bias_rows_kernel<<<grid, 256, 0, st>>>(bias, rows, N, ld, padded);
+    binattn::tc2::pad_bias_rows_kernel<<<grid, 256, 0, st>>>(bias, rows, N, bias_ld, ld, padded);
     if (int rc = launch_status("pad_bias_rows_kernel")) return rc;
     fbias = padded;
   }
@@ -284,8 +298,32 @@ int binattn_forward_ws(const uint32_t* q_bits, const uint32_t* k_bits, const flo
   BINATTN_CHECK_PTR(workspace);
   if (workspace_bytes < need)
     return fail(BINATTN_ERR_ARG, "workspace of %zu bytes is below the %zu this shape needs", workspace_bytes, need);
-  return forward_tma_ws(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out, workspace, need,
-                        nullptr, static_cast<cudaStream_t>(stream));
+  return forward_tma_ws(q_bits, k_bits, alpha_q, alpha_k, bias, N, v, softmax_scale, B, H, N, d, out, workspace,
+                        need, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int binattn_forward_bias_ld_ws(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
+                               const float* alpha_k, const uint16_t* bias, int bias_ld, const uint16_t* v,
+                               float softmax_scale, int B, int H, int N, int d, uint16_t* out, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  BINATTN_CHECK_PTR(bias);
+  if (int rc = check_forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out))
+    return rc;
+  if (bias_ld < N) return fail(BINATTN_ERR_ARG, "bias_ld = %d is below N = %d", bias_ld, N);
+  if (bias_ld == N)
+    return binattn_forward_ws(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out, workspace,
+                              workspace_bytes, stream);
+  const size_t need = binattn_forward_bias_ld_workspace_bytes(B, H, N, d, bias_ld);
+  if (!ws_path(d, N, true))
+    return fail(BINATTN_ERR_UNSUPPORTED, "a strided bias needs the TMA-fed pipeline (d %% 8 == 0, d <= 80); d = %d", d);
+  if (need) {
+    BINATTN_CHECK_PTR(workspace);
+    if (workspace_bytes < need)
+      return fail(BINATTN_ERR_ARG, "workspace of %zu bytes is below the %zu this shape needs", workspace_bytes,
+                  need);
+  }
+  return forward_tma_ws(q_bits, k_bits, alpha_q, alpha_k, bias, bias_ld, v, softmax_scale, B, H, N, d, out,
+                        workspace, need, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 size_t binattn_forward_fused_workspace_bytes(int B, int H, int N, int d, int q_dtype, int has_bias) {
@@ -315,8 +353,8 @@ int binattn_forward_fused_ws(const void* q, int q_dtype, const uint32_t* k_bits,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t fw = binattn_forward_workspace_bytes(B, H, N, d, bias != nullptr);
   if (fused_path(q_dtype, d, N, bias != nullptr))
-    return forward_tma_ws(nullptr, k_bits, nullptr, alpha_k, bias, v, softmax_scale, B, H, N, d, out, workspace, fw,
-                          static_cast<const uint16_t*>(q), st);
+    return forward_tma_ws(nullptr, k_bits, nullptr, alpha_k, bias, N, v, softmax_scale, B, H, N, d, out, workspace,
+                          fw, static_cast<const uint16_t*>(q), st);
   // Other shapes and fp32 Q: binattn_pack into the workspace, then the forward.
   char* ws = static_cast<char*>(workspace);
   const size_t tokens = static_cast<size_t>(B) * H * N;
@@ -376,6 +414,81 @@ int binattn_forward_static_ws(const uint32_t* q_bits, const uint32_t* k_bits, co
   if (int rc = static_workspace_addr(&ws)) return rc;
   return binattn_forward_ws(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out, ws,
                             kStaticWorkspaceBytes, stream);
+}
+
+int binattn_quantize_v(const uint16_t* v, int B, int H, int N, int d, int8_t* vq, float* scale, void* stream) {
+  BINATTN_CHECK_PTR(v);
+  BINATTN_CHECK_PTR(vq);
+  BINATTN_CHECK_PTR(scale);
+  if (int rc = check_shape(B, H, N, d)) return rc;
+  if (d % 8 != 0) return fail(BINATTN_ERR_UNSUPPORTED, "the 8-bit V code needs d %% 8 == 0 (d = %d)", d);
+  binattn::quantize_v_kernel<<<static_cast<unsigned>(B * H), binattn::kQvThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      v, N, d, 0, nullptr, vq, scale);
+  return launch_status("quantize_v_kernel");
+}
+
+namespace {
+// Workspace of binattn_forward_int8: V's tiled 8-bit code, its scales, the row
+// maxima, and with N % 8 != 0 the bias with padded rows.
+struct Int8Ws {
+  size_t vq, scale, mrow, pad, total;
+};
+Int8Ws int8_ws(int B, int H, int N, int d, bool has_bias) {
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t nkt = (static_cast<size_t>(N) + 63) / 64;
+  Int8Ws w;
+  w.vq = round256(BH * nkt * binattn::tc2::dv_for(d) * 64);
+  w.scale = round256(BH * d * 4);
+  w.mrow = round256(BH * N * 4);
+  w.pad = ws_pad_bytes(H, N, has_bias, N);
+  w.total = w.vq + w.scale + w.mrow + w.pad;
+  return w;
+}
+bool int8_path(int d, int N, bool has_bias) {
+  return binattn::tc2::supported(d, N, has_bias, false, has_bias ? padded_bias_ld(N) : 0);
+}
+}  // namespace
+
+size_t binattn_forward_int8_workspace_bytes(int B, int H, int N, int d, int has_bias) {
+  if (B < 1 || H < 1 || N < 1 || d < 1 || !int8_path(d, N, has_bias != 0)) return 0;
+  return int8_ws(B, H, N, d, has_bias != 0).total;
+}
+
+int binattn_forward_int8(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q, const float* alpha_k,
+                         const uint16_t* bias, const uint16_t* v, float softmax_scale, int B, int H, int N, int d,
+                         uint16_t* out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (int rc = check_forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out))
+    return rc;
+  if (!int8_path(d, N, bias != nullptr))
+    return fail(BINATTN_ERR_UNSUPPORTED, "the 8-bit P.V forward needs d %% 8 == 0 and d <= 80 (d = %d)", d);
+  BINATTN_CHECK_PTR(workspace);
+  const Int8Ws w = int8_ws(B, H, N, d, bias != nullptr);
+  if (workspace_bytes < w.total)
+    return fail(BINATTN_ERR_ARG, "workspace of %zu bytes is below the %zu this shape needs", workspace_bytes, w.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int8_t* vq8 = reinterpret_cast<int8_t*>(ws);
+  float* vscale = reinterpret_cast<float*>(ws + w.vq);
+  float* mrow = reinterpret_cast<float*>(ws + w.vq + w.scale);
+  const uint16_t* fbias = bias;
+  int ld = 0;
+  if (w.pad) {
+    ld = padded_bias_ld(N);
+    uint16_t* padded = reinterpret_cast<uint16_t*>(ws + w.vq + w.scale + w.mrow);
+    const long long rows = static_cast<long long>(H) * N;
+    binattn::tc2::pad_bias_rows_kernel<<<static_cast<unsigned>((rows * ld + 255) / 256), 256, 0, st>>>(
+        bias, rows, N, N, ld, padded);
+    if (int rc = launch_status("pad_bias_rows_kernel")) return rc;
+    fbias = padded;
+  }
+  binattn::quantize_v_kernel<<<static_cast<unsigned>(B * H), binattn::kQvThreads, 0, st>>>(
+      v, N, d, binattn::tc2::dv_for(d), vq8, nullptr, vscale);
+  if (int rc = launch_status("quantize_v_kernel")) return rc;
+  std::string msg;
+  if (int rc = binattn::forward_tc2_int8(q_bits, k_bits, alpha_q, alpha_k, fbias, ld, vq8, vscale, mrow,
+                                         softmax_scale, B, H, N, d, out, st, &msg))
+    return fail(rc, "%s", msg.c_str());
+  return ok();
 }
 
 int binattn_scores_debug(const uint32_t* q_bits, const uint32_t* k_bits, int B, int H, int N,

@@ -147,6 +147,12 @@ struct Params {
   // stall_after >= 0 the TMA producer of the 64-key pipeline issues nothing
   // from key tile stall_after on, so the stage's consumers time out.
   int stall_after = -1;
+  // 8-bit P.V (64-key pipeline): V's per-channel 8-bit code in the tiled
+  // operand layout (quantv.cuh), its scales [B,H,d], and the exact row max of
+  // the logits [B,H,N] (written by the row-max pass, read by the 8-bit pass).
+  const int8_t* vq8 = nullptr;
+  const float* vscale = nullptr;
+  float* mrow = nullptr;
 };
 
 // Named barrier 1 over the load-mode loader warps with an AND reduction.

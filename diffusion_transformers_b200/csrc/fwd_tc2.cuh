@@ -77,6 +77,8 @@ constexpr float kRescale = 5.545177444479562f;  // 8 ln 2: rescale only past a 2
 constexpr int kModeBin = 0;   // binary forward
 constexpr int kModeRef = 1;   // bf16 reference attention
 constexpr int kModeDump = 2;  // binary scores only (debug)
+constexpr int kModeMax = 3;   // 8-bit P.V, first pass: the exact row max of the logits
+constexpr int kModeI8 = 4;    // 8-bit P.V, second pass: u8 P (against that max) times s8 V
 
 // Shapes this pipeline takes (the caller falls back to the load-mode pipeline otherwise).
 // bias_ld: elements between bias rows (N, or a padded length; TMA needs % 8 == 0).
@@ -106,7 +108,8 @@ struct Layout {
   static constexpr int kBS = 4;                                  // bias stages (per t)
   static constexpr int kBiasTile = kRows * kKeys * 2;            // 16 KB
   static constexpr int kKTile = kMode == kModeRef ? kKeys * DV * 2 : kKeys * 96;
-  static constexpr int kVTile = kMode == kModeDump ? 0 : kKeys * DV * 2;
+  static constexpr int kVTile = (kMode == kModeDump || kMode == kModeMax) ? 0
+                                : kMode == kModeI8 ? kKeys * DV : kKeys * DV * 2;
   static constexpr int kBiasOff = 0;
   static constexpr int kK = kBiasOff + (kBias ? kBS * 2 * kBiasTile : 0);
   static constexpr int kV = kK + kKS * kKTile;
@@ -133,6 +136,24 @@ __device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor for kind::i8: unsigned 8-bit A, signed 8-bit B, s32 D,
+// both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
+  return (2u << 4) | (0u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[tmem] * B[smem], 8-bit integer operands (s32 accumulate).
+__device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}"
       ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -187,6 +208,10 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   using L = Layout<DV, kMode, kBias>;
   constexpr bool kRef = kMode == kModeRef;
   constexpr bool kDump = kMode == kModeDump;
+  constexpr bool kMax = kMode == kModeMax;
+  constexpr bool kI8 = kMode == kModeI8;
+  constexpr bool kF16PV = kMode == kModeBin || kRef;  // bf16 P.V from TMA-loaded V
+  constexpr bool kNoPV = kDump || kMax;
   constexpr int kKS = L::kKS, kBS = L::kBS;
   static_assert(DV % 16 == 0 && DV <= 96, "P.V N");
   static_assert(!kRef || DV <= 80, "reference Q_t columns");
@@ -229,7 +254,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   const int kq16 = (d + 15) / 16;              // reference QK^T MMAs (16 channels each)
 
   // ---------------------------------------------------------------- setup
-  if constexpr (!kDump) {
+  if constexpr (kF16PV) {
     // Channels >= d of every V stage (never written by TMA): channel d is 1.0
     // (the row-sum column), the rest 0. Reference K: pad channels 0.
     const int npad = (DV / 8 - dgroups) * kKeys;
@@ -250,7 +275,8 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kKS; ++s) {
-      mbar_init(&kv_full[s], kRef ? 1 : (kDump ? 32 : 33));
+      // the expander's 32 lanes, plus the arrive of the V copy
+      mbar_init(&kv_full[s], kRef ? 1 : (kNoPV ? 32 : 33));
       mbar_init(&kv_empty[s], 2);
     }
     for (int i = 0; i < kBS * 2; ++i) {
@@ -335,12 +361,12 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
 
   if (warp == kTmaWarp) {
     // --------------------------- V (and reference K), bias: one thread issues
-    if (lane == 0 && (!kDump || kBias)) {
+    if (lane == 0 && (!kNoPV || kBias)) {
       bool ok = true;
       for (int kt = 0; ok && kt < nkt; ++kt) {
         if (p.stall_after >= 0 && kt >= p.stall_after) break;  // test only
         const int j0 = key0 + kt * kKeys;
-        if constexpr (!kDump) {
+        if constexpr (kF16PV) {
           const int s = kt % kKS;
           if (kt >= kKS && !(ok = mbar_wait(&kv_empty[s], ((kt / kKS) - 1) & 1, abort))) break;
           mbar_arrive_expect_tx(&kv_full[s], static_cast<uint32_t>(dgroups * 1024 * (kRef ? 2 : 1)));
@@ -350,6 +376,14 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
             for (int g = 0; g < dgroups; ++g)
               tma_load_3d(smem + L::kK + s * L::kKTile + g * 1024, &tm_k, 8 * g, j0, bh, &kv_full[s]);
           }
+        } else if constexpr (kI8) {
+          // the tile's 8-bit V operand is one contiguous block of the tiled layout
+          const int s = kt % kKS;
+          if (kt >= kKS && !(ok = mbar_wait(&kv_empty[s], ((kt / kKS) - 1) & 1, abort))) break;
+          mbar_arrive_expect_tx(&kv_full[s], static_cast<uint32_t>(L::kVTile));
+          bulk_load(smem + L::kV + s * L::kVTile,
+                    p.vq8 + (static_cast<size_t>(bh) * nkt_all + kt_begin + kt) * L::kVTile,
+                    static_cast<uint32_t>(L::kVTile), &kv_full[s]);
         }
         if constexpr (kBias) {
           for (int t2 = 0; t2 < 2; ++t2) {
@@ -458,20 +492,28 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         const int bf = kt & 1;
         if (!(ok = mbar_wait(&p_full[tt * 2 + bf], (kt >> 1) & 1, abort))) break;
         tc_fence_after();
-        if constexpr (!kDump) {
+        if constexpr (kF16PV) {
           // O_tt += P_tt(kt) V(kt): A = P (bf16 pairs, 8 columns per 16 keys)
           const uint32_t v_base = smem_u32(smem + L::kV + s * L::kVTile);
 #pragma unroll
           for (int ks = 0; ks < kKeys / 16; ++ks)
             mma_ts(base_t + 128, base_t + 64 * bf + ks * 8, smem_desc(v_base + ks * 256, 128, 1024), kIdPV,
                    (kt > 0 || ks > 0));
+        } else if constexpr (kI8) {
+          // O_tt (s32) += P_tt(kt) V(kt): A = u8 P (4 keys per column, 8
+          // columns per 32 keys), B = s8 V, K-major, 32 keys per MMA
+          const uint32_t v_base = smem_u32(smem + L::kV + s * L::kVTile);
+#pragma unroll
+          for (int ks = 0; ks < kKeys / 32; ++ks)
+            mma_ts_i8(base_t + 128, base_t + 64 * bf + ks * 8, smem_desc(v_base + ks * 256, 128, 512),
+                      idesc_i8(kRows, DV), (kt > 0 || ks > 0));
         }
         mma_commit(&kv_empty[s]);  // this issuer's last use of stage s
         if (kt + 2 < nkt) {
           if (!(ok = stage_ready(kt + 2))) break;
           issue_qk(kt + 2);
           mma_commit(&s_full[tt * 2 + bf]);
-        } else if constexpr (!kDump) {
+        } else if constexpr (!kNoPV) {
           mma_commit(&o_done[tt * 2 + bf]);
         }
       }
@@ -488,7 +530,9 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
     const float ci = kRef ? p.scale : ((!kDump && row_valid) ? p.scale * aq_row : 0.f);
     const uint32_t o_col = tmem + lane_base + 256 * t + 128;
     const int r7 = r & 7;
+    // the running max; in the 8-bit pass, the row's exact max from the first pass
     float m = -INFINITY;
+    if constexpr (kI8) m = row_valid ? p.mrow[tok0 + row] : 0.f;
     bool ok = true;
     // Waits are made warp-uniform: the tcgen05.ld/st below are warp-collective.
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
@@ -545,9 +589,28 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       tmem_st16(p_col, pk);
     };
 
+    // 8-bit pass: u = rint(255 exp(logit - m)) of a 32-key chunk (m the row's
+    // exact max, so u <= 255), four keys per 32-bit TMEM column, lowest key in
+    // the lowest byte: the unsigned 8-bit A operand of the kind::i8 P.V
+    auto exps_u8 = [&](const uint32_t* xr, uint32_t p_col) {
+      const float* xf = reinterpret_cast<const float*>(xr);
+      uint32_t pk[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        uint32_t w = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t u = __float2uint_rn(ex2((xf[4 * e + k] - m) * kLog2e) * 255.f);
+          w |= (u < 255u ? u : 255u) << (8 * k);
+        }
+        pk[e] = w;
+      }
+      tmem_st8(p_col, pk);
+    };
+
     // The loop runs every key tile even after an error (with the work
     // skipped), so that each thread takes its part in every named barrier.
-    if (!kDump && t == 1) named_arrive(3, 2 * kSoftmaxPerTile);  // tile 0 takes the first exp turn
+    if (!kNoPV && t == 1) named_arrive(3, 2 * kSoftmaxPerTile);  // tile 0 takes the first exp turn
     for (int kt = 0; kt < nkt; ++kt) {
       const int s = kt % kKS;
       const int bf = kt & 1;
@@ -605,7 +668,9 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
           // than kRescale; until then every p = exp(logit - m) <= 2^8, and the
           // final division by l (summed against the same m) cancels the
           // offset. O_t holds l in column d, so one rescale covers both.
-          const bool grow = tmax > m + kRescale;
+          // The row-max pass only keeps the max; the 8-bit pass has it already.
+          const bool grow = kF16PV && tmax > m + kRescale;
+          if constexpr (kMax) m = fmaxf(m, tmax);
           if (__any_sync(0xffffffffu, grow)) {
             const float m_new = grow ? tmax : m;
             const float corr = grow ? ex2((m - m_new) * kLog2e) : 1.f;  // 0 while m is -inf
@@ -626,13 +691,22 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         // MUFU token: the exp phases of the two tiles alternate (named barriers
         // 3 and 4 over both tiles' softmax threads), so one tile's exps run
         // while the other computes its logits.
-        named_sync(3 + t, 2 * kSoftmaxPerTile);
-        if (ok) {
-          exps(xa, s_col);
-          exps(xb, s_col + 16);
-          if (kBias) mbar_arrive(&b_empty[bs * 2 + t]);
+        if constexpr (kMax) {
+          if (ok && kBias) mbar_arrive(&b_empty[bs * 2 + t]);
+        } else {
+          named_sync(3 + t, 2 * kSoftmaxPerTile);
+          if (ok) {
+            if constexpr (kI8) {
+              exps_u8(xa, s_col);
+              exps_u8(xb, s_col + 8);
+            } else {
+              exps(xa, s_col);
+              exps(xb, s_col + 16);
+            }
+            if (kBias) mbar_arrive(&b_empty[bs * 2 + t]);
+          }
+          if (!(t == 1 && kt == nkt - 1)) named_arrive(4 - t, 2 * kSoftmaxPerTile);  // pass the token on
         }
-        if (!(t == 1 && kt == nkt - 1)) named_arrive(4 - t, 2 * kSoftmaxPerTile);  // pass the token on
       }
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
@@ -641,7 +715,43 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         mbar_arrive(&p_full[t * 2 + bf]);
       }
     }
-    if constexpr (!kDump) {
+    if constexpr (kMax) {
+      if (ok && row_valid) p.mrow[tok0 + row] = m;
+    } else if constexpr (kI8) {
+      if (ok && wait_all(&o_done[t * 2 + ((nkt - 1) & 1)], 0)) {
+        tc_fence_after();
+        // O_c = s_c * acc_c / l with the s32 sums acc_c = sum_j u_j vq_jc and
+        // l = sum_j u_j (column d, the ones channel of the 8-bit V)
+        uint32_t lbits;
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(lbits) : "r"(o_col + d));
+        tmem_ld_wait();
+        const float inv = 1.f / static_cast<float>(static_cast<int>(lbits));
+        const float* vs = p.vscale + static_cast<size_t>(bh) * d;
+        uint16_t* orow = p.out + (tok0 + row) * d;
+#pragma unroll
+        for (int cc = 0; cc < DV; cc += 16) {
+          if (cc < d) {  // warp-uniform
+            uint32_t ov[16];
+            tmem_ld16(o_col + cc, ov);
+            tmem_ld_wait();
+            if (row_valid) {
+#pragma unroll
+              for (int e = 0; e < 16; e += 8) {
+                if (cc + e < d) {
+                  float f[8];
+#pragma unroll
+                  for (int k = 0; k < 8; ++k)
+                    f[k] = __ldg(vs + cc + e + k) * static_cast<float>(static_cast<int>(ov[e + k])) * inv;
+                  *reinterpret_cast<uint4*>(orow + cc + e) =
+                      make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                                 pack_bf16x2(f[6], f[7]));
+                }
+              }
+            }
+          }
+        }
+      }
+    } else if constexpr (!kDump) {
       if (ok && wait_all(&o_done[t * 2 + ((nkt - 1) & 1)], 0)) {
         tc_fence_after();
         uint32_t lbits;  // l = O_t column d
@@ -708,15 +818,15 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
 }
 
 // Bias rows padded to ld elements (ld % 8 == 0, pad 0), so that they are TMA
-// rows: out[(h * N + i) * ld + j] = j < N ? bias[(h * N + i) * N + j] : 0.
+// rows: out[(h * N + i) * ld + j] = j < N ? bias[(h * N + i) * src_ld + j] : 0.
 __global__ void __launch_bounds__(256) pad_bias_rows_kernel(const uint16_t* __restrict__ bias,
-                                                            long long rows, int N, int ld,
+                                                            long long rows, int N, int src_ld, int ld,
                                                             uint16_t* __restrict__ out) {
   const long long e = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
   if (e >= rows * ld) return;
   const long long row = e / ld;
   const int j = static_cast<int>(e - row * ld);
-  out[e] = j < N ? bias[row * N + j] : static_cast<uint16_t>(0);
+  out[e] = j < N ? bias[row * src_ld + j] : static_cast<uint16_t>(0);
 }
 
 // Joins the two key halves of split pairs: for row i with partials (O_h, m_h,
@@ -807,7 +917,8 @@ inline int launch(const tc::Params& prm, int ctas, cudaStream_t st, std::string*
   std::memset(&tm_bias, 0, sizeof tm_bias);
   std::memset(&tm_k, 0, sizeof tm_k);
   const cuuint64_t BH = static_cast<cuuint64_t>(prm.B) * prm.H;
-  if (kMode != kModeDump && !make_rows_map(&tm_v, prm.v, BH, prm.N, prm.d, "V", msg)) return BINATTN_ERR_CUDA;
+  if ((kMode == kModeBin || kMode == kModeRef) && !make_rows_map(&tm_v, prm.v, BH, prm.N, prm.d, "V", msg))
+    return BINATTN_ERR_CUDA;
   if (kMode == kModeRef && !make_rows_map(&tm_k, prm.k, BH, prm.N, prm.d, "K", msg)) return BINATTN_ERR_CUDA;
   if (kBias && !make_bias_map(&tm_bias, prm.bias, prm.H, prm.N, prm.bias_ld > 0 ? prm.bias_ld : prm.N, msg))
     return BINATTN_ERR_CUDA;
@@ -912,6 +1023,27 @@ inline int forward_tc2(const uint32_t* qb, const uint32_t* kb, const float* aq, 
     }
   }
   return BINATTN_OK;
+}
+
+// The 8-bit P.V forward on the 64-key pipeline: the row-max pass writes the
+// exact max of every row's logits to mrow, then the 8-bit pass forms
+// u = rint(255 exp(logit - max)) and O = s * (u . vq) / sum u with V's tiled
+// 8-bit code vq8 and scales vscale (quantize_v_kernel). No tail split.
+inline int forward_tc2_int8(const uint32_t* qb, const uint32_t* kb, const float* aq, const float* ak,
+                            const uint16_t* bias, int bias_ld, const int8_t* vq8, const float* vscale, float* mrow,
+                            float scale, int B, int H, int N, int d, uint16_t* out, cudaStream_t st,
+                            std::string* msg) {
+  tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, nullptr, out, nullptr, scale, B, H, N, d, bias_ld, 0, 0,
+                 nullptr};
+  prm.vq8 = vq8;
+  prm.vscale = vscale;
+  prm.mrow = mrow;
+  const int ctas = tc2::total_pairs(B, H, N);
+  if (int rc = bias ? tc2::dispatch_dv<tc2::kModeMax, true>(prm, ctas, st, msg)
+                    : tc2::dispatch_dv<tc2::kModeMax, false>(prm, ctas, st, msg))
+    return rc;
+  return bias ? tc2::dispatch_dv<tc2::kModeI8, true>(prm, ctas, st, msg)
+              : tc2::dispatch_dv<tc2::kModeI8, false>(prm, ctas, st, msg);
 }
 
 inline int scores_tc2(const uint32_t* qb, const uint32_t* kb, int B, int H, int N, int d, int32_t* S,

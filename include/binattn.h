@@ -168,6 +168,28 @@ int binattn_forward_ws(const uint32_t *q_bits, const uint32_t *k_bits,
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * binattn_forward_bias_ld_ws — binattn_forward_ws with the bias rows
+ * bias_ld >= N elements apart: element (h, i, j) of the bias is
+ * bias[(h * N + i) * bias_ld + j] (bf16, device, 16-byte aligned, not NULL).
+ * The bias is a learned parameter, fixed across calls: a caller that stores it
+ * once with bias_ld a multiple of 8 (binattn_padded_bias_ld(N)) lets the
+ * TMA-fed pipeline read it as it is, so no call pads it again; with any other
+ * bias_ld the rows are copied into the workspace as in binattn_forward_ws.
+ * Needs d % 8 == 0 and d <= 80 when bias_ld != N (BINATTN_ERR_UNSUPPORTED
+ * otherwise); bias_ld == N is binattn_forward_ws itself. Same result as
+ * binattn_forward_ws on the same bias values.
+ *   workspace  at least binattn_forward_bias_ld_workspace_bytes(...) bytes.
+ * Source: §2 methodology, the learnable bias b_ij added before the softmax.
+ */
+size_t binattn_forward_bias_ld_workspace_bytes(int B, int H, int N, int d, int bias_ld);
+int binattn_padded_bias_ld(int N);
+int binattn_forward_bias_ld_ws(const uint32_t *q_bits, const uint32_t *k_bits,
+                               const float *alpha_q, const float *alpha_k,
+                               const uint16_t *bias, int bias_ld, const uint16_t *v,
+                               float softmax_scale, int B, int H, int N, int d, uint16_t *out,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * binattn_forward_static_ws — binattn_forward_ws for callers that cannot
  * allocate device memory: a plug-in or hook that is handed its buffers by a
  * host framework whose caching allocator owns the device's memory, or a
@@ -241,6 +263,45 @@ int binattn_forward_engine(const uint32_t *q_bits, const uint32_t *k_bits,
                            const uint16_t *bias, const uint16_t *v, float softmax_scale,
                            int B, int H, int N, int d, uint16_t *out, int engine,
                            void *stream);
+
+/*
+ * binattn_quantize_v — the per-channel 8-bit code of V that the 8-bit P.V
+ * forward multiplies by: for each (b, h, channel c),
+ * scale[b,h,c] = max_j |V[b,h,j,c]| / 127 and
+ * vq[b,h,j,c] = rint(V[b,h,j,c] / scale[b,h,c]) (ties to even, clamped to
+ * [-127, 127]; 0 when the scale is 0), in fp32.
+ *   v      [B, H, N, d] bf16, device; d % 8 == 0 (else BINATTN_ERR_UNSUPPORTED).
+ *   vq     [B, H, N, d] int8, device, written.
+ *   scale  [B, H, d] fp32, device, written.
+ * Source: §2 hybrid quantisation (values in a per-channel 8-bit code).
+ */
+int binattn_quantize_v(const uint16_t *v, int B, int H, int N, int d, int8_t *vq, float *scale,
+                       void *stream);
+
+/*
+ * binattn_forward_int8 — the forward with an 8-bit P.V, the pages' hybrid
+ * variant: the scores, scale and bias as in binattn_forward; then
+ * u_ij = rint(255 * exp(logit_ij - max_j logit_ij)) (attention coefficients on
+ * [0, 1] in a static unsigned 8-bit code), V in its per-channel 8-bit code
+ * (binattn_quantize_v), and O[b,h,i,c] = scale[b,h,c] * sum_j u_ij vq_jc /
+ * sum_j u_ij, the products and sums exact in 32-bit integers
+ * (tcgen05.mma kind::i8, the successor of mma.s32.u8.s8.s32). Two passes over
+ * the keys: the first finds each row's exact max, so that no u exceeds 255
+ * and no integer sum is ever rescaled. Needs d % 8 == 0 and d <= 80
+ * (BINATTN_ERR_UNSUPPORTED otherwise); any N; bias [H, N, N] or NULL.
+ *   workspace  device, 16-byte aligned, at least
+ *              binattn_forward_int8_workspace_bytes(...) bytes (V's tiled
+ *              8-bit code, its scales, the row maxima and, for N % 8 != 0, a
+ *              padded copy of the bias), overwritten.
+ * Source: §2 hybrid quantisation; §2 hardware-aware implementation
+ * (mma.s32.u8.s8.s32).
+ */
+size_t binattn_forward_int8_workspace_bytes(int B, int H, int N, int d, int has_bias);
+int binattn_forward_int8(const uint32_t *q_bits, const uint32_t *k_bits,
+                         const float *alpha_q, const float *alpha_k,
+                         const uint16_t *bias, const uint16_t *v, float softmax_scale,
+                         int B, int H, int N, int d, uint16_t *out,
+                         void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * binattn_scores_debug — writes the integer scores S [B, H, N, N] (int32,

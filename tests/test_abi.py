@@ -66,6 +66,20 @@ def test_forward_host_validation(L):
     assert b"NULL" in L.binattn_last_error_message() or True
 
 
+def test_bias_ld_host_validation(L):
+    def fwd(bias=A, ld=24, d=64, N=16, ws=A, wsb=1 << 20):
+        return L.binattn_forward_bias_ld_ws(P(A), P(A), P(A), P(A), P(bias) if bias else None, ld, P(A),
+                                            ctypes.c_float(0.125), 1, 1, N, d, P(A), P(ws) if ws else None,
+                                            ctypes.c_size_t(wsb), None)
+    assert fwd(bias=0) == 1                 # the bias is required
+    assert fwd(ld=15) == 8                  # rows closer than N
+    assert fwd(d=33, ld=40) == 5            # a strided bias needs the TMA-fed pipeline
+    assert fwd(bias=A + 2) == 4
+    assert L.binattn_padded_bias_ld(197) == 200 and L.binattn_padded_bias_ld(200) == 200
+    assert L.binattn_padded_bias_ld(0) == 0
+    assert L.binattn_forward_bias_ld_workspace_bytes(1, 2, 197, 64, 150) == 0  # ld < N
+
+
 def test_pack_host_validation(L):
     def pack(x=A, dt=1, B=1, H=1, N=4, d=64, bits=A, alpha=A):
         return L.binattn_pack(P(x), dt, B, H, N, d, P(bits), P(alpha), None)

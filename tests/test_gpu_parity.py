@@ -358,3 +358,34 @@ def test_bounded_wait_runs_out_and_context_survives(orc, with_bias):
     ref = orc.forward(c["q"], c["k"], c["bias"] if with_bias else None, c["v"], c["softmax_scale"])
     r = run_path(c, engine="tc", with_bias=with_bias)
     check_o(bf16_to_f64(r["out"]), ref, f"after timeout bias={with_bias}")
+
+
+# ------------------------------------------ bias stored once with padded rows
+# A learned bias stored with rows bias_ld apart: with bias_ld % 8 == 0 the
+# TMA-fed pipeline reads it as it is (no padding kernel on the call), with any
+# other bias_ld the call pads it as binattn_forward_ws does. Either way O is
+# bit-identical to binattn_forward_ws on the same values, and meets the oracle.
+@pytest.mark.parametrize("shape", [(1, 2, 197, 64), (2, 3, 129, 72), (1, 2, 1001, 40), (2, 2, 256, 64)])
+def test_forward_bias_ld(orc, shape):
+    B, H, N, d = shape
+    c = make_custom(B, H, N, d, seed=13 * N + d, with_bias=True, bias_std=0.5)
+    q, k, v, bias = dev(c["q"]), dev(c["k"]), dev(c["v"]), dev(c["bias"])
+    qb, aq = binattn.pack(q)
+    kb, ak = binattn.pack(k)
+    want = binattn.forward_ws(qb, kb, aq, ak, bias, v, c["softmax_scale"])
+    ld8 = binattn.padded_bias_ld(N)
+    assert ld8 % 8 == 0 and N <= ld8 < N + 8
+    for ld in (ld8, ld8 + 3, ld8 + 8):
+        stored = torch.zeros((H, N, ld), dtype=torch.bfloat16, device="cuda")
+        stored[:, :, :N] = bias
+        stored[:, :, N:] = 7.0  # columns beyond N are never read
+        got = binattn.forward_bias_ld_ws(qb, kb, aq, ak, stored, v, c["softmax_scale"])
+        torch.cuda.synchronize()
+        binattn.device_status()
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16)), f"{shape} ld={ld}"
+        if ld % 8 == 0:  # no padded copy: only the split partials, as without a bias
+            assert binattn.lib().binattn_forward_bias_ld_workspace_bytes(B, H, N, d, ld) == \
+                binattn.workspace_bytes(B, H, N, d, False)
+    ref = orc.forward(c["q"], c["k"], c["bias"], c["v"], c["softmax_scale"])
+    check_o(bf16_to_f64(binattn.forward_bias_ld_ws(qb, kb, aq, ak, binattn.pad_bias(bias), v, c["softmax_scale"])),
+            ref, f"bias_ld {shape}")
