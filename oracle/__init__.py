@@ -64,11 +64,13 @@ class Oracle:
         lib.oracle_quantize_v.argtypes = [V, L, L, L, L, V, V]
         lib.oracle_forward_int8_rows.argtypes = [V, V, I, V, V, D, L, L, L, L, L, _i64p, V]
         lib.oracle_forward_int8.argtypes = [V, V, I, V, V, D, L, L, L, L, V]
+        lib.oracle_expand_relpos_bias.argtypes = [V, L, L, L, L, V]
         lib.oracle_num_threads.restype = I
         lib.oracle_set_num_threads.argtypes = [I]
         for f in ("oracle_pack", "oracle_scores_rows", "oracle_probs_rows",
                   "oracle_forward_rows", "oracle_forward", "oracle_forward_spread",
-                  "oracle_quantize_v", "oracle_forward_int8_rows", "oracle_forward_int8"):
+                  "oracle_quantize_v", "oracle_forward_int8_rows", "oracle_forward_int8",
+                  "oracle_expand_relpos_bias"):
             getattr(lib, f).restype = I
         self.lib = lib
 
@@ -237,6 +239,21 @@ class Oracle:
         if rc:
             raise RuntimeError(f"oracle_forward_int8 failed ({rc})")
         return O
+
+    # ----------------------------------------- the position-sensitive bias
+    def expand_relpos_bias(self, table, gh: int, gw: int, n_cls: int) -> np.ndarray:
+        """The dense bias [H, N, N] (bf16 bits), N = n_cls + gh * gw, of a
+        relative-position table [H, (2gh-1)(2gw-1) + 3 n_cls] (bf16 bits)."""
+        H, R = table.shape
+        if R != (2 * gh - 1) * (2 * gw - 1) + 3 * n_cls:
+            raise ValueError(f"table has {R} entries per head, expected {(2 * gh - 1) * (2 * gw - 1) + 3 * n_cls}")
+        t = self._bf16(table, "table", (H, R))
+        N = n_cls + gh * gw
+        out = np.zeros((H, N, N), dtype=np.uint16)
+        rc = self.lib.oracle_expand_relpos_bias(_ptr(t), H, gh, gw, n_cls, _ptr(out))
+        if rc:
+            raise RuntimeError(f"oracle_expand_relpos_bias failed ({rc})")
+        return out
 
 
 _default: Oracle | None = None

@@ -55,6 +55,18 @@
  *   9. O_ic = s_c * (sum_j u_ij vq_jc) / (sum_j u_ij), the row sum taken from
  *      the same 8-bit weights.
  *
+ * The position-sensitive bias ([ES] §2 "Mejora mediante Sesgo": the bias may
+ * be dense, position-sensitive or context-aware; [KO] §2 나-2) is read as a
+ * relative-position table, expanded to the dense bias by
+ * oracle_expand_relpos_bias:
+ *  10. tokens n_cls .. N - 1 are the patches of a gh x gw grid in row-major
+ *      order (patch p at row p / gw, column p % gw); n_cls (0 or 1) class
+ *      tokens come first. For two patches, bias[h, i, j] =
+ *      table[h, (y_i - y_j + gh - 1) * (2 gw - 1) + (x_i - x_j + gw - 1)];
+ *      with R0 = (2 gh - 1)(2 gw - 1), a class query and a patch key take
+ *      table[h, R0], a patch query and a class key table[h, R0 + 1], class
+ *      with class table[h, R0 + 2]. The table is bf16 [H, R0 + 3 n_cls].
+ *
  * Parity pins for each function live in the CPU test suite (exhaustive sign
  * predicate, packbits layout, Hamming identity, closed forms, invariants and an
  * independent numpy formulation on small cases).
@@ -524,4 +536,35 @@ int oracle_forward_int8(const void *q, const void *k, int qk_dtype,
     int rc = oracle_forward_int8_rows(q, k, qk_dtype, bias, v, softmax_scale, B, H, N, d, (long)T, rows, O);
     free(rows);
     return rc;
+}
+
+/* Step 10: the dense bias [H, N, N] (bf16 bits) of a relative-position table. */
+int oracle_expand_relpos_bias(const uint16_t *table, long H, long gh, long gw, long n_cls, uint16_t *bias)
+{
+    if (!table || !bias || H < 1 || gh < 1 || gw < 1 || n_cls < 0 || n_cls > 1)
+        return 1;
+    const long N = n_cls + gh * gw;
+    const long R0 = (2 * gh - 1) * (2 * gw - 1);
+    const long R = R0 + 3 * n_cls;
+    for (long h = 0; h < H; h++) {
+        for (long i = 0; i < N; i++) {
+            uint16_t *brow = bias + ((size_t)h * N + (size_t)i) * (size_t)N;
+            for (long j = 0; j < N; j++) {
+                long idx;
+                if (i < n_cls && j < n_cls)
+                    idx = R0 + 2;
+                else if (i < n_cls)
+                    idx = R0;
+                else if (j < n_cls)
+                    idx = R0 + 1;
+                else {
+                    const long pi = i - n_cls, pj = j - n_cls;
+                    const long dy = pi / gw - pj / gw, dx = pi % gw - pj % gw;
+                    idx = (dy + gh - 1) * (2 * gw - 1) + (dx + gw - 1);
+                }
+                brow[j] = table[(size_t)h * R + idx];
+            }
+        }
+    }
+    return 0;
 }

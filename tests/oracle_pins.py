@@ -441,6 +441,53 @@ def pin_int8_two_keys_closed_form(orc):
     assert np.array_equal(O1[0, :, 0], 0.125 * kk[0, :, 1]) and np.array_equal(O1[0, :, 1], 0.125 * kk[0, :, 0])
 
 
+# ------------------------------------------------ position-sensitive bias
+def pin_relpos_one_hot_counts(orc):
+    """A table that is 1 at one displacement (dy, dx) and 0 elsewhere expands
+    to a bias whose 1s are exactly the patch pairs at that displacement:
+    (gh - |dy|)(gw - |dx|) of them per head, each with y_i - y_j = dy and
+    x_i - x_j = dx; the class entries land on the class row and column."""
+    for gh, gw, n_cls in [(3, 4, 0), (4, 3, 1), (1, 5, 1), (5, 5, 0)]:
+        R0 = (2 * gh - 1) * (2 * gw - 1)
+        N = n_cls + gh * gw
+        for dy in range(-(gh - 1), gh):
+            for dx in range(-(gw - 1), gw):
+                t = np.zeros((1, R0 + 3 * n_cls), dtype=np.float32)
+                t[0, (dy + gh - 1) * (2 * gw - 1) + dx + gw - 1] = 1.0
+                b = _f64(orc.expand_relpos_bias(f32_to_bf16_bits(t), gh, gw, n_cls))[0]
+                ii, jj = np.nonzero(b)
+                assert len(ii) == (gh - abs(dy)) * (gw - abs(dx)), (gh, gw, dy, dx)
+                assert np.all(ii >= n_cls) and np.all(jj >= n_cls)
+                pi, pj = ii - n_cls, jj - n_cls
+                assert np.all(pi // gw - pj // gw == dy) and np.all(pi % gw - pj % gw == dx)
+        if n_cls:
+            for e, (i, j) in enumerate([(0, 5 % N or 1), (min(2, N - 1), 0), (0, 0)]):
+                t = np.zeros((1, R0 + 3), dtype=np.float32)
+                t[0, R0 + e] = 2.0
+                b = _f64(orc.expand_relpos_bias(f32_to_bf16_bits(t), gh, gw, 1))[0]
+                assert b[i, j] == 2.0
+                assert np.count_nonzero(b) == [N - 1, N - 1, 1][e]
+
+
+def pin_relpos_translation_invariance(orc):
+    """A random table: pairs of patches with the same displacement get the same
+    value, and every table entry of a head is reached (the map from
+    displacements to entries is onto), also per head."""
+    rng = np.random.default_rng(61)
+    gh, gw = 4, 6
+    R0 = (2 * gh - 1) * (2 * gw - 1)
+    t = f32_to_bf16_bits(rng.standard_normal((2, R0)).astype(np.float32))
+    b = _f64(orc.expand_relpos_bias(t, gh, gw, 0))
+    y, x = np.divmod(np.arange(gh * gw), gw)
+    dy, dx = y[:, None] - y[None, :], x[:, None] - x[None, :]
+    for h in range(2):
+        seen = {}
+        for a, c, v in zip(dy.ravel(), dx.ravel(), b[h].ravel()):
+            assert seen.setdefault((a, c), v) == v
+        assert len(seen) == R0
+        assert sorted(seen.values()) == sorted(_f64(t)[h].tolist())
+
+
 ALL_PINS = [
     pin_sign_predicate_exhaustive,
     pin_pack_layout_packbits,
@@ -464,4 +511,6 @@ ALL_PINS = [
     pin_quantize_v_closed_form,
     pin_int8_uniform_scores,
     pin_int8_two_keys_closed_form,
+    pin_relpos_one_hot_counts,
+    pin_relpos_translation_invariance,
 ]

@@ -68,6 +68,13 @@ MUTANTS = [
     ("8-bit row sum dropped",
      "O_rows[(size_t)r * d + c] = (double)s[bh * (size_t)d + c] * acc / usum;",
      "O_rows[(size_t)r * d + c] = (double)s[bh * (size_t)d + c] * acc / 255.0;"),
+    ("relative position with the key and query swapped",
+     "const long dy = pi / gw - pj / gw, dx = pi % gw - pj % gw;",
+     "const long dy = pj / gw - pi / gw, dx = pj % gw - pi % gw;"),
+    ("relative position rows of width gw instead of 2 gw - 1",
+     "idx = (dy + gh - 1) * (2 * gw - 1) + (dx + gw - 1);", "idx = (dy + gh - 1) * gw + (dx + gw - 1);"),
+    ("class entries swapped",
+     "idx = R0;\n", "idx = R0 + 1;\n"),
 ]
 
 
