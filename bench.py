@@ -611,6 +611,44 @@ def run_gpu(args, w_job, rank, world, local_rank):
             del iws
         binattn.device_status(stream)
 
+    # the position-sensitive bias: a relative-position table of the square
+    # patch grid (DiT's latent patches; no class token) instead of the dense
+    # [H, N, N] bias, same step and protocol
+    relpos = {}
+    g = int(round(math.sqrt(N)))
+    if args.engine == "auto" and g * g == N and d % 8 == 0 and d <= 80:
+        R = binattn.relpos_table_entries(g, g, 0)
+        trng = np.random.default_rng(rank_seed(w, rank) + 77)
+        table = torch.from_numpy((trng.standard_normal((H, R)) * 0.05).astype(np.float32)).to(dev).bfloat16()
+        rws = torch.empty(max(16, binattn.lib().binattn_forward_relpos_workspace_bytes(B, H, N, d)),
+                          dtype=torch.uint8, device=dev)
+        fr = lambda: binattn.forward_relpos(qb, kb, aq, ak, table, (g, g), 0, v, scale, workspace=rws, out=out,
+                                            stream=stream)
+        fr()
+        torch.cuda.synchronize()
+        barrier()
+        ev = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record(stream)
+            binattn.pack(q, qb, aq, stream)
+            binattn.pack(k, kb, ak, stream)
+            e1.record(stream)
+            fr()
+            e2.record(stream)
+            ev.append((e0, e1, e2))
+        torch.cuda.synchronize()
+        barrier()
+        binattn.device_status(stream)
+        rms = max_over_ranks(sum(b_.elapsed_time(c) for _, b_, c in ev) / len(ev))
+        relpos = {"grid": [g, g], "table_entries_per_head": R,
+                  "ms_per_step": round(max_over_ranks(sum(a.elapsed_time(c) for a, _, c in ev) / len(ev)), 5),
+                  "forward_ms": round(rms, 5), "call": "binattn_forward_relpos",
+                  "roofline": roofline_line(w, False, peaks, rms * 1e-3,
+                                            torch.cuda.get_device_properties(dev).multi_processor_count)}
+        del table, rws
+
     # in-build bf16 attention on the same shapes (speed reference)
     ref = None
     try:
@@ -691,6 +729,7 @@ def run_gpu(args, w_job, rank, world, local_rank):
                     "effective_tflops": round(a0["eff_flops"] / fwd0_s / 1e12, 2),
                     "roofline": roof0},
         "bf16_reference": ref,
+        "relpos_bias": relpos,
         "int8_pv": dict(int8, call="binattn_forward_int8 (V 8-bit code + row-max pass + 8-bit P.V pass)",
                         step="pack(Q) + pack(K) + binattn_forward_int8"),
         "other_workloads": others,

@@ -30,6 +30,7 @@ EXPORTS = (
     "binattn_last_error_message", "binattn_abi_version", "binattn_test_wait_timeout",
     "binattn_forward_bias_ld_workspace_bytes", "binattn_padded_bias_ld", "binattn_forward_bias_ld_ws",
     "binattn_quantize_v", "binattn_forward_int8_workspace_bytes", "binattn_forward_int8",
+    "binattn_forward_relpos_workspace_bytes", "binattn_forward_relpos",
 )
 
 
@@ -75,6 +76,10 @@ def lib() -> ctypes.CDLL:
     L.binattn_forward_int8_workspace_bytes.restype = ctypes.c_size_t
     L.binattn_forward_int8.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
     L.binattn_forward_int8.restype = I
+    L.binattn_forward_relpos_workspace_bytes.argtypes = [I, I, I, I]
+    L.binattn_forward_relpos_workspace_bytes.restype = ctypes.c_size_t
+    L.binattn_forward_relpos.argtypes = [P, P, P, P, P, I, I, I, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
+    L.binattn_forward_relpos.restype = I
     L.binattn_forward_fused_workspace_bytes.argtypes = [I, I, I, I, I, I]
     L.binattn_forward_fused_workspace_bytes.restype = ctypes.c_size_t
     L.binattn_forward_fused_ws.argtypes = [P, I, P, P, P, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
@@ -328,6 +333,39 @@ def forward_int8(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tens
         _check(lib().binattn_forward_int8(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k), _ptr(bias),
                                           _ptr(v), float(softmax_scale), B, H, N, d, _ptr(out), _ptr(workspace),
                                           ctypes.c_size_t(size), _stream(stream, dev)), "binattn_forward_int8")
+    return out
+
+
+def relpos_table_entries(gh: int, gw: int, n_cls: int) -> int:
+    """Entries per head of a relative-position table: (2gh-1)(2gw-1) + 3 n_cls."""
+    return (2 * gh - 1) * (2 * gw - 1) + 3 * n_cls
+
+
+def forward_relpos(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor, alpha_k: torch.Tensor,
+                   table: torch.Tensor, grid: tuple[int, int], n_cls: int, v: torch.Tensor, softmax_scale: float,
+                   workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """forward with the position-sensitive bias: a relative-position table
+    [H, relpos_table_entries(gh, gw, n_cls)] (bf16) of a gh x gw patch grid
+    after n_cls class tokens (binattn_forward_relpos)."""
+    B, H, N, d = v.shape
+    gh, gw = grid
+    _expect(table, "table", (H, relpos_table_entries(gh, gw, n_cls)), (torch.bfloat16,))
+    dev = _forward_args(q_bits, k_bits, alpha_q, alpha_k, None, v, out)
+    _device(table, v)
+    if workspace is not None:
+        _device(workspace, v)
+    need = int(lib().binattn_forward_relpos_workspace_bytes(B, H, N, d))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    size = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        _check(lib().binattn_forward_relpos(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k), _ptr(table),
+                                            int(gh), int(gw), int(n_cls), _ptr(v), float(softmax_scale), B, H, N, d,
+                                            _ptr(out), _ptr(workspace), ctypes.c_size_t(size), _stream(stream, dev)),
+               "binattn_forward_relpos")
     return out
 
 

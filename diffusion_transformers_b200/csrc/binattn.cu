@@ -491,6 +491,41 @@ int binattn_forward_int8(const uint32_t* q_bits, const uint32_t* k_bits, const f
   return ok();
 }
 
+size_t binattn_forward_relpos_workspace_bytes(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || d < 1 || !binattn::tc2::supported(d, N, false, false)) return 0;
+  return binattn::tc2::split_part_bytes(B, H, N, d);
+}
+
+int binattn_forward_relpos(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
+                           const float* alpha_k, const uint16_t* table, int gh, int gw, int n_cls,
+                           const uint16_t* v, float softmax_scale, int B, int H, int N, int d, uint16_t* out,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  BINATTN_CHECK_PTR(table);
+  if (int rc = check_forward_args(q_bits, k_bits, alpha_q, alpha_k, nullptr, v, softmax_scale, B, H, N, d, out))
+    return rc;
+  if (gh < 1 || gw < 1 || (n_cls != 0 && n_cls != 1) || static_cast<long long>(gh) * gw + n_cls != N)
+    return fail(BINATTN_ERR_SHAPE, "N = %d is not n_cls + gh * gw (%d + %d * %d)", N, n_cls, gh, gw);
+  const long long R = static_cast<long long>(2 * gh - 1) * (2 * gw - 1) + 3 * n_cls;
+  if (R > binattn::tc2::kRelTabMax)
+    return fail(BINATTN_ERR_UNSUPPORTED, "a %lld-entry table is more than the %d that fit in shared memory", R,
+                binattn::tc2::kRelTabMax);
+  if (!binattn::tc2::supported(d, N, false, false))
+    return fail(BINATTN_ERR_UNSUPPORTED, "the position-sensitive bias needs d %% 8 == 0 and d <= 80 (d = %d)", d);
+  const size_t need = binattn_forward_relpos_workspace_bytes(B, H, N, d);
+  if (need) {
+    BINATTN_CHECK_PTR(workspace);
+    if (workspace_bytes < need)
+      return fail(BINATTN_ERR_ARG, "workspace of %zu bytes is below the %zu this shape needs", workspace_bytes,
+                  need);
+  }
+  std::string msg;
+  if (int rc = binattn::forward_tc2_relpos(q_bits, k_bits, alpha_q, alpha_k, table, gh, gw, n_cls, v,
+                                           softmax_scale, B, H, N, d, out, static_cast<cudaStream_t>(stream), &msg,
+                                           need ? static_cast<float*>(workspace) : nullptr))
+    return fail(rc, "%s", msg.c_str());
+  return ok();
+}
+
 int binattn_scores_debug(const uint32_t* q_bits, const uint32_t* k_bits, int B, int H, int N,
                          int d, int32_t* S, int engine, void* stream) {
   BINATTN_CHECK_PTR(q_bits);

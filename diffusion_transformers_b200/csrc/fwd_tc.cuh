@@ -153,6 +153,11 @@ struct Params {
   const int8_t* vq8 = nullptr;
   const float* vscale = nullptr;
   float* mrow = nullptr;
+  // Position-sensitive bias (64-key pipeline): the relative-position table
+  // bf16 [H, rel_R] of a rel_gh x rel_gw patch grid after rel_ncls (0 or 1)
+  // class tokens, rel_R = (2 gh - 1)(2 gw - 1) + 3 ncls.
+  const uint16_t* rel_table = nullptr;
+  int rel_gh = 0, rel_gw = 0, rel_ncls = 0, rel_R = 0;
 };
 
 // Named barrier 1 over the load-mode loader warps with an AND reduction.

@@ -102,9 +102,18 @@ inline int dv_for(int d) { return d < 32 ? 32 : d < 64 ? 64 : d < 80 ? 80 : 96; 
 //  V      [kKS] 64 keys x DV bf16, MN-major: chunk (key j, group g of 8) at
 //         g * 1024 + j * 16 -> LBO = 128 (next 8 keys), SBO = 1024 (next 8 channels).
 //  ak     [kKS] 64 fp32.
-template <int DV, int kMode, bool kBias>
+// Bias kinds of the 64-key pipeline.
+constexpr int kNoBias = 0;
+constexpr int kDenseBias = 1;   // bf16 [H, N, N] (rows bias_ld apart), TMA boxes
+constexpr int kRelPosBias = 2;  // relative-position table [H, R] gathered from shared memory
+constexpr int kRelTabMax = 20480;  // table entries per head that fit beside the stages (fp32)
+constexpr int kClsKey = -(1 << 30);  // key offset that marks a class key
+
+template <int DV, int kMode, int kBiasKind>
 struct Layout {
-  static constexpr int kKS = kBias ? 4 : 8;                      // K / V / alpha_k stages
+  static constexpr bool kBias = kBiasKind == kDenseBias;
+  static constexpr bool kRel = kBiasKind == kRelPosBias;
+  static constexpr int kKS = (kBias || kRel) ? 4 : 8;            // K / V / alpha_k stages
   static constexpr int kBS = 4;                                  // bias stages (per t)
   static constexpr int kBiasTile = kRows * kKeys * 2;            // 16 KB
   static constexpr int kKTile = kMode == kModeRef ? kKeys * DV * 2 : kKeys * 96;
@@ -114,7 +123,9 @@ struct Layout {
   static constexpr int kK = kBiasOff + (kBias ? kBS * 2 * kBiasTile : 0);
   static constexpr int kV = kK + kKS * kKTile;
   static constexpr int kAk = kV + kKS * kVTile;
-  static constexpr int kBar = kAk + kKS * kKeys * 4;
+  static constexpr int kKo = kAk + kKS * kKeys * 4;               // relative-position key offsets
+  static constexpr int kTab = kKo + (kRel ? kKS * kKeys * 4 : 0);  // relative-position table (fp32)
+  static constexpr int kBar = kTab + (kRel ? kRelTabMax * 4 : 0);
   static constexpr int kNumBars = 48;
   static constexpr int kMisc = kBar + 8 * kNumBars;  // tmem base, abort flag
   static constexpr int kBytes = kMisc + 16;
@@ -201,11 +212,13 @@ __device__ __forceinline__ uint32_t e4m3_bytes(uint32_t word, int j0, int c0, in
   return v;
 }
 
-template <int DV, int kMode, bool kBias>
+template <int DV, int kMode, int kBiasKind>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
                const __grid_constant__ CUtensorMap tm_bias, const __grid_constant__ CUtensorMap tm_k) {
-  using L = Layout<DV, kMode, kBias>;
+  using L = Layout<DV, kMode, kBiasKind>;
+  constexpr bool kBias = L::kBias;  // dense bias
+  constexpr bool kRel = L::kRel;    // relative-position table
   constexpr bool kRef = kMode == kModeRef;
   constexpr bool kDump = kMode == kModeDump;
   constexpr bool kMax = kMode == kModeMax;
@@ -272,6 +285,12 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         *reinterpret_cast<uint4*>(smem + L::kK + s * L::kKTile + g * 1024 + kk * 16) = make_uint4(0, 0, 0, 0);
       }
     }
+  }
+  if constexpr (kRel) {
+    // this head's relative-position table, widened to fp32 once
+    float* tab = reinterpret_cast<float*>(smem + L::kTab);
+    const uint16_t* src_t = p.rel_table + static_cast<size_t>(h) * p.rel_R;
+    for (int e = threadIdx.x; e < p.rel_R; e += kThreads) tab[e] = bf16_bits_to_float(src_t[e]);
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kKS; ++s) {
@@ -405,6 +424,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       struct TileRegs {
         uint32_t wd[2][3];
         float ak[2];
+        int ko[2];
       };
       auto load_tile = [&](int kt, TileRegs& tr) {
 #pragma unroll
@@ -414,6 +434,12 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
 #pragma unroll
           for (int w = 0; w < 3; ++w) tr.wd[u][w] = (in && w < W) ? __ldg(p.kb + (tok0 + key) * W + w) : 0u;
           tr.ak[u] = (!kDump && in) ? __ldg(p.ak + tok0 + key) : 0.f;
+          if constexpr (kRel) {
+            // -(y_j (2 gw - 1) + x_j) for a patch key, so that a patch query's
+            // base plus it is the table entry of their displacement
+            const int pj = key - p.rel_ncls;
+            tr.ko[u] = !in ? 0 : pj < 0 ? kClsKey : -((pj / p.rel_gw) * (2 * p.rel_gw - 1) + pj % p.rel_gw);
+          }
         }
       };
       TileRegs cur, n1;
@@ -443,6 +469,11 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
           float* aks = reinterpret_cast<float*>(smem + L::kAk) + s * kKeys;
 #pragma unroll
           for (int u = 0; u < 2; ++u) aks[lane + 32 * u] = cur.ak[u];
+          if constexpr (kRel) {
+            int* kos = reinterpret_cast<int*>(smem + L::kKo) + s * kKeys;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) kos[lane + 32 * u] = cur.ko[u];
+          }
         }
         fence_proxy_async_smem();
         mbar_arrive(&kv_full[s]);
@@ -547,6 +578,23 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       return r1;
     };
     // logits of chunk c (32 keys, in place): S * alpha_k * (scale * alpha_q) + bias
+    // Position-sensitive bias: a patch query i reads table entry
+    // rel_base + ko_j for a patch key j (ko_j staged by the expander); a class
+    // query (and a row >= N, whose result is not stored) reads one fixed entry
+    // for every patch key; a class key reads rel_cls_key.
+    int rel_base = 0, rel_fixed = -1, rel_cls_key = 0;
+    if constexpr (kRel) {
+      const int R0 = (2 * p.rel_gh - 1) * (2 * p.rel_gw - 1);
+      const int pi = row - p.rel_ncls;
+      if (row_valid && pi >= 0) {
+        rel_base = (pi / p.rel_gw + p.rel_gh - 1) * (2 * p.rel_gw - 1) + pi % p.rel_gw + p.rel_gw - 1;
+        rel_cls_key = R0 + 1;
+      } else {
+        rel_fixed = row_valid ? R0 : 0;
+        rel_cls_key = row_valid ? R0 + 2 : 0;
+      }
+    }
+    const float* rel_tab = reinterpret_cast<const float*>(smem + L::kTab);
     auto logits = [&](uint32_t* xr, int c, const uint8_t* bsm, const float* aks) {
       float2* xs = reinterpret_cast<float2*>(xr);
       const float2 ci2 = make_float2(ci, ci);
@@ -561,6 +609,20 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             bv[e] = make_float2(__uint_as_float(rw[e] << 16), __uint_as_float(rw[e] & 0xFFFF0000u));
+        } else if constexpr (kRel) {
+          // the stage's key offsets follow its alpha_k (Layout: kKo = kAk + kKS * 64 * 4)
+          const int* kos = reinterpret_cast<const int*>(aks + kKS * kKeys) + kChunk * c + 8 * q;
+          const int4 o0 = *reinterpret_cast<const int4*>(kos);
+          const int4 o1 = *reinterpret_cast<const int4*>(kos + 4);
+          const int o[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+          float bb[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int idx = o[e] == kClsKey ? rel_cls_key : (rel_fixed >= 0 ? rel_fixed : rel_base + o[e]);
+            bb[e] = rel_tab[idx];
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) bv[e] = make_float2(bb[2 * e], bb[2 * e + 1]);
         }
         if constexpr (kRef) {
 #pragma unroll
@@ -910,8 +972,9 @@ inline bool make_bias_map(CUtensorMap* tm, const uint16_t* bias, cuuint64_t H, c
   return true;
 }
 
-template <int DV, int kMode, bool kBias>
+template <int DV, int kMode, int kBiasKind>
 inline int launch(const tc::Params& prm, int ctas, cudaStream_t st, std::string* msg) {
+  constexpr bool kBias = kBiasKind == kDenseBias;
   CUtensorMap tm_v, tm_bias, tm_k;
   std::memset(&tm_v, 0, sizeof tm_v);
   std::memset(&tm_bias, 0, sizeof tm_bias);
@@ -922,8 +985,8 @@ inline int launch(const tc::Params& prm, int ctas, cudaStream_t st, std::string*
   if (kMode == kModeRef && !make_rows_map(&tm_k, prm.k, BH, prm.N, prm.d, "K", msg)) return BINATTN_ERR_CUDA;
   if (kBias && !make_bias_map(&tm_bias, prm.bias, prm.H, prm.N, prm.bias_ld > 0 ? prm.bias_ld : prm.N, msg))
     return BINATTN_ERR_CUDA;
-  auto kern = fwd_tc2_kernel<DV, kMode, kBias>;
-  constexpr int smem = Layout<DV, kMode, kBias>::kLaunchBytes;
+  auto kern = fwd_tc2_kernel<DV, kMode, kBiasKind>;
+  constexpr int smem = Layout<DV, kMode, kBiasKind>::kLaunchBytes;
   static_assert(smem <= 227 * 1024, "shared memory over the sm_100 per-CTA limit");
   static std::atomic<uint64_t> configured{0};  // attribute set once per device and instantiation
   if (needs_setup(configured)) {
@@ -943,18 +1006,18 @@ inline int launch(const tc::Params& prm, int ctas, cudaStream_t st, std::string*
   return BINATTN_OK;
 }
 
-template <int kMode, bool kBias>
+template <int kMode, int kBiasKind>
 inline int dispatch_dv(const tc::Params& prm, int ctas, cudaStream_t st, std::string* msg) {
   switch (dv_for(prm.d)) {
-    case 32: return launch<32, kMode, kBias>(prm, ctas, st, msg);
-    case 64: return launch<64, kMode, kBias>(prm, ctas, st, msg);
-    case 80: return launch<80, kMode, kBias>(prm, ctas, st, msg);
+    case 32: return launch<32, kMode, kBiasKind>(prm, ctas, st, msg);
+    case 64: return launch<64, kMode, kBiasKind>(prm, ctas, st, msg);
+    case 80: return launch<80, kMode, kBiasKind>(prm, ctas, st, msg);
     default:
       if constexpr (kMode == kModeRef) {
         *msg = "reference attention on the 128-key pipeline needs d <= 72";
         return BINATTN_ERR_UNSUPPORTED;
       } else {
-        return launch<96, kMode, kBias>(prm, ctas, st, msg);
+        return launch<96, kMode, kBiasKind>(prm, ctas, st, msg);
       }
   }
 }
@@ -1003,8 +1066,8 @@ inline int forward_tc2(const uint32_t* qb, const uint32_t* kb, const float* aq, 
                  nullptr, qh, stall_after};
   const tc2::SplitPlan plan = part ? tc2::split_plan(B, H, N) : tc2::SplitPlan{tc2::total_pairs(B, H, N), 0};
   auto run = [&](int ctas) {
-    return bias ? tc2::dispatch_dv<tc2::kModeBin, true>(prm, ctas, st, msg)
-                : tc2::dispatch_dv<tc2::kModeBin, false>(prm, ctas, st, msg);
+    return bias ? tc2::dispatch_dv<tc2::kModeBin, tc2::kDenseBias>(prm, ctas, st, msg)
+                : tc2::dispatch_dv<tc2::kModeBin, tc2::kNoBias>(prm, ctas, st, msg);
   };
   if (plan.full > 0) {
     if (int rc = run(plan.full)) return rc;
@@ -1014,6 +1077,40 @@ inline int forward_tc2(const uint32_t* qb, const uint32_t* kb, const float* aq, 
     prm.split = 1;
     prm.part = part;
     if (int rc = run(2 * plan.tail)) return rc;
+    const int rows = plan.tail * 2 * tc2::kRows;
+    tc2::combine_halves_kernel<<<(rows + 255) / 256, 256, 0, st>>>(part, plan.full, plan.tail, B, H, N, d, out);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      *msg = std::string("combine_halves_kernel launch: ") + cudaGetErrorString(e);
+      return BINATTN_ERR_CUDA;
+    }
+  }
+  return BINATTN_OK;
+}
+
+// The binary forward with the position-sensitive bias: table bf16
+// [H, (2gh - 1)(2gw - 1) + 3 ncls] of a gh x gw patch grid after ncls class
+// tokens (N = ncls + gh * gw), gathered per key from shared memory instead of
+// a dense [H, N, N] read. part: as for forward_tc2 (tail split), or null.
+inline int forward_tc2_relpos(const uint32_t* qb, const uint32_t* kb, const float* aq, const float* ak,
+                              const uint16_t* table, int gh, int gw, int ncls, const uint16_t* v, float scale,
+                              int B, int H, int N, int d, uint16_t* out, cudaStream_t st, std::string* msg,
+                              float* part) {
+  tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, nullptr, v, out, nullptr, scale, B, H, N, d, 0, 0, 0, nullptr};
+  prm.rel_table = table;
+  prm.rel_gh = gh;
+  prm.rel_gw = gw;
+  prm.rel_ncls = ncls;
+  prm.rel_R = (2 * gh - 1) * (2 * gw - 1) + 3 * ncls;
+  const tc2::SplitPlan plan = part ? tc2::split_plan(B, H, N) : tc2::SplitPlan{tc2::total_pairs(B, H, N), 0};
+  if (plan.full > 0) {
+    if (int rc = tc2::dispatch_dv<tc2::kModeBin, tc2::kRelPosBias>(prm, plan.full, st, msg)) return rc;
+  }
+  if (plan.tail > 0) {
+    prm.pair_base = plan.full;
+    prm.split = 1;
+    prm.part = part;
+    if (int rc = tc2::dispatch_dv<tc2::kModeBin, tc2::kRelPosBias>(prm, 2 * plan.tail, st, msg)) return rc;
     const int rows = plan.tail * 2 * tc2::kRows;
     tc2::combine_halves_kernel<<<(rows + 255) / 256, 256, 0, st>>>(part, plan.full, plan.tail, B, H, N, d, out);
     cudaError_t e = cudaGetLastError();
@@ -1039,18 +1136,18 @@ inline int forward_tc2_int8(const uint32_t* qb, const uint32_t* kb, const float*
   prm.vscale = vscale;
   prm.mrow = mrow;
   const int ctas = tc2::total_pairs(B, H, N);
-  if (int rc = bias ? tc2::dispatch_dv<tc2::kModeMax, true>(prm, ctas, st, msg)
-                    : tc2::dispatch_dv<tc2::kModeMax, false>(prm, ctas, st, msg))
+  if (int rc = bias ? tc2::dispatch_dv<tc2::kModeMax, tc2::kDenseBias>(prm, ctas, st, msg)
+                    : tc2::dispatch_dv<tc2::kModeMax, tc2::kNoBias>(prm, ctas, st, msg))
     return rc;
-  return bias ? tc2::dispatch_dv<tc2::kModeI8, true>(prm, ctas, st, msg)
-              : tc2::dispatch_dv<tc2::kModeI8, false>(prm, ctas, st, msg);
+  return bias ? tc2::dispatch_dv<tc2::kModeI8, tc2::kDenseBias>(prm, ctas, st, msg)
+              : tc2::dispatch_dv<tc2::kModeI8, tc2::kNoBias>(prm, ctas, st, msg);
 }
 
 inline int scores_tc2(const uint32_t* qb, const uint32_t* kb, int B, int H, int N, int d, int32_t* S,
                       cudaStream_t st, std::string* msg) {
   tc::Params prm{qb, kb, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S, 0.f, B, H, N, d, 0, 0, 0,
                  nullptr};
-  return tc2::launch<32, tc2::kModeDump, false>(prm, tc2::total_pairs(B, H, N), st, msg);
+  return tc2::launch<32, tc2::kModeDump, tc2::kNoBias>(prm, tc2::total_pairs(B, H, N), st, msg);
 }
 
 inline int forward_ref_tc2(const uint16_t* q, const uint16_t* k, const uint16_t* bias, const uint16_t* v,
@@ -1059,8 +1156,8 @@ inline int forward_ref_tc2(const uint16_t* q, const uint16_t* k, const uint16_t*
   tc::Params prm{nullptr, nullptr, q, k, nullptr, nullptr, bias, v, out, nullptr, scale, B, H, N, d, 0, 0, 0,
                  nullptr};
   const int ctas = tc2::total_pairs(B, H, N);
-  return bias ? tc2::dispatch_dv<tc2::kModeRef, true>(prm, ctas, st, msg)
-              : tc2::dispatch_dv<tc2::kModeRef, false>(prm, ctas, st, msg);
+  return bias ? tc2::dispatch_dv<tc2::kModeRef, tc2::kDenseBias>(prm, ctas, st, msg)
+              : tc2::dispatch_dv<tc2::kModeRef, tc2::kNoBias>(prm, ctas, st, msg);
 }
 
 }  // namespace binattn

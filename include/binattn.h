@@ -304,6 +304,32 @@ int binattn_forward_int8(const uint32_t *q_bits, const uint32_t *k_bits,
                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * binattn_forward_relpos — binattn_forward with the position-sensitive form of
+ * the learnable bias instead of a dense [H, N, N] one: a relative-position
+ * table. The N tokens are n_cls (0 or 1) class tokens followed by the patches
+ * of a gh x gw grid in row-major order (N = n_cls + gh * gw, else
+ * BINATTN_ERR_SHAPE). With R0 = (2 gh - 1)(2 gw - 1), the bias of patch query
+ * i and patch key j is table[h, (y_i - y_j + gh - 1)(2 gw - 1) + x_i - x_j +
+ * gw - 1]; a class query with a patch key takes table[h, R0], a patch query
+ * with a class key table[h, R0 + 1], class with class table[h, R0 + 2].
+ *   table      bf16 [H, R0 + 3 n_cls], device, 16-byte aligned; at most
+ *              20480 entries per head (BINATTN_ERR_UNSUPPORTED beyond).
+ *   workspace  at least binattn_forward_relpos_workspace_bytes(...) bytes
+ *              (the split tail's partials; may be NULL when that is 0).
+ * Needs d % 8 == 0 and d <= 80. The result equals binattn_forward_ws with the
+ * dense bias that the table expands to, bit for bit; the table replaces the
+ * dense read of H N^2 bias elements by one of H R entries per CTA.
+ * Source: §2 bias enhancement (the bias may be dense, position-sensitive or
+ * context-aware).
+ */
+size_t binattn_forward_relpos_workspace_bytes(int B, int H, int N, int d);
+int binattn_forward_relpos(const uint32_t *q_bits, const uint32_t *k_bits,
+                           const float *alpha_q, const float *alpha_k,
+                           const uint16_t *table, int gh, int gw, int n_cls,
+                           const uint16_t *v, float softmax_scale, int B, int H, int N, int d,
+                           uint16_t *out, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * binattn_scores_debug — writes the integer scores S [B, H, N, N] (int32,
  * device) that engine `engine` computes inside the forward pass, using the same
  * kernel and score routine. For testing only: it materialises the N x N matrix.

@@ -80,6 +80,19 @@ def test_bias_ld_host_validation(L):
     assert L.binattn_forward_bias_ld_workspace_bytes(1, 2, 197, 64, 150) == 0  # ld < N
 
 
+def test_relpos_host_validation(L):
+    def fwd(table=A, gh=4, gw=4, ncls=0, N=16, d=64, ws=A):
+        return L.binattn_forward_relpos(P(A), P(A), P(A), P(A), P(table) if table else None, gh, gw, ncls, P(A),
+                                        ctypes.c_float(0.125), 1, 1, N, d, P(A), P(ws) if ws else None,
+                                        ctypes.c_size_t(1 << 20), None)
+    assert fwd(table=0) == 1
+    assert fwd(N=17) == 2                      # N must be n_cls + gh * gw
+    assert fwd(ncls=2, N=18) == 2              # at most one class token
+    assert fwd(gh=80, gw=80, N=6400) == 5      # 159^2 entries do not fit
+    assert fwd(d=33, N=16) == 5
+    assert fwd(table=A + 2) == 4
+
+
 def test_pack_host_validation(L):
     def pack(x=A, dt=1, B=1, H=1, N=4, d=64, bits=A, alpha=A):
         return L.binattn_pack(P(x), dt, B, H, N, d, P(bits), P(alpha), None)
