@@ -416,22 +416,41 @@ int binattn_forward_static_ws(const uint32_t* q_bits, const uint32_t* k_bits, co
                             kStaticWorkspaceBytes, stream);
 }
 
+namespace {
+// V's 8-bit code: the channel maxima into maxbits (zeroed first), the codes
+// (tiled with DV columns and / or plain), then the scales.
+int quantize_v_launch(const uint16_t* v, int B, int H, int N, int d, int DV, int* maxbits, int8_t* tiled,
+                      int8_t* plain, float* scale, cudaStream_t st) {
+  const size_t nmax = static_cast<size_t>(B) * H * d;
+  cudaError_t e = cudaMemsetAsync(maxbits, 0, nmax * sizeof(int), st);
+  if (e != cudaSuccess) return fail(BINATTN_ERR_CUDA, "memset of the V maxima: %s", cudaGetErrorString(e));
+  const dim3 gmax(static_cast<unsigned>(B * H), static_cast<unsigned>((N + binattn::kQvThreads - 1) / binattn::kQvThreads));
+  binattn::vmax_kernel<<<gmax, binattn::kQvThreads, 0, st>>>(v, N, d, maxbits);
+  if (int rc = launch_status("vmax_kernel")) return rc;
+  const dim3 gq(static_cast<unsigned>(B * H), static_cast<unsigned>((N + 63) / 64));
+  binattn::vquant_kernel<<<gq, binattn::kQvThreads, 0, st>>>(v, N, d, DV, maxbits, tiled, plain);
+  if (int rc = launch_status("vquant_kernel")) return rc;
+  binattn::vscale_kernel<<<static_cast<unsigned>((nmax + 255) / 256), 256, 0, st>>>(maxbits, static_cast<long long>(nmax), scale);
+  return launch_status("vscale_kernel");
+}
+}  // namespace
+
 int binattn_quantize_v(const uint16_t* v, int B, int H, int N, int d, int8_t* vq, float* scale, void* stream) {
   BINATTN_CHECK_PTR(v);
   BINATTN_CHECK_PTR(vq);
   BINATTN_CHECK_PTR(scale);
   if (int rc = check_shape(B, H, N, d)) return rc;
   if (d % 8 != 0) return fail(BINATTN_ERR_UNSUPPORTED, "the 8-bit V code needs d %% 8 == 0 (d = %d)", d);
-  binattn::quantize_v_kernel<<<static_cast<unsigned>(B * H), binattn::kQvThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      v, N, d, 0, nullptr, vq, scale);
-  return launch_status("quantize_v_kernel");
+  // the scales' buffer holds the maxima until the codes are written
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return quantize_v_launch(v, B, H, N, d, 0, reinterpret_cast<int*>(scale), nullptr, vq, scale, st);
 }
 
 namespace {
 // Workspace of binattn_forward_int8: V's tiled 8-bit code, its scales, the row
 // maxima, and with N % 8 != 0 the bias with padded rows.
 struct Int8Ws {
-  size_t vq, scale, mrow, pad, total;
+  size_t vq, scale, mrow, vmax, pad, total;
 };
 Int8Ws int8_ws(int B, int H, int N, int d, bool has_bias) {
   const size_t BH = static_cast<size_t>(B) * H;
@@ -440,8 +459,9 @@ Int8Ws int8_ws(int B, int H, int N, int d, bool has_bias) {
   w.vq = round256(BH * nkt * binattn::tc2::dv_for(d) * 64);
   w.scale = round256(BH * d * 4);
   w.mrow = round256(BH * N * 4);
+  w.vmax = round256(BH * d * 4);
   w.pad = ws_pad_bytes(H, N, has_bias, N);
-  w.total = w.vq + w.scale + w.mrow + w.pad;
+  w.total = w.vq + w.scale + w.mrow + w.vmax + w.pad;
   return w;
 }
 bool int8_path(int d, int N, bool has_bias) {
@@ -470,20 +490,19 @@ int binattn_forward_int8(const uint32_t* q_bits, const uint32_t* k_bits, const f
   int8_t* vq8 = reinterpret_cast<int8_t*>(ws);
   float* vscale = reinterpret_cast<float*>(ws + w.vq);
   float* mrow = reinterpret_cast<float*>(ws + w.vq + w.scale);
+  int* vmax = reinterpret_cast<int*>(ws + w.vq + w.scale + w.mrow);
   const uint16_t* fbias = bias;
   int ld = 0;
   if (w.pad) {
     ld = padded_bias_ld(N);
-    uint16_t* padded = reinterpret_cast<uint16_t*>(ws + w.vq + w.scale + w.mrow);
+    uint16_t* padded = reinterpret_cast<uint16_t*>(ws + w.vq + w.scale + w.mrow + w.vmax);
     const long long rows = static_cast<long long>(H) * N;
     binattn::tc2::pad_bias_rows_kernel<<<static_cast<unsigned>((rows * ld + 255) / 256), 256, 0, st>>>(
         bias, rows, N, N, ld, padded);
     if (int rc = launch_status("pad_bias_rows_kernel")) return rc;
     fbias = padded;
   }
-  binattn::quantize_v_kernel<<<static_cast<unsigned>(B * H), binattn::kQvThreads, 0, st>>>(
-      v, N, d, binattn::tc2::dv_for(d), vq8, nullptr, vscale);
-  if (int rc = launch_status("quantize_v_kernel")) return rc;
+  if (int rc = quantize_v_launch(v, B, H, N, d, binattn::tc2::dv_for(d), vmax, vq8, nullptr, vscale, st)) return rc;
   std::string msg;
   if (int rc = binattn::forward_tc2_int8(q_bits, k_bits, alpha_q, alpha_k, fbias, ld, vq8, vscale, mrow,
                                          softmax_scale, B, H, N, d, out, st, &msg))

@@ -105,14 +105,17 @@ inline int dv_for(int d) { return d < 32 ? 32 : d < 64 ? 64 : d < 80 ? 80 : 96; 
 // Bias kinds of the 64-key pipeline.
 constexpr int kNoBias = 0;
 constexpr int kDenseBias = 1;   // bf16 [H, N, N] (rows bias_ld apart), TMA boxes
-constexpr int kRelPosBias = 2;  // relative-position table [H, R] gathered from shared memory
+constexpr int kRelPosBias = 2;     // relative-position table [H, R] gathered from shared memory
+constexpr int kRelPosBiasCls = 3;  // the same with one class token before the patches
+constexpr int kRelPosBiasRows = 4; // no class token, grid rows a multiple of 32 keys: one run per chunk
 constexpr int kRelTabMax = 20480;  // table entries per head that fit beside the stages (fp32)
 constexpr int kClsKey = -(1 << 30);  // key offset that marks a class key
 
 template <int DV, int kMode, int kBiasKind>
 struct Layout {
   static constexpr bool kBias = kBiasKind == kDenseBias;
-  static constexpr bool kRel = kBiasKind == kRelPosBias;
+  static constexpr bool kRel = kBiasKind == kRelPosBias || kBiasKind == kRelPosBiasCls ||
+                               kBiasKind == kRelPosBiasRows;
   static constexpr int kKS = (kBias || kRel) ? 4 : 8;            // K / V / alpha_k stages
   static constexpr int kBS = 4;                                  // bias stages (per t)
   static constexpr int kBiasTile = kRows * kKeys * 2;            // 16 KB
@@ -219,6 +222,8 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   using L = Layout<DV, kMode, kBiasKind>;
   constexpr bool kBias = L::kBias;  // dense bias
   constexpr bool kRel = L::kRel;    // relative-position table
+  constexpr bool kRelCls = kBiasKind == kRelPosBiasCls;    // ... with a class token
+  constexpr bool kRelRows = kBiasKind == kRelPosBiasRows;  // ... read by runs of the table
   constexpr bool kRef = kMode == kModeRef;
   constexpr bool kDump = kMode == kModeDump;
   constexpr bool kMax = kMode == kModeMax;
@@ -434,7 +439,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
 #pragma unroll
           for (int w = 0; w < 3; ++w) tr.wd[u][w] = (in && w < W) ? __ldg(p.kb + (tok0 + key) * W + w) : 0u;
           tr.ak[u] = (!kDump && in) ? __ldg(p.ak + tok0 + key) : 0.f;
-          if constexpr (kRel) {
+          if constexpr (kRel && !kRelRows) {
             // -(y_j (2 gw - 1) + x_j) for a patch key, so that a patch query's
             // base plus it is the table entry of their displacement
             const int pj = key - p.rel_ncls;
@@ -469,7 +474,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
           float* aks = reinterpret_cast<float*>(smem + L::kAk) + s * kKeys;
 #pragma unroll
           for (int u = 0; u < 2; ++u) aks[lane + 32 * u] = cur.ak[u];
-          if constexpr (kRel) {
+          if constexpr (kRel && !kRelRows) {
             int* kos = reinterpret_cast<int*>(smem + L::kKo) + s * kKeys;
 #pragma unroll
             for (int u = 0; u < 2; ++u) kos[lane + 32 * u] = cur.ko[u];
@@ -586,16 +591,21 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
     if constexpr (kRel) {
       const int R0 = (2 * p.rel_gh - 1) * (2 * p.rel_gw - 1);
       const int pi = row - p.rel_ncls;
-      if (row_valid && pi >= 0) {
-        rel_base = (pi / p.rel_gw + p.rel_gh - 1) * (2 * p.rel_gw - 1) + pi % p.rel_gw + p.rel_gw - 1;
-        rel_cls_key = R0 + 1;
-      } else {
-        rel_fixed = row_valid ? R0 : 0;
-        rel_cls_key = row_valid ? R0 + 2 : 0;
+      // a row >= N takes patch 0's base (its result is not stored; every
+      // index it forms is still inside the table)
+      const int pb = (row_valid && pi >= 0) ? pi : 0;
+      rel_base = (pb / p.rel_gw + p.rel_gh - 1) * (2 * p.rel_gw - 1) + pb % p.rel_gw + p.rel_gw - 1;
+      if constexpr (kRelCls) {
+        if (row_valid && pi >= 0) {
+          rel_cls_key = R0 + 1;
+        } else {
+          rel_fixed = row_valid ? R0 : 0;
+          rel_cls_key = row_valid ? R0 + 2 : 0;
+        }
       }
     }
     const float* rel_tab = reinterpret_cast<const float*>(smem + L::kTab);
-    auto logits = [&](uint32_t* xr, int c, const uint8_t* bsm, const float* aks) {
+    auto logits = [&](uint32_t* xr, int c, const uint8_t* bsm, const float* aks, int jtile) {
       float2* xs = reinterpret_cast<float2*>(xr);
       const float2 ci2 = make_float2(ci, ci);
 #pragma unroll
@@ -610,6 +620,15 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
           for (int e = 0; e < 4; ++e)
             bv[e] = make_float2(__uint_as_float(rw[e] << 16), __uint_as_float(rw[e] & 0xFFFF0000u));
         } else if constexpr (kRel) {
+          if constexpr (kRelRows) {
+            // the chunk's 32 keys lie in one grid row, so key e of the chunk
+            // reads entry rp - e; a chunk beyond N (wholly masked) reads the
+            // last real chunk's entries instead
+            const int jc = min(jtile + kChunk * c, N - kChunk);
+            const float* rp = rel_tab + rel_base - (jc / p.rel_gw) * (2 * p.rel_gw - 1) - jc % p.rel_gw;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) bv[e] = make_float2(rp[-(8 * q + 2 * e)], rp[-(8 * q + 2 * e + 1)]);
+          } else {
           // the stage's key offsets follow its alpha_k (Layout: kKo = kAk + kKS * 64 * 4)
           const int* kos = reinterpret_cast<const int*>(aks + kKS * kKeys) + kChunk * c + 8 * q;
           const int4 o0 = *reinterpret_cast<const int4*>(kos);
@@ -618,11 +637,14 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
           float bb[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const int idx = o[e] == kClsKey ? rel_cls_key : (rel_fixed >= 0 ? rel_fixed : rel_base + o[e]);
-            bb[e] = rel_tab[idx];
+            if constexpr (kRelCls)
+              bb[e] = rel_tab[o[e] == kClsKey ? rel_cls_key : (rel_fixed >= 0 ? rel_fixed : rel_base + o[e])];
+            else
+              bb[e] = rel_tab[rel_base + o[e]];
           }
 #pragma unroll
           for (int e = 0; e < 4; ++e) bv[e] = make_float2(bb[2 * e], bb[2 * e + 1]);
+          }
         }
         if constexpr (kRef) {
 #pragma unroll
@@ -654,18 +676,26 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
     // 8-bit pass: u = rint(255 exp(logit - m)) of a 32-key chunk (m the row's
     // exact max, so u <= 255), four keys per 32-bit TMEM column, lowest key in
     // the lowest byte: the unsigned 8-bit A operand of the kind::i8 P.V
+    // The rounding runs on the FMA pipe: y = 255 p + 1.5 * 2^23 (one fused
+    // multiply-add, rounded to nearest even) holds rint(255 p) in its low
+    // mantissa bits, since 0 <= 255 p <= 255 sits where the ulp is 1; the low
+    // bytes of four such words are then gathered by byte permutes.
     auto exps_u8 = [&](const uint32_t* xr, uint32_t p_col) {
-      const float* xf = reinterpret_cast<const float*>(xr);
+      const float2* xs = reinterpret_cast<const float2*>(xr);
+      const float2 l2e2 = make_float2(kLog2e, kLog2e);
+      const float2 nm2 = make_float2(-m * kLog2e, -m * kLog2e);
+      const float2 k255 = make_float2(255.f, 255.f);
+      const float2 magic = make_float2(12582912.f, 12582912.f);
       uint32_t pk[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t u = __float2uint_rn(ex2((xf[4 * e + k] - m) * kLog2e) * 255.f);
-          w |= (u < 255u ? u : 255u) << (8 * k);
-        }
-        pk[e] = w;
+        const float2 a0 = __ffma2_rn(xs[2 * e], l2e2, nm2);
+        const float2 a1 = __ffma2_rn(xs[2 * e + 1], l2e2, nm2);
+        const float2 y0 = __ffma2_rn(make_float2(ex2(a0.x), ex2(a0.y)), k255, magic);
+        const float2 y1 = __ffma2_rn(make_float2(ex2(a1.x), ex2(a1.y)), k255, magic);
+        const uint32_t lo = __byte_perm(__float_as_uint(y0.x), __float_as_uint(y0.y), 0x0040);
+        const uint32_t hi = __byte_perm(__float_as_uint(y1.x), __float_as_uint(y1.y), 0x0040);
+        pk[e] = __byte_perm(lo, hi, 0x5410);
       }
       tmem_st8(p_col, pk);
     };
@@ -700,8 +730,8 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         if (ok) {
           const uint8_t* bsm = smem + L::kBiasOff + (bs * 2 + t) * L::kBiasTile + r * 128;
           const float* aks = reinterpret_cast<const float*>(smem + L::kAk) + s * kKeys;
-          logits(xa, 0, bsm, aks);
-          logits(xb, 1, bsm, aks);
+          logits(xa, 0, bsm, aks, key0 + kt * kKeys);
+          logits(xb, 1, bsm, aks, key0 + kt * kKeys);
           float* x0 = reinterpret_cast<float*>(xa);
           float* x1 = reinterpret_cast<float*>(xb);
           const int jt = key0 + kt * kKeys;
@@ -1103,14 +1133,23 @@ inline int forward_tc2_relpos(const uint32_t* qb, const uint32_t* kb, const floa
   prm.rel_ncls = ncls;
   prm.rel_R = (2 * gh - 1) * (2 * gw - 1) + 3 * ncls;
   const tc2::SplitPlan plan = part ? tc2::split_plan(B, H, N) : tc2::SplitPlan{tc2::total_pairs(B, H, N), 0};
+  // grid rows a whole number of 32-key chunks and no class token: every chunk
+  // of keys is one run of the table (N is then a multiple of 32, so a chunk is
+  // wholly below N or wholly beyond it)
+  const bool rows = ncls == 0 && gw % tc2::kChunk == 0;
+  auto run = [&](int ctas) {
+    return ncls   ? tc2::dispatch_dv<tc2::kModeBin, tc2::kRelPosBiasCls>(prm, ctas, st, msg)
+           : rows ? tc2::dispatch_dv<tc2::kModeBin, tc2::kRelPosBiasRows>(prm, ctas, st, msg)
+                  : tc2::dispatch_dv<tc2::kModeBin, tc2::kRelPosBias>(prm, ctas, st, msg);
+  };
   if (plan.full > 0) {
-    if (int rc = tc2::dispatch_dv<tc2::kModeBin, tc2::kRelPosBias>(prm, plan.full, st, msg)) return rc;
+    if (int rc = run(plan.full)) return rc;
   }
   if (plan.tail > 0) {
     prm.pair_base = plan.full;
     prm.split = 1;
     prm.part = part;
-    if (int rc = tc2::dispatch_dv<tc2::kModeBin, tc2::kRelPosBias>(prm, 2 * plan.tail, st, msg)) return rc;
+    if (int rc = run(2 * plan.tail)) return rc;
     const int rows = plan.tail * 2 * tc2::kRows;
     tc2::combine_halves_kernel<<<(rows + 255) / 256, 256, 0, st>>>(part, plan.full, plan.tail, B, H, N, d, out);
     cudaError_t e = cudaGetLastError();

@@ -124,35 +124,18 @@ __device__ __forceinline__ void pack_row_bf16_w(const uint16_t* __restrict__ row
 }
 
 // bf16 rows with d % 8 == 0 (every token a whole number of 16-byte chunks):
-// a block stages kRowsTokens consecutive tokens, one contiguous byte range,
-// into shared memory with coalesced 16-byte loads, token tk at chunk
-// tk * pitch (pitch = d/8 rounded up to odd, so that the 8 threads of a
-// shared-memory wavefront read 8 different bank groups); then each thread packs
-// one token from there with pack_row_chunks.
-constexpr int kRowsTokens = 128;
+// one thread per token (pack_row_bf16), all of its row's 16-byte loads in
+// flight at once.
+constexpr int kRowsTokens = 256;
 template <int W>
 __global__ void __launch_bounds__(kRowsTokens)
 pack_bf16_rows_kernel(const uint16_t* __restrict__ x, long long n_tokens, int d,
                       uint32_t* __restrict__ bits, float* __restrict__ alpha) {
-  __shared__ uint4 stage[kRowsTokens * (4 * W + 1)];
-  const long long t0 = static_cast<long long>(blockIdx.x) * kRowsTokens;
-  const int ntok = static_cast<int>(min(static_cast<long long>(kRowsTokens), n_tokens - t0));
-  const int ng = d / 8;
-  const int pitch = ng | 1;
-  const uint4* src = reinterpret_cast<const uint4*>(x + t0 * d);
-  for (int c = threadIdx.x; c < ntok * ng; c += kRowsTokens) {
-    const int tk = c / ng;
-    stage[tk * pitch + (c - tk * ng)] = __ldg(src + c);
-  }
-  __syncthreads();
-  if (static_cast<int>(threadIdx.x) >= ntok) return;
-  uint4 v[4 * W];
-#pragma unroll
-  for (int g = 0; g < 4 * W; ++g) v[g] = g < ng ? stage[threadIdx.x * pitch + g] : make_uint4(0, 0, 0, 0);
+  const long long t = static_cast<long long>(blockIdx.x) * kRowsTokens + threadIdx.x;
+  if (t >= n_tokens) return;
   uint32_t words[W];
   float a;
-  pack_row_chunks<W>(v, d, words, a);
-  const long long t = t0 + threadIdx.x;
+  pack_row_bf16<W>(x + t * d, d, words, a);
 #pragma unroll
   for (int w = 0; w < W; ++w) bits[t * W + w] = words[w];
   alpha[t] = a;
