@@ -21,6 +21,7 @@ path) on a bounded sample of the same workload on the host cores.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -60,6 +61,9 @@ def parse():
     ap.add_argument("--profile-once", action="store_true",
                     help="run --warmup plain steps (with bias) and exit: the command profiled by ncu")
     ap.add_argument("--no-bias", action="store_true", help="with --profile-once: steps without bias")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="with --profile-once: replace the workload's batch B (a small case for multi-pass "
+                         "ncu captures)")
     return ap.parse_args()
 
 
@@ -143,8 +147,8 @@ def roofline_line(w, with_bias, peaks, fwd_s, n_sm=148, sm_mhz=None):
 # back into null. The digest covers the code only (comments removed, runs of
 # white space collapsed), so an edit of a comment keeps the capture valid.
 NCU_TRAFFIC = {
-    "sources_sha256": "583f2e64017821cf280786dffad1769301b411b431bdb25bf90831377d9331e6",
-    "bytes_per_call": {"dit_xl_1024/bias": 590_076_672},
+    "sources_sha256": "f5ce3cff18430b2c164e2e5db74163c3746f6a5678da86493858c84906573943",
+    "bytes_per_call": {"dit_xl_1024/bias": 590_075_904},
 }
 
 _C_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'|//[^\n]*|/\*.*?\*/', re.S)
@@ -436,7 +440,6 @@ def rank_inputs(w, rank, world, shard_mode):
     """This rank's workload and inputs. Replicas: the whole workload on its own
     seed. Heads: one batch (the workload's seed on every rank) of which this
     rank holds heads head_range(H, world, rank) only, bias slice included."""
-    import dataclasses
 
     from diffusion_transformers_b200 import shard
     if shard_mode == "heads" and world > 1:
@@ -779,6 +782,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     w = WORKLOADS[args.workload]
+    if args.batch is not None:
+        if not args.profile_once or args.batch < 1:
+            raise SystemExit("--batch B (B >= 1) goes with --profile-once only")
+        w = dataclasses.replace(w, B=args.batch)
     if args.impl == "reference":
         run_reference(args, w, rank)
         return

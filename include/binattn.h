@@ -204,7 +204,11 @@ int binattn_forward_bias_ld_ws(const uint32_t *q_bits, const uint32_t *k_bits,
  * any library.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current) and keeps it; make that
- *    first call before any stream capture that includes this call.
+ *    first call before any stream capture that includes this call. The kept
+ *    address belongs to the device's current context: after cudaDeviceReset
+ *    on a device that this call has used, the library's kernel set-up and
+ *    this address are stale, and the library must not be used on that device
+ *    again in the same process.
  *  - Shapes whose binattn_forward_workspace_bytes exceeds 32 MiB return
  *    BINATTN_ERR_UNSUPPORTED before anything is launched (for example a bias
  *    with N % 8 != 0 and H * N * roundup(N, 8) * 2 > 32 MiB).
