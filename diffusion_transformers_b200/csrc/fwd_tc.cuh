@@ -158,6 +158,10 @@ struct Params {
   // class tokens, rel_R = (2 gh - 1)(2 gw - 1) + 3 ncls.
   const uint16_t* rel_table = nullptr;
   int rel_gh = 0, rel_gw = 0, rel_ncls = 0, rel_R = 0;
+  // 64-key pipeline without split: the launch covers pairs pair_base ..
+  // pair_base + npairs - 1, CTA c taking c, c + gridDim.x, ... (a persistent
+  // launch of fewer CTAs than pairs); 0: one pair per CTA.
+  int npairs = 0;
 };
 
 // Named barrier 1 over the load-mode loader warps with an AND reduction.

@@ -9,7 +9,10 @@
 //
 // Shapes: d % 8 == 0, d <= 80; with a bias also N % 8 == 0 (the bias rows are
 // TMA rows). One CTA (12 warps, one per SM) owns 256 query rows of one (b, h)
-// as two 128-row tiles t = 0, 1 and streams the keys in tiles of 64:
+// as two 128-row tiles t = 0, 1 and streams the keys in tiles of 64. A launch
+// of fewer CTAs than such pairs (one per SM) is persistent: each CTA takes
+// several pairs in turn, keeping its tensor memory and barriers, and its
+// shared-memory rings run on from one pair's key tiles into the next's.
 //   warps 0-7  softmax: warps 4t..4t+3 for tile t, one thread per query row
 //              (TMEM lane).
 //   warp 8, 9  MMA issuers, one thread each: warp 8 + t issues for tile t.
@@ -245,25 +248,43 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   uint64_t* p_full = bars + 36;    // [2 t][2 b] softmax t published P (128 arrivals) -> issuer t
   uint64_t* o_done = bars + 40;    // [2 t][2 b] P.V commit of the last two tiles (no QK^T follows)
   uint64_t* drain = bars + 44;     // [2 t] error path only
+  uint64_t* q_ready = bars + 46;   // [2 t] softmax t staged the pair's Q_t (128 arrivals) -> issuer t
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Batch entries sharing a bias tile (same h and query tile) are adjacent in
-  // launch order, so the bias tile is fetched from HBM once.
-  // 256-row pair of this CTA (b fastest, then the query tile, then h), and
-  // with split, which half of the key tiles it takes.
+  // Work items are 256-row pairs, numbered b fastest, then the query tile,
+  // then h: batch entries sharing a bias tile (same h and query tile) are
+  // adjacent, so CTAs running side by side fetch it from HBM once.
+  // Without split, CTA c takes pairs pair_base + c + i * gridDim.x, i = 0, 1,
+  // ..., below pair_base + npairs (npairs == 0: one pair per CTA). A CTA that
+  // takes several pairs keeps its tensor memory, barriers and staged pads,
+  // and its shared-memory rings run on across pairs, so the next pair's first
+  // tiles load while the current pair finishes. With split, CTA 2i + half
+  // takes one key half of pair pair_base + i. The position-sensitive bias
+  // stages one head's table once, so its launches take one pair per CTA.
   const int nq = (p.N + 2 * kRows - 1) / (2 * kRows);
-  const int pidx = p.pair_base + (p.split ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x));
   const int half = p.split ? static_cast<int>(blockIdx.x & 1) : 0;
-  const int b = pidx % p.B;
-  const int qt = (pidx / p.B) % nq;
-  const int h = pidx / (p.B * nq);
-  const int bh = b * p.H + h;
+  const int G = static_cast<int>(gridDim.x);
+  const int npairs = p.npairs > 0 ? p.npairs : G;
+  const int n_items = (p.split || kRel) ? 1 : max(0, (npairs - static_cast<int>(blockIdx.x) + G - 1) / G);
+  struct Item {
+    int pidx, h, bh, q0;
+    size_t tok0;
+  };
+  auto item = [&](int it) {
+    Item w;
+    w.pidx = p.pair_base + (p.split ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x) + it * G);
+    const int b = w.pidx % p.B;
+    const int qt = (w.pidx / p.B) % nq;
+    w.h = w.pidx / (p.B * nq);
+    w.bh = b * p.H + w.h;
+    w.tok0 = static_cast<size_t>(w.bh) * p.N;
+    w.q0 = qt * 2 * kRows;
+    return w;
+  };
   const int N = p.N, d = p.d;
   const int W = (d + 31) / 32;                 // sign words per token (binary)
-  const size_t tok0 = static_cast<size_t>(bh) * N;
-  const int q0 = qt * 2 * kRows;
   const int nkt_all = (N + kKeys - 1) / kKeys;
   const int kt_begin = p.split && half ? nkt_all / 2 : 0;
   const int nkt = p.split ? (half ? nkt_all - nkt_all / 2 : nkt_all / 2) : nkt_all;  // tiles of this CTA
@@ -294,7 +315,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   if constexpr (kRel) {
     // this head's relative-position table, widened to fp32 once
     float* tab = reinterpret_cast<float*>(smem + L::kTab);
-    const uint16_t* src_t = p.rel_table + static_cast<size_t>(h) * p.rel_R;
+    const uint16_t* src_t = p.rel_table + static_cast<size_t>(item(0).h) * p.rel_R;
     for (int e = threadIdx.x; e < p.rel_R; e += kThreads) tab[e] = bf16_bits_to_float(src_t[e]);
   }
   if (threadIdx.x == 0) {
@@ -314,6 +335,8 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
     }
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
+    mbar_init(&q_ready[0], kSoftmaxPerTile);
+    mbar_init(&q_ready[1], kSoftmaxPerTile);
     *abort = 0;
     fence_mbar_init();
   }
@@ -326,16 +349,15 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Softmax threads: this thread's query row; Q_t operand row into TMEM.
   // Softmax warp w < 8: tile t = w / 4, rows 32 (w % 4) .. + 31 (the warp's
   // TMEM lane quadrant), one thread per row.
   const int t = warp >> 2;
   const int r = ((warp & 3) << 5) | lane;    // row within the tile = TMEM lane
-  const int row = q0 + t * kRows + r;
-  const bool row_valid = warp < kSoftmaxWarps && row < N;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  float aq_row = 0.f;  // alpha_q of this thread's row (binary forward)
-  if (warp < kSoftmaxWarps) {
+  // Softmax threads, once per pair: this thread's row of Q_t into TMEM, and
+  // alpha_q of the row (binary forward), returned.
+  auto stage_q = [&](const Item& w, int row, bool row_valid) {
+    float aq_row = 0.f;
     if constexpr (kRef) {
       // bf16 pairs: column c2 holds channels 2 c2 (low half) and 2 c2 + 1
       const uint32_t qcol = tmem + lane_base + 256 * t + 128 + DV;
@@ -345,7 +367,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         for (int h2 = 0; h2 < 2; ++h2) {
           uint4 val = make_uint4(0, 0, 0, 0);
           if (row_valid && 8 * (c + h2) < d)
-            val = *reinterpret_cast<const uint4*>(p.q + (tok0 + row) * d + 8 * (c + h2));
+            val = *reinterpret_cast<const uint4*>(p.q + (w.tok0 + row) * d + 8 * (c + h2));
           wv[4 * h2 + 0] = val.x;
           wv[4 * h2 + 1] = val.y;
           wv[4 * h2 + 2] = val.z;
@@ -360,61 +382,72 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       uint32_t qw[3] = {0u, 0u, 0u};
       if (row_valid && !kDump) {
         if (p.qh) {
-          pack_row_bf16_w(p.qh + (tok0 + row) * d, d, W, qw, aq_row);  // Q binarised here
+          pack_row_bf16_w(p.qh + (w.tok0 + row) * d, d, W, qw, aq_row);  // Q binarised here
         } else {
-          for (int w = 0; w < W; ++w) qw[w] = p.qb[(tok0 + row) * W + w];
-          aq_row = p.aq[tok0 + row];
+          for (int k = 0; k < W; ++k) qw[k] = p.qb[(w.tok0 + row) * W + k];
+          aq_row = p.aq[w.tok0 + row];
         }
       } else if (row_valid) {
-        for (int w = 0; w < W; ++w) qw[w] = p.qb[(tok0 + row) * W + w];
+        for (int k = 0; k < W; ++k) qw[k] = p.qb[(w.tok0 + row) * W + k];
       }
-      for (int w = 0; w < W; ++w) {
-        const uint32_t word = w == 0 ? qw[0] : w == 1 ? qw[1] : qw[2];
+      for (int k = 0; k < W; ++k) {
+        const uint32_t word = k == 0 ? qw[0] : k == 1 ? qw[1] : qw[2];
         uint32_t wv[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) wv[j] = row_valid ? e4m3_bytes(word, 4 * j, 32 * w + 4 * j, d, true) : 0u;
-        tmem_st8(qcol + 8 * w, wv);
+        for (int j = 0; j < 8; ++j) wv[j] = row_valid ? e4m3_bytes(word, 4 * j, 32 * k + 4 * j, d, true) : 0u;
+        tmem_st8(qcol + 8 * k, wv);
       }
     }
     tmem_st_wait();
     tc_fence_before();
-  }
+    return aq_row;
+  };
   fence_proxy_async_smem();
   __syncthreads();
   tc_fence_after();
 
   if (warp == kTmaWarp) {
     // --------------------------- V (and reference K), bias: one thread issues
+    // Ring slots and phases follow the tile count g over all of the CTA's
+    // pairs (g = it * nkt + kt), as in every role below.
     if (lane == 0 && (!kNoPV || kBias)) {
       bool ok = true;
-      for (int kt = 0; ok && kt < nkt; ++kt) {
-        if (p.stall_after >= 0 && kt >= p.stall_after) break;  // test only
-        const int j0 = key0 + kt * kKeys;
-        if constexpr (kF16PV) {
-          const int s = kt % kKS;
-          if (kt >= kKS && !(ok = mbar_wait(&kv_empty[s], ((kt / kKS) - 1) & 1, abort))) break;
-          mbar_arrive_expect_tx(&kv_full[s], static_cast<uint32_t>(dgroups * 1024 * (kRef ? 2 : 1)));
-          for (int g = 0; g < dgroups; ++g)
-            tma_load_3d(smem + L::kV + s * L::kVTile + g * 1024, &tm_v, 8 * g, j0, bh, &kv_full[s]);
-          if constexpr (kRef) {
-            for (int g = 0; g < dgroups; ++g)
-              tma_load_3d(smem + L::kK + s * L::kKTile + g * 1024, &tm_k, 8 * g, j0, bh, &kv_full[s]);
+      for (int it = 0; ok && it < n_items; ++it) {
+        const Item w = item(it);
+        for (int kt = 0; ok && kt < nkt; ++kt) {
+          const int g = it * nkt + kt;
+          if (p.stall_after >= 0 && g >= p.stall_after) {  // test only
+            ok = false;
+            break;
           }
-        } else if constexpr (kI8) {
-          // the tile's 8-bit V operand is one contiguous block of the tiled layout
-          const int s = kt % kKS;
-          if (kt >= kKS && !(ok = mbar_wait(&kv_empty[s], ((kt / kKS) - 1) & 1, abort))) break;
-          mbar_arrive_expect_tx(&kv_full[s], static_cast<uint32_t>(L::kVTile));
-          bulk_load(smem + L::kV + s * L::kVTile,
-                    p.vq8 + (static_cast<size_t>(bh) * nkt_all + kt_begin + kt) * L::kVTile,
-                    static_cast<uint32_t>(L::kVTile), &kv_full[s]);
-        }
-        if constexpr (kBias) {
-          for (int t2 = 0; t2 < 2; ++t2) {
-            const int i = (kt % kBS) * 2 + t2;
-            if (kt >= kBS && !(ok = mbar_wait(&b_empty[i], ((kt / kBS) - 1) & 1, abort))) break;
-            mbar_arrive_expect_tx(&b_full[i], L::kBiasTile);
-            tma_load_3d(smem + L::kBiasOff + i * L::kBiasTile, &tm_bias, j0, q0 + t2 * kRows, h, &b_full[i]);
+          const int j0 = key0 + kt * kKeys;
+          if constexpr (kF16PV) {
+            const int s = g % kKS;
+            if (g >= kKS && !(ok = mbar_wait(&kv_empty[s], ((g / kKS) - 1) & 1, abort))) break;
+            mbar_arrive_expect_tx(&kv_full[s], static_cast<uint32_t>(dgroups * 1024 * (kRef ? 2 : 1)));
+            for (int c = 0; c < dgroups; ++c)
+              tma_load_3d(smem + L::kV + s * L::kVTile + c * 1024, &tm_v, 8 * c, j0, w.bh, &kv_full[s]);
+            if constexpr (kRef) {
+              for (int c = 0; c < dgroups; ++c)
+                tma_load_3d(smem + L::kK + s * L::kKTile + c * 1024, &tm_k, 8 * c, j0, w.bh, &kv_full[s]);
+            }
+          } else if constexpr (kI8) {
+            // the tile's 8-bit V operand is one contiguous block of the tiled layout
+            const int s = g % kKS;
+            if (g >= kKS && !(ok = mbar_wait(&kv_empty[s], ((g / kKS) - 1) & 1, abort))) break;
+            mbar_arrive_expect_tx(&kv_full[s], static_cast<uint32_t>(L::kVTile));
+            bulk_load(smem + L::kV + s * L::kVTile,
+                      p.vq8 + (static_cast<size_t>(w.bh) * nkt_all + kt_begin + kt) * L::kVTile,
+                      static_cast<uint32_t>(L::kVTile), &kv_full[s]);
+          }
+          if constexpr (kBias) {
+            for (int t2 = 0; t2 < 2; ++t2) {
+              const int i = (g % kBS) * 2 + t2;
+              if (g >= kBS && !(ok = mbar_wait(&b_empty[i], ((g / kBS) - 1) & 1, abort))) break;
+              mbar_arrive_expect_tx(&b_full[i], L::kBiasTile);
+              tma_load_3d(smem + L::kBiasOff + i * L::kBiasTile, &tm_bias, j0, w.q0 + t2 * kRows, w.h,
+                          &b_full[i]);
+            }
           }
         }
       }
@@ -431,11 +464,15 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         float ak[2];
         int ko[2];
       };
-      auto load_tile = [&](int kt, TileRegs& tr) {
+      // tile g of the CTA's sequence: key tile g % nkt of pair g / nkt
+      const int g_end = n_items * nkt;
+      auto load_tile = [&](int g, TileRegs& tr) {
+        const int kt = nkt > 0 ? g % nkt : 0;
+        const size_t tok0 = g < g_end ? item(g / nkt).tok0 : 0;
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int key = key0 + kt * kKeys + lane + 32 * u;
-          const bool in = kt < nkt && key < N;
+          const bool in = g < g_end && key < N;
 #pragma unroll
           for (int w = 0; w < 3; ++w) tr.wd[u][w] = (in && w < W) ? __ldg(p.kb + (tok0 + key) * W + w) : 0u;
           tr.ak[u] = (!kDump && in) ? __ldg(p.ak + tok0 + key) : 0.f;
@@ -450,11 +487,11 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       TileRegs cur, n1;
       load_tile(0, cur);
       load_tile(1, n1);
-      for (int kt = 0; kt < nkt; ++kt) {
+      for (int g = 0; g < g_end; ++g) {
         TileRegs n2;
-        load_tile(kt + 2, n2);
-        const int s = kt % kKS;
-        const bool ok = kt < kKS || mbar_wait(&kv_empty[s], ((kt / kKS) - 1) & 1, abort);
+        load_tile(g + 2, n2);
+        const int s = g % kKS;
+        const bool ok = g < kKS || mbar_wait(&kv_empty[s], ((g / kKS) - 1) & 1, abort);
         if (!__all_sync(0xffffffffu, ok)) break;
         uint8_t* ks = smem + L::kK + s * L::kKTile;
 #pragma unroll
@@ -494,10 +531,10 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       constexpr uint32_t kIdPV = idesc_bf16(kRows, DV, true);
       const uint32_t kb_sbo = kRef ? 128u : static_cast<uint32_t>(8 * 32 * W);
       const uint32_t base_t = tmem + 256 * tt;
-      // S_tt^(kt%2) = Q_tt K(kt)^T
-      auto issue_qk = [&](int kt) {
-        const uint32_t k_base = smem_u32(smem + L::kK + (kt % kKS) * L::kKTile);
-        const uint32_t d_col = base_t + 64 * (kt & 1);
+      // S_tt^(g%2) = Q_tt K(g)^T for tile g of the CTA's sequence
+      auto issue_qk = [&](int g) {
+        const uint32_t k_base = smem_u32(smem + L::kK + (g % kKS) * L::kKTile);
+        const uint32_t d_col = base_t + 64 * (g & 1);
         if constexpr (kRef) {
           for (int ks = 0; ks < kq16; ++ks)
             mma_ts(d_col, base_t + 128 + DV + ks * 8, smem_desc(k_base + ks * 2048, 1024, kb_sbo), kIdQK, ks > 0);
@@ -511,46 +548,54 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       // stage with alpha_k and, with a bias, this tile's bias box. The issuer
       // waits for them and then arrives on s_full itself (release), so the
       // softmax threads' single wait on s_full also covers alpha_k and the bias.
-      auto stage_ready = [&](int kt) {
-        if (!mbar_wait(&kv_full[kt % kKS], (kt / kKS) & 1, abort)) return false;
-        if (kBias && !mbar_wait(&b_full[(kt % kBS) * 2 + tt], (kt / kBS) & 1, abort)) return false;
-        mbar_arrive(&s_full[tt * 2 + (kt & 1)]);
+      auto stage_ready = [&](int g) {
+        if (!mbar_wait(&kv_full[g % kKS], (g / kKS) & 1, abort)) return false;
+        if (kBias && !mbar_wait(&b_full[(g % kBS) * 2 + tt], (g / kBS) & 1, abort)) return false;
+        mbar_arrive(&s_full[tt * 2 + (g & 1)]);
         tc_fence_after();
         return true;
       };
-      for (int kt = 0; ok && kt < 2 && kt < nkt; ++kt) {
-        if (!(ok = stage_ready(kt))) break;
-        issue_qk(kt);
-        mma_commit(&s_full[tt * 2 + (kt & 1)]);
-      }
-      for (int kt = 0; ok && kt < nkt; ++kt) {
-        const int s = kt % kKS;
-        const int bf = kt & 1;
-        if (!(ok = mbar_wait(&p_full[tt * 2 + bf], (kt >> 1) & 1, abort))) break;
+      for (int it = 0; ok && it < n_items; ++it) {
+        // Q_tt of the pair is in TMEM (and, from the second pair on, the
+        // softmax threads have read the previous pair's O)
+        if (!(ok = mbar_wait(&q_ready[tt], it & 1, abort))) break;
         tc_fence_after();
-        if constexpr (kF16PV) {
-          // O_tt += P_tt(kt) V(kt): A = P (bf16 pairs, 8 columns per 16 keys)
-          const uint32_t v_base = smem_u32(smem + L::kV + s * L::kVTile);
-#pragma unroll
-          for (int ks = 0; ks < kKeys / 16; ++ks)
-            mma_ts(base_t + 128, base_t + 64 * bf + ks * 8, smem_desc(v_base + ks * 256, 128, 1024), kIdPV,
-                   (kt > 0 || ks > 0));
-        } else if constexpr (kI8) {
-          // O_tt (s32) += P_tt(kt) V(kt): A = u8 P (4 keys per column, 8
-          // columns per 32 keys), B = s8 V, K-major, 32 keys per MMA
-          const uint32_t v_base = smem_u32(smem + L::kV + s * L::kVTile);
-#pragma unroll
-          for (int ks = 0; ks < kKeys / 32; ++ks)
-            mma_ts_i8(base_t + 128, base_t + 64 * bf + ks * 8, smem_desc(v_base + ks * 256, 128, 512),
-                      idesc_i8(kRows, DV), (kt > 0 || ks > 0));
+        const int g0 = it * nkt;
+        for (int kt = 0; ok && kt < 2 && kt < nkt; ++kt) {
+          if (!(ok = stage_ready(g0 + kt))) break;
+          issue_qk(g0 + kt);
+          mma_commit(&s_full[tt * 2 + ((g0 + kt) & 1)]);
         }
-        mma_commit(&kv_empty[s]);  // this issuer's last use of stage s
-        if (kt + 2 < nkt) {
-          if (!(ok = stage_ready(kt + 2))) break;
-          issue_qk(kt + 2);
-          mma_commit(&s_full[tt * 2 + bf]);
-        } else if constexpr (!kNoPV) {
-          mma_commit(&o_done[tt * 2 + bf]);
+        for (int kt = 0; ok && kt < nkt; ++kt) {
+          const int g = g0 + kt;
+          const int s = g % kKS;
+          const int bf = g & 1;
+          if (!(ok = mbar_wait(&p_full[tt * 2 + bf], (g >> 1) & 1, abort))) break;
+          tc_fence_after();
+          if constexpr (kF16PV) {
+            // O_tt += P_tt(kt) V(kt): A = P (bf16 pairs, 8 columns per 16 keys)
+            const uint32_t v_base = smem_u32(smem + L::kV + s * L::kVTile);
+#pragma unroll
+            for (int ks = 0; ks < kKeys / 16; ++ks)
+              mma_ts(base_t + 128, base_t + 64 * bf + ks * 8, smem_desc(v_base + ks * 256, 128, 1024), kIdPV,
+                     (kt > 0 || ks > 0));
+          } else if constexpr (kI8) {
+            // O_tt (s32) += P_tt(kt) V(kt): A = u8 P (4 keys per column, 8
+            // columns per 32 keys), B = s8 V, K-major, 32 keys per MMA
+            const uint32_t v_base = smem_u32(smem + L::kV + s * L::kVTile);
+#pragma unroll
+            for (int ks = 0; ks < kKeys / 32; ++ks)
+              mma_ts_i8(base_t + 128, base_t + 64 * bf + ks * 8, smem_desc(v_base + ks * 256, 128, 512),
+                        idesc_i8(kRows, DV), (kt > 0 || ks > 0));
+          }
+          mma_commit(&kv_empty[s]);  // this issuer's last use of stage s
+          if (kt + 2 < nkt) {
+            if (!(ok = stage_ready(g + 2))) break;
+            issue_qk(g + 2);
+            mma_commit(&s_full[tt * 2 + bf]);
+          } else if constexpr (!kNoPV) {
+            mma_commit(&o_done[tt * 2 + bf]);
+          }
         }
       }
       {  // wait (bounded) for every MMA of this thread before TMEM is freed
@@ -562,23 +607,30 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- softmax
-    // per-row factor of the logit: scale * alpha_q (binary) or scale (reference)
-    const float ci = kRef ? p.scale : ((!kDump && row_valid) ? p.scale * aq_row : 0.f);
     const uint32_t o_col = tmem + lane_base + 256 * t + 128;
     const int r7 = r & 7;
-    // the running max; in the 8-bit pass, the row's exact max from the first pass
+    // Per pair (set at the top of each): the thread's row, the per-row factor
+    // of the logit (scale * alpha_q, binary; scale, reference) and the running
+    // max (in the 8-bit pass, the row's exact max from the first pass).
+    int row = 0;
+    bool row_valid = false;
+    size_t tok0 = 0;
+    float ci = 0.f;
     float m = -INFINITY;
-    if constexpr (kI8) m = row_valid ? p.mrow[tok0 + row] : 0.f;
     bool ok = true;
     // Waits are made warp-uniform: the tcgen05.ld/st below are warp-collective.
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
     };
-    // P.V of tile kt - 1 is complete once QK^T(kt + 1) (issued after it by the
-    // same thread) is, or, for the last tile, once its own commit lands.
-    auto wait_pv_prev = [&](int kt) {
-      const bool r1 = kt + 1 < nkt ? wait_all(&s_full[t * 2 + ((kt + 1) & 1)], ((kt + 1) >> 1) & 1)
-                                   : wait_all(&o_done[t * 2 + ((kt - 1) & 1)], 0);
+    // o_done[t][b] completes once per pair for each b when a pair has two or
+    // more key tiles; with one, the pairs alternate between the two buffers.
+    auto od_parity = [&](int it) { return static_cast<uint32_t>((nkt >= 2 ? it : it >> 1) & 1); };
+    // P.V of tile g - 1 (key tile kt - 1 of pair it) is complete once
+    // QK^T(g + 1) (issued after it by the same thread) is, or, for the pair's
+    // last tile, once its own commit lands.
+    auto wait_pv_prev = [&](int g, int kt, int it) {
+      const bool r1 = kt + 1 < nkt ? wait_all(&s_full[t * 2 + ((g + 1) & 1)], ((g + 1) >> 1) & 1)
+                                   : wait_all(&o_done[t * 2 + ((g - 1) & 1)], od_parity(it));
       tc_fence_after();
       return r1;
     };
@@ -588,7 +640,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
     // query (and a row >= N, whose result is not stored) reads one fixed entry
     // for every patch key; a class key reads rel_cls_key.
     int rel_base = 0, rel_fixed = -1, rel_cls_key = 0;
-    if constexpr (kRel) {
+    auto rel_setup = [&]() {
       const int R0 = (2 * p.rel_gh - 1) * (2 * p.rel_gw - 1);
       const int pi = row - p.rel_ncls;
       // a row >= N takes patch 0's base (its result is not stored; every
@@ -603,7 +655,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
           rel_cls_key = row_valid ? R0 + 2 : 0;
         }
       }
-    }
+    };
     const float* rel_tab = reinterpret_cast<const float*>(smem + L::kTab);
     auto logits = [&](uint32_t* xr, int c, const uint8_t* bsm, const float* aks, int jtile) {
       float2* xs = reinterpret_cast<float2*>(xr);
@@ -702,13 +754,31 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
 
     // The loop runs every key tile even after an error (with the work
     // skipped), so that each thread takes its part in every named barrier.
-    if (!kNoPV && t == 1) named_arrive(3, 2 * kSoftmaxPerTile);  // tile 0 takes the first exp turn
+    if (!kNoPV && t == 1 && n_items > 0) named_arrive(3, 2 * kSoftmaxPerTile);  // tile 0 takes the first exp turn
+    const int g_end = n_items * nkt;
+    for (int it = 0; it < n_items; ++it) {
+    const Item w = item(it);
+    tok0 = w.tok0;
+    row = w.q0 + t * kRows + r;
+    row_valid = row < N;
+    {
+      // Q_t of the pair into TMEM; the issuer waits for all 128 rows. From
+      // the second pair on, the previous pair's epilogue has read O_t (its
+      // last P.V waited for), so the pair's first P.V may overwrite it.
+      const float aq_row = ok ? stage_q(w, row, row_valid) : 0.f;
+      mbar_arrive(&q_ready[t]);
+      ci = kRef ? p.scale : ((!kDump && row_valid) ? p.scale * aq_row : 0.f);
+    }
+    m = -INFINITY;
+    if constexpr (kI8) m = row_valid ? p.mrow[tok0 + row] : 0.f;
+    if constexpr (kRel) rel_setup();
     for (int kt = 0; kt < nkt; ++kt) {
-      const int s = kt % kKS;
-      const int bf = kt & 1;
-      const int bs = kt % kBS;
-      // scores, alpha_k and the bias tile of kt (see the issuer's stage_ready)
-      if (ok) ok = wait_all(&s_full[t * 2 + bf], (kt >> 1) & 1);
+      const int g = it * nkt + kt;  // tile of the CTA's sequence: ring slots and phases
+      const int s = g % kKS;
+      const int bf = g & 1;
+      const int bs = g % kBS;
+      // scores, alpha_k and the bias tile of g (see the issuer's stage_ready)
+      if (ok) ok = wait_all(&s_full[t * 2 + bf], (g >> 1) & 1);
       tc_fence_after();
       const uint32_t s_col = tmem + lane_base + 256 * t + 64 * bf;
       uint32_t xa[kChunk], xb[kChunk];
@@ -766,7 +836,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
           if (__any_sync(0xffffffffu, grow)) {
             const float m_new = grow ? tmax : m;
             const float corr = grow ? ex2((m - m_new) * kLog2e) : 1.f;  // 0 while m is -inf
-            if (kt > 0 && (ok = wait_pv_prev(kt))) {
+            if (kt > 0 && (ok = wait_pv_prev(g, kt, it))) {
 #pragma unroll
               for (int cc = 0; cc < DV; cc += 16) {
                 uint32_t ov[16];
@@ -797,7 +867,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
             }
             if (kBias) mbar_arrive(&b_empty[bs * 2 + t]);
           }
-          if (!(t == 1 && kt == nkt - 1)) named_arrive(4 - t, 2 * kSoftmaxPerTile);  // pass the token on
+          if (!(t == 1 && g == g_end - 1)) named_arrive(4 - t, 2 * kSoftmaxPerTile);  // pass the token on
         }
       }
       ok = __all_sync(0xffffffffu, ok);
@@ -810,7 +880,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
     if constexpr (kMax) {
       if (ok && row_valid) p.mrow[tok0 + row] = m;
     } else if constexpr (kI8) {
-      if (ok && wait_all(&o_done[t * 2 + ((nkt - 1) & 1)], 0)) {
+      if (ok && wait_all(&o_done[t * 2 + ((it * nkt + nkt - 1) & 1)], od_parity(it))) {
         tc_fence_after();
         // O_c = s_c * acc_c / l with the s32 sums acc_c = sum_j u_j vq_jc and
         // l = sum_j u_j (column d, the ones channel of the 8-bit V)
@@ -818,7 +888,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(lbits) : "r"(o_col + d));
         tmem_ld_wait();
         const float inv = 1.f / static_cast<float>(static_cast<int>(lbits));
-        const float* vs = p.vscale + static_cast<size_t>(bh) * d;
+        const float* vs = p.vscale + static_cast<size_t>(item(it).bh) * d;
         uint16_t* orow = p.out + (tok0 + row) * d;
 #pragma unroll
         for (int cc = 0; cc < DV; cc += 16) {
@@ -844,7 +914,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         }
       }
     } else if constexpr (!kDump) {
-      if (ok && wait_all(&o_done[t * 2 + ((nkt - 1) & 1)], 0)) {
+      if (ok && wait_all(&o_done[t * 2 + ((it * nkt + nkt - 1) & 1)], od_parity(it))) {
         tc_fence_after();
         uint32_t lbits;  // l = O_t column d
         asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(lbits) : "r"(o_col + d));
@@ -855,7 +925,8 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
           // ((slot * 2 + half) * (d + 2) + c) * 256 + r256, so that a warp's 32
           // rows store (and the combine kernel loads) 128 contiguous bytes
           const int r256 = t * kRows + r;
-          float* dst = p.part + static_cast<size_t>((pidx - p.pair_base) * 2 + half) * (d + 2) * (2 * kRows) + r256;
+          // (a split launch takes one pair per CTA: pair_base + blockIdx.x / 2)
+          float* dst = p.part + static_cast<size_t>((blockIdx.x >> 1) * 2 + half) * (d + 2) * (2 * kRows) + r256;
           for (int cc = 0; cc < d; cc += 8) {  // warp-uniform trip count: the loads are collective
             uint32_t ov[8];
             tmem_ld8(o_col + cc, ov);
@@ -896,6 +967,7 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         }
       }
     }
+    }  // pairs
   }
 
   // ------------------------------------------------------------- teardown
@@ -1078,6 +1150,32 @@ inline SplitPlan split_plan(int B, int H, int N) {
   if (full == 0 || tail == 0 || 2 * tail > nsm || (N + kKeys - 1) / kKeys < 32) return {P, 0};
   return {full, tail};
 }
+// The grid of a launch over P whole pairs of N keys. With at most
+// kPersistMaxTiles key tiles per pair it is persistent: one CTA per SM (each
+// CTA holds all of its SM's tensor memory), CTA c taking pairs c, c + S, ...;
+// sets prm.npairs and returns the CTA count. Longer pairs run one per CTA
+// (npairs = 0, P CTAs), and so does a launch without a device to ask.
+// Measured (one B200): persistent grids cut DeiT-B (4 key tiles) by 13%,
+// ViT-L/16 (10) by 8% and DiT-XL/2 512 px (16) by 4%; at 64 key tiles they
+// gain nothing with the bf16 P.V and lose 13-20% in the two 8-bit P.V passes,
+// whose bias reads are closer to the HBM bound: a CTA launched as another
+// ends starts beside the CTA launched just before it, which reads the same
+// bias tiles for the other batch entry, while persistent CTAs drift apart
+// over their pairs and lose part of that L2 reuse.
+constexpr int kPersistMaxTiles = 16;
+inline int grid_for(tc::Params& prm, int P) {
+  prm.npairs = 0;
+  if ((prm.N + kKeys - 1) / kKeys > kPersistMaxTiles) return P;
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      nsm <= 0) {
+    cudaGetLastError();
+    return P;
+  }
+  if (P <= nsm) return P;
+  prm.npairs = P;
+  return nsm;
+}
 // Bytes of the partial results of the split pairs (fp32 O, m, l per row and half).
 inline size_t split_part_bytes(int B, int H, int N, int d) {
   const SplitPlan pl = split_plan(B, H, N);
@@ -1099,8 +1197,8 @@ inline int forward_tc2(const uint32_t* qb, const uint32_t* kb, const float* aq, 
     return bias ? tc2::dispatch_dv<tc2::kModeBin, tc2::kDenseBias>(prm, ctas, st, msg)
                 : tc2::dispatch_dv<tc2::kModeBin, tc2::kNoBias>(prm, ctas, st, msg);
   };
-  if (plan.full > 0) {
-    if (int rc = run(plan.full)) return rc;
+  if (plan.full > 0) {  // (a split launch takes one pair per CTA and ignores npairs)
+    if (int rc = run(tc2::grid_for(prm, plan.full))) return rc;
   }
   if (plan.tail > 0) {
     prm.pair_base = plan.full;
@@ -1174,7 +1272,7 @@ inline int forward_tc2_int8(const uint32_t* qb, const uint32_t* kb, const float*
   prm.vq8 = vq8;
   prm.vscale = vscale;
   prm.mrow = mrow;
-  const int ctas = tc2::total_pairs(B, H, N);
+  const int ctas = tc2::grid_for(prm, tc2::total_pairs(B, H, N));
   if (int rc = bias ? tc2::dispatch_dv<tc2::kModeMax, tc2::kDenseBias>(prm, ctas, st, msg)
                     : tc2::dispatch_dv<tc2::kModeMax, tc2::kNoBias>(prm, ctas, st, msg))
     return rc;
@@ -1186,7 +1284,8 @@ inline int scores_tc2(const uint32_t* qb, const uint32_t* kb, int B, int H, int 
                       cudaStream_t st, std::string* msg) {
   tc::Params prm{qb, kb, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S, 0.f, B, H, N, d, 0, 0, 0,
                  nullptr};
-  return tc2::launch<32, tc2::kModeDump, tc2::kNoBias>(prm, tc2::total_pairs(B, H, N), st, msg);
+  return tc2::launch<32, tc2::kModeDump, tc2::kNoBias>(prm, tc2::grid_for(prm, tc2::total_pairs(B, H, N)), st,
+                                                       msg);
 }
 
 inline int forward_ref_tc2(const uint16_t* q, const uint16_t* k, const uint16_t* bias, const uint16_t* v,
@@ -1194,7 +1293,7 @@ inline int forward_ref_tc2(const uint16_t* q, const uint16_t* k, const uint16_t*
                            std::string* msg) {
   tc::Params prm{nullptr, nullptr, q, k, nullptr, nullptr, bias, v, out, nullptr, scale, B, H, N, d, 0, 0, 0,
                  nullptr};
-  const int ctas = tc2::total_pairs(B, H, N);
+  const int ctas = tc2::grid_for(prm, tc2::total_pairs(B, H, N));
   return bias ? tc2::dispatch_dv<tc2::kModeRef, tc2::kDenseBias>(prm, ctas, st, msg)
               : tc2::dispatch_dv<tc2::kModeRef, tc2::kNoBias>(prm, ctas, st, msg);
 }

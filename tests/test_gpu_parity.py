@@ -389,3 +389,33 @@ def test_forward_bias_ld(orc, shape):
     ref = orc.forward(c["q"], c["k"], c["bias"], c["v"], c["softmax_scale"])
     check_o(bf16_to_f64(binattn.forward_bias_ld_ws(qb, kb, aq, ak, binattn.pad_bias(bias), v, c["softmax_scale"])),
             ref, f"bias_ld {shape}")
+
+
+# ------------------------------------- persistent launches: several pairs per CTA
+# With more 256-row pairs than SMs, the 64-key pipeline runs one CTA per SM,
+# each taking pairs c, c + S, ... in turn with its rings running on across
+# them. One, two and three key tiles per pair (with one, the pairs alternate
+# between the two P.V completion barriers), 320 pairs: every output row, the
+# dense-bias forward, both 8-bit P.V passes and the score dump of that pipeline.
+@pytest.mark.parametrize("shape", [(16, 20, 56, 64), (8, 40, 96, 72), (4, 80, 136, 32)])
+def test_persistent_many_pairs(orc, shape):
+    B, H, N, d = shape
+    c = make_custom(B, H, N, d, seed=7 * N + d, with_bias=True, bias_std=0.5, zeros_frac=0.05)
+    q, k, v, bias = dev(c["q"]), dev(c["k"]), dev(c["v"]), dev(c["bias"])
+    qb, aq = binattn.pack(q)
+    kb, ak = binattn.pack(k)
+    S = binattn.scores_debug(qb, kb, d, engine="tc_biased").cpu().numpy()
+    assert np.array_equal(S, orc.scores(c["q"], c["k"])), f"scores {shape}"
+    o = binattn.forward(qb, kb, aq, ak, bias, v, c["softmax_scale"], engine="tc")
+    o_ws = binattn.forward_ws(qb, kb, aq, ak, bias, v, c["softmax_scale"])
+    o8 = binattn.forward_int8(qb, kb, aq, ak, bias, v, c["softmax_scale"])
+    o8n = binattn.forward_int8(qb, kb, aq, ak, None, v, c["softmax_scale"])
+    torch.cuda.synchronize()
+    binattn.device_status()
+    ref, spread = orc.forward_spread(c["q"], c["k"], c["bias"], c["v"], c["softmax_scale"])
+    check_o(bf16_to_f64(o), ref, f"persistent {shape}", spread=spread)
+    assert torch.equal(o.view(torch.int16), o_ws.view(torch.int16)), f"forward_ws {shape}"
+    check_o(bf16_to_f64(o8), orc.forward_int8(c["q"], c["k"], c["bias"], c["v"], c["softmax_scale"]),
+            f"persistent int8 {shape}")
+    check_o(bf16_to_f64(o8n), orc.forward_int8(c["q"], c["k"], None, c["v"], c["softmax_scale"]),
+            f"persistent int8 no bias {shape}")
