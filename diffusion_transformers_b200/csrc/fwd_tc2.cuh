@@ -464,15 +464,23 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         float ak[2];
         int ko[2];
       };
-      // tile g of the CTA's sequence: key tile g % nkt of pair g / nkt
+      // The tiles of the CTA's sequence in order: key tile kt_l of pair it_l
+      // is loaded next (tok_l: the pair's first token), past the end zeros.
       const int g_end = n_items * nkt;
-      auto load_tile = [&](int g, TileRegs& tr) {
-        const int kt = nkt > 0 ? g % nkt : 0;
-        const size_t tok0 = g < g_end ? item(g / nkt).tok0 : 0;
+      int it_l = 0, kt_l = 0;
+      size_t tok_l = n_items > 0 ? item(0).tok0 : 0;
+      auto load_next = [&](TileRegs& tr) {
+        const bool live = it_l < n_items;
+        const size_t tok0 = tok_l;
+        const int kt = kt_l;
+        if (live && ++kt_l == nkt) {
+          kt_l = 0;
+          if (++it_l < n_items) tok_l = item(it_l).tok0;
+        }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int key = key0 + kt * kKeys + lane + 32 * u;
-          const bool in = g < g_end && key < N;
+          const bool in = live && key < N;
 #pragma unroll
           for (int w = 0; w < 3; ++w) tr.wd[u][w] = (in && w < W) ? __ldg(p.kb + (tok0 + key) * W + w) : 0u;
           tr.ak[u] = (!kDump && in) ? __ldg(p.ak + tok0 + key) : 0.f;
@@ -485,11 +493,11 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         }
       };
       TileRegs cur, n1;
-      load_tile(0, cur);
-      load_tile(1, n1);
+      load_next(cur);
+      load_next(n1);
       for (int g = 0; g < g_end; ++g) {
         TileRegs n2;
-        load_tile(g + 2, n2);
+        load_next(n2);
         const int s = g % kKS;
         const bool ok = g < kKS || mbar_wait(&kv_empty[s], ((g / kKS) - 1) & 1, abort);
         if (!__all_sync(0xffffffffu, ok)) break;
@@ -1150,22 +1158,15 @@ inline SplitPlan split_plan(int B, int H, int N) {
   if (full == 0 || tail == 0 || 2 * tail > nsm || (N + kKeys - 1) / kKeys < 32) return {P, 0};
   return {full, tail};
 }
-// The grid of a launch over P whole pairs of N keys. With at most
-// kPersistMaxTiles key tiles per pair it is persistent: one CTA per SM (each
-// CTA holds all of its SM's tensor memory), CTA c taking pairs c, c + S, ...;
-// sets prm.npairs and returns the CTA count. Longer pairs run one per CTA
-// (npairs = 0, P CTAs), and so does a launch without a device to ask.
-// Measured (one B200): persistent grids cut DeiT-B (4 key tiles) by 13%,
-// ViT-L/16 (10) by 8% and DiT-XL/2 512 px (16) by 4%; at 64 key tiles they
-// gain nothing with the bf16 P.V and lose 13-20% in the two 8-bit P.V passes,
-// whose bias reads are closer to the HBM bound: a CTA launched as another
-// ends starts beside the CTA launched just before it, which reads the same
-// bias tiles for the other batch entry, while persistent CTAs drift apart
-// over their pairs and lose part of that L2 reuse.
-constexpr int kPersistMaxTiles = 16;
+// The grid of a launch over P whole pairs: with more pairs than SMs it is
+// persistent, one CTA per SM (each CTA holds all of its SM's tensor memory),
+// CTA c taking pairs c, c + S, ...; sets prm.npairs and returns the CTA
+// count. Otherwise, or without a device to ask, one pair per CTA (npairs = 0).
+// Measured on one B200 against one pair per CTA: DeiT-B -16%, ViT-L/16 -9%,
+// DiT-XL/2 512 px -6%, DiT-XL/2 1024 px (its 444 whole pairs) -1%, and the
+// same or better for both 8-bit P.V passes.
 inline int grid_for(tc::Params& prm, int P) {
   prm.npairs = 0;
-  if ((prm.N + kKeys - 1) / kKeys > kPersistMaxTiles) return P;
   int dev = 0, nsm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       nsm <= 0) {
