@@ -355,8 +355,10 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
   const int r = ((warp & 3) << 5) | lane;    // row within the tile = TMEM lane
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   // Softmax threads, once per pair: this thread's row of Q_t into TMEM, and
-  // alpha_q of the row (binary forward), returned.
-  auto stage_q = [&](const Item& w, int row, bool row_valid) {
+  // alpha_q of the row (binary forward), returned. A binary forward from
+  // binattn_pack's output takes the row's sign words and alpha_q in qw / aq,
+  // loaded one pair ahead (fetch_qbits below).
+  auto stage_q = [&](const Item& w, int row, bool row_valid, const uint32_t (&qw_in)[3], float aq_in) {
     float aq_row = 0.f;
     if constexpr (kRef) {
       // bf16 pairs: column c2 holds channels 2 c2 (low half) and 2 c2 + 1
@@ -379,17 +381,10 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       // e4m3 bytes: column c4 holds channels 4 c4 .. 4 c4 + 3 (lowest byte first);
       // pad channels (>= d) are 0 so they add nothing to the score.
       const uint32_t qcol = tmem + lane_base + 256 * t + kQColBin;
-      uint32_t qw[3] = {0u, 0u, 0u};
-      if (row_valid && !kDump) {
-        if (p.qh) {
-          pack_row_bf16_w(p.qh + (w.tok0 + row) * d, d, W, qw, aq_row);  // Q binarised here
-        } else {
-          for (int k = 0; k < W; ++k) qw[k] = p.qb[(w.tok0 + row) * W + k];
-          aq_row = p.aq[w.tok0 + row];
-        }
-      } else if (row_valid) {
-        for (int k = 0; k < W; ++k) qw[k] = p.qb[(w.tok0 + row) * W + k];
-      }
+      uint32_t qw[3] = {qw_in[0], qw_in[1], qw_in[2]};
+      aq_row = aq_in;
+      if (row_valid && !kDump && p.qh)
+        pack_row_bf16_w(p.qh + (w.tok0 + row) * d, d, W, qw, aq_row);  // Q binarised here
       for (int k = 0; k < W; ++k) {
         const uint32_t word = k == 0 ? qw[0] : k == 1 ? qw[1] : qw[2];
         uint32_t wv[8];
@@ -764,6 +759,24 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
     // skipped), so that each thread takes its part in every named barrier.
     if (!kNoPV && t == 1 && n_items > 0) named_arrive(3, 2 * kSoftmaxPerTile);  // tile 0 takes the first exp turn
     const int g_end = n_items * nkt;
+    // the sign words and alpha_q of this thread's row in pair it2 (zeros for
+    // a row >= N, past the last pair, and where stage_q does not take them)
+    uint32_t qn[3];
+    float aqn;
+    auto fetch_qbits = [&](int it2, uint32_t (&qw)[3], float& a) {
+      qw[0] = qw[1] = qw[2] = 0u;
+      a = 0.f;
+      if (kRef || p.qh != nullptr || it2 >= n_items) return;
+      const Item w2 = item(it2);
+      const int row2 = w2.q0 + t * kRows + r;
+      if (row2 < N) {
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+          if (k < W) qw[k] = __ldg(p.qb + (w2.tok0 + row2) * W + k);
+        if (!kDump) a = __ldg(p.aq + w2.tok0 + row2);
+      }
+    };
+    fetch_qbits(0, qn, aqn);
     for (int it = 0; it < n_items; ++it) {
     const Item w = item(it);
     tok0 = w.tok0;
@@ -773,9 +786,10 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
       // Q_t of the pair into TMEM; the issuer waits for all 128 rows. From
       // the second pair on, the previous pair's epilogue has read O_t (its
       // last P.V waited for), so the pair's first P.V may overwrite it.
-      const float aq_row = ok ? stage_q(w, row, row_valid) : 0.f;
+      const float aq_row = ok ? stage_q(w, row, row_valid, qn, aqn) : 0.f;
       mbar_arrive(&q_ready[t]);
       ci = kRef ? p.scale : ((!kDump && row_valid) ? p.scale * aq_row : 0.f);
+      fetch_qbits(it + 1, qn, aqn);  // in flight through this pair
     }
     m = -INFINITY;
     if constexpr (kI8) m = row_valid ? p.mrow[tok0 + row] : 0.f;
