@@ -287,6 +287,31 @@ def cpu_oracle_sample(w, with_bias, target_s, inp=None):
                        f"{b3 * 1e3:.3f} ms per row), extrapolated to all rows as prep + rows x per-row")
 
 
+def cpu_oracle_all(skip, target_s=1.5, single_core=("tiny", "deit_b")):
+    """The oracle on every other workload (with its bias), all host cores, a
+    bounded sample of about target_s each; single-core as well on the small
+    ones. Reported beside the GPU numbers, never timed against them."""
+    import oracle
+    orc = oracle.get()
+    cores = orc.num_threads()
+    out = {}
+    for name in sorted(WORKLOADS):
+        if name == skip:
+            continue
+        w = WORKLOADS[name]
+        inp = make_inputs(w, with_bias=True)
+        r = cpu_oracle_sample(w, True, target_s, inp)
+        out[name] = {"ms": round(r["value"], 3), "cores": r["cores"], "sample": r["sample"]}
+        if name in single_core:
+            orc.set_num_threads(1)
+            try:
+                r1 = cpu_oracle_sample(w, True, target_s, inp)
+            finally:
+                orc.set_num_threads(cores)
+            out[name]["single_core_ms"] = round(r1["value"], 3)
+    return out
+
+
 # ------------------------------------------------------------------ ranks
 def rank_seed(w, rank):
     """Every rank draws its own batch of the workload (weak scaling): rank 0
@@ -773,6 +798,7 @@ def run_gpu(args, w_job, rank, world, local_rank):
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(w, True, args.cpu_seconds, inp)
+        line["cpu_oracle_workloads"] = cpu_oracle_all(w.name)
     print(json.dumps(line), flush=True)
 
 
