@@ -61,6 +61,9 @@ def parse():
     ap.add_argument("--profile-once", action="store_true",
                     help="run --warmup plain steps (with bias) and exit: the command profiled by ncu")
     ap.add_argument("--no-bias", action="store_true", help="with --profile-once: steps without bias")
+    ap.add_argument("--profile-path", default="dense", choices=["dense", "int8", "relpos"],
+                    help="with --profile-once: the forward call the steps make (dense or no bias, the 8-bit P.V "
+                         "forward, the position-sensitive bias)")
     ap.add_argument("--batch", type=int, default=None,
                     help="with --profile-once: replace the workload's batch B (a small case for multi-pass "
                          "ncu captures)")
@@ -147,8 +150,8 @@ def roofline_line(w, with_bias, peaks, fwd_s, n_sm=148, sm_mhz=None):
 # back into null. The digest covers the code only (comments removed, runs of
 # white space collapsed), so an edit of a comment keeps the capture valid.
 NCU_TRAFFIC = {
-    "sources_sha256": "f5ce3cff18430b2c164e2e5db74163c3746f6a5678da86493858c84906573943",
-    "bytes_per_call": {"dit_xl_1024/bias": 590_075_904},
+    "sources_sha256": "e9e3ca022ab5da25352252f5e348eb9323258245cbdd3c226e05851a3f987387",
+    "bytes_per_call": {"dit_xl_1024/bias": 588_929_024},
 }
 
 _C_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'|//[^\n]*|/\*.*?\*/', re.S)
@@ -546,8 +549,28 @@ def run_gpu(args, w_job, rank, world, local_rank):
         return max_over_ranks_of(x, world, dev)
 
     if args.profile_once:
+        b = None if args.no_bias else bias
+        if args.profile_path == "int8":
+            iws = torch.empty(max(16, binattn.int8_workspace_bytes(B, H, N, d, b is not None)), dtype=torch.uint8,
+                              device=dev)
+            call = lambda: binattn.forward_int8(qb, kb, aq, ak, b, v, scale, workspace=iws, out=out, stream=stream)
+        elif args.profile_path == "relpos":
+            g = int(round(math.sqrt(N)))
+            if g * g != N:
+                raise SystemExit("--profile-path relpos needs a square patch grid (N = g * g)")
+            trng = np.random.default_rng(rank_seed(w, rank) + 77)
+            table = torch.from_numpy((trng.standard_normal((H, binattn.relpos_table_entries(g, g, 0))) * 0.05)
+                                     .astype(np.float32)).to(dev).bfloat16()
+            rws = torch.empty(max(16, binattn.lib().binattn_forward_relpos_workspace_bytes(B, H, N, d)),
+                              dtype=torch.uint8, device=dev)
+            call = lambda: binattn.forward_relpos(qb, kb, aq, ak, table, (g, g), 0, v, scale, workspace=rws,
+                                                  out=out, stream=stream)
+        else:
+            call = lambda: fwd(b)
         for _ in range(args.warmup):
-            step(None if args.no_bias else bias)
+            binattn.pack(q, qb, aq, stream)
+            binattn.pack(k, kb, ak, stream)
+            call()
         torch.cuda.synchronize()
         binattn.device_status(stream)
         return
