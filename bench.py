@@ -700,21 +700,34 @@ def run_gpu(args, w_job, rank, world, local_rank):
                                             torch.cuda.get_device_properties(dev).multi_processor_count)}
         del table, rws
 
-    # in-build bf16 attention on the same shapes (speed reference)
+    # in-build bf16 attention on the same shapes (speed reference), with the
+    # binary forward's launch plan (binattn_ref_bf16_forward_ws: persistent
+    # whole pairs, split tail) and, beside it, without the workspace
     ref = None
     try:
-        binattn.ref_bf16_forward(q, k, bias, v, scale, out=out, stream=stream)
-        torch.cuda.synchronize()
-        ev = []
-        for _ in range(args.steps):
-            flush.fill_(1)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            binattn.ref_bf16_forward(q, k, bias, v, scale, out=out, stream=stream)
-            e1.record(stream)
-            ev.append((e0, e1))
-        torch.cuda.synchronize()
-        ref = {"forward_ms": max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / len(ev))}
+        rws = torch.empty(max(16, binattn.lib().binattn_ref_bf16_forward_workspace_bytes(B, H, N, d, 1)),
+                          dtype=torch.uint8, device=dev)
+        variants = (("ws", lambda: binattn.ref_bf16_forward_ws(q, k, bias, v, scale, workspace=rws, out=out,
+                                                                stream=stream)),
+                    ("plain", lambda: binattn.ref_bf16_forward(q, k, bias, v, scale, out=out, stream=stream)))
+        ref_ms = {}
+        for name, f in variants:
+            f()
+            torch.cuda.synchronize()
+            ev = []
+            for _ in range(args.steps):
+                flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                f()
+                e1.record(stream)
+                ev.append((e0, e1))
+            torch.cuda.synchronize()
+            ref_ms[name] = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / len(ev))
+        binattn.device_status(stream)
+        ref = {"forward_ms": round(ref_ms["ws"], 5), "call": "binattn_ref_bf16_forward_ws",
+               "without_split_ms": round(ref_ms["plain"], 5)}
+        del rws
     except Exception as exc:  # not built for this engine/shape
         ref = {"unavailable": str(exc).splitlines()[0]}
 

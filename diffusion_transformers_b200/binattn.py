@@ -31,6 +31,7 @@ EXPORTS = (
     "binattn_forward_bias_ld_workspace_bytes", "binattn_padded_bias_ld", "binattn_forward_bias_ld_ws",
     "binattn_quantize_v", "binattn_forward_int8_workspace_bytes", "binattn_forward_int8",
     "binattn_forward_relpos_workspace_bytes", "binattn_forward_relpos",
+    "binattn_ref_bf16_forward_workspace_bytes", "binattn_ref_bf16_forward_ws",
 )
 
 
@@ -85,6 +86,10 @@ def lib() -> ctypes.CDLL:
     L.binattn_forward_fused_ws.argtypes = [P, I, P, P, P, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
     L.binattn_scores_debug.argtypes = [P, P, I, I, I, I, P, I, P]
     L.binattn_ref_bf16_forward.argtypes = [P, P, P, P, F, I, I, I, I, P, P]
+    L.binattn_ref_bf16_forward_workspace_bytes.argtypes = [I, I, I, I, I]
+    L.binattn_ref_bf16_forward_workspace_bytes.restype = ctypes.c_size_t
+    L.binattn_ref_bf16_forward_ws.argtypes = [P, P, P, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
+    L.binattn_ref_bf16_forward_ws.restype = I
     L.binattn_test_wait_timeout.argtypes = [P, P, P, P, P, P, F, I, I, I, I, P, I, P]
     L.binattn_device_status.argtypes = [P]
     L.binattn_strerror.argtypes = [I]
@@ -432,6 +437,33 @@ def ref_bf16_forward(q: torch.Tensor, k: torch.Tensor, bias: torch.Tensor | None
         _check(lib().binattn_ref_bf16_forward(_ptr(q), _ptr(k), _ptr(bias), _ptr(v), float(softmax_scale),
                                               B, H, N, d, _ptr(out), _stream(stream, dev)),
                "binattn_ref_bf16_forward")
+    return out
+
+
+def ref_bf16_forward_ws(q: torch.Tensor, k: torch.Tensor, bias: torch.Tensor | None, v: torch.Tensor,
+                        softmax_scale: float, workspace: torch.Tensor | None = None,
+                        out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """ref_bf16_forward with the long-sequence launch plan of forward_ws (a
+    short last wave split by key halves); workspace of
+    binattn_ref_bf16_forward_workspace_bytes, allocated here when None."""
+    B, H, N, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        _expect(t, name, (B, H, N, d), (torch.bfloat16,))
+    _expect(bias, "bias", (H, N, N), (torch.bfloat16,))
+    dev = _device(q, k, bias, v, out)
+    if workspace is not None:
+        _device(workspace, v)
+    need = int(lib().binattn_ref_bf16_forward_workspace_bytes(B, H, N, d, bias is not None))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    size = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        _check(lib().binattn_ref_bf16_forward_ws(_ptr(q), _ptr(k), _ptr(bias), _ptr(v), float(softmax_scale),
+                                                 B, H, N, d, _ptr(out), _ptr(workspace), ctypes.c_size_t(size),
+                                                 _stream(stream, dev)),
+               "binattn_ref_bf16_forward_ws")
     return out
 
 

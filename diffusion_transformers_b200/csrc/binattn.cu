@@ -585,9 +585,9 @@ int binattn_scores_debug(const uint32_t* q_bits, const uint32_t* k_bits, int B, 
   }
 }
 
-int binattn_ref_bf16_forward(const uint16_t* q, const uint16_t* k, const uint16_t* bias,
-                             const uint16_t* v, float softmax_scale, int B, int H, int N, int d,
-                             uint16_t* out, void* stream) {
+static int ref_bf16_forward(const uint16_t* q, const uint16_t* k, const uint16_t* bias, const uint16_t* v,
+                            float softmax_scale, int B, int H, int N, int d, uint16_t* out, float* part,
+                            void* stream) {
   BINATTN_CHECK_PTR(q);
   BINATTN_CHECK_PTR(k);
   BINATTN_CHECK_PTR(v);
@@ -600,11 +600,38 @@ int binattn_ref_bf16_forward(const uint16_t* q, const uint16_t* k, const uint16_
   std::string msg;
   int rc = binattn::tc2::supported(d, N, bias != nullptr, true)
                ? binattn::forward_ref_tc2(q, k, bias, v, softmax_scale, B, H, N, d, out,
-                                          static_cast<cudaStream_t>(stream), &msg)
+                                          static_cast<cudaStream_t>(stream), &msg, part)
                : binattn::forward_ref_bf16(q, k, bias, v, softmax_scale, B, H, N, d, out,
                                            static_cast<cudaStream_t>(stream), &msg);
   if (rc) return fail(rc, "%s", msg.c_str());
   return ok();
+}
+
+int binattn_ref_bf16_forward(const uint16_t* q, const uint16_t* k, const uint16_t* bias,
+                             const uint16_t* v, float softmax_scale, int B, int H, int N, int d,
+                             uint16_t* out, void* stream) {
+  return ref_bf16_forward(q, k, bias, v, softmax_scale, B, H, N, d, out, nullptr, stream);
+}
+
+size_t binattn_ref_bf16_forward_workspace_bytes(int B, int H, int N, int d, int has_bias) {
+  if (B < 1 || H < 1 || N < 1 || d < 1 || !binattn::tc2::supported(d, N, has_bias != 0, true)) return 0;
+  return binattn::tc2::split_part_bytes(B, H, N, d);
+}
+
+int binattn_ref_bf16_forward_ws(const uint16_t* q, const uint16_t* k, const uint16_t* bias, const uint16_t* v,
+                                float softmax_scale, int B, int H, int N, int d, uint16_t* out,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  const size_t need = (B >= 1 && H >= 1 && N >= 1 && d >= 1)
+                          ? binattn_ref_bf16_forward_workspace_bytes(B, H, N, d, bias != nullptr)
+                          : 0;
+  if (need) {
+    BINATTN_CHECK_PTR(workspace);
+    if (workspace_bytes < need)
+      return fail(BINATTN_ERR_ARG, "workspace of %zu bytes is below the %zu this shape needs", workspace_bytes,
+                  need);
+  }
+  return ref_bf16_forward(q, k, bias, v, softmax_scale, B, H, N, d, out,
+                          need ? static_cast<float*>(workspace) : nullptr, stream);
 }
 
 int binattn_test_wait_timeout(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,

@@ -1197,6 +1197,36 @@ inline size_t split_part_bytes(int B, int H, int N, int d) {
   return static_cast<size_t>(pl.tail) * 2 * kRows * 2 * (d + 2) * 4;
 }
 
+// One forward over all pairs of a call. With `part` (split_part_bytes of
+// workspace) and a split plan, the whole pairs run as one launch and the tail
+// pairs as two key halves each, joined by combine_halves_kernel; without,
+// every pair runs whole. run(ctas) launches the kernel with prm. persistent:
+// the whole-pair launch may take several pairs per CTA (grid_for); a kernel
+// that stages per-head data keeps one pair per CTA.
+template <class Run>
+inline int run_pairs(tc::Params& prm, float* part, bool persistent, Run run, cudaStream_t st, std::string* msg) {
+  const int B = prm.B, H = prm.H, N = prm.N, d = prm.d;
+  const SplitPlan plan = part ? split_plan(B, H, N) : SplitPlan{total_pairs(B, H, N), 0};
+  if (plan.full > 0) {  // (a split launch takes one pair per CTA and ignores npairs)
+    prm.npairs = 0;
+    if (int rc = run(persistent ? grid_for(prm, plan.full) : plan.full)) return rc;
+  }
+  if (plan.tail > 0) {
+    prm.pair_base = plan.full;
+    prm.split = 1;
+    prm.part = part;
+    if (int rc = run(2 * plan.tail)) return rc;
+    const int rows = plan.tail * 2 * kRows;
+    combine_halves_kernel<<<(rows + 255) / 256, 256, 0, st>>>(part, plan.full, plan.tail, B, H, N, d, prm.out);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      *msg = std::string("combine_halves_kernel launch: ") + cudaGetErrorString(e);
+      return BINATTN_ERR_CUDA;
+    }
+  }
+  return BINATTN_OK;
+}
+
 }  // namespace tc2
 
 // part: workspace for the tail split (tc2::split_part_bytes), or null for no split.
@@ -1207,28 +1237,11 @@ inline int forward_tc2(const uint32_t* qb, const uint32_t* kb, const float* aq, 
                        float* part = nullptr, const uint16_t* qh = nullptr, int stall_after = -1) {
   tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d, bias_ld, 0, 0,
                  nullptr, qh, stall_after};
-  const tc2::SplitPlan plan = part ? tc2::split_plan(B, H, N) : tc2::SplitPlan{tc2::total_pairs(B, H, N), 0};
   auto run = [&](int ctas) {
     return bias ? tc2::dispatch_dv<tc2::kModeBin, tc2::kDenseBias>(prm, ctas, st, msg)
                 : tc2::dispatch_dv<tc2::kModeBin, tc2::kNoBias>(prm, ctas, st, msg);
   };
-  if (plan.full > 0) {  // (a split launch takes one pair per CTA and ignores npairs)
-    if (int rc = run(tc2::grid_for(prm, plan.full))) return rc;
-  }
-  if (plan.tail > 0) {
-    prm.pair_base = plan.full;
-    prm.split = 1;
-    prm.part = part;
-    if (int rc = run(2 * plan.tail)) return rc;
-    const int rows = plan.tail * 2 * tc2::kRows;
-    tc2::combine_halves_kernel<<<(rows + 255) / 256, 256, 0, st>>>(part, plan.full, plan.tail, B, H, N, d, out);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) {
-      *msg = std::string("combine_halves_kernel launch: ") + cudaGetErrorString(e);
-      return BINATTN_ERR_CUDA;
-    }
-  }
-  return BINATTN_OK;
+  return tc2::run_pairs(prm, part, true, run, st, msg);
 }
 
 // The binary forward with the position-sensitive bias: table bf16
@@ -1245,7 +1258,6 @@ inline int forward_tc2_relpos(const uint32_t* qb, const uint32_t* kb, const floa
   prm.rel_gw = gw;
   prm.rel_ncls = ncls;
   prm.rel_R = (2 * gh - 1) * (2 * gw - 1) + 3 * ncls;
-  const tc2::SplitPlan plan = part ? tc2::split_plan(B, H, N) : tc2::SplitPlan{tc2::total_pairs(B, H, N), 0};
   // grid rows a whole number of 32-key chunks and no class token: every chunk
   // of keys is one run of the table (N is then a multiple of 32, so a chunk is
   // wholly below N or wholly beyond it)
@@ -1255,23 +1267,8 @@ inline int forward_tc2_relpos(const uint32_t* qb, const uint32_t* kb, const floa
            : rows ? tc2::dispatch_dv<tc2::kModeBin, tc2::kRelPosBiasRows>(prm, ctas, st, msg)
                   : tc2::dispatch_dv<tc2::kModeBin, tc2::kRelPosBias>(prm, ctas, st, msg);
   };
-  if (plan.full > 0) {
-    if (int rc = run(plan.full)) return rc;
-  }
-  if (plan.tail > 0) {
-    prm.pair_base = plan.full;
-    prm.split = 1;
-    prm.part = part;
-    if (int rc = run(2 * plan.tail)) return rc;
-    const int rows = plan.tail * 2 * tc2::kRows;
-    tc2::combine_halves_kernel<<<(rows + 255) / 256, 256, 0, st>>>(part, plan.full, plan.tail, B, H, N, d, out);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) {
-      *msg = std::string("combine_halves_kernel launch: ") + cudaGetErrorString(e);
-      return BINATTN_ERR_CUDA;
-    }
-  }
-  return BINATTN_OK;
+  // one pair per CTA: the kernel stages one head's table
+  return tc2::run_pairs(prm, part, false, run, st, msg);
 }
 
 // The 8-bit P.V forward on the 64-key pipeline: the row-max pass writes the
@@ -1303,14 +1300,17 @@ inline int scores_tc2(const uint32_t* qb, const uint32_t* kb, int B, int H, int 
                                                        msg);
 }
 
+// part: workspace for the tail split (tc2::split_part_bytes), or null.
 inline int forward_ref_tc2(const uint16_t* q, const uint16_t* k, const uint16_t* bias, const uint16_t* v,
                            float scale, int B, int H, int N, int d, uint16_t* out, cudaStream_t st,
-                           std::string* msg) {
+                           std::string* msg, float* part = nullptr) {
   tc::Params prm{nullptr, nullptr, q, k, nullptr, nullptr, bias, v, out, nullptr, scale, B, H, N, d, 0, 0, 0,
                  nullptr};
-  const int ctas = tc2::grid_for(prm, tc2::total_pairs(B, H, N));
-  return bias ? tc2::dispatch_dv<tc2::kModeRef, tc2::kDenseBias>(prm, ctas, st, msg)
-              : tc2::dispatch_dv<tc2::kModeRef, tc2::kNoBias>(prm, ctas, st, msg);
+  auto run = [&](int ctas) {
+    return bias ? tc2::dispatch_dv<tc2::kModeRef, tc2::kDenseBias>(prm, ctas, st, msg)
+                : tc2::dispatch_dv<tc2::kModeRef, tc2::kNoBias>(prm, ctas, st, msg);
+  };
+  return tc2::run_pairs(prm, part, true, run, st, msg);
 }
 
 }  // namespace binattn

@@ -809,28 +809,12 @@ inline int forward_tc3(const uint32_t* qb, const uint32_t* kb, const float* aq, 
                        float* part = nullptr, const uint16_t* qh = nullptr) {
   tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d, bias_ld, 0, 0,
                  nullptr, qh};
-  const tc2::SplitPlan plan = part ? tc2::split_plan(B, H, N) : tc2::SplitPlan{tc2::total_pairs(B, H, N), 0};
   auto run = [&](int ctas) {
     return bias ? tc3::dispatch_dv<tc3::kModeBin, true>(prm, ctas, st, msg)
                 : tc3::dispatch_dv<tc3::kModeBin, false>(prm, ctas, st, msg);
   };
-  if (plan.full > 0) {
-    if (int rc = run(plan.full)) return rc;
-  }
-  if (plan.tail > 0) {
-    prm.pair_base = plan.full;
-    prm.split = 1;
-    prm.part = part;
-    if (int rc = run(2 * plan.tail)) return rc;
-    const int rows = plan.tail * 2 * tc2::kRows;
-    tc2::combine_halves_kernel<<<(rows + 255) / 256, 256, 0, st>>>(part, plan.full, plan.tail, B, H, N, d, out);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) {
-      *msg = std::string("combine_halves_kernel launch: ") + cudaGetErrorString(e);
-      return BINATTN_ERR_CUDA;
-    }
-  }
-  return BINATTN_OK;
+  // one pair per CTA (this pipeline has no persistent loop)
+  return tc2::run_pairs(prm, part, false, run, st, msg);
 }
 
 }  // namespace binattn

@@ -359,6 +359,28 @@ int binattn_ref_bf16_forward(const uint16_t *q, const uint16_t *k,
                              uint16_t *out, void *stream);
 
 /*
+ * binattn_ref_bf16_forward_ws — the same reference with the long-sequence
+ * launch plan of binattn_forward_ws: where a short last wave of 256-row
+ * pairs would leave SMs idle, those pairs run as two key halves each, joined
+ * by a combine kernel, so that the reference and the binary forward are
+ * timed with the same plan. Arguments as binattn_ref_bf16_forward, plus:
+ *   workspace        device, caller-owned, 16-byte aligned, at least
+ *                    binattn_ref_bf16_forward_workspace_bytes(B, H, N, d,
+ *                    bias != NULL) bytes (it holds the halves' partial
+ *                    results); may be NULL when that is 0. Contents need no
+ *                    initialisation and are overwritten.
+ *   workspace_bytes  its size.
+ * Errors: as binattn_ref_bf16_forward; BINATTN_ERR_NULL / _ALIGN / _ARG for a
+ * missing, misaligned or short workspace.
+ */
+size_t binattn_ref_bf16_forward_workspace_bytes(int B, int H, int N, int d, int has_bias);
+int binattn_ref_bf16_forward_ws(const uint16_t *q, const uint16_t *k,
+                                const uint16_t *bias, const uint16_t *v,
+                                float softmax_scale, int B, int H, int N, int d,
+                                uint16_t *out, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/*
  * binattn_test_wait_timeout — test only: the binary forward on the 64-key
  * pipeline (d % 8 == 0, d <= 80; with a bias, N % 8 == 0), arguments as for
  * binattn_forward, except that its TMA producer issues nothing from key tile

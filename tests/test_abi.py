@@ -120,6 +120,25 @@ def test_scores_and_ref_host_validation(L):
                                       P(A), None) == 8
 
 
+def test_ref_ws_host_validation(L):
+    def rws(ws=A, size=1 << 30, N=4096, d=72, bias=A):
+        return L.binattn_ref_bf16_forward_ws(P(A), P(A), P(bias) if bias else None, P(A), ctypes.c_float(0.125),
+                                             2, 16, N, d, P(A), P(ws) if ws else None, ctypes.c_size_t(size), None)
+    # the reference's workspace is the split partials of the binary forward's
+    # plan (none on a shape the TMA-fed reference does not take)
+    assert L.binattn_ref_bf16_forward_workspace_bytes(2, 16, 4096, 72, 1) == _expected_ws(2, 16, 4096, 72, False)
+    assert L.binattn_ref_bf16_forward_workspace_bytes(2, 16, 4096, 80, 1) == 0
+    assert L.binattn_ref_bf16_forward_workspace_bytes(0, 16, 4096, 72, 1) == 0
+    assert rws(d=33) == 5
+    assert rws(bias=A + 2) == 4
+    assert rws(N=0) == 2
+    need = L.binattn_ref_bf16_forward_workspace_bytes(2, 16, 4096, 72, 1)
+    if need:  # only with a device to ask for the SM count
+        assert rws(ws=0) == 1
+        assert rws(ws=A + 8) == 4
+        assert rws(size=need - 1) == 8
+
+
 def test_last_error_message_is_specific(L):
     assert _fwd(L, v=A + 8) == 4
     assert b"v is not 16-byte aligned" in L.binattn_last_error_message()
@@ -304,6 +323,10 @@ def test_binding_marshals_every_call(monkeypatch):
     assert S.shape == (B, H, N, N) and calls[-1][1][2:6] == (B, H, N, d)
     binattn.ref_bf16_forward(q, q, None, v, 0.25)
     assert calls[-1][0] == "binattn_ref_bf16_forward" and calls[-1][1][5:9] == (B, H, N, d)
+    binattn.ref_bf16_forward_ws(q, q, bias, v, 0.25, workspace=torch.zeros(64, dtype=torch.uint8))
+    name, args = calls[-1]
+    assert name == "binattn_ref_bf16_forward_ws" and args[5:9] == (B, H, N, d) and args[11].value == 64
+    assert args[2].value == bias.data_ptr()
 
 
 @pytest.mark.parametrize("lang,std", [("c", "c99"), ("c++", "c++11")])

@@ -74,3 +74,26 @@ def test_ref_attention_full_size_sampled(name, with_bias):
     ref = numpy_attention(inp["q"], inp["k"], inp["v"], inp["bias"], inp["softmax_scale"], rows)
     vmax = float(np.abs(bf16_bits_to_f32(inp["v"])).max())
     check_ref(bf16_to_f64(got), ref, vmax, f"ref {name} bias={with_bias}")
+
+
+# binattn_ref_bf16_forward_ws runs the reference with the binary forward's
+# launch plan: at DiT-XL/2 1024 px the pairs of heads 14 and 15 are in the
+# split tail (two key halves joined by the combine kernel). Rows there, and
+# elsewhere, against the fp64 attention.
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_ref_attention_ws_split_tail(with_bias):
+    inp = make_inputs("dit_xl_1024", with_bias=with_bias)
+    B, H, N, d = inp["B"], inp["H"], inp["N"], inp["d"]
+    bias = dev(inp["bias"]) if with_bias else None
+    out = binattn.ref_bf16_forward_ws(dev(inp["q"]), dev(inp["k"]), bias, dev(inp["v"]), inp["softmax_scale"])
+    torch.cuda.synchronize()
+    binattn.device_status()
+    rng = np.random.default_rng(11)
+    tail = [(b * H + h) * N + i for b, h, i in zip(rng.integers(0, B, 24), rng.integers(14, 16, 24),
+                                                  rng.integers(0, N, 24))]
+    rows = np.concatenate([np.array(tail, dtype=np.int64), sample_rows(B, H, N, 16, seed=5)])
+    got = out.view(B * H * N, d)[torch.from_numpy(rows).cuda()]
+    ref = numpy_attention(inp["q"], inp["k"], inp["v"], inp["bias"] if with_bias else None,
+                          inp["softmax_scale"], rows)
+    vmax = float(np.abs(bf16_bits_to_f32(inp["v"])).max())
+    check_ref(bf16_to_f64(got), ref, vmax, f"ref_ws dit_xl_1024 bias={with_bias}")
