@@ -42,6 +42,19 @@ def test_pack_exact(orc, shape, qk_dtype):
     np.testing.assert_allclose(alpha.cpu().numpy().astype(np.float64), oa, rtol=1e-6, atol=0)
 
 
+# bf16 tokens of whole 16-byte chunks (one thread per token, the arithmetic
+# of the forward's own binarisation of Q): every d % 8 == 0 up to 128, with
+# ragged last blocks; bits exact, alpha within 1e-6.
+@pytest.mark.parametrize("d", [8, 16, 24, 40, 56, 64, 72, 80, 88, 104, 120, 128])
+def test_pack_rows_every_chunk_count(orc, d):
+    for N in (1, 193, 1000):
+        c = make_custom(2, 3, N, d, seed=N + d, zeros_frac=0.05)
+        bits, alpha = binattn.pack(dev(c["q"]))
+        ob, oa = orc.pack(c["q"])
+        assert np.array_equal(bits.cpu().numpy().view(np.uint32), ob), (N, d)
+        np.testing.assert_allclose(alpha.cpu().numpy().astype(np.float64), oa, rtol=1e-6, atol=0)
+
+
 @pytest.mark.parametrize("name", ["tiny", "deit_b", "vit_l384", "dit_xl_512", "dit_xl_1024"])
 def test_pack_exact_full_size(orc, name):
     inp = make_inputs(name, with_bias=False)
