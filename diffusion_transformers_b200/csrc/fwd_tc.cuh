@@ -843,14 +843,22 @@ struct TensorMaps {
   CUtensorMap v, ak, bias, k;
 };
 
-// One [BH][N][d] bf16 tensor as boxes of 8 channels x 64 keys: each box is one
-// column of 16-byte chunks of the no-swizzle operand layouts above.
+// One [BH][N][d] bf16 tensor as boxes of 8 channels x box_keys keys: each box
+// is one column of 16-byte chunks of the no-swizzle operand layouts of the
+// tensor-core pipelines. Keys >= N of the last tile are outside the box's
+// (b, h) plane and read as 0. Every TMA-fed pipeline builds its V (and
+// reference K) maps here.
 inline bool make_rows_map(EncodeTiledFn enc, CUtensorMap* tm, const uint16_t* base, cuuint64_t BH,
-                          cuuint64_t N, cuuint64_t d, const char* what, std::string* msg) {
+                          cuuint64_t N, cuuint64_t d, const char* what, std::string* msg,
+                          cuuint32_t box_keys = kKeys) {
+  if (!enc) {
+    *msg = "cuTensorMapEncodeTiled entry point unavailable";
+    return false;
+  }
   const cuuint32_t es[3] = {1, 1, 1};
   const cuuint64_t dims[3] = {d, N, BH};
   const cuuint64_t strides[2] = {d * 2, N * d * 2};
-  const cuuint32_t box[3] = {8, kKeys, 1};
+  const cuuint32_t box[3] = {8, box_keys, 1};
   CUresult rc = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(base), dims, strides,
                     box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

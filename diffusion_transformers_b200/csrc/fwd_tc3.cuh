@@ -711,28 +711,10 @@ fwd_tc3_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
 }
 
 // ------------------------------------------------------------------- host
-// One [BH][N][d] bf16 tensor as boxes of 8 channels x 128 keys (one column of
-// 16-byte chunks of the no-swizzle operand layouts above). Keys >= N of the
-// last tile are outside the box's (b, h) plane and read as 0.
+// V as boxes of 8 channels x 128 keys (tc::make_rows_map).
 inline bool make_rows_map(CUtensorMap* tm, const uint16_t* base, cuuint64_t BH, cuuint64_t N, cuuint64_t d,
                           const char* what, std::string* msg) {
-  tc::EncodeTiledFn enc = tc::encode_fn();
-  if (!enc) {
-    *msg = "cuTensorMapEncodeTiled entry point unavailable";
-    return false;
-  }
-  const cuuint32_t es[3] = {1, 1, 1};
-  const cuuint64_t dims[3] = {d, N, BH};
-  const cuuint64_t strides[2] = {d * 2, N * d * 2};
-  const cuuint32_t box[3] = {8, kKeys, 1};
-  CUresult rc = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(base), dims, strides, box,
-                    es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (rc != CUDA_SUCCESS) {
-    *msg = std::string("tensor map (") + what + ") rejected: " + std::to_string(rc);
-    return false;
-  }
-  return true;
+  return tc::make_rows_map(tc::encode_fn(), tm, base, BH, N, d, what, msg, kKeys);
 }
 
 template <int DV, int kMode, bool kBias>
