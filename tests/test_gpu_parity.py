@@ -432,3 +432,41 @@ def test_persistent_many_pairs(orc, shape):
             f"persistent int8 {shape}")
     check_o(bf16_to_f64(o8n), orc.forward_int8(c["q"], c["k"], None, c["v"], c["softmax_scale"]),
             f"persistent int8 no bias {shape}")
+
+
+# ------------------------------------------------------------- maximum sizes
+# The host accepts N <= 65535 and B * H <= 65535. At N = 65535 (512 key tiles
+# of the 128-key pipeline, a ragged last tile of 127 keys) sampled rows of the
+# tensor-core and CUDA-core forwards meet the oracle. At B * H = 65535 with
+# N = 8, the 64-key pipeline with a bias runs 65535 pairs on a persistent grid
+# (about 443 pairs per CTA, one key tile each) and the 128-key one without a
+# bias 65535 CTAs: every row against the oracle.
+def test_max_sequence_length(orc):
+    B, H, N, d = 1, 1, 65535, 64
+    c = make_custom(B, H, N, d, seed=65535, with_bias=False, zeros_frac=0.01)
+    q, k, v = dev(c["q"]), dev(c["k"]), dev(c["v"])
+    qb, aq = binattn.pack(q)
+    kb, ak = binattn.pack(k)
+    rows = np.concatenate([np.arange(4), np.arange(N - 4, N), sample_rows(B, H, N, 24, seed=3)])
+    ref = orc.forward_rows(c["q"], c["k"], None, c["v"], c["softmax_scale"], rows)
+    for engine in ("tc", "simt"):
+        out = binattn.forward(qb, kb, aq, ak, None, v, c["softmax_scale"], engine=engine)
+        torch.cuda.synchronize()
+        binattn.device_status()
+        got = out.view(B * H * N, d)[torch.from_numpy(rows).cuda()]
+        check_o(bf16_to_f64(got), ref, f"N = 65535 {engine}")
+
+
+@pytest.mark.parametrize("B,H,with_bias", [(65535, 1, False), (1, 65535, True), (65535, 1, True)])
+def test_max_batch_heads(orc, B, H, with_bias):
+    N, d = 8, 64
+    c = make_custom(B, H, N, d, seed=B + 2 * H, with_bias=with_bias, bias_std=0.5)
+    q, k, v = dev(c["q"]), dev(c["k"]), dev(c["v"])
+    bias = dev(c["bias"]) if with_bias else None
+    qb, aq = binattn.pack(q)
+    kb, ak = binattn.pack(k)
+    out = binattn.forward(qb, kb, aq, ak, bias, v, c["softmax_scale"], engine="tc")
+    torch.cuda.synchronize()
+    binattn.device_status()
+    ref = orc.forward(c["q"], c["k"], c["bias"] if with_bias else None, c["v"], c["softmax_scale"])
+    check_o(bf16_to_f64(out), ref, f"B={B} H={H} bias={with_bias}")
