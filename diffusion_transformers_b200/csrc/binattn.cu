@@ -263,9 +263,7 @@ int forward_tma_ws(const uint32_t* q_bits, const uint32_t* k_bits, const float* 
   if (pad) {
     ld = padded_bias_ld(N);
     uint16_t* padded = static_cast<uint16_t*>(workspace);
-    const long long rows = static_cast<long long>(H) * N;
-    const unsigned grid = static_cast<unsigned>((rows * ld + 255) / 256);
-    binattn::tc2::pad_bias_rows_kernel<<<grid, 256, 0, st>>>(bias, rows, N, bias_ld, ld, padded);
+    binattn::tc2::pad_bias_rows(bias, static_cast<long long>(H) * N, N, bias_ld, ld, padded, st);
     if (int rc = launch_status("pad_bias_rows_kernel")) return rc;
     fbias = padded;
   }
@@ -496,9 +494,7 @@ int binattn_forward_int8(const uint32_t* q_bits, const uint32_t* k_bits, const f
   if (w.pad) {
     ld = padded_bias_ld(N);
     uint16_t* padded = reinterpret_cast<uint16_t*>(ws + w.vq + w.scale + w.mrow + w.vmax);
-    const long long rows = static_cast<long long>(H) * N;
-    binattn::tc2::pad_bias_rows_kernel<<<static_cast<unsigned>((rows * ld + 255) / 256), 256, 0, st>>>(
-        bias, rows, N, N, ld, padded);
+    binattn::tc2::pad_bias_rows(bias, static_cast<long long>(H) * N, N, N, ld, padded, st);
     if (int rc = launch_status("pad_bias_rows_kernel")) return rc;
     fbias = padded;
   }

@@ -1005,14 +1005,40 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
 
 // Bias rows padded to ld elements (ld % 8 == 0, pad 0), so that they are TMA
 // rows: out[(h * N + i) * ld + j] = j < N ? bias[(h * N + i) * src_ld + j] : 0.
+// One warp per row (grid-stride over rows): lane c writes 16-byte chunk c of
+// the padded row (out is 16-byte aligned, ld % 8 == 0), reading its 8 source
+// elements with consecutive 2-byte loads across the warp (a source row starts
+// at any element).
 __global__ void __launch_bounds__(256) pad_bias_rows_kernel(const uint16_t* __restrict__ bias,
                                                             long long rows, int N, int src_ld, int ld,
                                                             uint16_t* __restrict__ out) {
-  const long long e = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
-  if (e >= rows * ld) return;
-  const long long row = e / ld;
-  const int j = static_cast<int>(e - row * ld);
-  out[e] = j < N ? bias[row * src_ld + j] : static_cast<uint16_t>(0);
+  const int lane = threadIdx.x & 31;
+  const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
+  const int chunks = ld / 8;
+  for (long long row = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); row < rows;
+       row += nwarps) {
+    const uint16_t* src = bias + row * src_ld;
+    uint4* dst = reinterpret_cast<uint4*>(out + row * ld);
+    for (int c = lane; c < chunks; c += 32) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 8 * c + 2 * e;
+        const uint32_t lo = j < N ? __ldg(src + j) : 0u;
+        const uint32_t hi = j + 1 < N ? __ldg(src + j + 1) : 0u;
+        w[e] = lo | (hi << 16);
+      }
+      dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+// Launches pad_bias_rows_kernel over rows rows: 8 warps per block, at most
+// 8 blocks per SM of a 148-SM part (the kernel strides over the rest).
+inline void pad_bias_rows(const uint16_t* bias, long long rows, int N, int src_ld, int ld, uint16_t* out,
+                          cudaStream_t st) {
+  const long long blocks = (rows + 7) / 8;
+  const unsigned grid = static_cast<unsigned>(blocks < 148 * 8 ? blocks : 148 * 8);
+  pad_bias_rows_kernel<<<grid, 256, 0, st>>>(bias, rows, N, src_ld, ld, out);
 }
 
 // Joins the two key halves of split pairs: for row i with partials (O_h, m_h,
