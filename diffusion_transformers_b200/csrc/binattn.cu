@@ -15,7 +15,6 @@
 #include "fwd_simt.cuh"
 #include "fwd_tc.cuh"
 #include "fwd_tc2.cuh"
-#include "fwd_tc3.cuh"
 #include "quantv.cuh"
 
 namespace {
@@ -188,14 +187,10 @@ int binattn_forward_engine(const uint32_t* q_bits, const uint32_t* k_bits, const
       if (!binattn::tc_supported(d))
         return fail(BINATTN_ERR_UNSUPPORTED, "engine %d needs d %% 8 == 0 (d = %d)", engine, d);
       std::string msg;
-      // TC: e4m3 +-1 operands where the shape allows, on the pipeline that
-      // measured fastest for it (128-key tiles without a bias, 64-key tiles
-      // with one); other shapes use bf16 +-1 operands
+      // TC: e4m3 +-1 operands on the TMA-fed 64-key pipeline where the shape
+      // allows (with or without a bias); other shapes use bf16 +-1 operands
       int rc;
-      if (engine == BINATTN_ENGINE_TC && !bias && binattn::tc3::supported(d, N, false))
-        rc = binattn::forward_tc3(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out, st,
-                                  &msg);
-      else if (engine == BINATTN_ENGINE_TC && binattn::tc2::supported(d, N, bias != nullptr, false))
+      if (engine == BINATTN_ENGINE_TC && binattn::tc2::supported(d, N, bias != nullptr, false))
         rc = binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out, st,
                                   &msg);
       else
@@ -224,7 +219,7 @@ namespace {
 // pad is rounded up to 256 bytes.
 int padded_bias_ld(int N) { return (N + 7) / 8 * 8; }
 bool ws_path(int d, int N, bool has_bias) {
-  return binattn::tc3::supported(d, N, has_bias, has_bias ? padded_bias_ld(N) : 0);
+  return binattn::tc2::supported(d, N, has_bias, false, has_bias ? padded_bias_ld(N) : 0);
 }
 // Bytes of the padded bias copy: needed when the bias rows (bias_ld elements
 // apart) are not TMA rows.
@@ -269,10 +264,8 @@ int forward_tma_ws(const uint32_t* q_bits, const uint32_t* k_bits, const float* 
   }
   float* part = need > pad ? reinterpret_cast<float*>(static_cast<char*>(workspace) + pad) : nullptr;
   std::string msg;
-  int rc = fbias ? binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, fbias, v, softmax_scale, B, H, N, d,
-                                        out, st, &msg, ld, part, qh)
-                 : binattn::forward_tc3(q_bits, k_bits, alpha_q, alpha_k, fbias, v, softmax_scale, B, H, N, d,
-                                        out, st, &msg, ld, part, qh);
+  int rc = binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, fbias, v, softmax_scale, B, H, N, d, out, st,
+                                &msg, ld, part, qh);
   if (rc) return fail(rc, "%s", msg.c_str());
   return ok();
 }
@@ -563,13 +556,11 @@ int binattn_scores_debug(const uint32_t* q_bits, const uint32_t* k_bits, int B, 
     case BINATTN_ENGINE_TC_BIASED: {
       if (!binattn::tc_supported(d))
         return fail(BINATTN_ERR_UNSUPPORTED, "engine TC needs d %% 8 == 0 (d = %d)", d);
-      // the kernel the TC forward runs for this shape: without a bias the
-      // 128-key pipeline, with one the 64-key pipeline, else the load-mode one
+      // the kernel the TC forward runs for this shape: the TMA-fed 64-key
+      // pipeline, else the load-mode one
       std::string msg;
       int rc;
-      if (engine == BINATTN_ENGINE_TC && binattn::tc3::supported(d, N, false))
-        rc = binattn::scores_tc3(q_bits, k_bits, B, H, N, d, S, st, &msg);
-      else if (binattn::tc2::supported(d, N, false, false))
+      if (binattn::tc2::supported(d, N, false, false))
         rc = binattn::scores_tc2(q_bits, k_bits, B, H, N, d, S, st, &msg);
       else
         rc = binattn::scores_tc(q_bits, k_bits, B, H, N, d, S, st, &msg);

@@ -133,7 +133,7 @@ struct Params {
   float scale;
   int B, H, N, d;
   int bias_ld;  // elements between bias rows (N, or the padded row length); 0 means N
-  // 128-key-tile pipeline only: CTAs cover 256-row pairs pair_base + blockIdx.x
+  // 64-key TMA-fed pipeline only: CTAs cover 256-row pairs pair_base + blockIdx.x
   // (split == 0), or, with split == 1, CTA 2i + h covers key half h of pair
   // pair_base + i and writes partial results to `part`.
   int pair_base;

@@ -1146,7 +1146,7 @@ inline int dispatch_dv(const tc::Params& prm, int ctas, cudaStream_t st, std::st
     case 80: return launch<80, kMode, kBiasKind>(prm, ctas, st, msg);
     default:
       if constexpr (kMode == kModeRef) {
-        *msg = "reference attention on the 128-key pipeline needs d <= 72";
+        *msg = "the reference attention on this pipeline needs d <= 72";
         return BINATTN_ERR_UNSUPPORTED;
       } else {
         return launch<96, kMode, kBiasKind>(prm, ctas, st, msg);

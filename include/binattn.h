@@ -85,8 +85,11 @@ typedef enum {
     BINATTN_ENGINE_SIMT = 1,
     BINATTN_ENGINE_POPC_TC = 2,
     BINATTN_ENGINE_TC = 3,
-    /* binattn_scores_debug only: the scores of the TC engine as a forward WITH
-     * a bias computes them (BINATTN_ENGINE_TC: as one without a bias). */
+    /* binattn_scores_debug only: the scores of the TC engine as a forward
+     * with a bias computes them. With and without a bias the TC forward now
+     * runs the same kernel, so this gives the same scores as
+     * BINATTN_ENGINE_TC; the code is kept so that callers that name it still
+     * work. */
     BINATTN_ENGINE_TC_BIASED = 4
 } binattn_engine;
 
@@ -337,10 +340,9 @@ int binattn_forward_relpos(const uint32_t *q_bits, const uint32_t *k_bits,
  * binattn_scores_debug — writes the integer scores S [B, H, N, N] (int32,
  * device) that engine `engine` computes inside the forward pass, using the same
  * kernel and score routine. For testing only: it materialises the N x N matrix.
- * The TC engine runs different kernels with and without a bias:
- * BINATTN_ENGINE_TC gives the scores of the kernel a forward without a bias
- * runs, BINATTN_ENGINE_TC_BIASED those of the kernel a forward with a bias
- * runs, for this shape.
+ * BINATTN_ENGINE_TC and BINATTN_ENGINE_TC_BIASED give the scores of the
+ * kernel the TC forward runs for this shape (the TMA-fed 64-key pipeline for
+ * d % 8 == 0, d <= 80; else the load-mode one).
  * Source: §2, S_ij = d - 2 * popcount(q_i XOR k_j) (identical pad bits add 0).
  */
 int binattn_scores_debug(const uint32_t *q_bits, const uint32_t *k_bits,

@@ -68,9 +68,8 @@ def test_pack_exact_full_size(orc, name):
 # --------------------------------------------------------------- scores (a3, a8)
 # The POPC_TC forward uses the same __popc routine as SIMT (one debug kernel);
 # the TC engine has its own tensor-core score routines and needs d % 8 == 0:
-# "tc" dumps from the kernel a forward without a bias runs (the 128-key
-# pipeline where it applies), "tc_biased" from the one a forward with a bias
-# runs (the 64-key pipeline).
+# "tc" and "tc_biased" dump the scores of the kernel the TC forward runs (the
+# TMA-fed 64-key pipeline where it applies, with or without a bias).
 TC_SCORE_ENGINES = ["tc", "tc_biased"]
 SCORE_CASES = [(s, e) for s in SMALL_SHAPES + ODD_D_SHAPES for e in ["simt"] + TC_SCORE_ENGINES
                if e == "simt" or s[3] % 8 == 0]
@@ -153,8 +152,7 @@ def test_forward_special_cases(orc, engine):
 
 # Keys whose scale alpha_k grows with the key index: every later key tile has
 # larger logits, so the running max grows tile after tile and O (with l) is
-# rescaled again and again, in both pipelines (no bias: 128-key tiles; bias:
-# 64-key tiles), on a ragged N.
+# rescaled again and again, with and without a bias, on a ragged N.
 @pytest.mark.parametrize("with_bias", [False, True])
 @pytest.mark.parametrize("d", [64, 72])
 def test_forward_growing_max(orc, with_bias, d):
@@ -435,12 +433,12 @@ def test_persistent_many_pairs(orc, shape):
 
 
 # ------------------------------------------------------------- maximum sizes
-# The host accepts N <= 65535 and B * H <= 65535. At N = 65535 (512 key tiles
-# of the 128-key pipeline, a ragged last tile of 127 keys) sampled rows of the
-# tensor-core and CUDA-core forwards meet the oracle. At B * H = 65535 with
-# N = 8, the 64-key pipeline with a bias runs 65535 pairs on a persistent grid
-# (about 443 pairs per CTA, one key tile each) and the 128-key one without a
-# bias 65535 CTAs: every row against the oracle.
+# The host accepts N <= 65535 and B * H <= 65535. At N = 65535 (1024 key
+# tiles of 64, a ragged last tile of 63 keys, on a persistent grid of 256
+# pairs) sampled rows of the tensor-core and CUDA-core forwards meet the
+# oracle. At B * H = 65535 with N = 8, the forward runs 65535 pairs on a
+# persistent grid (about 443 pairs per CTA, one key tile each), with and
+# without a bias: every row against the oracle.
 def test_max_sequence_length(orc):
     B, H, N, d = 1, 1, 65535, 64
     c = make_custom(B, H, N, d, seed=65535, with_bias=False, zeros_frac=0.01)
