@@ -129,6 +129,12 @@ int binattn_pack(const void *x, int dtype, int B, int H, int N, int d,
  * before a bf16 x bf16 -> fp32 P.V on the tensor-core engines (fp32 P on SIMT);
  * normalisation by the fp32 row sum in the epilogue.
  * No mask: every query attends to all N keys (vision / diffusion self-attention).
+ * Speed: for d % 8 == 0, d <= 80 this runs the TMA-fed tensor-core pipeline,
+ * except with a bias whose rows are not a multiple of 8 elements (N % 8 != 0,
+ * e.g. N = 197 or 577): TMA cannot read such rows, so that call reads the bias
+ * with plain loads at a few per cent of the roofline. Give such a bias a
+ * workspace (binattn_forward_ws pads it per call) or store it once with padded
+ * rows (binattn_forward_bias_ld_ws).
  */
 int binattn_forward(const uint32_t *q_bits, const uint32_t *k_bits,
                     const float *alpha_q, const float *alpha_k,
