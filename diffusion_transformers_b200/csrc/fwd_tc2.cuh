@@ -389,7 +389,9 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         const uint32_t word = k == 0 ? qw[0] : k == 1 ? qw[1] : qw[2];
         uint32_t wv[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) wv[j] = row_valid ? e4m3_bytes(word, 4 * j, 32 * k + 4 * j, d, true) : 0u;
+        // four channels per column (e4m3_nibble); d % 8 == 0, so a column is
+        // wholly below d or wholly padding (0)
+        for (int j = 0; j < 8; ++j) wv[j] = (row_valid && 32 * k + 4 * j < d) ? e4m3_nibble(word >> (4 * j)) : 0u;
         tmem_st8(qcol + 8 * k, wv);
       }
     }
@@ -965,16 +967,19 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
         } else {
         const float inv = 1.f / __uint_as_float(lbits);
         uint16_t* orow = p.out + (tok0 + row) * d;
+        // two column blocks of 16 per wait, so that the tensor-memory latency
+        // is paid once per 32 columns
 #pragma unroll
-        for (int cc = 0; cc < DV; cc += 16) {
+        for (int cc = 0; cc < DV; cc += 32) {
           if (cc < d) {  // warp-uniform: d is the same for every thread
-            uint32_t ov[16];
-            tmem_ld16(o_col + cc, ov);
+            uint32_t ov[32];
+            tmem_ld16(o_col + cc, *reinterpret_cast<uint32_t(*)[16]>(ov));
+            if (cc + 16 < DV && cc + 16 < d) tmem_ld16(o_col + cc + 16, *reinterpret_cast<uint32_t(*)[16]>(ov + 16));
             tmem_ld_wait();
             if (row_valid) {
 #pragma unroll
-              for (int e = 0; e < 16; e += 8) {
-                if (cc + e < d) {
+              for (int e = 0; e < 32; e += 8) {
+                if (cc + e < DV && cc + e < d) {
                   uint4 o4;
                   o4.x = pack_bf16x2(__uint_as_float(ov[e + 0]) * inv, __uint_as_float(ov[e + 1]) * inv);
                   o4.y = pack_bf16x2(__uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
