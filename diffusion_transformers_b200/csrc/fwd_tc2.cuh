@@ -1,6 +1,7 @@
 // fwd_tc2.cuh — the TMA-fed forward pipeline with e4m3 +-1 operands for the
-// binary QK^T: binary forward, its debug-scores variant, and the bf16
-// reference attention on the same pipeline.
+// binary QK^T: the binary forward (with a dense bias, a relative-position
+// table bias, or none), its 8-bit P.V passes, its debug-scores variant, and
+// the bf16 reference attention on the same pipeline.
 //
 // Source: "BinaryAttention: One-Bit QK-Attention for Vision and Diffusion
 // Transformers", §2 methodology (scaled binary Q/K, XNOR/popcount similarity,
@@ -40,6 +41,10 @@
 // Binary scores: Q and K bits become e4m3 +1.0 (0x38) / -1.0 (0xB8), pad
 // channels of Q are 0, and the fp32 accumulator holds the exact integer
 // d - 2 popcount(q XOR k) (kind::f8f6f4, K = 32 channels per MMA).
+//
+// Per pair the softmax threads stage Q_t (its sign words loaded one pair
+// ahead) and hand it to the issuer through q_ready; the issuer then starts
+// the pair's first two QK^T.
 //
 // Softmax per row, fp32, one thread per row: logit = (S alpha_k)
 // (scale alpha_q) + bias; the tile's max is settled before any exp; the
