@@ -61,9 +61,9 @@ def parse():
     ap.add_argument("--profile-once", action="store_true",
                     help="run --warmup plain steps (with bias) and exit: the command profiled by ncu")
     ap.add_argument("--no-bias", action="store_true", help="with --profile-once: steps without bias")
-    ap.add_argument("--profile-path", default="dense", choices=["dense", "int8", "relpos"],
+    ap.add_argument("--profile-path", default="dense", choices=["dense", "int8", "relpos", "sample"],
                     help="with --profile-once: the forward call the steps make (dense or no bias, the 8-bit P.V "
-                         "forward, the position-sensitive bias)")
+                         "forward, the position-sensitive bias, one dense bias per batch entry)")
     ap.add_argument("--batch", type=int, default=None,
                     help="with --profile-once: replace the workload's batch B (a small case for multi-pass "
                          "ncu captures)")
@@ -80,16 +80,17 @@ def workload_config(w, with_bias=True):
     }
 
 
-def algorithmic(w, with_bias=True):
+def algorithmic(w, with_bias=True, bias_per_sample=False):
     """Per-launch algorithmic work of the forward kernel (one (b,h,i,j) pair =
-    2d binary ops for QK, 2d flops for P.V)."""
+    2d binary ops for QK, 2d flops for P.V). bias_per_sample: one dense bias
+    per batch entry ([B, H, N, N], the context-aware form) instead of [H, N, N]."""
     BH, N, d = w.B * w.H, w.N, w.d
     pairs = BH * N * N
     W = (d + 31) // 32
     bytes_ = (2 * BH * N * W * 4          # q_bits, k_bits
               + 2 * BH * N * 4            # alpha_q, alpha_k
               + 2 * BH * N * d * 2        # V read, O written
-              + (w.H * N * N * 2 if with_bias else 0))  # bias, once
+              + ((BH if bias_per_sample else w.H) * N * N * 2 if with_bias else 0))  # bias, once
     pack_bytes = 2 * (BH * N * d * 2 + BH * N * W * 4 + BH * N * 4)
     return dict(pairs=pairs, qk_ops=2 * d * pairs, pv_flops=2 * d * pairs,
                 eff_flops=4 * d * pairs, bytes=bytes_, pack_bytes=pack_bytes)
@@ -103,13 +104,13 @@ E4M3_OVER_BF16 = 2.0
 MUFU_EXP_PER_CLK_PER_SM = 16  # ex2 throughput of the special-function unit
 
 
-def roofline_terms(w, with_bias, peaks, n_sm=148, sm_mhz=None):
+def roofline_terms(w, with_bias, peaks, n_sm=148, sm_mhz=None, bias_per_sample=False):
     """Roofline of one forward call: T_roof = max(T_mem, T_QK + T_PV), with
     T_mem = algorithmic bytes / HBM peak, T_PV = P.V flops / bf16 peak and
     T_QK = binary QK ops / e4m3 peak (the pipe the scores run on). The exp
     floor (one ex2 per pair on the special-function unit) is reported beside
     it; it is not part of T_roof."""
-    a = algorithmic(w, with_bias)
+    a = algorithmic(w, with_bias, bias_per_sample)
     bf16 = peaks["bf16_tflops"] * 1e12
     e4m3 = E4M3_OVER_BF16 * bf16
     t_mem = a["bytes"] / (peaks["hbm_gbs"] * 1e9)
@@ -123,12 +124,12 @@ def roofline_terms(w, with_bias, peaks, n_sm=148, sm_mhz=None):
                 tensor_peak_tflops=(a["qk_ops"] + a["pv_flops"]) / t_tensor / 1e12, work=a)
 
 
-def roofline_line(w, with_bias, peaks, fwd_s, n_sm=148, sm_mhz=None):
+def roofline_line(w, with_bias, peaks, fwd_s, n_sm=148, sm_mhz=None, bias_per_sample=False):
     """The bench line's roofline object for a forward call of fwd_s seconds:
     frac = T_roof / fwd_s. Bound hbm: achieved = algorithmic bytes / time
     against the HBM peak. Bound tensor: achieved = (QK ops + P.V flops) / time
     against the blended peak (QK ops + P.V flops) / (T_QK + T_PV)."""
-    r = roofline_terms(w, with_bias, peaks, n_sm, sm_mhz)
+    r = roofline_terms(w, with_bias, peaks, n_sm, sm_mhz, bias_per_sample)
     a = r["work"]
     if r["bound"] == "hbm":
         achieved, peak, unit = a["bytes"] / fwd_s / 1e9, peaks["hbm_gbs"], "GB/s"
@@ -145,13 +146,14 @@ def roofline_line(w, with_bias, peaks, fwd_s, n_sm=148, sm_mhz=None):
 # DRAM traffic of one forward call from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum summed over the launches the call makes at dit_xl_1024
 # with bias: the full-wave launch, the key-split tail launch and the combine; the
-# summary is profiles/fwd_tc2_dit_xl_1024_bias.md), valid only for the kernel
+# summary is profiles/fwd_tc2_dit_xl_1024_bias.md; "sample_bias" is the same call
+# with one bias per batch entry, profiles/sample_bias_dit_xl_1024.md), valid only for the kernel
 # sources it was taken on: any change to their code turns the reported traffic
 # back into null. The digest covers the code only (comments removed, runs of
 # white space collapsed), so an edit of a comment keeps the capture valid.
 NCU_TRAFFIC = {
-    "sources_sha256": "d32271b7085f3bb77ed855fefae5027c05f47146adb951dd77cfe743cd173c64",
-    "bytes_per_call": {"dit_xl_1024/bias": 588_367_616},
+    "sources_sha256": "9db1fb6cea252ee688aca9260fec0d6498dee55b041dd7b426fb35016c103357",
+    "bytes_per_call": {"dit_xl_1024/bias": 588_756_480, "dit_xl_1024/sample_bias": 1_126_140_672},
 }
 
 _C_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'|//[^\n]*|/\*.*?\*/', re.S)
@@ -595,6 +597,14 @@ def run_gpu(args, w_job, rank, world, local_rank):
                               dtype=torch.uint8, device=dev)
             call = lambda: binattn.forward_relpos(qb, kb, aq, ak, table, (g, g), 0, v, scale, workspace=rws,
                                                   out=out, stream=stream)
+        elif args.profile_path == "sample":
+            if b is None:
+                raise SystemExit("--profile-path sample needs the bias")
+            sb = torch.cat([torch.roll(b, -i, dims=0).unsqueeze(0) for i in range(B)])
+            sws = torch.empty(max(16, binattn.lib().binattn_forward_sample_bias_workspace_bytes(B, H, N, d, N)),
+                              dtype=torch.uint8, device=dev)
+            call = lambda: binattn.forward_sample_bias_ws(qb, kb, aq, ak, sb, v, scale, workspace=sws, out=out,
+                                                          stream=stream)
         else:
             call = lambda: fwd(b)
         for _ in range(args.warmup):
@@ -730,6 +740,44 @@ def run_gpu(args, w_job, rank, world, local_rank):
                                             torch.cuda.get_device_properties(dev).multi_processor_count)}
         del table, rws
 
+    # the context-aware form of the bias: one dense bias per batch entry
+    # (binattn_forward_sample_bias_ws), entry b the workload's bias with its
+    # heads rotated by b; same step and protocol. B times the bias bytes.
+    sample_bias = {}
+    if args.engine == "auto" and d % 8 == 0 and d <= 80 and bias is not None:
+        sb = torch.cat([torch.roll(bias, -i, dims=0).unsqueeze(0) for i in range(B)])
+        sws = torch.empty(max(16, binattn.lib().binattn_forward_sample_bias_workspace_bytes(B, H, N, d, N)),
+                          dtype=torch.uint8, device=dev)
+        fs = lambda: binattn.forward_sample_bias_ws(qb, kb, aq, ak, sb, v, scale, workspace=sws, out=out,
+                                                    stream=stream)
+        fs()
+        torch.cuda.synchronize()
+        barrier()
+        ev = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record(stream)
+            binattn.pack(q, qb, aq, stream)
+            binattn.pack(k, kb, ak, stream)
+            e1.record(stream)
+            fs()
+            e2.record(stream)
+            ev.append((e0, e1, e2))
+        torch.cuda.synchronize()
+        barrier()
+        binattn.device_status(stream)
+        sms = max_over_ranks(sum(b_.elapsed_time(c) for _, b_, c in ev) / len(ev))
+        sample_bias = {"bias_shape": [B, H, N, N], "call": "binattn_forward_sample_bias_ws",
+                       "ms_per_step": round(max_over_ranks(sum(a.elapsed_time(c) for a, _, c in ev) / len(ev)), 5),
+                       "forward_ms": round(sms, 5),
+                       "roofline": roofline_line(w, True, peaks, sms * 1e-3,
+                                                 torch.cuda.get_device_properties(dev).multi_processor_count,
+                                                 bias_per_sample=True)
+                       | {"traffic": ncu_traffic(f"{w.name}/sample_bias"),
+                          "algorithmic_bytes": algorithmic(w, True, bias_per_sample=True)["bytes"]}}
+        del sb, sws
+
     # in-build bf16 attention on the same shapes (speed reference), with the
     # binary forward's launch plan (binattn_ref_bf16_forward_ws: persistent
     # whole pairs, split tail) and, beside it, without the workspace
@@ -840,6 +888,7 @@ def run_gpu(args, w_job, rank, world, local_rank):
                     "roofline": roof0},
         "bf16_reference": ref,
         "relpos_bias": relpos,
+        "per_sample_bias": sample_bias,
         "int8_pv": dict(int8, call="binattn_forward_int8 (V 8-bit code + row-max pass + 8-bit P.V pass)",
                         step="pack(Q) + pack(K) + binattn_forward_int8"),
         "other_workloads": others,

@@ -32,6 +32,7 @@ EXPORTS = (
     "binattn_quantize_v", "binattn_forward_int8_workspace_bytes", "binattn_forward_int8",
     "binattn_forward_relpos_workspace_bytes", "binattn_forward_relpos",
     "binattn_ref_bf16_forward_workspace_bytes", "binattn_ref_bf16_forward_ws",
+    "binattn_forward_sample_bias_workspace_bytes", "binattn_forward_sample_bias_ws",
 )
 
 
@@ -71,6 +72,10 @@ def lib() -> ctypes.CDLL:
     L.binattn_padded_bias_ld.restype = I
     L.binattn_forward_bias_ld_ws.argtypes = [P, P, P, P, P, I, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
     L.binattn_forward_bias_ld_ws.restype = I
+    L.binattn_forward_sample_bias_workspace_bytes.argtypes = [I, I, I, I, I]
+    L.binattn_forward_sample_bias_workspace_bytes.restype = ctypes.c_size_t
+    L.binattn_forward_sample_bias_ws.argtypes = [P, P, P, P, P, I, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
+    L.binattn_forward_sample_bias_ws.restype = I
     L.binattn_quantize_v.argtypes = [P, I, I, I, I, P, P, P]
     L.binattn_quantize_v.restype = I
     L.binattn_forward_int8_workspace_bytes.argtypes = [I, I, I, I, I]
@@ -299,6 +304,37 @@ def forward_bias_ld_ws(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torc
                                                 ld, _ptr(v), float(softmax_scale), B, H, N, d, _ptr(out),
                                                 _ptr(workspace), ctypes.c_size_t(size), _stream(stream, dev)),
                "binattn_forward_bias_ld_ws")
+    return out
+
+
+def forward_sample_bias_ws(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor,
+                           alpha_k: torch.Tensor, bias: torch.Tensor, v: torch.Tensor, softmax_scale: float,
+                           workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                           stream=None) -> torch.Tensor:
+    """forward_ws with one bias per batch entry (a context-aware bias, computed
+    per sample): bias [B, H, N, ld], ld >= N (only its first N columns are read)."""
+    B, H, N, d = v.shape
+    if bias.dim() != 4 or tuple(bias.shape[:3]) != (B, H, N) or bias.shape[3] < N:
+        raise ValueError(f"bias must be [B={B}, H={H}, N={N}, ld >= N], got {tuple(bias.shape)}")
+    if bias.dtype != torch.bfloat16 or not bias.is_contiguous():
+        raise TypeError("bias must be a contiguous bfloat16 tensor")
+    ld = bias.shape[3]
+    dev = _forward_args(q_bits, k_bits, alpha_q, alpha_k, None, v, out)
+    _device(bias, v)
+    if workspace is not None:
+        _device(workspace, v)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    need = int(lib().binattn_forward_sample_bias_workspace_bytes(B, H, N, d, ld))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    size = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        _check(lib().binattn_forward_sample_bias_ws(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k),
+                                                    _ptr(bias), ld, _ptr(v), float(softmax_scale), B, H, N, d,
+                                                    _ptr(out), _ptr(workspace), ctypes.c_size_t(size),
+                                                    _stream(stream, dev)),
+               "binattn_forward_sample_bias_ws")
     return out
 
 

@@ -222,14 +222,16 @@ bool ws_path(int d, int N, bool has_bias) {
   return binattn::tc2::supported(d, N, has_bias, false, has_bias ? padded_bias_ld(N) : 0);
 }
 // Bytes of the padded bias copy: needed when the bias rows (bias_ld elements
-// apart) are not TMA rows.
-size_t ws_pad_bytes(int H, int N, bool has_bias, int bias_ld) {
+// apart) are not TMA rows. bias_heads: H for a shared bias [H, N, N], B * H
+// for one bias per batch entry.
+size_t ws_pad_bytes(long long bias_heads, int N, bool has_bias, int bias_ld) {
   if (!has_bias || bias_ld % 8 == 0) return 0;
-  return (static_cast<size_t>(H) * N * padded_bias_ld(N) * 2 + 255) / 256 * 256;
+  return (static_cast<size_t>(bias_heads) * N * padded_bias_ld(N) * 2 + 255) / 256 * 256;
 }
-size_t ws_bytes(int B, int H, int N, int d, bool has_bias, int bias_ld) {
+size_t ws_bytes(int B, int H, int N, int d, bool has_bias, int bias_ld, bool per_sample = false) {
   if (B < 1 || H < 1 || N < 1 || d < 1 || !ws_path(d, N, has_bias)) return 0;
-  return ws_pad_bytes(H, N, has_bias, bias_ld) + binattn::tc2::split_part_bytes(B, H, N, d);
+  const long long bias_heads = per_sample ? static_cast<long long>(B) * H : H;
+  return ws_pad_bytes(bias_heads, N, has_bias, bias_ld) + binattn::tc2::split_part_bytes(B, H, N, d);
 }
 }  // namespace
 
@@ -248,24 +250,27 @@ namespace {
 // The TMA-fed forward with a workspace (ws_path(d, N, bias) holds): bias rows
 // padded into the workspace when N % 8 != 0, a short last wave split by key
 // halves, and with qh set, Q binarised inside the kernel.
-// bias_ld: elements between the caller's bias rows (>= N).
+// bias_ld: elements between the caller's bias rows (>= N). per_sample: the
+// bias is [B, H, N, bias_ld] (one per batch entry), not [H, N, bias_ld].
 int forward_tma_ws(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q, const float* alpha_k,
                    const uint16_t* bias, int bias_ld, const uint16_t* v, float softmax_scale, int B, int H, int N,
-                   int d, uint16_t* out, void* workspace, size_t need, const uint16_t* qh, cudaStream_t st) {
-  const size_t pad = ws_pad_bytes(H, N, bias != nullptr, bias_ld);
+                   int d, uint16_t* out, void* workspace, size_t need, const uint16_t* qh, cudaStream_t st,
+                   bool per_sample = false) {
+  const long long bias_heads = per_sample ? static_cast<long long>(B) * H : H;
+  const size_t pad = ws_pad_bytes(bias_heads, N, bias != nullptr, bias_ld);
   const uint16_t* fbias = bias;
   int ld = bias_ld == N ? 0 : bias_ld;
   if (pad) {
     ld = padded_bias_ld(N);
     uint16_t* padded = static_cast<uint16_t*>(workspace);
-    binattn::tc2::pad_bias_rows(bias, static_cast<long long>(H) * N, N, bias_ld, ld, padded, st);
+    binattn::tc2::pad_bias_rows(bias, bias_heads * N, N, bias_ld, ld, padded, st);
     if (int rc = launch_status("pad_bias_rows_kernel")) return rc;
     fbias = padded;
   }
   float* part = need > pad ? reinterpret_cast<float*>(static_cast<char*>(workspace) + pad) : nullptr;
   std::string msg;
   int rc = binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, fbias, v, softmax_scale, B, H, N, d, out, st,
-                                &msg, ld, part, qh);
+                                &msg, ld, part, qh, -1, per_sample);
   if (rc) return fail(rc, "%s", msg.c_str());
   return ok();
 }
@@ -315,6 +320,33 @@ int binattn_forward_bias_ld_ws(const uint32_t* q_bits, const uint32_t* k_bits, c
   }
   return forward_tma_ws(q_bits, k_bits, alpha_q, alpha_k, bias, bias_ld, v, softmax_scale, B, H, N, d, out,
                         workspace, need, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+size_t binattn_forward_sample_bias_workspace_bytes(int B, int H, int N, int d, int bias_ld) {
+  if (bias_ld < N) return 0;
+  return ws_bytes(B, H, N, d, true, bias_ld, true);
+}
+
+int binattn_forward_sample_bias_ws(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q,
+                                   const float* alpha_k, const uint16_t* bias, int bias_ld, const uint16_t* v,
+                                   float softmax_scale, int B, int H, int N, int d, uint16_t* out, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  BINATTN_CHECK_PTR(bias);
+  if (int rc = check_forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out))
+    return rc;
+  if (bias_ld < N) return fail(BINATTN_ERR_ARG, "bias_ld = %d is below N = %d", bias_ld, N);
+  if (!ws_path(d, N, true))
+    return fail(BINATTN_ERR_UNSUPPORTED,
+                "a per-sample bias needs the TMA-fed pipeline (d %% 8 == 0, d <= 80); d = %d", d);
+  const size_t need = binattn_forward_sample_bias_workspace_bytes(B, H, N, d, bias_ld);
+  if (need) {
+    BINATTN_CHECK_PTR(workspace);
+    if (workspace_bytes < need)
+      return fail(BINATTN_ERR_ARG, "workspace of %zu bytes is below the %zu this shape needs", workspace_bytes,
+                  need);
+  }
+  return forward_tma_ws(q_bits, k_bits, alpha_q, alpha_k, bias, bias_ld, v, softmax_scale, B, H, N, d, out,
+                        workspace, need, nullptr, static_cast<cudaStream_t>(stream), true);
 }
 
 size_t binattn_forward_fused_workspace_bytes(int B, int H, int N, int d, int q_dtype, int has_bias) {

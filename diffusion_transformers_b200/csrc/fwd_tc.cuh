@@ -162,6 +162,10 @@ struct Params {
   // pair_base + npairs - 1, CTA c taking c, c + gridDim.x, ... (a persistent
   // launch of fewer CTAs than pairs); 0: one pair per CTA.
   int npairs = 0;
+  // 64-key pipeline, dense bias: 1 when each batch entry has its own bias
+  // [B, H, N rows] (a context-aware bias, computed per sample), read at row
+  // (b * H + h) * N + i; 0 when the batch shares one bias [H, N rows].
+  int bias_per_sample = 0;
 };
 
 // Named barrier 1 over the load-mode loader warps with an AND reduction.

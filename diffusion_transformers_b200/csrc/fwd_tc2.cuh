@@ -447,8 +447,8 @@ fwd_tc2_kernel(const tc::Params p, const __grid_constant__ CUtensorMap tm_v,
               const int i = (g % kBS) * 2 + t2;
               if (g >= kBS && !(ok = mbar_wait(&b_empty[i], ((g / kBS) - 1) & 1, abort))) break;
               mbar_arrive_expect_tx(&b_full[i], L::kBiasTile);
-              tma_load_3d(smem + L::kBiasOff + i * L::kBiasTile, &tm_bias, j0, w.q0 + t2 * kRows, w.h,
-                          &b_full[i]);
+              tma_load_3d(smem + L::kBiasOff + i * L::kBiasTile, &tm_bias, j0, w.q0 + t2 * kRows,
+                          p.bias_per_sample ? w.bh : w.h, &b_full[i]);
             }
           }
         }
@@ -1091,8 +1091,9 @@ inline bool make_rows_map(CUtensorMap* tm, const uint16_t* base, cuuint64_t BH, 
   return tc::make_rows_map(tc::encode_fn(), tm, base, BH, N, d, what, msg, kKeys);
 }
 
-// bias [H][N rows][N keys] bf16, rows ld elements apart (ld % 8 == 0), as boxes of
-// 64 keys x 128 rows, 128B swizzle.
+// bias [H][N rows][N keys] bf16 (or [B * H][N][N], one bias per batch entry),
+// rows ld elements apart (ld % 8 == 0), as boxes of 64 keys x 128 rows, 128B
+// swizzle.
 inline bool make_bias_map(CUtensorMap* tm, const uint16_t* bias, cuuint64_t H, cuuint64_t N,
                           cuuint64_t ld, std::string* msg) {
   tc::EncodeTiledFn enc = tc::encode_fn();
@@ -1125,7 +1126,8 @@ inline int launch(const tc::Params& prm, int ctas, cudaStream_t st, std::string*
   if ((kMode == kModeBin || kMode == kModeRef) && !make_rows_map(&tm_v, prm.v, BH, prm.N, prm.d, "V", msg))
     return BINATTN_ERR_CUDA;
   if (kMode == kModeRef && !make_rows_map(&tm_k, prm.k, BH, prm.N, prm.d, "K", msg)) return BINATTN_ERR_CUDA;
-  if (kBias && !make_bias_map(&tm_bias, prm.bias, prm.H, prm.N, prm.bias_ld > 0 ? prm.bias_ld : prm.N, msg))
+  if (kBias && !make_bias_map(&tm_bias, prm.bias, prm.bias_per_sample ? BH : prm.H, prm.N,
+                              prm.bias_ld > 0 ? prm.bias_ld : prm.N, msg))
     return BINATTN_ERR_CUDA;
   auto kern = fwd_tc2_kernel<DV, kMode, kBiasKind>;
   constexpr int smem = Layout<DV, kMode, kBiasKind>::kLaunchBytes;
@@ -1249,12 +1251,15 @@ inline int run_pairs(tc::Params& prm, float* part, bool persistent, Run run, cud
 
 // part: workspace for the tail split (tc2::split_part_bytes), or null for no split.
 // qh: bf16 Q for a forward that binarises Q itself (qb, aq then unused), or null.
+// bias_per_sample: the bias is [B, H, N, N] (one per batch entry), not [H, N, N].
 inline int forward_tc2(const uint32_t* qb, const uint32_t* kb, const float* aq, const float* ak,
                        const uint16_t* bias, const uint16_t* v, float scale, int B, int H, int N, int d,
                        uint16_t* out, cudaStream_t st, std::string* msg, int bias_ld = 0,
-                       float* part = nullptr, const uint16_t* qh = nullptr, int stall_after = -1) {
+                       float* part = nullptr, const uint16_t* qh = nullptr, int stall_after = -1,
+                       bool bias_per_sample = false) {
   tc::Params prm{qb, kb, nullptr, nullptr, aq, ak, bias, v, out, nullptr, scale, B, H, N, d, bias_ld, 0, 0,
                  nullptr, qh, stall_after};
+  prm.bias_per_sample = bias_per_sample ? 1 : 0;
   auto run = [&](int ctas) {
     return bias ? tc2::dispatch_dv<tc2::kModeBin, tc2::kDenseBias>(prm, ctas, st, msg)
                 : tc2::dispatch_dv<tc2::kModeBin, tc2::kNoBias>(prm, ctas, st, msg);

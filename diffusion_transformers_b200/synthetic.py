@@ -146,3 +146,20 @@ def make_custom(B: int, H: int, N: int, d: int, seed: int, qk_dtype: str = "bf16
         k = f32_to_bf16_bits(k)
     return dict(q=q, k=k, v=f32_to_bf16_bits(v), bias=bias, B=B, H=H, N=N, d=d,
                 softmax_scale=1.0 / math.sqrt(d), qk_dtype=qk_dtype, name=f"custom{B}x{H}x{N}x{d}")
+
+
+def per_sample_bias(B: int, H: int, N: int, seed: int, bias_std: float = 0.5,
+                    base: np.ndarray | None = None) -> np.ndarray:
+    """One dense bias per batch entry, bf16 bits [B, H, N, N]: the stand-in for a
+    context-aware bias, which differs from sample to sample.
+
+    Without ``base``: B independent N(0, bias_std^2) draws. With ``base`` (bf16
+    bits [H, N, N], e.g. a workload's shared bias): entry b is ``base`` with its
+    heads rotated by b, distinct per sample without a second draw of N^2 values
+    per head (used at full size).
+    """
+    if base is not None:
+        assert base.shape == (H, N, N)
+        return np.stack([np.roll(base, -b, axis=0) for b in range(B)])
+    rng = np.random.default_rng(seed)
+    return f32_to_bf16_bits(rng.standard_normal(size=(B, H, N, N), dtype=np.float32) * np.float32(bias_std))

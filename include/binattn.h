@@ -317,6 +317,36 @@ int binattn_forward_int8(const uint32_t *q_bits, const uint32_t *k_bits,
                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * binattn_forward_sample_bias_ws — binattn_forward_ws with one bias per batch
+ * entry: bias bf16 [B, H, N, bias_ld] (device, 16-byte aligned, not NULL),
+ * element (b, h, i, j) at bias[((b * H + h) * N + i) * bias_ld + j], bias_ld
+ * >= N. This is the context-aware form of the learnable bias: a bias computed
+ * from each sample's own content differs from sample to sample, so the
+ * forward takes the result of that computation, whatever it is, as a dense
+ * bias per batch entry. The logit of row (b, h, i), key j is
+ * softmax_scale * alpha_q * alpha_k * S_ij + bias[b, h, i, j].
+ * With bias_ld % 8 == 0 the kernel reads the rows as they are; otherwise they
+ * are first copied into the workspace with rows padded to 8 elements.
+ *   workspace  at least binattn_forward_sample_bias_workspace_bytes(...) bytes
+ *              (the padded copy, B * H * N * roundup(N, 8) * 2 bytes when
+ *              bias_ld % 8 != 0, and the split tail's partials); may be NULL
+ *              when that size is 0.
+ * Needs d % 8 == 0 and d <= 80 (BINATTN_ERR_UNSUPPORTED otherwise);
+ * BINATTN_ERR_ARG when bias_ld < N or the workspace is too small; otherwise
+ * errors as binattn_forward. With the same bias in every batch entry the
+ * result equals binattn_forward_ws on that bias, bit for bit.
+ * Source: §2 bias enhancement (the bias may be dense, position-sensitive or
+ * context-aware).
+ */
+size_t binattn_forward_sample_bias_workspace_bytes(int B, int H, int N, int d, int bias_ld);
+int binattn_forward_sample_bias_ws(const uint32_t *q_bits, const uint32_t *k_bits,
+                                   const float *alpha_q, const float *alpha_k,
+                                   const uint16_t *bias, int bias_ld, const uint16_t *v,
+                                   float softmax_scale, int B, int H, int N, int d,
+                                   uint16_t *out, void *workspace, size_t workspace_bytes,
+                                   void *stream);
+
+/*
  * binattn_forward_relpos — binattn_forward with the position-sensitive form of
  * the learnable bias instead of a dense [H, N, N] one: a relative-position
  * table. The N tokens are n_cls (0 or 1) class tokens followed by the patches

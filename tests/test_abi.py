@@ -80,6 +80,28 @@ def test_bias_ld_host_validation(L):
     assert L.binattn_forward_bias_ld_workspace_bytes(1, 2, 197, 64, 150) == 0  # ld < N
 
 
+def test_sample_bias_host_validation(L):
+    def fwd(bias=A, ld=16, d=64, N=16, ws=A, wsb=1 << 20, B=2, H=3):
+        return L.binattn_forward_sample_bias_ws(P(A), P(A), P(A), P(A), P(bias) if bias else None, ld, P(A),
+                                                ctypes.c_float(0.125), B, H, N, d, P(A), P(ws) if ws else None,
+                                                ctypes.c_size_t(wsb), None)
+    assert fwd(bias=0) == 1                 # the bias is required
+    assert fwd(ld=15) == 8                  # rows closer than N
+    assert fwd(d=33) == 5                   # only the TMA-fed pipeline takes it
+    assert fwd(d=96) == 5
+    assert fwd(bias=A + 2) == 4
+    assert fwd(ws=0, N=197, ld=197) == 1    # the padded copy needs a workspace
+    assert fwd(N=197, ld=197, wsb=100) == 8
+    assert b"workspace" in L.binattn_last_error_message()
+    assert L.binattn_forward_sample_bias_workspace_bytes(2, 3, 197, 64, 150) == 0  # ld < N
+    # the padded copy holds B * H bias matrices, not H
+    for B, H, N, d, ld in [(64, 12, 197, 64, 197), (2, 16, 4096, 72, 4096), (3, 2, 300, 8, 301), (1, 19, 2048, 72, 2048)]:
+        pad = 0 if ld % 8 == 0 else (B * H * N * ((N + 7) // 8 * 8) * 2 + 255) // 256 * 256
+        shared = L.binattn_forward_bias_ld_workspace_bytes(B, H, N, d, ld)
+        shared_pad = 0 if ld % 8 == 0 else (H * N * ((N + 7) // 8 * 8) * 2 + 255) // 256 * 256
+        assert L.binattn_forward_sample_bias_workspace_bytes(B, H, N, d, ld) == pad + shared - shared_pad
+
+
 def test_relpos_host_validation(L):
     def fwd(table=A, gh=4, gw=4, ncls=0, N=16, d=64, ws=A):
         return L.binattn_forward_relpos(P(A), P(A), P(A), P(A), P(table) if table else None, gh, gw, ncls, P(A),
@@ -327,6 +349,13 @@ def test_binding_marshals_every_call(monkeypatch):
     name, args = calls[-1]
     assert name == "binattn_ref_bf16_forward_ws" and args[5:9] == (B, H, N, d) and args[11].value == 64
     assert args[2].value == bias.data_ptr()
+    sbias = torch.zeros(B, H, N, N + 7, **bf)
+    binattn.forward_sample_bias_ws(qb, qb, aq, aq, sbias, v, 0.25, workspace=torch.zeros(32, dtype=torch.uint8))
+    name, args = calls[-1]
+    assert name == "binattn_forward_sample_bias_ws" and args[5] == N + 7 and args[8:12] == (B, H, N, d)
+    assert args[4].value == sbias.data_ptr() and args[14].value == 32
+    with pytest.raises(ValueError, match="bias must be"):
+        binattn.forward_sample_bias_ws(qb, qb, aq, aq, bias, v, 0.25)
 
 
 @pytest.mark.parametrize("lang,std", [("c", "c99"), ("c++", "c++11")])

@@ -123,6 +123,8 @@ def test_algorithmic_work_matches_the_hand_figures():
         assert abs(a["pv_flops"] / 1e9 / gflop - 1) < 5e-3, name
         assert a["eff_flops"] == 2 * a["pv_flops"] == a["pv_flops"] + a["qk_ops"]
     assert round(bench.algorithmic(WORKLOADS["dit_xl_1024"], False)["bytes"] / 1e6, 1) == 41.9
+    # one bias per batch entry: 2 x 16 x 4096^2 bf16 values (1073.7 MB) in place of 536.9 MB
+    assert round(bench.algorithmic(WORKLOADS["dit_xl_1024"], True, bias_per_sample=True)["bytes"] / 1e6, 1) == 1115.7
 
 
 def test_rank_inputs_heads_shard_one_batch():
