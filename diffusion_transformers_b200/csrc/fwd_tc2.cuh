@@ -1,7 +1,8 @@
 // fwd_tc2.cuh — the TMA-fed forward pipeline with e4m3 +-1 operands for the
-// binary QK^T: the binary forward (with a dense bias, a relative-position
-// table bias, or none), its 8-bit P.V passes, its debug-scores variant, and
-// the bf16 reference attention on the same pipeline.
+// binary QK^T: the binary forward (with a dense bias shared over the batch or
+// one per batch entry, a relative-position table bias, or none), its 8-bit P.V
+// passes, its debug-scores variant, and the bf16 reference attention on the
+// same pipeline.
 //
 // Source: "BinaryAttention: One-Bit QK-Attention for Vision and Diffusion
 // Transformers", §2 methodology (scaled binary Q/K, XNOR/popcount similarity,
