@@ -8,7 +8,9 @@ softmax; one [N, N] plane per head is this library's reading of its shape).
 So one forward splits across g ranks with no exchange
 step: rank r takes heads [h0, h1) = [r*H//g, (r+1)*H//g), holds only its
 slices Q, K, V [B, h1-h0, N, d] and bias [h1-h0, N, N] (the dense bias, the
-largest tensor of the call, is never replicated), and computes O[:, h0:h1].
+largest tensor of the call, is never replicated; a per-sample bias
+[B, H, N, N] is sliced the same way on its head axis), and computes
+O[:, h0:h1].
 O stays sharded where the next layer consumes it; gather_heads() puts it back
 together on every rank for callers that want it whole.
 
@@ -45,12 +47,15 @@ def slice_heads(x, h0: int, h1: int, axis: int):
 
 def shard_inputs(inp: dict, world: int, rank: int) -> dict:
     """This rank's part of a make_inputs() dictionary: Q, K, V sliced on the
-    head axis, the bias on its first axis, H replaced by the slice's size."""
+    head axis, the bias on its head axis (the first of a shared [H, N, N]
+    bias, the second of a per-sample [B, H, N, N] one), H replaced by the
+    slice's size."""
     h0, h1 = head_range(inp["H"], world, rank)
     out = dict(inp)
     for key in ("q", "k", "v"):
         out[key] = slice_heads(inp[key], h0, h1, 1)
-    out["bias"] = slice_heads(inp.get("bias"), h0, h1, 0)
+    bias = inp.get("bias")
+    out["bias"] = slice_heads(bias, h0, h1, 1 if bias is not None and bias.ndim == 4 else 0)
     out["H"] = h1 - h0
     out["heads"] = (h0, h1)
     return out

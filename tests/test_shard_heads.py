@@ -3,7 +3,8 @@
 Every (b, h) is independent, so each rank computes its heads' slice with the
 oracle and the gathered result must equal the unsharded oracle bit for bit
 (the oracle computes every query row the same way whatever else is in the
-call). Two gloo ranks, even and uneven head counts.
+call). Two gloo ranks, even and uneven head counts, a shared bias and one
+bias per batch entry.
 """
 import os
 import socket
@@ -42,6 +43,11 @@ def test_shard_inputs_slices_the_head_axes():
     assert np.array_equal(s["q"], c["q"][:, 2:5]) and s["q"].flags.c_contiguous
     assert np.array_equal(s["bias"], c["bias"][2:5])
     assert shard.shard_inputs(dict(c, bias=None), 2, 0)["bias"] is None
+    # one bias per batch entry [B, H, N, N]: sliced on its head axis
+    from diffusion_transformers_b200.synthetic import per_sample_bias
+    pb = per_sample_bias(2, 5, 16, seed=3)
+    sp = shard.shard_inputs(dict(c, bias=pb), 2, 1)
+    assert np.array_equal(sp["bias"], pb[:, 2:5]) and sp["bias"].flags.c_contiguous
 
 
 def _free_port():
@@ -50,7 +56,16 @@ def _free_port():
         return sk.getsockname()[1]
 
 
-def _worker(rank, world, port, H, out):
+def _oracle_forward(orc, c, bias, scale):
+    """The oracle's forward; a per-sample bias [B, H, N, N] runs it per batch
+    entry with that entry's bias."""
+    if bias is None or bias.ndim == 3:
+        return orc.forward(c["q"], c["k"], bias, c["v"], scale)
+    return np.concatenate([orc.forward(c["q"][b:b + 1], c["k"][b:b + 1], bias[b], c["v"][b:b + 1], scale)
+                           for b in range(bias.shape[0])])
+
+
+def _worker(rank, world, port, H, per_sample, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import datetime
 
@@ -63,21 +78,24 @@ def _worker(rank, world, port, H, out):
         orc.set_num_threads(1)
         c = make_custom(2, H, 40, 72, seed=17, with_bias=True, bias_std=0.5)
         c["H"] = H
+        if per_sample:
+            from diffusion_transformers_b200.synthetic import per_sample_bias
+            c["bias"] = per_sample_bias(2, H, 40, seed=19)
         mine = shard.shard_inputs(c, world, rank)  # this rank holds only its slices
-        o_local = orc.forward(mine["q"], mine["k"], mine["bias"], mine["v"], c["softmax_scale"])
+        o_local = _oracle_forward(orc, mine, mine["bias"], c["softmax_scale"])
         o = shard.gather_heads(torch.from_numpy(o_local), H, world, rank)
-        full = orc.forward(c["q"], c["k"], c["bias"], c["v"], c["softmax_scale"])
+        full = _oracle_forward(orc, c, c["bias"], c["softmax_scale"])
         out[rank] = (bool(np.array_equal(o.numpy(), full)), tuple(o.shape), mine["heads"])
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("H", [4, 5])
-def test_two_ranks_gather_equals_unsharded_oracle(H):
+@pytest.mark.parametrize("H,per_sample", [(4, False), (5, False), (5, True)])
+def test_two_ranks_gather_equals_unsharded_oracle(H, per_sample):
     world = 2
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.start_processes(_worker, args=(world, _free_port(), H, out), nprocs=world, join=True,
+    mp.start_processes(_worker, args=(world, _free_port(), H, per_sample, out), nprocs=world, join=True,
                        start_method="spawn")
     for r in range(world):
         same, shape, heads = out[r]
