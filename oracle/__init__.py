@@ -65,12 +65,13 @@ class Oracle:
         lib.oracle_forward_int8_rows.argtypes = [V, V, I, V, V, D, L, L, L, L, L, _i64p, V]
         lib.oracle_forward_int8.argtypes = [V, V, I, V, V, D, L, L, L, L, V]
         lib.oracle_expand_relpos_bias.argtypes = [V, L, L, L, L, V]
+        lib.oracle_backward.argtypes = [V, V, I, V, V, V, D, L, L, L, L, V, V, V, V]
         lib.oracle_num_threads.restype = I
         lib.oracle_set_num_threads.argtypes = [I]
         for f in ("oracle_pack", "oracle_scores_rows", "oracle_probs_rows",
                   "oracle_forward_rows", "oracle_forward", "oracle_forward_spread",
                   "oracle_quantize_v", "oracle_forward_int8_rows", "oracle_forward_int8",
-                  "oracle_expand_relpos_bias"):
+                  "oracle_expand_relpos_bias", "oracle_backward"):
             getattr(lib, f).restype = I
         self.lib = lib
 
@@ -254,6 +255,28 @@ class Oracle:
         if rc:
             raise RuntimeError(f"oracle_expand_relpos_bias failed ({rc})")
         return out
+
+
+    # ------------------------------------------------------------ backward
+    def backward(self, q, k, bias, v, dO, softmax_scale, with_dbias: bool = True):
+        """Gradients for an upstream gradient dO (bf16 bits [B,H,N,d]): dV, ds,
+        dt fp64 [B,H,N,d] (ds, dt with respect to the scaled binary Q and K,
+        s = alpha_q sign(q), t = alpha_k sign(k)) and dbias fp64 [H,N,N] summed
+        over the batch (None unless with_dbias)."""
+        B, H, N, d = q.shape
+        q, k = self._qk(q, k)
+        v = self._bf16(v, "v", (B, H, N, d))
+        g = self._bf16(dO, "dO", (B, H, N, d))
+        b = self._bf16(bias, "bias", (H, N, N))
+        dV = np.zeros((B, H, N, d), dtype=np.float64)
+        ds = np.zeros((B, H, N, d), dtype=np.float64)
+        dt = np.zeros((B, H, N, d), dtype=np.float64)
+        db = np.zeros((H, N, N), dtype=np.float64) if with_dbias else None
+        rc = self.lib.oracle_backward(_ptr(q), _ptr(k), self._dtype_code(q), _ptr(b), _ptr(v), _ptr(g),
+                                      float(softmax_scale), B, H, N, d, _ptr(dV), _ptr(ds), _ptr(dt), _ptr(db))
+        if rc:
+            raise RuntimeError(f"oracle_backward failed ({rc})")
+        return dV, ds, dt, db
 
 
 _default: Oracle | None = None

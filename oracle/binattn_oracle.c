@@ -67,6 +67,22 @@
  *      table[h, R0], a patch query and a class key table[h, R0 + 1], class
  *      with class table[h, R0 + 2]. The table is bf16 [H, R0 + 3 n_cls].
  *
+ * The backward (oracle_backward) gives the gradients of a loss that the
+ * forward fixes exactly, for an upstream gradient dO = dLoss/dO (bf16
+ * [B, H, N, d]). With s_i = alpha_q_i * sigma(q_i) and t_j = alpha_k_j *
+ * sigma(k_j), the scaled binary representations of [ES] §2, the logit of
+ * step 4 is softmax_scale * <s_i, t_j> + bias[h, i, j], and:
+ *  11. dV_j = sum_i P_ij * dO_i;
+ *  12. dP_ij = <dO_i, V_j> and D_i = sum_j P_ij * dP_ij;
+ *  13. dlogit_ij = P_ij * (dP_ij - D_i), the softmax's Jacobian applied to dP;
+ *  14. ds_i = softmax_scale * sum_j dlogit_ij * t_j and
+ *      dt_j = softmax_scale * sum_i dlogit_ij * s_i;
+ *  15. dbias[h, i, j] = sum_b dlogit_bhij (one bias serves every b).
+ * Training ([ES] §2 "Entrenamiento y Optimización": quantisation-aware
+ * training with self-distillation; [KO] §2 다) also needs the gradient through
+ * sigma and the mean to q and k; the pages give no estimator for it, so the
+ * backward stops at s and t. Under the straight-through reading, dq = ds.
+ *
  * Parity pins for each function live in the CPU test suite (exhaustive sign
  * predicate, packbits layout, Hamming identity, closed forms, invariants and an
  * independent numpy formulation on small cases).
@@ -567,4 +583,92 @@ int oracle_expand_relpos_bias(const uint16_t *table, long H, long gh, long gw, l
         }
     }
     return 0;
+}
+
+/*
+ * Steps 11-15: gradients of the forward for an upstream gradient dO (bf16
+ * [B, H, N, d]), all fp64: dV, ds, dt [B, H, N, d] and, when dbias is not
+ * NULL, dbias [H, N, N] summed over b. bias is bf16 [H, N, N] or NULL (zero).
+ * Every (b, h) is computed with its full N x N matrices P and dlogit; the
+ * batch entries of one head run in order, so dbias sums them in order b.
+ */
+int oracle_backward(const void *q, const void *k, int qk_dtype, const uint16_t *bias,
+                    const uint16_t *v, const uint16_t *dO, double softmax_scale,
+                    long B, long H, long N, long d,
+                    double *dV, double *ds, double *dt, double *dbias)
+{
+    if (!q || !k || !v || !dO || !dV || !ds || !dt || d < 1 || N < 1 || B < 1 || H < 1)
+        return 1;
+    prep_t p;
+    if (prep_init(&p, q, k, qk_dtype, B, H, N, d)) {
+        prep_free(&p);
+        return 3;
+    }
+    int err = 0;
+    long h;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (h = 0; h < H; h++) {
+        double *P = (double *)malloc(sizeof(double) * (size_t)N * N);
+        double *dL = (double *)malloc(sizeof(double) * (size_t)N * N);
+        if (!P || !dL) {
+            free(P); free(dL);
+#pragma omp atomic write
+            err = 4;
+            continue;
+        }
+        if (dbias)
+            for (size_t e = 0; e < (size_t)N * N; e++)
+                dbias[(size_t)h * N * N + e] = 0.0;
+        for (long b = 0; b < B; b++) {
+            const size_t tok0 = ((size_t)b * H + (size_t)h) * (size_t)N; /* token of (b, h, 0) */
+            /* steps 3-5: the probabilities of every row */
+            for (long i = 0; i < N; i++)
+                probs_row(&p, tok0 + (size_t)i, bias, softmax_scale, P + (size_t)i * N);
+            /* steps 12-13 */
+            for (long i = 0; i < N; i++) {
+                double Di = 0.0;
+                for (long j = 0; j < N; j++) {
+                    double dP = 0.0;
+                    for (long c = 0; c < d; c++)
+                        dP += load_elem(dO, ORACLE_BF16, (tok0 + i) * d + c) *
+                              load_elem(v, ORACLE_BF16, (tok0 + j) * d + c);
+                    dL[(size_t)i * N + j] = dP;
+                    Di += P[(size_t)i * N + j] * dP;
+                }
+                for (long j = 0; j < N; j++)
+                    dL[(size_t)i * N + j] = P[(size_t)i * N + j] * (dL[(size_t)i * N + j] - Di);
+            }
+            /* step 11 */
+            for (long j = 0; j < N; j++)
+                for (long c = 0; c < d; c++) {
+                    double acc = 0.0;
+                    for (long i = 0; i < N; i++)
+                        acc += P[(size_t)i * N + j] * load_elem(dO, ORACLE_BF16, (tok0 + i) * d + c);
+                    dV[(tok0 + j) * d + c] = acc;
+                }
+            /* step 14: t_j = alpha_k_j sigma(k_j), s_i = alpha_q_i sigma(q_i) */
+            for (long i = 0; i < N; i++)
+                for (long c = 0; c < d; c++) {
+                    double acc = 0.0;
+                    for (long j = 0; j < N; j++)
+                        acc += dL[(size_t)i * N + j] * p.ak[tok0 + j] * p.sk[(tok0 + j) * d + c];
+                    ds[(tok0 + i) * d + c] = softmax_scale * acc;
+                }
+            for (long j = 0; j < N; j++)
+                for (long c = 0; c < d; c++) {
+                    double acc = 0.0;
+                    for (long i = 0; i < N; i++)
+                        acc += dL[(size_t)i * N + j] * p.aq[tok0 + i] * p.sq[(tok0 + i) * d + c];
+                    dt[(tok0 + j) * d + c] = softmax_scale * acc;
+                }
+            /* step 15 */
+            if (dbias)
+                for (size_t e = 0; e < (size_t)N * N; e++)
+                    dbias[(size_t)h * N * N + e] += dL[e];
+        }
+        free(P);
+        free(dL);
+    }
+    prep_free(&p);
+    return err;
 }

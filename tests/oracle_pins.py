@@ -488,6 +488,125 @@ def pin_relpos_translation_invariance(orc):
         assert sorted(seen.values()) == sorted(_f64(t)[h].tolist())
 
 
+# ---------------------------------------------------- the backward (row f4)
+def _loss(orc, q, k, bias, v, dO, scale) -> float:
+    """The scalar loss sum(dO * O) whose gradients the backward returns."""
+    return float((orc.forward(q, k, bias, v, scale) * _f64(dO)).sum())
+
+
+def _grad_of_definition(q, k, bias, v, dO, scale, H, N):
+    """Gradients of sum(dO * O) by torch's automatic differentiation (fp64) of
+    the forward's matrix form, with s = alpha_q sign(q), t = alpha_k sign(k),
+    V and the bias as the leaves."""
+    import torch
+    qf, kf = _f64(q), _f64(k)
+    s = torch.tensor(np.abs(qf).mean(-1)[..., None] * np.where(qf >= 0, 1.0, -1.0), requires_grad=True)
+    t = torch.tensor(np.abs(kf).mean(-1)[..., None] * np.where(kf >= 0, 1.0, -1.0), requires_grad=True)
+    V = torch.tensor(_f64(v), requires_grad=True)
+    b = torch.tensor(_f64(bias) if bias is not None else np.zeros((H, N, N)), requires_grad=True)
+    L = scale * (s @ t.transpose(-1, -2)) + b
+    O = torch.softmax(L, dim=-1) @ V
+    (O * torch.tensor(_f64(dO))).sum().backward()
+    return V.grad.numpy(), s.grad.numpy(), t.grad.numpy(), b.grad.numpy()
+
+
+def pin_backward_autograd(orc):
+    """dV, ds, dt and dbias (summed over the batch) equal what automatic
+    differentiation of the forward's definition gives, on small shapes with
+    and without a bias (a zero bias still has a gradient)."""
+    rng = np.random.default_rng(41)
+    for (B, H, N, d) in [(1, 1, 1, 1), (2, 2, 3, 5), (1, 3, 8, 72), (2, 1, 8, 33), (3, 2, 7, 64)]:
+        for with_bias in (False, True):
+            c = make_custom(B, H, N, d, seed=int(rng.integers(1 << 30)), qk_dtype="bf16",
+                            with_bias=with_bias, bias_std=0.7, zeros_frac=0.1)
+            dO = f32_to_bf16_bits(rng.standard_normal((B, H, N, d)).astype(np.float32))
+            got = orc.backward(c["q"], c["k"], c["bias"], c["v"], dO, c["softmax_scale"])
+            want = _grad_of_definition(c["q"], c["k"], c["bias"], c["v"], dO, c["softmax_scale"], H, N)
+            for name, g, w in zip(("dV", "ds", "dt", "dbias"), got, want):
+                assert g.shape == w.shape, name
+                assert np.allclose(g, w, rtol=1e-10, atol=1e-13), f"{name} differs from autograd at {B,H,N,d}"
+
+
+def pin_backward_invariants(orc):
+    """Rows of dlogit (so of dbias) sum to 0, because softmax rows sum to 1;
+    sum_j dV_j = sum_i dO_i; at softmax_scale 0 the scaled binary Q and K get
+    no gradient, and with no bias the attention is uniform, so dV_j is the
+    mean of dO over the rows; doubling dO doubles every gradient."""
+    B, H, N, d = 2, 2, 37, 40
+    c = make_custom(B, H, N, d, seed=5, with_bias=True, bias_std=0.8)
+    rng = np.random.default_rng(6)
+    dO = f32_to_bf16_bits(rng.standard_normal((B, H, N, d)).astype(np.float32))
+    dV, ds, dt, db = orc.backward(c["q"], c["k"], c["bias"], c["v"], dO, c["softmax_scale"])
+    assert np.abs(db.sum(-1)).max() <= 1e-13 * max(1.0, np.abs(db).max()) * N, "dbias rows do not sum to 0"
+    assert np.allclose(dV.sum(2), _f64(dO).sum(2), rtol=1e-12, atol=1e-12), "sum_j dV_j != sum_i dO_i"
+    _, ds0, dt0, _ = orc.backward(c["q"], c["k"], c["bias"], c["v"], dO, 0.0)
+    assert not ds0.any() and not dt0.any(), "scale 0 must give ds = dt = 0"
+    dV0, _, _, _ = orc.backward(c["q"], c["k"], None, c["v"], dO, 0.0)
+    want = np.broadcast_to(_f64(dO).mean(2, keepdims=True), dV0.shape)
+    assert np.allclose(dV0, want, rtol=1e-13, atol=1e-15), "uniform attention: dV_j != mean_i dO_i"
+    dO2 = f32_to_bf16_bits(2 * bf16_bits_to_f32(dO))  # exact in bf16
+    for g1, g2 in zip(orc.backward(c["q"], c["k"], c["bias"], c["v"], dO, c["softmax_scale"]),
+                      orc.backward(c["q"], c["k"], c["bias"], c["v"], dO2, c["softmax_scale"])):
+        assert np.allclose(g2, 2 * g1, rtol=1e-13, atol=1e-15), "not linear in dO"
+
+
+def pin_backward_finite_differences(orc):
+    """Differences of the forward oracle's loss sum(dO * O), on inputs with
+    few significant bits so that every perturbed input below is exact:
+    - the loss is linear in V, so one step of V_jc gives dV_jc exactly;
+    - scaling query row i by lambda scales alpha_q_i (its signs stay), so
+      dloss/dlambda = <ds_i, s_i>; likewise key row j gives <dt_j, t_j>;
+    - adding delta to the bias column of key j in every row of head h gives
+      sum_i dbias[h, i, j].
+    The last three use Richardson extrapolation of central differences."""
+    B, H, N, d = 1, 2, 12, 24
+    rng = np.random.default_rng(77)
+    q = (rng.integers(-120, 121, size=(B, H, N, d)) / 64).astype(np.float32)
+    k = (rng.integers(-120, 121, size=(B, H, N, d)) / 64).astype(np.float32)
+    v = f32_to_bf16_bits((rng.integers(-60, 61, size=(B, H, N, d)) / 16).astype(np.float32))
+    bias = f32_to_bf16_bits((rng.integers(-200, 201, size=(H, N, N)) / 256).astype(np.float32))
+    dO = f32_to_bf16_bits(rng.standard_normal((B, H, N, d)).astype(np.float32))
+    scale = 0.3
+    dV, ds, dt, db = orc.backward(q, k, bias, v, dO, scale)
+    base = _loss(orc, q, k, bias, v, dO, scale)
+
+    def richardson(f, e):
+        d1 = (f(e) - f(-e)) / (2 * e)
+        d2 = (f(2 * e) - f(-2 * e)) / (4 * e)
+        return (4 * d1 - d2) / 3
+
+    for (h, j, c_) in [(0, 0, 0), (1, 11, 23), (1, 5, 7)]:
+        v2 = bf16_bits_to_f32(v).copy()
+        v2[0, h, j, c_] += np.float32(1 / 16)
+        fd = (_loss(orc, q, k, bias, f32_to_bf16_bits(v2), dO, scale) - base) * 16
+        assert abs(fd - dV[0, h, j, c_]) <= 1e-9 * (1 + abs(fd)), f"dV[{h},{j},{c_}]"
+    s = np.abs(q.astype(np.float64)).mean(-1)[..., None] * np.where(q >= 0, 1.0, -1.0)
+    t = np.abs(k.astype(np.float64)).mean(-1)[..., None] * np.where(k >= 0, 1.0, -1.0)
+    e = 2.0 ** -12
+    for (h, i) in [(0, 0), (1, 7), (0, 11)]:
+        def fq(x, h=h, i=i):
+            q2 = q.copy()
+            q2[0, h, i] = q[0, h, i] * np.float32(1 + x)
+            return _loss(orc, q2, k, bias, v, dO, scale)
+
+        def fk(x, h=h, i=i):
+            k2 = k.copy()
+            k2[0, h, i] = k[0, h, i] * np.float32(1 + x)
+            return _loss(orc, q, k2, bias, v, dO, scale)
+        want_q = float((ds[0, h, i] * s[0, h, i]).sum())
+        want_k = float((dt[0, h, i] * t[0, h, i]).sum())
+        assert abs(richardson(fq, e) - want_q) <= 1e-8 * (1 + abs(want_q)), f"<ds, s> at row {h},{i}"
+        assert abs(richardson(fk, e) - want_k) <= 1e-8 * (1 + abs(want_k)), f"<dt, t> at row {h},{i}"
+    delta = 2.0 ** -8
+    for (h, j) in [(0, 0), (1, 6), (1, 11)]:
+        def fb(x, h=h, j=j):
+            b2 = bf16_bits_to_f32(bias).copy()
+            b2[h, :, j] += np.float32(x)
+            return _loss(orc, q, k, f32_to_bf16_bits(b2), v, dO, scale)
+        want_b = float(db[h, :, j].sum())
+        assert abs(richardson(fb, delta) - want_b) <= 1e-7 * (1 + abs(want_b)), f"dbias column {h},{j}"
+
+
 ALL_PINS = [
     pin_sign_predicate_exhaustive,
     pin_pack_layout_packbits,
@@ -513,4 +632,7 @@ ALL_PINS = [
     pin_int8_two_keys_closed_form,
     pin_relpos_one_hot_counts,
     pin_relpos_translation_invariance,
+    pin_backward_autograd,
+    pin_backward_invariants,
+    pin_backward_finite_differences,
 ]

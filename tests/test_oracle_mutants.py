@@ -75,6 +75,24 @@ MUTANTS = [
      "idx = (dy + gh - 1) * (2 * gw - 1) + (dx + gw - 1);", "idx = (dy + gh - 1) * gw + (dx + gw - 1);"),
     ("class entries swapped",
      "idx = R0;\n", "idx = R0 + 1;\n"),
+    ("backward without the softmax's D_i term",
+     "dL[(size_t)i * N + j] = P[(size_t)i * N + j] * (dL[(size_t)i * N + j] - Di);",
+     "dL[(size_t)i * N + j] = P[(size_t)i * N + j] * dL[(size_t)i * N + j];"),
+    ("dV from the transposed probabilities",
+     "acc += P[(size_t)i * N + j] * load_elem(dO,", "acc += P[(size_t)j * N + i] * load_elem(dO,"),
+    ("ds without softmax_scale",
+     "ds[(tok0 + i) * d + c] = softmax_scale * acc;", "ds[(tok0 + i) * d + c] = acc;"),
+    ("ds against the query's own signs",
+     "acc += dL[(size_t)i * N + j] * p.ak[tok0 + j] * p.sk[(tok0 + j) * d + c];",
+     "acc += dL[(size_t)i * N + j] * p.ak[tok0 + j] * p.sq[(tok0 + i) * d + c];"),
+    ("dt from the rows of dlogit",
+     "acc += dL[(size_t)i * N + j] * p.aq[tok0 + i] * p.sq[(tok0 + i) * d + c];",
+     "acc += dL[(size_t)j * N + i] * p.aq[tok0 + i] * p.sq[(tok0 + i) * d + c];"),
+    ("dbias of the last batch entry only",
+     "dbias[(size_t)h * N * N + e] += dL[e];", "dbias[(size_t)h * N * N + e] = dL[e];"),
+    ("dbias transposed",
+     "dbias[(size_t)h * N * N + e] += dL[e];",
+     "dbias[(size_t)h * N * N + (e % N) * N + e / N] += dL[e];"),
 ]
 
 
