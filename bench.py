@@ -96,6 +96,20 @@ def algorithmic(w, with_bias=True, bias_per_sample=False):
                 eff_flops=4 * d * pairs, bytes=bytes_, pack_bytes=pack_bytes)
 
 
+def algorithmic_backward(w):
+    """Algorithmic work of one backward call with the dense bias: the packed Q
+    and K, alphas, V and dO read once, the bias read once, dV, ds, dt (fp32)
+    and dbias (fp32, summed over b) written once; one binary QK^T recomputed
+    (2d ops per pair) and four products of the P.V kind (dP, dV, ds, dt: 2d
+    flops per pair each)."""
+    BH, N, d = w.B * w.H, w.N, w.d
+    pairs = BH * N * N
+    W = (d + 31) // 32
+    bytes_ = (2 * BH * N * W * 4 + 2 * BH * N * 4 + 2 * BH * N * d * 2 + w.H * N * N * 2
+              + 3 * BH * N * d * 4 + w.H * N * N * 4)
+    return dict(pairs=pairs, qk_ops=2 * d * pairs, pv_like_flops=8 * d * pairs, bytes=bytes_)
+
+
 # The binary QK^T runs on tcgen05.mma kind::f8f6f4 with e4m3 +-1 operands. Its
 # dense rate is twice the bf16 rate (NVIDIA's nominal 4.5 against 2.25 PFLOP/s
 # per GPU; on this part an e4m3 M=128 N=128 K=32 MMA and a bf16 M=128 N=128
@@ -146,14 +160,15 @@ def roofline_line(w, with_bias, peaks, fwd_s, n_sm=148, sm_mhz=None, bias_per_sa
 # DRAM traffic of one forward call from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum summed over the launches the call makes at dit_xl_1024
 # with bias: the full-wave launch, the key-split tail launch and the combine; the
-# summary is profiles/fwd_tc2_dit_xl_1024_bias.md; "sample_bias" is the same call
-# with one bias per batch entry, profiles/sample_bias_dit_xl_1024.md), valid only for the kernel
+# summary is profiles/fwd_tc2_dit_xl_1024_bias.md; the same call with one bias per
+# batch entry was captured on earlier sources, profiles/sample_bias_dit_xl_1024.md),
+# valid only for the kernel
 # sources it was taken on: any change to their code turns the reported traffic
 # back into null. The digest covers the code only (comments removed, runs of
 # white space collapsed), so an edit of a comment keeps the capture valid.
 NCU_TRAFFIC = {
-    "sources_sha256": "9db1fb6cea252ee688aca9260fec0d6498dee55b041dd7b426fb35016c103357",
-    "bytes_per_call": {"dit_xl_1024/bias": 588_756_480, "dit_xl_1024/sample_bias": 1_126_140_672},
+    "sources_sha256": "83b3d65fe546d7e5c9b94a48d41a5bf70cd6c61a101ce6082a566e9918cb02a2",
+    "bytes_per_call": {"dit_xl_1024/bias": 588_474_624},
 }
 
 _C_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'|//[^\n]*|/\*.*?\*/', re.S)
@@ -778,6 +793,45 @@ def run_gpu(args, w_job, rank, world, local_rank):
                           "algorithmic_bytes": algorithmic(w, True, bias_per_sample=True)["bytes"]}}
         del sb, sws
 
+    # the backward (binattn_backward: dV, the gradients of the scaled binary
+    # Q and K, and dbias summed over the batch) for an upstream gradient dO,
+    # timed over a few calls with a cold L2
+    backward = None
+    try:
+        grng = np.random.default_rng(rank_seed(w, rank) + 99)
+        gO = torch.from_numpy(grng.standard_normal((B, H, N, d), dtype=np.float32)).to(dev).bfloat16()
+        bws = torch.empty(max(16, binattn.lib().binattn_backward_workspace_bytes(B, H, N, d)), dtype=torch.uint8,
+                          device=dev)
+        fb = lambda: binattn.backward(qb, kb, aq, ak, bias, v, gO, scale, workspace=bws, stream=stream)
+        fb()
+        torch.cuda.synchronize()
+        barrier()
+        ev = []
+        for _ in range(min(args.steps, 3)):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fb()
+            e1.record(stream)
+            ev.append((e0, e1))
+        torch.cuda.synchronize()
+        barrier()
+        binattn.device_status(stream)
+        bms = max_over_ranks(sum(a.elapsed_time(c) for a, c in ev) / len(ev))
+        ab = algorithmic_backward(w)
+        t_mem = ab["bytes"] / (peaks["hbm_gbs"] * 1e9)
+        t_tensor = ab["pv_like_flops"] / (peaks["bf16_tflops"] * 1e12) + \
+            ab["qk_ops"] / (E4M3_OVER_BF16 * peaks["bf16_tflops"] * 1e12)
+        t_roof = max(t_mem, t_tensor)
+        backward = {"call": "binattn_backward (CUDA cores: rows kernel, columns kernel)", "ms": round(bms, 4),
+                    "calls_timed": len(ev), "algorithmic_bytes": ab["bytes"],
+                    "roofline": {"bound": "hbm" if t_mem >= t_tensor else "tensor",
+                                 "t_roof_us": round(t_roof * 1e6, 2), "t_mem_us": round(t_mem * 1e6, 2),
+                                 "t_tensor_us": round(t_tensor * 1e6, 2), "frac": round(t_roof / (bms * 1e-3), 5)}}
+        del gO, bws
+    except Exception as exc:  # reported, not fatal: the forward's numbers stand on their own
+        backward = {"unavailable": str(exc).splitlines()[0]}
+
     # in-build bf16 attention on the same shapes (speed reference), with the
     # binary forward's launch plan (binattn_ref_bf16_forward_ws: persistent
     # whole pairs, split tail) and, beside it, without the workspace
@@ -889,6 +943,7 @@ def run_gpu(args, w_job, rank, world, local_rank):
         "bf16_reference": ref,
         "relpos_bias": relpos,
         "per_sample_bias": sample_bias,
+        "backward": backward,
         "int8_pv": dict(int8, call="binattn_forward_int8 (V 8-bit code + row-max pass + 8-bit P.V pass)",
                         step="pack(Q) + pack(K) + binattn_forward_int8"),
         "other_workloads": others,

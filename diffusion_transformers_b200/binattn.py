@@ -33,6 +33,7 @@ EXPORTS = (
     "binattn_forward_relpos_workspace_bytes", "binattn_forward_relpos",
     "binattn_ref_bf16_forward_workspace_bytes", "binattn_ref_bf16_forward_ws",
     "binattn_forward_sample_bias_workspace_bytes", "binattn_forward_sample_bias_ws",
+    "binattn_backward_workspace_bytes", "binattn_backward",
 )
 
 
@@ -76,6 +77,10 @@ def lib() -> ctypes.CDLL:
     L.binattn_forward_sample_bias_workspace_bytes.restype = ctypes.c_size_t
     L.binattn_forward_sample_bias_ws.argtypes = [P, P, P, P, P, I, P, F, I, I, I, I, P, P, ctypes.c_size_t, P]
     L.binattn_forward_sample_bias_ws.restype = I
+    L.binattn_backward_workspace_bytes.argtypes = [I, I, I, I]
+    L.binattn_backward_workspace_bytes.restype = ctypes.c_size_t
+    L.binattn_backward.argtypes = [P, P, P, P, P, P, P, F, I, I, I, I, P, P, P, P, P, ctypes.c_size_t, P]
+    L.binattn_backward.restype = I
     L.binattn_quantize_v.argtypes = [P, I, I, I, I, P, P, P]
     L.binattn_quantize_v.restype = I
     L.binattn_forward_int8_workspace_bytes.argtypes = [I, I, I, I, I]
@@ -336,6 +341,34 @@ def forward_sample_bias_ws(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: 
                                                     _stream(stream, dev)),
                "binattn_forward_sample_bias_ws")
     return out
+
+
+def backward(q_bits: torch.Tensor, k_bits: torch.Tensor, alpha_q: torch.Tensor, alpha_k: torch.Tensor,
+             bias: torch.Tensor | None, v: torch.Tensor, dO: torch.Tensor, softmax_scale: float,
+             with_dbias: bool = True, workspace: torch.Tensor | None = None, stream=None):
+    """Gradients of the forward for an upstream gradient dO (bf16 [B,H,N,d]):
+    (dV, ds, dt, dbias), dV/ds/dt fp32 [B,H,N,d] (ds, dt with respect to the
+    scaled binary Q and K, alpha * sign), dbias fp32 [H,N,N] summed over the
+    batch, or None without with_dbias."""
+    B, H, N, d = v.shape
+    dev = _forward_args(q_bits, k_bits, alpha_q, alpha_k, bias, v, None)
+    _expect(dO, "dO", (B, H, N, d), (torch.bfloat16,))
+    _device(dO, v)
+    if workspace is not None:
+        _device(workspace, v)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dV, ds, dt = (torch.empty((B, H, N, d), **f32) for _ in range(3))
+    dbias = torch.empty((H, N, N), **f32) if with_dbias else None
+    need = int(lib().binattn_backward_workspace_bytes(B, H, N, d))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    size = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        _check(lib().binattn_backward(_ptr(q_bits), _ptr(k_bits), _ptr(alpha_q), _ptr(alpha_k), _ptr(bias), _ptr(v),
+                                      _ptr(dO), float(softmax_scale), B, H, N, d, _ptr(dV), _ptr(ds), _ptr(dt),
+                                      _ptr(dbias), _ptr(workspace), ctypes.c_size_t(size), _stream(stream, dev)),
+               "binattn_backward")
+    return dV, ds, dt, dbias
 
 
 def quantize_v(v: torch.Tensor, stream=None):

@@ -16,6 +16,7 @@
 #include "fwd_tc.cuh"
 #include "fwd_tc2.cuh"
 #include "quantv.cuh"
+#include "bwd_simt.cuh"
 
 namespace {
 
@@ -666,6 +667,42 @@ int binattn_test_wait_timeout(const uint32_t* q_bits, const uint32_t* k_bits, co
   const int rc = binattn::forward_tc2(q_bits, k_bits, alpha_q, alpha_k, bias, v, softmax_scale, B, H, N, d, out,
                                       static_cast<cudaStream_t>(stream), &msg, 0, nullptr, nullptr, stall_after);
   if (rc) return fail(rc, "%s", msg.c_str());
+  return ok();
+}
+
+size_t binattn_backward_workspace_bytes(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || d < 1 || d > 128 || static_cast<long long>(B) * H > 65535 || N > 65535) return 0;
+  // LSE and D, one float each per query row
+  return (2 * static_cast<size_t>(B) * H * N * sizeof(float) + 255) / 256 * 256;
+}
+
+int binattn_backward(const uint32_t* q_bits, const uint32_t* k_bits, const float* alpha_q, const float* alpha_k,
+                     const uint16_t* bias, const uint16_t* v, const uint16_t* dO, float softmax_scale, int B, int H,
+                     int N, int d, float* dV, float* ds, float* dt, float* dbias, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  BINATTN_CHECK_PTR(q_bits);
+  BINATTN_CHECK_PTR(k_bits);
+  BINATTN_CHECK_PTR(alpha_q);
+  BINATTN_CHECK_PTR(alpha_k);
+  BINATTN_CHECK_PTR(v);
+  BINATTN_CHECK_PTR(dO);
+  BINATTN_CHECK_PTR(dV);
+  BINATTN_CHECK_PTR(ds);
+  BINATTN_CHECK_PTR(dt);
+  BINATTN_CHECK_PTR(workspace);
+  if (bias && !aligned16(bias)) return fail(BINATTN_ERR_ALIGN, "bias is not 16-byte aligned");
+  if (dbias && !aligned16(dbias)) return fail(BINATTN_ERR_ALIGN, "dbias is not 16-byte aligned");
+  if (!std::isfinite(softmax_scale)) return fail(BINATTN_ERR_ARG, "softmax_scale is not finite");
+  if (int rc = check_shape(B, H, N, d)) return rc;
+  const size_t need = binattn_backward_workspace_bytes(B, H, N, d);
+  if (workspace_bytes < need)
+    return fail(BINATTN_ERR_ARG, "workspace of %zu bytes is below the %zu this shape needs", workspace_bytes, need);
+  float* lse = static_cast<float*>(workspace);
+  float* D = lse + static_cast<size_t>(B) * H * N;
+  std::string msg;
+  if (binattn::bwd::backward(q_bits, k_bits, alpha_q, alpha_k, bias, v, dO, softmax_scale, B, H, N, d, dV, ds, dt,
+                             dbias, lse, D, static_cast<cudaStream_t>(stream), &msg))
+    return fail(BINATTN_ERR_CUDA, "%s", msg.c_str());
   return ok();
 }
 

@@ -163,3 +163,10 @@ def per_sample_bias(B: int, H: int, N: int, seed: int, bias_std: float = 0.5,
         return np.stack([np.roll(base, -b, axis=0) for b in range(B)])
     rng = np.random.default_rng(seed)
     return f32_to_bf16_bits(rng.standard_normal(size=(B, H, N, N), dtype=np.float32) * np.float32(bias_std))
+
+
+def upstream_grad(B: int, H: int, N: int, d: int, seed: int) -> np.ndarray:
+    """An upstream gradient dLoss/dO for the backward, bf16 bits [B, H, N, d]:
+    N(0, 1) draws from default_rng(seed)."""
+    rng = np.random.default_rng(seed)
+    return f32_to_bf16_bits(rng.standard_normal(size=(B, H, N, d), dtype=np.float32))

@@ -373,6 +373,41 @@ int binattn_forward_relpos(const uint32_t *q_bits, const uint32_t *k_bits,
                            uint16_t *out, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * binattn_backward — the gradients of the forward (binattn_forward's result,
+ * with exact fp32 softmax weights) for an upstream gradient dO = dLoss/dO.
+ * With c = softmax_scale, s_i = alpha_q_i * sign(q_i) and t_j = alpha_k_j *
+ * sign(k_j) (the scaled binary Q and K), logit_ij = c <s_i, t_j> + bias[h,i,j]
+ * and P = softmax_j(logit):
+ *   dV_j = sum_i P_ij dO_i
+ *   dlogit_ij = P_ij (<dO_i, V_j> - D_i),  D_i = sum_j P_ij <dO_i, V_j>
+ *   ds_i = c sum_j dlogit_ij t_j,  dt_j = c sum_i dlogit_ij s_i
+ *   dbias[h, i, j] = sum_b dlogit_bhij
+ * The gradient stops at s and t: how it reaches q and k through sign and the
+ * mean (the estimator of quantisation-aware training) is the caller's choice;
+ * with the straight-through estimator dq = ds and dk = dt.
+ *   q_bits, k_bits, alpha_q, alpha_k, bias, v   as binattn_forward.
+ *   dO     bf16 [B, H, N, d], device.
+ *   dV, ds, dt   fp32 [B, H, N, d], device, written.
+ *   dbias  fp32 [H, N, N], device, written (the gradient of a zero bias when
+ *          bias is NULL); NULL skips it. The sum over b runs in order b, so
+ *          the result does not depend on scheduling.
+ *   workspace  device, 16-byte aligned, at least
+ *          binattn_backward_workspace_bytes(B, H, N, d) bytes (the row
+ *          log-sum-exp and D, one float each per query row).
+ * Any d in 1..128. Runs on CUDA cores. Errors as binattn_forward, plus
+ * BINATTN_ERR_ARG for a workspace that is too small. Asynchronous on stream.
+ * Source: §2 methodology (the forward's steps) and its training bullet
+ * (quantisation-aware training with self-distillation, which needs them).
+ */
+size_t binattn_backward_workspace_bytes(int B, int H, int N, int d);
+int binattn_backward(const uint32_t *q_bits, const uint32_t *k_bits,
+                     const float *alpha_q, const float *alpha_k,
+                     const uint16_t *bias, const uint16_t *v, const uint16_t *dO,
+                     float softmax_scale, int B, int H, int N, int d,
+                     float *dV, float *ds, float *dt, float *dbias,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * binattn_scores_debug — writes the integer scores S [B, H, N, N] (int32,
  * device) that engine `engine` computes inside the forward pass, using the same
  * kernel and score routine. For testing only: it materialises the N x N matrix.

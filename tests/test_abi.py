@@ -102,6 +102,31 @@ def test_sample_bias_host_validation(L):
         assert L.binattn_forward_sample_bias_workspace_bytes(B, H, N, d, ld) == pad + shared - shared_pad
 
 
+def test_backward_host_validation(L):
+    def bwd(q=A, dO=A, dV=A, ds=A, dt=A, dbias=A, bias=None, ws=A, wsb=1 << 20, B=1, H=2, N=16, d=64,
+            scale=0.125):
+        return L.binattn_backward(P(q), P(A), P(A), P(A), P(bias) if bias else None, P(A), P(dO) if dO else None,
+                                  ctypes.c_float(scale), B, H, N, d, P(dV) if dV else None, P(ds) if ds else None,
+                                  P(dt) if dt else None, P(dbias) if dbias else None, P(ws) if ws else None,
+                                  ctypes.c_size_t(wsb), None)
+    assert bwd(q=0) == 1
+    assert bwd(dO=0) == 1
+    assert bwd(dV=0) == 1 and bwd(ds=0) == 1 and bwd(dt=0) == 1
+    assert bwd(ws=0) == 1                      # the workspace holds LSE and D
+    assert bwd(dbias=A + 4) == 4
+    assert bwd(bias=A + 2) == 4
+    assert bwd(dV=A + 8) == 4
+    assert bwd(N=0) == 2 and bwd(d=129) == 2 and bwd(B=300, H=300) == 2
+    assert bwd(scale=math.nan) == 8
+    assert bwd(wsb=255) == 8
+    assert b"workspace" in L.binattn_last_error_message()
+    # one float of LSE and one of D per query row, rounded up to 256 bytes
+    assert L.binattn_backward_workspace_bytes(1, 2, 16, 64) == 256
+    assert L.binattn_backward_workspace_bytes(2, 16, 4096, 72) == 2 * 2 * 16 * 4096 * 4
+    assert L.binattn_backward_workspace_bytes(3, 5, 7, 1) == (2 * 3 * 5 * 7 * 4 + 255) // 256 * 256
+    assert L.binattn_backward_workspace_bytes(1, 1, 16, 129) == 0
+
+
 def test_relpos_host_validation(L):
     def fwd(table=A, gh=4, gw=4, ncls=0, N=16, d=64, ws=A):
         return L.binattn_forward_relpos(P(A), P(A), P(A), P(A), P(table) if table else None, gh, gw, ncls, P(A),
@@ -356,6 +381,13 @@ def test_binding_marshals_every_call(monkeypatch):
     assert args[4].value == sbias.data_ptr() and args[14].value == 32
     with pytest.raises(ValueError, match="bias must be"):
         binattn.forward_sample_bias_ws(qb, qb, aq, aq, bias, v, 0.25)
+    dV, ds, dt, db = binattn.backward(qb, qb, aq, aq, bias, v, q, 0.25)
+    name, args = calls[-1]
+    assert name == "binattn_backward" and args[8:12] == (B, H, N, d) and args[7] == 0.25
+    assert args[6].value == q.data_ptr() and args[12].value == dV.data_ptr() and args[15].value == db.data_ptr()
+    assert dV.dtype == torch.float32 and dV.shape == (B, H, N, d) and db.shape == (H, N, N)
+    binattn.backward(qb, qb, aq, aq, None, v, q, 0.25, with_dbias=False)
+    assert calls[-1][1][4] is None and calls[-1][1][15] is None
 
 
 @pytest.mark.parametrize("lang,std", [("c", "c99"), ("c++", "c++11")])
