@@ -40,7 +40,8 @@ constexpr int kT = 64;       // threads per block: query rows (rows kernel) or k
 constexpr int kTile = 64;    // keys (rows kernel) or query rows (cols kernel) staged per tile
 constexpr int kPitch = 65;   // pitch of the [channel][thread] arrays
 
-// Shared-memory floats of each kernel for head dim d (W sign words per token).
+// Dynamic shared memory of each kernel, in bytes, for head dim d (at most 4
+// sign words per token).
 inline size_t rows_smem_bytes(int d) {
   const size_t floats = 2 * static_cast<size_t>(d) * kPitch  // dO^T, ds accumulators
                         + static_cast<size_t>(kTile) * d     // V of the key tile
