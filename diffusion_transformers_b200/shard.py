@@ -12,7 +12,8 @@ largest tensor of the call, is never replicated; a per-sample bias
 [B, H, N, N] is sliced the same way on its head axis), and computes
 O[:, h0:h1].
 O stays sharded where the next layer consumes it; gather_heads() puts it back
-together on every rank for callers that want it whole.
+together on every rank for callers that want it whole. The backward splits the
+same way: a rank's dV, ds, dt and dbias are those of its heads.
 
 Host logic only: the kernels see an ordinary call with H = h1 - h0.
 """

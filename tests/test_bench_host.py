@@ -125,6 +125,11 @@ def test_algorithmic_work_matches_the_hand_figures():
     assert round(bench.algorithmic(WORKLOADS["dit_xl_1024"], False)["bytes"] / 1e6, 1) == 41.9
     # one bias per batch entry: 2 x 16 x 4096^2 bf16 values (1073.7 MB) in place of 536.9 MB
     assert round(bench.algorithmic(WORKLOADS["dit_xl_1024"], True, bias_per_sample=True)["bytes"] / 1e6, 1) == 1115.7
+    # the backward at DiT-1024: bits 3.1 MB + alphas 1.0 MB + V and dO 37.7 MB + bias 536.9 MB read,
+    # dV, ds, dt 113.2 MB + dbias (fp32) 1073.7 MB written; 4 products of 2d flops per pair
+    ab = bench.algorithmic_backward(WORKLOADS["dit_xl_1024"])
+    assert round(ab["bytes"] / 1e6, 1) == 1765.8
+    assert ab["pv_like_flops"] == 4 * 77_309_411_328 and ab["qk_ops"] == 77_309_411_328
 
 
 def test_rank_inputs_heads_shard_one_batch():

@@ -90,6 +90,48 @@ def _worker(rank, world, port, H, per_sample, out):
         dist.destroy_process_group()
 
 
+def _bwd_worker(rank, world, port, H, out):
+    # the backward partitions by heads the same way: each rank's dV, ds, dt
+    # [B, h1-h0, N, d] and dbias [h1-h0, N, N] (its heads' bias, summed over
+    # b on the rank) gathered on the head axis equal the unsharded backward
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import oracle
+    from diffusion_transformers_b200.synthetic import make_custom, upstream_grad
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    try:
+        orc = oracle.get()
+        orc.set_num_threads(1)
+        c = make_custom(2, H, 24, 40, seed=23, with_bias=True, bias_std=0.5)
+        c["H"] = H
+        c["dO"] = upstream_grad(2, H, 24, 40, seed=24)
+        mine = shard.shard_inputs(c, world, rank)
+        dO_mine = shard.slice_heads(c["dO"], *mine["heads"], 1)
+        g = orc.backward(mine["q"], mine["k"], mine["bias"], mine["v"], dO_mine, c["softmax_scale"])
+        full = orc.backward(c["q"], c["k"], c["bias"], c["v"], c["dO"], c["softmax_scale"])
+        same = []
+        for x, w in zip(g[:3], full[:3]):
+            same.append(bool(np.array_equal(shard.gather_heads(torch.from_numpy(x), H, world, rank).numpy(), w)))
+        # dbias carries heads on its first axis: gather it as [1, h1-h0, N, N]
+        db = shard.gather_heads(torch.from_numpy(g[3][None]), H, world, rank)[0].numpy()
+        same.append(bool(np.array_equal(db, full[3])))
+        out[rank] = tuple(same)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_backward_gather_equals_unsharded_oracle():
+    world, H = 2, 5
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_bwd_worker, args=(world, _free_port(), H, out), nprocs=world, join=True,
+                       start_method="spawn")
+    for r in range(world):
+        assert out[r] == (True, True, True, True), f"rank {r}: gathered gradients differ {out[r]}"
+
+
 @pytest.mark.parametrize("H,per_sample", [(4, False), (5, False), (5, True)])
 def test_two_ranks_gather_equals_unsharded_oracle(H, per_sample):
     world = 2
