@@ -1,5 +1,6 @@
 /*
- * binattn.h — C ABI of the BinaryAttention forward pass for NVIDIA B200 (sm_100a).
+ * binattn.h — C ABI of the BinaryAttention forward pass (and its backward) for
+ * NVIDIA B200 (sm_100a).
  *
  * The method ("BinaryAttention: One-Bit QK-Attention for Vision and Diffusion
  * Transformers", technical summaries, §2 Methodology) replaces the query/key
