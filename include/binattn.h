@@ -336,8 +336,8 @@ int binattn_forward_int8(const uint32_t *q_bits, const uint32_t *k_bits,
  * BINATTN_ERR_ARG when bias_ld < N or the workspace is too small; otherwise
  * errors as binattn_forward. With the same bias in every batch entry the
  * result equals binattn_forward_ws on that bias, bit for bit.
- * Source: §2 bias enhancement (the bias may be dense, position-sensitive or
- * context-aware).
+ * Source: §2 bias enhancement (dense, position-sensitive and context-aware
+ * forms of the bias are named).
  */
 size_t binattn_forward_sample_bias_workspace_bytes(int B, int H, int N, int d, int bias_ld);
 int binattn_forward_sample_bias_ws(const uint32_t *q_bits, const uint32_t *k_bits,
@@ -363,8 +363,8 @@ int binattn_forward_sample_bias_ws(const uint32_t *q_bits, const uint32_t *k_bit
  * Needs d % 8 == 0 and d <= 80. The result equals binattn_forward_ws with the
  * dense bias that the table expands to, bit for bit; the table replaces the
  * dense read of H N^2 bias elements by one of H R entries per CTA.
- * Source: §2 bias enhancement (the bias may be dense, position-sensitive or
- * context-aware).
+ * Source: §2 bias enhancement (dense, position-sensitive and context-aware
+ * forms of the bias are named).
  */
 size_t binattn_forward_relpos_workspace_bytes(int B, int H, int N, int d);
 int binattn_forward_relpos(const uint32_t *q_bits, const uint32_t *k_bits,

@@ -55,8 +55,8 @@
  *   9. O_ic = s_c * (sum_j u_ij vq_jc) / (sum_j u_ij), the row sum taken from
  *      the same 8-bit weights.
  *
- * The position-sensitive bias ([ES] §2 "Mejora mediante Sesgo": the bias may
- * be dense, position-sensitive or context-aware; [KO] §2 나-2) is read as a
+ * The position-sensitive bias ([ES] §2 "Mejora mediante Sesgo", which names
+ * dense, position-sensitive and context-aware forms; [KO] §2 나-2) is read as a
  * relative-position table, expanded to the dense bias by
  * oracle_expand_relpos_bias:
  *  10. tokens n_cls .. N - 1 are the patches of a gh x gw grid in row-major
